@@ -1,0 +1,222 @@
+"""ctypes wrapper of the C oracle (kq_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline / reference arm of ``bench.py`` use this module.  The product package
+never imports it.  It holds no arithmetic of its own: every function marshals
+numpy arrays into the C oracle and back.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kq_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libkq_oracle.so")
+
+F32 = 0
+BF16 = 1
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (plain -O2, no FMA contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < max(
+        os.path.getmtime(_SRC), os.path.getmtime(os.path.join(_HERE, "kq_oracle.h"))
+    ):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.kqo_factor.argtypes = [ctypes.c_float] * 3 + [P]
+        L.kqo_factor_inverse.argtypes = [ctypes.c_float] * 3 + [P]
+        L.kqo_kron.argtypes = [P, I, P, I, P]
+        L.kqo_expand_f64.argtypes = [P, I64, I, P]
+        L.kqo_expand.argtypes = [P, I64, I, I, P]
+        L.kqo_bf16_from_f64.argtypes = [ctypes.c_double]
+        L.kqo_bf16_from_f64.restype = ctypes.c_uint16
+        L.kqo_hadamard.argtypes = [I, P]
+        L.kqo_e8m0.argtypes = [ctypes.c_float]
+        L.kqo_e8m0.restype = I
+        L.kqo_e8m0_many.argtypes = [P, I64, P]
+        L.kqo_e8m0_many.restype = None
+        L.kqo_e2m1.argtypes = [ctypes.c_float]
+        L.kqo_e2m1.restype = I
+        L.kqo_e2m1_value.argtypes = [I]
+        L.kqo_e2m1_value.restype = ctypes.c_double
+        L.kqo_e2m1_pack.argtypes = [P, I64, P]
+        L.kqo_transform.argtypes = [P, I64, I64, I64, P, I, P]
+        L.kqo_mx_quantize.argtypes = [P, I64, I64, P, P]
+        L.kqo_quantize.argtypes = [P, I64, I64, I64, P, I, P, P]
+        L.kqo_smooth_quantize.argtypes = [P, I64, I64, I64, P, P, P]
+        L.kqo_fwht_quantize.argtypes = [P, I64, I64, I64, P, P]
+        L.kqo_dequantize.argtypes = [P, P, I64, I64, P, I, P]
+        for name in ("kqo_factor", "kqo_factor_inverse", "kqo_kron", "kqo_expand_f64", "kqo_expand",
+                     "kqo_hadamard", "kqo_e2m1_pack", "kqo_transform", "kqo_mx_quantize", "kqo_quantize",
+                     "kqo_smooth_quantize", "kqo_fwht_quantize", "kqo_dequantize"):
+            getattr(L, name).restype = None
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bf16_bits(x: np.ndarray) -> np.ndarray:
+    assert x.dtype == np.uint16, "activations are passed as bf16 bit patterns (uint16)"
+    return np.ascontiguousarray(x)
+
+
+def factor(l: float, u: float, v: float, inverse: bool = False) -> np.ndarray:
+    F = np.zeros(4, np.float64)
+    (lib().kqo_factor_inverse if inverse else lib().kqo_factor)(l, u, v, _p(F))
+    return F.reshape(2, 2)
+
+
+def kron(A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    A = np.ascontiguousarray(A, np.float64)
+    B = np.ascontiguousarray(B, np.float64)
+    out = np.zeros((A.shape[0] * B.shape[0],) * 2, np.float64)
+    lib().kqo_kron(_p(A), A.shape[0], _p(B), B.shape[0], _p(out))
+    return out
+
+
+def expand_f64(params: np.ndarray, inverse: bool = False) -> np.ndarray:
+    params = np.ascontiguousarray(params, np.float32).reshape(-1, 5, 3)
+    nb = params.shape[0]
+    K = np.zeros((nb, 32, 32), np.float64)
+    lib().kqo_expand_f64(_p(params), nb, int(inverse), _p(K))
+    return K
+
+
+def expand(params: np.ndarray, dtype: int = F32, inverse: bool = False) -> np.ndarray:
+    """fp32 matrices (dtype F32) or bf16 bit patterns as uint16 (dtype BF16)."""
+    params = np.ascontiguousarray(params, np.float32).reshape(-1, 5, 3)
+    nb = params.shape[0]
+    out = np.zeros((nb, 32, 32), np.float32 if dtype == F32 else np.uint16)
+    lib().kqo_expand(_p(params), nb, int(inverse), dtype, _p(out))
+    return out
+
+
+def bf16_from_f64(a: float) -> int:
+    return int(lib().kqo_bf16_from_f64(float(a)))
+
+
+def hadamard(n: int) -> np.ndarray:
+    H = np.zeros((1 << n, 1 << n), np.float64)
+    lib().kqo_hadamard(n, _p(H))
+    return H
+
+
+def e8m0(amax: float) -> int:
+    return int(lib().kqo_e8m0(float(amax)))
+
+
+def e8m0_many(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a, np.float32).reshape(-1)
+    out = np.zeros(a.size, np.uint8)
+    lib().kqo_e8m0_many(_p(a), a.size, _p(out))
+    return out
+
+
+def e2m1(v: float) -> int:
+    return int(lib().kqo_e2m1(float(v)))
+
+
+def e2m1_value(code: int) -> float:
+    return float(lib().kqo_e2m1_value(int(code)))
+
+
+def e2m1_pack(v: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(v, np.float32).reshape(-1)
+    out = np.zeros(v.size // 2, np.uint8)
+    lib().kqo_e2m1_pack(_p(v), v.size, _p(out))
+    return out
+
+
+def _mats_dtype(mats: np.ndarray) -> int:
+    if mats.dtype == np.float32:
+        return F32
+    if mats.dtype == np.uint16:
+        return BF16
+    raise TypeError("mats must be float32 or bf16 bits (uint16)")
+
+
+def transform(x: np.ndarray, mats: np.ndarray, d: int | None = None) -> np.ndarray:
+    x = _bf16_bits(x)
+    M, ldx = x.shape
+    d = ldx if d is None else d
+    mats = np.ascontiguousarray(mats)
+    y = np.zeros((M, d), np.float32)
+    lib().kqo_transform(_p(x), M, d, ldx, _p(mats), _mats_dtype(mats), _p(y))
+    return y
+
+
+def mx_quantize(y: np.ndarray):
+    y = np.ascontiguousarray(y, np.float32)
+    M, d = y.shape
+    q = np.zeros((M, d // 2), np.uint8)
+    s = np.zeros((M, d // 32), np.uint8)
+    lib().kqo_mx_quantize(_p(y), M, d, _p(q), _p(s))
+    return q, s
+
+
+def quantize(x: np.ndarray, mats: np.ndarray, d: int | None = None):
+    x = _bf16_bits(x)
+    M, ldx = x.shape
+    d = ldx if d is None else d
+    mats = np.ascontiguousarray(mats)
+    q = np.zeros((M, d // 2), np.uint8)
+    s = np.zeros((M, d // 32), np.uint8)
+    lib().kqo_quantize(_p(x), M, d, ldx, _p(mats), _mats_dtype(mats), _p(q), _p(s))
+    return q, s
+
+
+def smooth_quantize(x: np.ndarray, inv_s: np.ndarray, d: int | None = None):
+    x = _bf16_bits(x)
+    M, ldx = x.shape
+    d = ldx if d is None else d
+    inv_s = np.ascontiguousarray(inv_s, np.float32)
+    q = np.zeros((M, d // 2), np.uint8)
+    s = np.zeros((M, d // 32), np.uint8)
+    lib().kqo_smooth_quantize(_p(x), M, d, ldx, _p(inv_s), _p(q), _p(s))
+    return q, s
+
+
+def fwht_quantize(x: np.ndarray, d: int | None = None):
+    x = _bf16_bits(x)
+    M, ldx = x.shape
+    d = ldx if d is None else d
+    q = np.zeros((M, d // 2), np.uint8)
+    s = np.zeros((M, d // 32), np.uint8)
+    lib().kqo_fwht_quantize(_p(x), M, d, ldx, _p(q), _p(s))
+    return q, s
+
+
+def dequantize(q: np.ndarray, scales: np.ndarray, inv_mats: np.ndarray | None = None) -> np.ndarray:
+    q = np.ascontiguousarray(q, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    M, d = q.shape[0], q.shape[1] * 2
+    out = np.zeros((M, d), np.float64)
+    if inv_mats is None:
+        lib().kqo_dequantize(_p(q), _p(scales), M, d, None, F32, _p(out))
+    else:
+        inv_mats = np.ascontiguousarray(inv_mats)
+        lib().kqo_dequantize(_p(q), _p(scales), M, d, _p(inv_mats), _mats_dtype(inv_mats), _p(out))
+    return out

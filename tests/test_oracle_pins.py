@@ -1,0 +1,430 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each test checks one oracle function against a closed form, a textbook
+identity, a library routine used as a step, a brute force on small inputs, or a
+value printed on the pages (tests/golden/).  A dropped term, a wrong sign, a
+transposed operand or a swapped factor order in the oracle fails at least one.
+"""
+from __future__ import annotations
+
+import itertools
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from mxfp4_activations_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+E2M1_MAGS = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+# ---------------------------------------------------------------- helpers (independent formulations)
+
+def brute_e2m1(v: np.ndarray) -> np.ndarray:
+    """Nearest E2M1 magnitude by exhaustive distance search; on equal distance the
+    code with mantissa bit 0 (even code) wins; magnitudes above the largest grid
+    value saturate to it; sign bit from the sign of v."""
+    v = np.asarray(v, np.float32)
+    a = np.minimum(np.abs(v.astype(np.float64)), E2M1_MAGS[-1])
+    best = np.full(a.shape, np.inf)
+    code = np.zeros(a.shape, np.int64)
+    for c, g in enumerate(E2M1_MAGS):
+        dist = np.abs(a - g)
+        take = (dist < best) | ((dist == best) & (c % 2 == 0))
+        best = np.where(take, dist, best)
+        code = np.where(take, c, code)
+    return code | (np.signbit(v).astype(np.int64) << 3)
+
+
+def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
+    packed = np.asarray(packed, np.uint8).reshape(-1)
+    out = np.empty(packed.size * 2, np.int64)
+    out[0::2] = packed & 0xF
+    out[1::2] = packed >> 4
+    return out
+
+
+def f32_exponent_field(a: np.ndarray) -> np.ndarray:
+    return ((np.asarray(a, np.float32).view(np.uint32) >> 23) & 0xFF).astype(np.int64)
+
+
+def e8m0_from_bits(amax: np.ndarray) -> np.ndarray:
+    """floor(log2 amax) from the fp32 bit fields: normal -> field - 127,
+    subnormal -> index of the top set mantissa bit - 149; then e = that - 2,
+    clamped to [-127, 127], byte = e + 127; amax = 0 -> 0."""
+    a = np.asarray(amax, np.float32)
+    bits = a.view(np.uint32).astype(np.int64)
+    field = (bits >> 23) & 0xFF
+    mant = bits & 0x7FFFFF
+    top = np.zeros_like(mant)
+    for k in range(23):
+        top = np.where((mant >> k) & 1 == 1, k, top)
+    flog = np.where(field > 0, field - 127, top - 149)
+    e = np.clip(flog - 2, -127, 127)
+    byte = e + 127
+    return np.where(a == 0, 0, byte)
+
+
+def lu_numpy(l, u, v):
+    L = np.array([[1.0, 0.0], [float(l), 1.0]])
+    U = np.array([[float(u), float(v)], [0.0, 1.0 / float(u)]])
+    return L @ U
+
+
+def f32_round_fraction(q: Fraction) -> np.float32:
+    """Correct rounding of an exact rational to fp32 (nearest, ties to even),
+    by bracketing between adjacent fp32 values."""
+    if q == 0:
+        return np.float32(0.0)
+    f = np.float32(float(q))  # within one ulp
+    lo = f if Fraction(float(f)) <= q else np.nextafter(f, np.float32(-np.inf))
+    hi = np.nextafter(lo, np.float32(np.inf))
+    dlo, dhi = q - Fraction(float(lo)), Fraction(float(hi)) - q
+    if dlo < dhi:
+        return lo
+    if dhi < dlo:
+        return hi
+    return lo if (lo.view(np.uint32) & 1) == 0 else hi
+
+
+def bf16_bits_to_frac(h: int) -> Fraction:
+    return Fraction(float(np.array([h << 16], np.uint32).view(np.float32)[0]))
+
+
+# ---------------------------------------------------------------- E2M1 element rounding (C5)
+
+def test_e2m1_golden_grid(orc):
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "e2m1_grid.txt")) if l.strip() and not l.startswith("#")]
+    for r in rows:
+        if r[0] == "tie":
+            v, code = float(r[1]), int(r[2])
+            assert orc.e2m1(v) == code, r
+            assert orc.e2m1(-v) == code | 8, r
+        else:
+            code, val = int(r[0]), float(r[1])
+            assert orc.e2m1_value(code) == val and math.copysign(1, orc.e2m1_value(code)) == math.copysign(1, val)
+            assert orc.e2m1(val) == code  # every representable value maps to itself (incl. -0 -> 8)
+
+
+def test_e2m1_exhaustive_core_binades(orc):
+    """Every fp32 pattern with |v| in [2^-3, 2^3) (all midpoints, neighbours of
+    midpoints and saturation region), both signs, against the brute force."""
+    lo = np.float32(0.125).view(np.uint32)
+    hi = np.float32(8.0).view(np.uint32)
+    step = 1 << 23
+    for start in range(int(lo), int(hi), step):
+        pos = np.arange(start, min(start + step, int(hi)), dtype=np.uint32)
+        for bits in (pos, pos | np.uint32(0x80000000)):
+            v = bits.view(np.float32)
+            got = unpack_nibbles(orc.e2m1_pack(v))
+            want = brute_e2m1(v)
+            bad = np.nonzero(got != want)[0]
+            assert bad.size == 0, (v[bad[:5]], got[bad[:5]], want[bad[:5]])
+
+
+def test_e2m1_random_patterns_and_specials(orc):
+    rng = np.random.default_rng(123)
+    bits = rng.integers(0, 2**32, size=1 << 21, dtype=np.uint64).astype(np.uint32)
+    v = bits.view(np.float32)
+    v = v[np.isfinite(v)]
+    specials = np.array([0.0, -0.0, 1e-45, -1e-45, 1.17549435e-38, 0.2499999, 0.2500001, 5.9999995, 6.0,
+                         6.0000005, 7.0, 1e30, -1e30, 3.4028235e38, -3.4028235e38], np.float32)
+    v = np.concatenate([v, specials]).astype(np.float32)
+    if v.size % 2:
+        v = v[:-1]
+    got = unpack_nibbles(orc.e2m1_pack(v))
+    assert np.array_equal(got, brute_e2m1(v))
+
+
+def test_e2m1_pack_nibble_order(orc):
+    # byte k = code(v[2k]) | code(v[2k+1]) << 4
+    p = orc.e2m1_pack(np.array([0.5, 6.0, -1.0, 0.0], np.float32))
+    assert list(p) == [0x71, 0x0A]
+
+
+# ---------------------------------------------------------------- E8M0 shared scale (C4)
+
+def test_e8m0_every_exponent_field(orc):
+    rng = np.random.default_rng(7)
+    mants = np.concatenate([[0, 1, 2, (1 << 22), (1 << 23) - 2, (1 << 23) - 1],
+                            rng.integers(0, 1 << 23, size=250)]).astype(np.uint32)
+    fields = np.arange(0, 255, dtype=np.uint32)
+    bits = (fields[:, None] << 23) | mants[None, :]
+    a = bits.reshape(-1).view(np.float32)
+    assert np.array_equal(orc.e8m0_many(a).astype(np.int64), e8m0_from_bits(a))
+
+
+def test_e8m0_closed_forms(orc):
+    # powers of two map exactly: amax = 2^k -> e = k - 2
+    for k in range(-124, 128):
+        assert orc.e8m0(math.ldexp(1.0, k)) == max(k - 2, -127) + 127
+    assert orc.e8m0(0.0) == 0
+    assert orc.e8m0(float("inf")) == 0xFF and orc.e8m0(float("nan")) == 0xFF
+    assert orc.e8m0(4.0) == 127 and orc.e8m0(np.nextafter(np.float32(4.0), np.float32(0))) == 126
+    assert orc.e8m0(7.999999) == 127 and orc.e8m0(8.0) == 128
+
+
+# ---------------------------------------------------------------- bf16 rounding of the expanded matrix
+
+def test_bf16_from_f64_against_bracketing(orc):
+    rng = np.random.default_rng(11)
+    vals = list(rng.normal(0, 1, 3000) * np.exp2(rng.integers(-140, 120, 3000)))
+    # exact bf16 midpoints (ties) and their neighbours
+    for h in rng.integers(1, 0x7F7F, 500):
+        a = float(bf16_bits_to_frac(int(h)))
+        b = float(bf16_bits_to_frac(int(h) + 1))
+        m = 0.5 * (a + b)
+        vals += [m, np.nextafter(m, 0), np.nextafter(m, np.inf), -m]
+    vals += [0.0, -0.0, 1e-45, 3.0e38, 3.4e38, 3.3961e38, 1e-40, -1e-41]
+    for a in vals:
+        got = orc.bf16_from_f64(a)
+        q = Fraction(abs(a))
+        # bracket |a| between adjacent bf16 patterns (patterns are monotone in value)
+        f = np.array([abs(a)], np.float32)  # nearest fp32, then truncate to bf16
+        h = int(f.view(np.uint32)[0] >> 16)
+        cands = [c for c in (h - 1, h, h + 1, h + 2) if 0 <= c <= 0x7F80]
+        best = None
+        for c in cands:
+            cv = bf16_bits_to_frac(c) if c < 0x7F80 else Fraction(2) ** 128
+            dist = abs(cv - q)
+            if best is None or dist < best[0] or (dist == best[0] and c % 2 == 0):
+                best = (dist, c)
+        want = best[1] | (0x8000 if math.copysign(1, a) < 0 else 0)
+        assert got == want, (a, hex(got), hex(want))
+
+
+# ---------------------------------------------------------------- factors and Kronecker expansion (C1, C2)
+
+def test_factor_is_lu_product_with_unit_det(orc):
+    rng = np.random.default_rng(3)
+    for l, u, v in rng.normal(0, 1, (200, 3)).astype(np.float32):
+        if abs(u) < 1e-3:
+            continue
+        F = orc.factor(l, u, v)
+        assert np.array_equal(F, lu_numpy(l, u, v))
+        assert abs(np.linalg.det(F) - 1.0) < 1e-12 * max(1.0, np.abs(F).max() ** 2)
+        Fi = orc.factor(l, u, v, inverse=True)
+        assert np.allclose(Fi, np.linalg.inv(F), rtol=1e-12, atol=1e-12 * np.abs(F).max() ** 2)
+
+
+def test_expand_matches_numpy_kron_and_bit_convention(orc):
+    params = inputs.lu_params(6, seed=5)
+    K = orc.expand_f64(params)
+    for b in range(6):
+        Fs = [lu_numpy(*params[b, k]) for k in range(5)]
+        ref = Fs[0]
+        for F in Fs[1:]:
+            ref = np.kron(ref, F)
+        assert np.allclose(K[b], ref, rtol=1e-14, atol=0)
+        # entry-wise: K[i][j] = prod_k F_k[bit(4-k) of i][bit(4-k) of j]  (F0 on the top bit)
+        for i, j in itertools.product(range(32), range(32)):
+            prod = 1.0
+            for k in range(5):
+                prod *= Fs[k][(i >> (4 - k)) & 1, (j >> (4 - k)) & 1]
+            assert abs(K[b, i, j] - prod) <= 1e-14 * abs(prod)
+
+
+def test_oracle_kron_against_numpy(orc):
+    rng = np.random.default_rng(9)
+    A = rng.normal(size=(2, 2))
+    B = rng.normal(size=(4, 4))
+    assert np.array_equal(orc.kron(A, B), np.kron(A, B))
+
+
+def test_param_count_is_3log2n_and_under_half_of_per_channel():
+    # "five 2x2 unit-determinant LU factors (15 parameters per block)" and
+    # 3 log2(n) per block; "less than half the parameters of per-channel scaling"
+    p = inputs.lu_params(36, seed=0)
+    assert p.shape == (36, 5, 3) and p[0].size == 15 == 3 * int(math.log2(32))
+    d = 1152
+    assert (d // 32) * 15 < d / 2
+
+
+def test_det_is_one(orc):
+    params = inputs.lu_params(64, seed=21)
+    K = orc.expand_f64(params)
+    dets = np.linalg.det(K)
+    assert np.all(np.abs(dets - 1.0) < 1e-9)
+    K32 = orc.expand(params).astype(np.float64)
+    assert np.all(np.abs(np.linalg.det(K32) - 1.0) < 1e-5)
+
+
+def test_inverse_is_kron_of_factor_inverses(orc):
+    params = inputs.lu_params(32, seed=22)
+    K = orc.expand_f64(params)
+    Ki = orc.expand_f64(params, inverse=True)
+    assert np.allclose(Ki, np.linalg.inv(K), rtol=0, atol=1e-12)
+    eye = np.broadcast_to(np.eye(32), K.shape)
+    assert np.abs(K @ Ki - eye).max() < 1e-12
+
+
+def test_round_trip_fp32_below_1e_5(orc):
+    params = inputs.lu_params(36, seed=23)
+    K32 = orc.expand(params).astype(np.float32)
+    Ki32 = orc.expand(params, inverse=True).astype(np.float32)
+    x = np.random.default_rng(24).standard_normal((64, 36, 32)).astype(np.float32)
+    y = np.einsum("rbi,bij->rbj", x, K32).astype(np.float32)
+    xr = np.einsum("rbj,bji->rbi", y, Ki32).astype(np.float32)
+    err = np.abs(xr - x).max(axis=-1) / np.abs(x).max(axis=-1)
+    assert err.max() < 1e-5
+
+
+def test_bf16_expand_is_rounding_of_fp64(orc):
+    params = inputs.lu_params(8, seed=25)
+    K = orc.expand_f64(params)
+    Kb = orc.expand(params, dtype=orc.BF16)
+    # every bf16 entry is the nearest bf16 of the fp64 entry (checked with the
+    # independent bracketing of test_bf16_from_f64_against_bracketing on a sample)
+    vals = inputs.bf16_bits_to_f32(Kb).astype(np.float64)
+    spacing = np.exp2(np.floor(np.log2(np.abs(K))) - 7)
+    assert np.all(np.abs(vals - K) <= 0.5 * spacing)
+
+
+# ---------------------------------------------------------------- Hadamard initialisation and Lemma 1
+
+def sylvester_closed_form(n: int) -> np.ndarray:
+    N = 1 << n
+    i = np.arange(N)
+    pc = np.vectorize(lambda t: bin(t).count("1"))(i[:, None] & i[None, :])
+    return np.where(pc % 2 == 0, 1.0, -1.0) * 2.0 ** (-n / 2)
+
+
+def test_hadamard_matches_golden_h2_and_closed_form(orc):
+    lines = [l.split() for l in open(os.path.join(GOLDEN, "hadamard_h2.txt")) if l.strip() and not l.startswith("#")]
+    norm = float(lines[0][1])
+    H2 = norm * np.array([[float(t) for t in r] for r in lines[1:]])
+    assert np.allclose(orc.hadamard(1), H2, rtol=0, atol=4e-16)
+    for n in (2, 3, 5):
+        H = orc.hadamard(n)
+        assert np.allclose(H, sylvester_closed_form(n), rtol=0, atol=1e-15)
+        assert np.allclose(H @ H.T, np.eye(1 << n), atol=1e-14)  # eq. 2: H H^T = I
+
+
+def test_hadamard_init_reproduces_h32_up_to_signs(orc):
+    K = orc.expand_f64(inputs.hadamard_params(1))[0]
+    D = np.diag([(-1.0) ** bin(i).count("1") for i in range(32)])
+    H32 = sylvester_closed_form(5)
+    assert np.abs(K - D @ H32).max() < 1e-6  # only fp32 rounding of 1/sqrt2 in the params
+    assert np.allclose(np.abs(K), 2.0 ** -2.5, rtol=5e-7, atol=0)  # fp32 params: 1/u - u != u exactly
+    assert np.abs(K @ K.T - np.eye(32)).max() < 1e-6
+    # the FWHT comparison path uses fp32(H_32): entries are +-fp32(2^-2.5)
+    assert np.all(np.abs(orc.hadamard(5).astype(np.float32)) == np.float32(2.0 ** -2.5))
+
+
+def test_lemma1_norm_and_spread(orc):
+    params = inputs.hadamard_params(1)
+    K32 = orc.expand(params)
+    rng = np.random.default_rng(31)
+    for c in range(32):
+        alpha = float(rng.choice([1.0, 3.5, -20.0, 96.0]))
+        x = np.zeros((1, 32), np.float32)
+        x[0, c] = alpha
+        y = orc.transform(inputs.f32_to_bf16_bits(x), K32)[0].astype(np.float64)
+        assert abs(np.linalg.norm(y) - abs(alpha)) < 1e-6 * abs(alpha)
+        assert np.allclose(np.abs(y), abs(alpha) / math.sqrt(32), rtol=1e-6)
+
+
+def test_lemma1_golden_quantized_onehot(orc):
+    K32 = orc.expand(inputs.hadamard_params(1))
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "lemma1_onehot.txt")) if l.strip() and not l.startswith("#")]
+    for c, byte, hexcodes in rows:
+        x = np.zeros((1, 32), np.float32)
+        x[0, int(c)] = 32.0
+        q, s = orc.quantize(inputs.f32_to_bf16_bits(x), K32)
+        assert s[0, 0] == int(byte)
+        assert q[0].tobytes().hex() == hexcodes
+
+
+# ---------------------------------------------------------------- transform and end-to-end quantize, brute force (C3..C6)
+
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_transform_exact_rational_brute_force(orc, dtype):
+    rng = np.random.default_rng(41 + dtype)
+    M, d = 3, 64
+    x = inputs.f32_to_bf16_bits((rng.standard_t(3, (M, d)) * rng.choice([1, 100], (M, d))).astype(np.float32))
+    params = inputs.lu_params(d // 32, seed=42)
+    mats = orc.expand(params, dtype=dtype)
+    y = orc.transform(x, mats)
+    matf = mats if dtype == 0 else inputs.bf16_bits_to_f32(mats)
+    for r in range(M):
+        for b in range(d // 32):
+            xs = [bf16_bits_to_frac(int(h)) for h in x[r, 32 * b:32 * b + 32]]
+            for j in range(32):
+                exact = sum(xs[i] * Fraction(float(matf[b, i, j])) for i in range(32))
+                assert y[r, 32 * b + j] == f32_round_fraction(exact), (r, b, j)
+
+
+def test_quantize_end_to_end_brute_force(orc):
+    rng = np.random.default_rng(51)
+    M, d = 4, 96
+    x = inputs.f32_to_bf16_bits((rng.standard_normal((M, d)) * 3).astype(np.float32))
+    x[1, 32:64] = 0  # an all-zero block
+    x[2, 5] = inputs.f32_to_bf16_bits(np.array([200.0], np.float32))[0]
+    params = inputs.lu_params(d // 32, seed=52)
+    K32 = orc.expand(params)
+    q, s = orc.quantize(x, K32)
+    for r in range(M):
+        for b in range(d // 32):
+            xs = [bf16_bits_to_frac(int(h)) for h in x[r, 32 * b:32 * b + 32]]
+            y = np.array([f32_round_fraction(sum(xs[i] * Fraction(float(K32[b, i, j])) for i in range(32)))
+                          for j in range(32)], np.float32)
+            byte = int(e8m0_from_bits(np.array([np.abs(y).max()], np.float32))[0])
+            assert s[r, b] == byte
+            v = (y.astype(np.float64) * 2.0 ** (127 - byte)).astype(np.float32)
+            assert np.array_equal(unpack_nibbles(q[r, 16 * b:16 * b + 16]), brute_e2m1(v))
+
+
+def test_nonfinite_block_rule(orc):
+    y = np.zeros((1, 64), np.float32)
+    y[0, 3] = np.inf
+    y[0, 40] = 1.0
+    q, s = orc.mx_quantize(y)
+    assert s[0, 0] == 0xFF and not q[0, :16].any()
+    assert s[0, 1] == orc.e8m0(1.0)
+
+
+def test_dequantize_is_grid_value_times_scale(orc):
+    rng = np.random.default_rng(61)
+    y = (rng.standard_normal((8, 64)) * np.exp2(rng.integers(-10, 10, (8, 1)))).astype(np.float32)
+    q, s = orc.mx_quantize(y)
+    yh = orc.dequantize(q, s)
+    codes = unpack_nibbles(q.reshape(-1)).reshape(8, 64)
+    scale = np.exp2(np.repeat(s.astype(np.int64) - 127, 32, axis=1).astype(np.float64))
+    sign = np.where(codes >= 8, -1.0, 1.0)
+    assert np.array_equal(yh, sign * E2M1_MAGS[codes & 7] * scale)
+    # the error of each element is at most half a grid step (or the saturation gap)
+    assert np.all(np.abs(yh - y) <= np.maximum(1.0 * scale, np.abs(y) - 6 * scale + 1e-30))
+
+
+def test_dequantize_with_inverse_undoes_transform(orc):
+    params = inputs.lu_params(4, seed=62)
+    K32, Ki32 = orc.expand(params), orc.expand(params, inverse=True)
+    y = np.random.default_rng(63).standard_normal((5, 128)).astype(np.float32)
+    q, s = orc.mx_quantize(y)
+    yh = orc.dequantize(q, s)
+    xh = orc.dequantize(q, s, inv_mats=Ki32)
+    ref = np.einsum("rbj,bji->rbi", yh.reshape(5, 4, 32), Ki32.astype(np.float64)).reshape(5, 128)
+    assert np.allclose(xh, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_smooth_is_single_rounding_of_product(orc):
+    rng = np.random.default_rng(71)
+    x = inputs.f32_to_bf16_bits(rng.standard_normal((6, 64)).astype(np.float32) * 7)
+    inv_s = rng.uniform(0.01, 3.0, 64).astype(np.float32)
+    q, s = orc.smooth_quantize(x, inv_s)
+    y = inputs.bf16_bits_to_f32(x) * inv_s[None, :]  # fp32 multiply: one IEEE rounding
+    q2, s2 = orc.mx_quantize(y.astype(np.float32))
+    assert np.array_equal(q, q2) and np.array_equal(s, s2)
+
+
+def test_fwht_equals_kroquant_with_sylvester_matrix(orc):
+    rng = np.random.default_rng(81)
+    x = inputs.f32_to_bf16_bits(rng.standard_normal((7, 96)).astype(np.float32))
+    q, s = orc.fwht_quantize(x)
+    H = np.broadcast_to(sylvester_closed_form(5).astype(np.float32), (3, 32, 32)).copy()
+    q2, s2 = orc.quantize(x, H)
+    assert np.array_equal(q, q2) and np.array_equal(s, s2)
