@@ -1,0 +1,562 @@
+#!/usr/bin/env python3
+"""Throughput of the KroQuant online activation quantizer on B200.
+
+One step = one pass of the whole hot path (load, block transform, amax, E8M0
+scale, E2M1 round, pack, store) over the FLUX.1-schnell-shaped activations of
+one denoising step: M = 4608 tokens at d = 3072 and at d = 12288 (bf16, Student-t
+nu = 3, 0.5 % outlier channels x100, seeded synthetic data).  The metric is
+quantizer GB/s with algorithmic bytes (2 B in + 0.5 B codes + 1/32 B scales per
+element), its fraction of HBM bandwidth, and tokens/s.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py --sweep   # KroQuant vs per-channel scaling vs FWHT, every shape
+
+Multi-GPU (torchrun, one process per GPU): rows are independent, each rank
+quantizes its own batch (weak scaling, no collective on the data path); time is
+the max over ranks.  ``--impl reference`` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mxfp4_activations_b200 import inputs  # noqa: E402
+
+FLUX_M = 4608
+FLUX_DS = (3072, 12288)
+BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 32.0
+PROFILE_JSON = os.path.join(ROOT, "profiles", "kq_quant_flux_traffic.json")
+KERNEL_SOURCES = ["mxfp4_activations_b200/csrc/kq_quant.cuh", "mxfp4_activations_b200/csrc/kq_common.cuh",
+                  "mxfp4_activations_b200/csrc/kq_lib.cu"]
+
+
+def algo_bytes(M: int, d: int) -> float:
+    return BYTES_PER_ELEM * M * d
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def recorded_traffic():
+    """dram bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    if not os.path.exists(PROFILE_JSON):
+        return None
+    with open(PROFILE_JSON) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_step")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+class QuantStep:
+    """Device-resident buffers for one step over every d, rotated over n copies."""
+
+    def __init__(self, torch, kq, xs_host, params_host, n_copies: int, device):
+        self.torch = torch
+        self.kq = kq
+        self.lib = kq.load()
+        self.items = []
+        for d, x, params in zip(FLUX_DS, xs_host, params_host):
+            p = torch.from_numpy(params).to(device)
+            mats = kq.kq_expand_blocks(p)
+            fac = kq.kq_expand_factored(p)
+            x0 = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+            copies = [x0] + [x0.clone() for _ in range(n_copies - 1)]
+            M = x.shape[0]
+            qs = [torch.empty((M, d // 2), dtype=torch.uint8, device=device) for _ in range(n_copies)]
+            ss = [torch.empty((M, d // 32), dtype=torch.uint8, device=device) for _ in range(n_copies)]
+            inv_s = torch.from_numpy(inputs.smooth_inv_scale(x)).to(device)
+            self.items.append(dict(d=d, M=M, params=p, mats=mats, fac=fac, x=copies, q=qs, s=ss, inv_s=inv_s))
+        self.n = n_copies
+        self.stream = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+    def launch(self, it: int, item: dict, kind: str = "kroquant"):
+        c = it % self.n
+        x, q, s = item["x"][c], item["q"][c], item["s"][c]
+        M, d = item["M"], item["d"]
+        if kind == "kroquant":
+            st = self.lib.kq_quantize(x.data_ptr(), M, d, d, item["mats"].data_ptr(), 0, item["fac"].data_ptr(),
+                                      q.data_ptr(), s.data_ptr(), 2, self.stream)
+        elif kind == "smooth":
+            st = self.lib.kq_ref_smooth_quantize(x.data_ptr(), M, d, d, item["inv_s"].data_ptr(), q.data_ptr(),
+                                                 s.data_ptr(), self.stream)
+        else:
+            st = self.lib.kq_ref_fwht_quantize(x.data_ptr(), M, d, d, q.data_ptr(), s.data_ptr(), self.stream)
+        if st != 0:
+            raise RuntimeError(f"{kind} launch failed: {self.lib.kq_status_string(st).decode()}")
+
+    def bytes_per_step(self) -> float:
+        return sum(algo_bytes(it["M"], it["d"]) for it in self.items)
+
+
+def timed(torch, step: QuantStep, K: int, kind: str, per_launch: bool):
+    """K steps bracketed by events; optional events around every launch."""
+    ev = torch.cuda.Event
+    if per_launch:
+        marks = [[(ev(enable_timing=True), ev(enable_timing=True)) for _ in step.items] for _ in range(K)]
+    start, stop = ev(enable_timing=True), ev(enable_timing=True)
+    start.record()
+    for it in range(K):
+        for j, item in enumerate(step.items):
+            if per_launch:
+                marks[it][j][0].record()
+            step.launch(it, item, kind)
+            if per_launch:
+                marks[it][j][1].record()
+    stop.record()
+    stop.synchronize()
+    total_ms = start.elapsed_time(stop)
+    launch_ms = None
+    if per_launch:
+        launch_ms = [sum(a.elapsed_time(b) for a, b in (marks[i][j] for i in range(K))) for j in range(len(step.items))]
+    return total_ms, launch_ms
+
+
+def e2e_run(torch, kq, step: QuantStep, xs_host, K: int):
+    """Same metric through the public API with host buffers: every step copies
+    that step's activations from pinned host memory, quantizes, and reads the
+    codes and scales back to pinned host memory."""
+    dev = step.items[0]["x"][0].device
+    hx = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in xs_host]
+    hq = [torch.empty((it["M"], it["d"] // 2), dtype=torch.uint8).pin_memory() for it in step.items]
+    hs = [torch.empty((it["M"], it["d"] // 32), dtype=torch.uint8).pin_memory() for it in step.items]
+    dx = [torch.empty(x.shape, dtype=torch.int16, device=dev) for x in xs_host]
+    h2d = sum(x.nbytes for x in xs_host)
+    d2h = sum(t.numel() for t in hq) + sum(t.numel() for t in hs)
+
+    def one():
+        for j, it in enumerate(step.items):
+            dx[j].copy_(hx[j], non_blocking=True)
+            q, s = kq.kq_quantize(dx[j].view(torch.bfloat16), it["mats"], it["fac"], variant="butterfly",
+                                  q=it["q"][0], scales=it["s"][0])
+            hq[j].copy_(q, non_blocking=True)
+            hs[j].copy_(s, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(K):
+        one()
+    t1.record()
+    t1.synchronize()
+    ms = t0.elapsed_time(t1)
+    return ms, h2d, d2h
+
+
+def run_gpu(args) -> None:
+    import torch
+    import torch.distributed as dist
+
+    import mxfp4_activations_b200 as kq
+    from mxfp4_activations_b200 import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", init_method="env://", timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else 0)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    kq.load()
+
+    # inputs: each rank draws its own batch (weak scaling); seeds differ by rank
+    xs, ps = [], []
+    for d in FLUX_DS:
+        x, p = inputs.config_case("flux", d)
+        if rank:
+            x = inputs.activations(FLUX_M, d, "t3", seed=[3, d, 0, rank], outlier_frac=0.005,
+                                   outlier_scale=(100.0, 100.0))
+        xs.append(x)
+        ps.append(p)
+    step = QuantStep(torch, kq, xs, ps, n_copies=4, device=device)
+    bytes_step = step.bytes_per_step()
+    resident_mb = 4 * sum(x.nbytes for x in xs) / 1e6
+
+    for it in range(args.warmup):
+        for item in step.items:
+            step.launch(it, item)
+    torch.cuda.synchronize()
+    err = kq.kq_get_device_error(clear=True)
+    if err != 0:
+        raise RuntimeError(f"device error after warm-up: {kq.kq_status_string(err)}")
+
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or 0) if world == 1 else local
+    with ClockSampler(gpu_index) as clk:
+        # untimed soak so that the clock record covers a loaded GPU, then the timed K steps
+        t_end = time.time() + 1.0
+        it = 0
+        while time.time() < t_end:
+            for item in step.items:
+                step.launch(it, item)
+            it += 1
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        total_ms, launch_ms = timed(torch, step, args.steps, "kroquant", per_launch=True)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    if world > 1:
+        t = torch.tensor([total_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    err = kq.kq_get_device_error(clear=True)
+    if err != 0:
+        raise RuntimeError(f"device error in timed region: {kq.kq_status_string(err)}")
+
+    # comparison kernels on the same inputs (after the timed region)
+    comp = {}
+    for kind in ("smooth", "fwht", "kroquant"):
+        timed(torch, step, 20, kind, per_launch=False)
+        ms, lm = timed(torch, step, max(50, args.steps), kind, per_launch=True)
+        n = max(50, args.steps)
+        comp[kind] = {"gbs": bytes_step * n / (sum(lm) * 1e-3) / 1e9,
+                      "us_per_launch": {str(it["d"]): lm[j] * 1e3 / n for j, it in enumerate(step.items)}}
+
+    e2e_ms, h2d, d2h = e2e_run(torch, kq, step, xs, max(3, min(args.steps, 20)))
+    e2e_steps = max(3, min(args.steps, 20))
+
+    if world > 1:
+        dist.barrier()
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    peaks = measured_peaks()
+    value = world * bytes_step * args.steps / (total_ms * 1e-3) / 1e9
+    launch_total_ms = sum(launch_ms)
+    achieved = bytes_step * args.steps / (launch_total_ms * 1e-3) / 1e9
+    traffic = recorded_traffic()
+    clocks = clk.summary()
+    out = {
+        "metric": "quantizer GB/s (bf16 in + FP4/E8M0 out) and % of B200 HBM peak; tokens/s",
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": "FLUX.1-schnell-shaped activations, M=4608 tokens x d in {3072, 12288} bf16, "
+                        "Student-t(3) with 0.5% outlier channels x100, per-block LU params Hadamard+N(0,0.05)",
+            "M": FLUX_M, "d": list(FLUX_DS), "variant": "butterfly",
+            "l2": f"inputs rotated over 4 device copies ({resident_mb:.0f} MB > 126 MB L2)",
+            "parallelism": f"dp{world} (rows sharded, no collective)",
+        },
+        "tokens_per_s": round(world * FLUX_M * args.steps / (total_ms * 1e-3), 1),
+        "hbm_frac_measured": round(value / world / peaks["hbm_gbs"], 4),
+        "hbm_frac_nominal_8tbs": round(value / world / 8000.0, 4),
+        "roofline": {
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
+            "traffic": traffic,
+            "algorithmic_bytes_per_step": bytes_step,
+            "us_per_launch": {str(it["d"]): round(launch_ms[j] * 1e3 / args.steps, 3)
+                              for j, it in enumerate(step.items)},
+        },
+        "comparison": {k: {"gbs": round(v["gbs"], 1),
+                           "us_per_launch": {dk: round(dv, 3) for dk, dv in v["us_per_launch"].items()}}
+                       for k, v in comp.items()},
+        "e2e": {"value": round(bytes_step * e2e_steps / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "tokens_per_s": round(FLUX_M * e2e_steps / (e2e_ms * 1e-3), 1)},
+        "gpu_launches": len(FLUX_DS) * args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
+
+def flux_oracle_data():
+    from oracle import oracle as orc
+
+    orc.build()
+    data = []
+    for d in FLUX_DS:
+        x, p = inputs.config_case("flux", d)
+        data.append((x, orc.expand(p)))
+    return data
+
+
+def oracle_sample(seconds: float, data=None):
+    """Time the oracle on the leading rows of the same FLUX workload; the row
+    count grows (up to all M rows, then whole repeated passes) until the sample
+    takes about `seconds` of single-thread CPU work."""
+    from oracle import oracle as orc
+
+    data = data or flux_oracle_data()
+    rows, passes = 8, 1
+    while True:
+        t0 = time.perf_counter()
+        for _ in range(passes):
+            for x, K in data:
+                orc.quantize(np.ascontiguousarray(x[:rows]), K)
+        dt = time.perf_counter() - t0
+        if dt >= 0.8 * seconds:
+            break
+        grow = seconds / max(dt, 1e-3) * 1.05
+        if rows < FLUX_M:
+            rows = min(FLUX_M, max(rows * 2, int(rows * grow)))
+        else:
+            passes = max(passes + 1, int(passes * grow))
+    nbytes = sum(algo_bytes(rows, d) for d in FLUX_DS) * passes
+    return nbytes / dt / 1e9, rows, passes, dt
+
+
+def cpu_baseline(seconds: float) -> dict:
+    gbs, rows, passes, dt = oracle_sample(seconds)
+    return {"value": round(gbs, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{passes} pass(es) over {rows} of 4608 rows of each FLUX shape (d=3072 and d=12288), "
+                      f"{dt:.1f} s of single-thread C oracle, same algorithmic-byte numerator"}
+
+
+def run_reference(args) -> None:
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    # each step: a bounded sample of the workload, sized so that W + K steps end in minutes
+    per_step = max(0.5, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
+    from oracle import oracle as orc
+
+    data = flux_oracle_data()
+    _, rows, _, _ = oracle_sample(per_step, data)
+
+    def one():
+        for x, K in data:
+            orc.quantize(np.ascontiguousarray(x[:rows]), K)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    dt = time.perf_counter() - t0
+    nbytes = sum(algo_bytes(rows, d) for d in FLUX_DS) * args.steps
+    gbs = nbytes / dt / 1e9
+    sample = f"{rows} rows of each FLUX shape (d=3072, d=12288) per step, single-thread C oracle"
+    out = {
+        "impl": "reference",
+        "metric": "quantizer GB/s (bf16 in + FP4/E8M0 out) and % of B200 HBM peak; tokens/s",
+        "value": round(gbs, 6), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3 / max(1, args.steps), 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "FLUX.1-schnell-shaped activations, M=4608 tokens x d in {3072, 12288} bf16 "
+                               "(bounded row sample per step)", "M": FLUX_M, "d": list(FLUX_DS)},
+        "tokens_per_s": round(rows * args.steps / dt, 3),
+        "cpu_baseline": {"value": round(gbs, 6), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(gbs, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+# ---------------------------------------------------------------- sweep (config 4 and the named configs)
+
+def run_sweep(args) -> None:
+    import torch
+
+    import mxfp4_activations_b200 as kq
+    from mxfp4_activations_b200 import build
+
+    build.build()
+    kq.load()
+    lib = kq.load()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    cases = [(name, M, d) for name, c in inputs.CONFIGS.items() for d in c["ds"] for M in [c["M"]]]
+    cases += [("sweep", M, d) for M in inputs.SWEEP_M for d in inputs.SWEEP_D]
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    for name, M, d in cases:
+        x, p = inputs.sweep_case(M, d) if name == "sweep" else inputs.config_case(name, d)
+        xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+        pd = torch.from_numpy(p).cuda()
+        mats, fac = kq.kq_expand_blocks(pd), kq.kq_expand_factored(pd)
+        inv_s = torch.from_numpy(inputs.smooth_inv_scale(x)).cuda()
+        q = torch.empty((M, d // 2), dtype=torch.uint8, device="cuda")
+        s = torch.empty((M, d // 32), dtype=torch.uint8, device="cuda")
+        calls = {
+            "kroquant": lambda: lib.kq_quantize(xd.data_ptr(), M, d, d, mats.data_ptr(), 0, fac.data_ptr(),
+                                                q.data_ptr(), s.data_ptr(), 2, stream),
+            "smooth": lambda: lib.kq_ref_smooth_quantize(xd.data_ptr(), M, d, d, inv_s.data_ptr(), q.data_ptr(),
+                                                         s.data_ptr(), stream),
+            "fwht": lambda: lib.kq_ref_fwht_quantize(xd.data_ptr(), M, d, d, q.data_ptr(), s.data_ptr(), stream),
+        }
+        res = {}
+        reps = 30 if M * d < 2**26 else 10
+        for kind, fn in calls.items():
+            for _ in range(3):
+                assert fn() == 0
+            times = []
+            for _ in range(reps):
+                flush.fill_(1.0)  # evict L2 between launches
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                assert fn() == 0
+                b.record()
+                b.synchronize()
+                times.append(a.elapsed_time(b) * 1e3)
+            med = statistics.median(times)
+            res[kind] = {"us_median": round(med, 3), "us_best": round(min(times), 3),
+                         "gbs_median": round(algo_bytes(M, d) / (med * 1e-6) / 1e9, 1)}
+        line = {"sweep": name, "M": M, "d": d, "bytes": algo_bytes(M, d), **res,
+                "kroquant_vs_smooth_speed": round(res["smooth"]["us_median"] / res["kroquant"]["us_median"], 3),
+                "kroquant_vs_fwht_speed": round(res["fwht"]["us_median"] / res["kroquant"]["us_median"], 3)}
+        print(json.dumps(line), flush=True)
+        del xd, q, s
+    assert kq.kq_get_device_error(clear=True) == 0
+
+
+def run_profile(args) -> None:
+    """Small fixed launch sequence for ncu: every kernel kind on both FLUX
+    shapes, `--steps` times each, no soak, no clocks, no host-buffer pass."""
+    import torch
+
+    import mxfp4_activations_b200 as kq
+    from mxfp4_activations_b200 import build
+
+    build.build()
+    kq.load()
+    xs, ps = zip(*(inputs.config_case("flux", d) for d in FLUX_DS))
+    step = QuantStep(torch, kq, list(xs), list(ps), n_copies=1, device=torch.device("cuda", 0))
+    kinds = args.profile_kinds.split(",")
+    for kind in kinds:
+        for it in range(args.steps):
+            for item in step.items:
+                step.launch(it, item, kind)
+    torch.cuda.synchronize()
+    assert kq.kq_get_device_error(clear=True) == 0
+    print(json.dumps({"profile": kinds, "launches": len(kinds) * args.steps * len(FLUX_DS)}))
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["kq", "reference"], default="kq")
+    ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--profile", action="store_true", help="short launch sequence for ncu")
+    ap.add_argument("--profile-kinds", default="kroquant,smooth,fwht")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
+    elif args.profile:
+        run_profile(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,184 @@
+/*
+ * kq.h -- C ABI of the B200 (sm_100a) KroQuant online activation quantizer.
+ *
+ * The method (cited by page title and section):
+ *   [KQ-sum] "KroQuant: Kronecker-Structured Block Transforms for Efficient
+ *            Post-Training Quantization of Diffusion Transformers", research-map
+ *            summary page, sections "Approach", "Key results", "Limitations".
+ *   [KQ-abs] the KroQuant abstract (reprinted on two paper-listing pages).
+ *   [LRQ]    "LRQ-DiT: Log-Rotation Post-Training Quantization of Diffusion
+ *            Transformers", Sec. 3.2 eq. (2)-(3).
+ * Every 32-element block of a bf16 activation row is multiplied by its own
+ * learned invertible 32x32 matrix K_b = F0 (x) F1 (x) F2 (x) F3 (x) F4, each F_k a
+ * 2x2 unit-determinant LU factor (15 parameters per block) [KQ-sum, Approach],
+ * and the result is quantized to MXFP4 ("W4A4 (MXFP4e2)" [KQ-abs]): E2M1
+ * codes plus one E8M0 scale per 32 elements.
+ *
+ * Conventions fixed by this library (readings where the pages are silent):
+ *   params  fp32 [nb][5][3]: (l, u, v) of factor k; F_k = L U with
+ *           L = [[1,0],[l,1]], U = [[u,v],[0,1/u]]; F0 acts on the most
+ *           significant bit of the index inside the block.
+ *   y = x K (row vector, as X H in [LRQ] eq. 2); y_j is the fp32 rounding of the
+ *           exact sum over the block, K being the matrices given to kq_quantize.
+ *   scale   e = floor(log2 max|y|) - 2 clamped to [-127,127]; byte e + 127;
+ *           a block with max|y| = 0 has byte 0; a block holding a non-finite y
+ *           has byte 0xFF and zero codes.
+ *   codes   v = y 2^-e rounded to E2M1 (nearest, ties to even code, saturating
+ *           at 6, sign kept: a negative v that rounds to 0 gives code 0x8);
+ *           byte k of a row holds element 2k in its low nibble.
+ *
+ * Ownership: the caller owns every buffer (device memory unless stated).  No
+ * entry point allocates, frees or synchronises; all device work is enqueued on
+ * the given stream.  Argument errors are returned before anything is launched.
+ * A launch failure returns KQ_ERR_CUDA.  Kernels that wait on asynchronous
+ * copies bound every wait; a wait that runs out records a flag that
+ * kq_get_device_error() reports.
+ */
+#ifndef KQ_H
+#define KQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define KQ_API __attribute__((visibility("default")))
+#else
+#define KQ_API
+#endif
+
+/* Same type as cudaStream_t / CUstream; NULL is the legacy default stream. */
+typedef struct CUstream_st* kq_stream_t;
+
+typedef enum {
+  KQ_OK = 0,
+  KQ_ERR_INVALID_ARG = 1, /* NULL pointer where one is required, bad enum, negative size */
+  KQ_ERR_SHAPE = 2,       /* d not a multiple of 32, ldx < d, odd n, size overflow      */
+  KQ_ERR_ALIGN = 3,       /* a pointer or a row stride breaks the alignment stated below */
+  KQ_ERR_SINGULAR = 4,    /* a factor had u == 0 (reported by kq_get_device_error)      */
+  KQ_ERR_UNSUPPORTED = 5, /* variant / dtype combination not provided                   */
+  KQ_ERR_CUDA = 6,        /* a CUDA call failed (launch, attribute, tensor map)         */
+  KQ_ERR_DEVICE_TIMEOUT = 7 /* a kernel gave up a bounded wait (kq_get_device_error)    */
+} kq_status;
+
+typedef enum { KQ_F32 = 0, KQ_BF16 = 1 } kq_dtype;
+
+/* Which kernel computes the block transform inside kq_quantize.
+ *   KQ_VAR_BUTTERFLY: 5-stage 2x2 butterfly over registers (needs KQ_F32
+ *                     matrices and the factored form from kq_expand_factored).
+ *   KQ_VAR_MMA:       tensor-core product with the dense block matrix.
+ *   KQ_VAR_AUTO:      the faster provided variant for the shape and dtype. */
+typedef enum { KQ_VAR_AUTO = 0, KQ_VAR_MMA = 1, KQ_VAR_BUTTERFLY = 2 } kq_variant;
+
+#define KQ_BLOCK 32          /* elements per block / per E8M0 scale                */
+#define KQ_NFACTORS 5        /* 2x2 factors per block                              */
+#define KQ_PARAMS_PER_BLOCK 15
+#define KQ_FACTORED_FLOATS 48 /* floats per block in the factored form            */
+
+/* ---------------------------------------------------------------- set-up (once per layer)
+ *
+ * kq_expand_blocks -- [KQ-sum, Approach]: K_b = F0 (x) F1 (x) F2 (x) F3 (x) F4
+ * from the 15 LU parameters of each block; with inverse != 0,
+ * K_b^-1 = F0^-1 (x) ... (x) F4^-1 (det F_k = 1, so F^-1 = [[d,-b],[-c,a]]).
+ *   params  device fp32 [nb][5][3], 4-byte aligned.
+ *   nb      number of blocks (>= 0; 0 is a no-op).
+ *   mats    device [nb][32][32] row-major (row = input index i, column = output
+ *           index j, so y_j = sum_i x_i mats[i][j]); fp32 (KQ_F32) or bf16 bits
+ *           (KQ_BF16), 4-byte aligned.  Every entry is computed in fp64 and
+ *           rounded once (to nearest even) to out_dtype.
+ * A factor with u == 0 yields non-finite entries and sets the device flag
+ * read by kq_get_device_error() (KQ_ERR_SINGULAR).
+ */
+KQ_API kq_status kq_expand_blocks(const float* params, int64_t nb, int inverse, kq_dtype out_dtype,
+                           void* mats, kq_stream_t stream);
+
+/* kq_expand_factored -- the same K_b in the form the butterfly kernel applies:
+ * F_k = M_k diag(a_k, d_k) with M_k = [[1, b_k/d_k],[c_k/a_k, 1]], so that
+ * K_b = (M_0 (x) ... (x) M_4) D_b with D_b = diag_j prod_k (a_k or d_k).
+ *   factored  device fp32 [nb][48], 16-byte aligned:
+ *             [0..4]  c_k/a_k   [5..9] b_k/d_k   [10..41] D_b[j]
+ *             [42]    max_ij |K_b[i][j]| rounded up   [43] 1.0 when the block
+ *             must use the exact fp64 path (some d_k == 0 or a ratio overflows)
+ *             [44]    absolute error allowance for fp32-subnormal results
+ *             [45..47] zero.  Coefficients are fp64 values rounded once.
+ */
+KQ_API kq_status kq_expand_factored(const float* params, int64_t nb, float* factored, kq_stream_t stream);
+
+/* ---------------------------------------------------------------- hot path
+ *
+ * kq_quantize -- [KQ-abs]: each 32-element block goes through its own
+ * transform, then MXFP4 ("W4A4 (MXFP4e2)"): y = x K_b, one E8M0 scale and 32
+ * E2M1 codes per block, in one pass over x.
+ *   x        device bf16 bits [M][ldx]; 16-byte aligned; ldx % 8 == 0; ldx >= d.
+ *   M        rows (tokens) >= 0 (0 is a no-op);  d = channels, d % 32 == 0.
+ *   mats     device [d/32][32][32] from kq_expand_blocks in mat_dtype.  The
+ *            output is defined by these matrices (see the header comment).
+ *   factored device [d/32][48] from kq_expand_factored for the same params, or
+ *            NULL; required by KQ_VAR_BUTTERFLY.
+ *   q        device [M][d/2] packed E2M1 codes, 16-byte aligned.
+ *   scales   device [M][d/32] E8M0 bytes.
+ * The butterfly variant computes y in fp32, bounds its rounding error from the
+ * block's L1 norm and max|K_b|, and recomputes in fp64 (summing in increasing i)
+ * exactly those scales and codes that the bound cannot certify, so its output
+ * equals the fp64 definition.
+ */
+KQ_API kq_status kq_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const void* mats,
+                      kq_dtype mat_dtype, const float* factored, uint8_t* q, uint8_t* scales,
+                      kq_variant variant, kq_stream_t stream);
+
+/* kq_dequantize -- inverse of the MXFP4 step [KQ-abs]: yhat_j = E2M1(code_j) *
+ * 2^(byte-127) (byte 0xFF gives NaN), and, when inv_mats != NULL, the block
+ * transform is undone, xhat = yhat K_b^-1 (the activation side of [LRQ] eq. 2).
+ *   q, scales  device, as produced by kq_quantize ([M][d/2], [M][d/32]); q 16-byte aligned.
+ *   inv_mats   device [d/32][32][32] in mat_dtype (kq_expand_blocks, inverse=1) or NULL.
+ *   out        device [M][d] in out_dtype (fp32 or bf16 bits), 16-byte aligned.
+ * Without inv_mats the fp32 result is exact; with it, the fp32 sum has the
+ * rounding error of 32 fused multiply-adds.
+ */
+KQ_API kq_status kq_dequantize(const uint8_t* q, const uint8_t* scales, int64_t M, int64_t d,
+                        const void* inv_mats, kq_dtype mat_dtype, void* out, kq_dtype out_dtype,
+                        kq_stream_t stream);
+
+/* ---------------------------------------------------------------- comparison points
+ *
+ * kq_ref_smooth_quantize -- per-channel scaling (SmoothQuant) then MXFP4, the
+ * cheaper comparison kernel of [KQ-sum, Key results] and [KQ-abs]:
+ * y_j = fp32(x_j * inv_s[j]).  Same layouts and alignment as kq_quantize;
+ * inv_s is device fp32 [d], 16-byte aligned.
+ */
+KQ_API kq_status kq_ref_smooth_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const float* inv_s,
+                                 uint8_t* q, uint8_t* scales, kq_stream_t stream);
+
+/* kq_ref_fwht_quantize -- fixed 32-point Hadamard then MXFP4, the FWHT
+ * comparison point of [KQ-sum, Key results]: every block is multiplied by the
+ * normalised Sylvester matrix H_32 of [LRQ] eq. 3 rounded to fp32, with the same
+ * exactness guarantee as the butterfly variant of kq_quantize. */
+KQ_API kq_status kq_ref_fwht_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, uint8_t* q,
+                               uint8_t* scales, kq_stream_t stream);
+
+/* kq_e2m1_pack -- the element step of MXFP4 alone: out[k] = code(v[2k]) |
+ * code(v[2k+1]) << 4 for already scaled fp32 values (same rounding as
+ * kq_quantize).  v device fp32 [n], out device [n/2]; n even. */
+KQ_API kq_status kq_e2m1_pack(const float* v, int64_t n, uint8_t* out, kq_stream_t stream);
+
+/* ---------------------------------------------------------------- status
+ *
+ * kq_get_device_error -- synchronises the current device and reports the
+ * flags kernels on it have recorded: KQ_ERR_DEVICE_TIMEOUT (a bounded wait ran
+ * out), KQ_ERR_SINGULAR (a factor with u == 0), else KQ_OK.  clear != 0 resets
+ * the flags.  Returns KQ_ERR_CUDA if the device cannot be read. */
+KQ_API kq_status kq_get_device_error(int clear);
+
+/* Static, human-readable name of a status code. */
+KQ_API const char* kq_status_string(kq_status status);
+
+/* ABI version of this header (major * 100 + minor). */
+KQ_API int kq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KQ_H */

@@ -1,1 +1,52 @@
-"""B200-native KroQuant online activation quantizer (placeholder, filled below)."""
+"""B200-native (sm_100a) KroQuant online activation quantizer.
+
+Every 32-element block of a bf16 activation row is multiplied by its own
+Kronecker-structured 32x32 transform (five 2x2 unit-determinant LU factors,
+15 parameters per block) and quantized to MXFP4 (E2M1 codes + one E8M0 scale
+per block), as described on the "KroQuant: Kronecker-Structured Block
+Transforms for Efficient Post-Training Quantization of Diffusion Transformers"
+pages.  The work is done by libkq.so (include/kq.h); this package is its
+thin ctypes binding plus seeded input generators (``inputs``).
+"""
+from ._lib import (  # noqa: F401
+    EXPORTED,
+    KQError,
+    kq_abi_version,
+    kq_dequantize,
+    kq_e2m1_pack,
+    kq_expand_blocks,
+    kq_expand_factored,
+    kq_get_device_error,
+    kq_quantize,
+    kq_ref_fwht_quantize,
+    kq_ref_smooth_quantize,
+    kq_status_string,
+    load,
+)
+
+
+class BlockTransform:
+    """The per-layer set-up of one KroQuant transform: the LU parameters
+    [d/32, 5, 3] expanded once into the dense block matrices (fp32 and bf16), their
+    inverses and the butterfly (factored) form, then reused for every call."""
+
+    def __init__(self, params):
+        self.params = params.contiguous()
+        self.mats = kq_expand_blocks(self.params)
+        self.factored = kq_expand_factored(self.params)
+        self._inv = None
+
+    @property
+    def inverse_mats(self):
+        if self._inv is None:
+            self._inv = kq_expand_blocks(self.params, inverse=True)
+        return self._inv
+
+    def quantize(self, x, variant: str = "auto", q=None, scales=None):
+        return kq_quantize(x, self.mats, self.factored, variant=variant, q=q, scales=scales)
+
+    def dequantize(self, q, scales, undo_transform: bool = True, out_dtype=None):
+        import torch
+
+        return kq_dequantize(q, scales, self.inverse_mats if undo_transform else None,
+                             out_dtype=out_dtype or torch.float32)

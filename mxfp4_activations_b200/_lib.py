@@ -1,0 +1,213 @@
+"""ctypes binding of libkq.so (include/kq.h).
+
+Argument marshalling only: every function checks tensor dtypes, devices and
+shapes, passes raw device pointers and the current CUDA stream to the C ABI
+and raises on a non-zero status.  There is no fallback: if libkq.so is missing
+or a call fails, an exception says so.  PyTorch provides device memory and
+streams; all arithmetic runs in the library's kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkq.so")
+
+KQ_F32, KQ_BF16 = 0, 1
+VARIANTS = {"auto": 0, "mma": 1, "butterfly": 2}
+STATUS = {
+    0: "KQ_OK", 1: "KQ_ERR_INVALID_ARG", 2: "KQ_ERR_SHAPE", 3: "KQ_ERR_ALIGN", 4: "KQ_ERR_SINGULAR",
+    5: "KQ_ERR_UNSUPPORTED", 6: "KQ_ERR_CUDA", 7: "KQ_ERR_DEVICE_TIMEOUT",
+}
+EXPORTED = (
+    "kq_expand_blocks", "kq_expand_factored", "kq_quantize", "kq_dequantize", "kq_ref_smooth_quantize",
+    "kq_ref_fwht_quantize", "kq_e2m1_pack", "kq_get_device_error", "kq_status_string", "kq_abi_version",
+)
+
+
+class KQError(RuntimeError):
+    def __init__(self, fn: str, status: int, message: str):
+        super().__init__(f"{fn} failed: {message}")
+        self.status = status
+        self.status_name = STATUS.get(status, str(status))
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libkq.so (built by mxfp4_activations_b200.build); raises if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"libkq.so not found at {path}: build it with `python -m mxfp4_activations_b200.build` "
+            "(there is no CPU fallback)")
+    L = ctypes.CDLL(path)
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    sig = {
+        "kq_expand_blocks": [P, I64, I, I, P, P],
+        "kq_expand_factored": [P, I64, P, P],
+        "kq_quantize": [P, I64, I64, I64, P, I, P, P, P, I, P],
+        "kq_dequantize": [P, P, I64, I64, P, I, P, I, P],
+        "kq_ref_smooth_quantize": [P, I64, I64, I64, P, P, P, P],
+        "kq_ref_fwht_quantize": [P, I64, I64, I64, P, P, P],
+        "kq_e2m1_pack": [P, I64, P, P],
+        "kq_get_device_error": [I],
+        "kq_status_string": [I],
+        "kq_abi_version": [],
+    }
+    for name, args in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = I
+    L.kq_status_string.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        msg = load().kq_status_string(status).decode()
+        raise KQError(fn, status, msg)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _cuda(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _mat_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KQ_F32
+    if t.dtype in (torch.bfloat16, torch.int16, torch.uint16):
+        return KQ_BF16
+    raise TypeError("matrices must be float32 or bfloat16")
+
+
+def _rows(x: torch.Tensor, name: str = "x"):
+    """(M, d, ldx) of a 2-D bf16 activation whose rows may be strided."""
+    if x.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError(f"{name} must be bfloat16 (or its 16-bit patterns)")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError(f"{name} must be 2-D with unit column stride")
+    return x.shape[0], x.shape[1], x.stride(0)
+
+
+# ---------------------------------------------------------------- set-up
+
+def kq_expand_blocks(params: torch.Tensor, inverse: bool = False, dtype: torch.dtype = torch.float32,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    _cuda(params, "params")
+    params = params.contiguous()
+    if params.dtype != torch.float32 or params.numel() % 15 != 0:
+        raise ValueError("params must be float32 [nb, 5, 3]")
+    nb = params.numel() // 15
+    if out is None:
+        out = torch.empty((nb, 32, 32), dtype=dtype, device=params.device)
+    _check("kq_expand_blocks", load().kq_expand_blocks(_ptr(params), nb, int(bool(inverse)), _mat_dtype(out),
+                                                         _ptr(out), _stream(params.device)))
+    return out
+
+
+def kq_expand_factored(params: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    _cuda(params, "params")
+    params = params.contiguous()
+    if params.dtype != torch.float32 or params.numel() % 15 != 0:
+        raise ValueError("params must be float32 [nb, 5, 3]")
+    nb = params.numel() // 15
+    if out is None:
+        out = torch.empty((nb, 48), dtype=torch.float32, device=params.device)
+    _check("kq_expand_factored", load().kq_expand_factored(_ptr(params), nb, _ptr(out), _stream(params.device)))
+    return out
+
+
+# ---------------------------------------------------------------- hot path
+
+def _outputs(x: torch.Tensor, M: int, d: int, q, scales):
+    if q is None:
+        q = torch.empty((M, d // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((M, d // 32), dtype=torch.uint8, device=x.device)
+    if q.dtype != torch.uint8 or scales.dtype != torch.uint8 or not q.is_contiguous() or not scales.is_contiguous():
+        raise ValueError("q and scales must be contiguous uint8")
+    if q.numel() < M * (d // 2) or scales.numel() < M * (d // 32):
+        raise ValueError("q or scales too small")
+    return q, scales
+
+
+def kq_quantize(x: torch.Tensor, mats: torch.Tensor, factored: torch.Tensor | None = None, variant: str = "auto",
+                q: torch.Tensor | None = None, scales: torch.Tensor | None = None):
+    """MXFP4 of x K_b per 32-element block -> (codes uint8 [M, d/2], E8M0 uint8 [M, d/32])."""
+    _cuda(x, "x")
+    M, d, ldx = _rows(x)
+    q, scales = _outputs(x, M, d, q, scales)
+    _check("kq_quantize", load().kq_quantize(_ptr(x), M, d, ldx, _ptr(mats), _mat_dtype(mats), _ptr(factored),
+                                             _ptr(q), _ptr(scales), VARIANTS[variant], _stream(x.device)))
+    return q, scales
+
+
+def kq_dequantize(q: torch.Tensor, scales: torch.Tensor, inv_mats: torch.Tensor | None = None,
+                  out_dtype: torch.dtype = torch.float32, out: torch.Tensor | None = None) -> torch.Tensor:
+    _cuda(q, "q")
+    M, d = q.shape[0], q.shape[1] * 2
+    if out is None:
+        out = torch.empty((M, d), dtype=out_dtype, device=q.device)
+    mdt = _mat_dtype(inv_mats) if inv_mats is not None else KQ_F32
+    _check("kq_dequantize", load().kq_dequantize(_ptr(q), _ptr(scales), M, d, _ptr(inv_mats), mdt, _ptr(out),
+                                                 _mat_dtype(out), _stream(q.device)))
+    return out
+
+
+def kq_ref_smooth_quantize(x: torch.Tensor, inv_s: torch.Tensor, q=None, scales=None):
+    _cuda(x, "x")
+    M, d, ldx = _rows(x)
+    q, scales = _outputs(x, M, d, q, scales)
+    _check("kq_ref_smooth_quantize", load().kq_ref_smooth_quantize(_ptr(x), M, d, ldx, _ptr(inv_s), _ptr(q),
+                                                                   _ptr(scales), _stream(x.device)))
+    return q, scales
+
+
+def kq_ref_fwht_quantize(x: torch.Tensor, q=None, scales=None):
+    _cuda(x, "x")
+    M, d, ldx = _rows(x)
+    q, scales = _outputs(x, M, d, q, scales)
+    _check("kq_ref_fwht_quantize", load().kq_ref_fwht_quantize(_ptr(x), M, d, ldx, _ptr(q), _ptr(scales),
+                                                               _stream(x.device)))
+    return q, scales
+
+
+def kq_e2m1_pack(v: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    _cuda(v, "v")
+    v = v.contiguous()
+    if v.dtype != torch.float32:
+        raise TypeError("v must be float32")
+    if out is None:
+        out = torch.empty(v.numel() // 2, dtype=torch.uint8, device=v.device)
+    _check("kq_e2m1_pack", load().kq_e2m1_pack(_ptr(v), v.numel(), _ptr(out), _stream(v.device)))
+    return out
+
+
+def kq_get_device_error(clear: bool = True) -> int:
+    """Synchronises the current device; returns the kq_status of recorded device flags."""
+    return int(load().kq_get_device_error(int(bool(clear))))
+
+
+def kq_status_string(status: int) -> str:
+    return load().kq_status_string(int(status)).decode()
+
+
+def kq_abi_version() -> int:
+    return int(load().kq_abi_version())

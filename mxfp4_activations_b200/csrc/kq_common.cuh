@@ -1,0 +1,149 @@
+// kq_common.cuh -- device helpers shared by the kernels of libkq (sm_100a only).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libkq is written for sm_100a (B200) only"
+#endif
+
+namespace kq {
+
+constexpr int kBlock = 32;            // elements per MX block
+constexpr int kFactored = 48;         // floats per block in the factored form
+
+// Flags recorded by kernels (read and cleared by kq_get_device_error).
+constexpr unsigned kDevErrTimeout = 1u;
+constexpr unsigned kDevErrSingular = 2u;
+
+// One status word per device; only flag bits are ever OR-ed into it.
+__device__ unsigned int g_dev_error;
+
+__device__ __forceinline__ void record_error(unsigned bits) { atomicOr(&g_dev_error, bits); }
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
+
+// E2M1 codes of 8 fp32 values: nibble e of the result holds the code of v[e].
+// cvt.rn.satfinite.e2m1x2.f32 d, a, b puts a's code in the high nibble of d.
+__device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v3, float v4, float v5,
+                                           float v6, float v7) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c3, %8, %7;\n\t"
+      "mov.b32 %0, {c0, c1, c2, c3};\n\t}"
+      : "=r"(r)
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+  return r;
+}
+
+// E2M1 code of one value (low nibble).
+__device__ __forceinline__ uint32_t e2m1_one(float v) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 c0;\n\t.reg .b16 h;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c0, %1, %1;\n\t"
+      "cvt.u16.u8 h, c0;\n\t"
+      "cvt.u32.u16 %0, h;\n\t}"
+      : "=r"(r)
+      : "f"(v));
+  return r & 0xFu;
+}
+
+// E8M0 byte of a non-negative finite block maximum m: floor(log2 m) - 2 clamped
+// at -127, plus 127, which is max(exponent field - 2, 0) for every m >= 0.
+__device__ __forceinline__ int e8m0_byte(float m) {
+  const int ef = int(__float_as_uint(m) >> 23);
+  return ef > 2 ? ef - 2 : 0;
+}
+// 2^-e for a scale byte in [0, 252]: an fp32 with exponent field 254 - byte.
+__device__ __forceinline__ float inv_scale_of_byte(int byte) { return __uint_as_float(uint32_t(254 - byte) << 23); }
+
+// max with NaN propagation (a NaN anywhere makes the block maximum NaN).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---------------------------------------------------------------- mbarrier / TMA (no multicast)
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+// Make freshly initialised barriers visible to the other threads and to the
+// asynchronous (TMA) proxy.
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Returns false (and
+// records kDevErrTimeout) when it has not completed after limit_ns.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > limit_ns) {
+      record_error(kDevErrTimeout);
+      return false;
+    }
+  }
+}
+
+// 3-D tiled TMA load (coordinates innermost first) completing on an mbarrier.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0,
+                                            int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+      "[%2];" ::"r"(smem_addr(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+}  // namespace kq

@@ -1,0 +1,144 @@
+// kq_expand.cuh -- set-up kernels: LU parameters -> block matrices / factored form.
+//
+// "KroQuant: Kronecker-Structured Block Transforms ...", Approach: each 32x32
+// block transform is the Kronecker product of five 2x2 unit-determinant LU
+// factors (15 parameters per block).  Factor k of block b is F = L U with
+// L = [[1,0],[l,1]], U = [[u,v],[0,1/u]], (l,u,v) = params[b][k]; F0 is the
+// outermost factor (it acts on the top bit of the index inside the block).
+// All set-up arithmetic is fp64 with explicit IEEE operations, rounded once.
+#pragma once
+
+#include "kq_common.cuh"
+
+namespace kq {
+
+// F = L U written as the 2x2 matrix product (row r, column c of F is
+// L[r][0] U[0][c] + L[r][1] U[1][c], zero terms included, so signed zeros
+// follow the same IEEE rules as the product written out).
+__device__ __forceinline__ void lu_factor(const float* __restrict__ prm, double F[4]) {
+  const double l = prm[0], u = prm[1], v = prm[2];
+  const double L[4] = {1.0, 0.0, l, 1.0};
+  const double U[4] = {u, v, 0.0, __ddiv_rn(1.0, u)};
+#pragma unroll
+  for (int r = 0; r < 2; r++)
+#pragma unroll
+    for (int c = 0; c < 2; c++)
+      F[2 * r + c] = __dadd_rn(__dmul_rn(L[2 * r], U[c]), __dmul_rn(L[2 * r + 1], U[2 + c]));
+}
+
+// F^-1 = U^-1 L^-1, U^-1 = [[1/u, -v],[0, u]], L^-1 = [[1,0],[-l,1]].
+__device__ __forceinline__ void lu_factor_inverse(const float* __restrict__ prm, double F[4]) {
+  const double l = prm[0], u = prm[1], v = prm[2];
+  const double Ui[4] = {__ddiv_rn(1.0, u), -v, 0.0, u};
+  const double Li[4] = {1.0, 0.0, -l, 1.0};
+#pragma unroll
+  for (int r = 0; r < 2; r++)
+#pragma unroll
+    for (int c = 0; c < 2; c++)
+      F[2 * r + c] = __dadd_rn(__dmul_rn(Ui[2 * r], Li[c]), __dmul_rn(Ui[2 * r + 1], Li[2 + c]));
+}
+
+// Round-to-nearest-even of a double to bf16 bits, from the definition: the
+// spacing of bf16 values around |a| is 2^(max(E,-126) - 7), E = floor(log2 |a|).
+__device__ __forceinline__ uint16_t bf16_rne_from_f64(double a) {
+  if (isnan(a)) return 0x7FC0;
+  const uint16_t sign = signbit(a) ? 0x8000 : 0;
+  const double m = fabs(a);
+  if (m == 0.0) return sign;
+  if (isinf(m)) return sign | 0x7F80;
+  int E = int((__double_as_longlong(m) >> 52) & 0x7FF) - 1023;  // fp64 subnormals: far below bf16
+  if (E < -126) E = -126;
+  const int qe = E - 7;
+  const double n = scalbn(m, -qe);  // exact
+  double k = floor(n);
+  const double fr = n - k;
+  if (fr > 0.5 || (fr == 0.5 && fmod(k, 2.0) != 0.0)) k += 1.0;
+  const float r = float(scalbn(k, qe));  // exact (or +inf past the largest bf16)
+  return sign | uint16_t(__float_as_uint(r) >> 16);
+}
+
+// One thread per matrix entry: K[i][j] = F0[i4][j4] (F1[i3][j3] (F2 (F3 F4))),
+// the Kronecker product assembled from the innermost factor outward.
+__global__ void expand_kernel(const float* __restrict__ params, int64_t nb, int inverse, int out_bf16,
+                              void* __restrict__ mats) {
+  const int64_t gid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gid >= nb * 1024) return;
+  const int64_t b = gid >> 10;
+  const int i = int(gid >> 5) & 31, j = int(gid) & 31;
+  double F[5][4];
+  bool singular = false;
+#pragma unroll
+  for (int k = 0; k < 5; k++) {
+    const float* prm = params + b * 15 + 3 * k;
+    if (prm[1] == 0.0f) singular = true;
+    if (inverse)
+      lu_factor_inverse(prm, F[k]);
+    else
+      lu_factor(prm, F[k]);
+  }
+  double acc = F[4][2 * (i & 1) + (j & 1)];
+#pragma unroll
+  for (int k = 3; k >= 0; k--) {
+    const int bi = (i >> (4 - k)) & 1, bj = (j >> (4 - k)) & 1;
+    acc = __dmul_rn(F[k][2 * bi + bj], acc);
+  }
+  if (singular && i == 0 && j == 0) record_error(kDevErrSingular);
+  if (out_bf16)
+    static_cast<uint16_t*>(mats)[gid] = bf16_rne_from_f64(acc);
+  else
+    static_cast<float*>(mats)[gid] = __double2float_rn(acc);
+}
+
+// One thread per block: the butterfly form F_k = M_k diag(a_k, d_k).
+__global__ void expand_factored_kernel(const float* __restrict__ params, int64_t nb, float* __restrict__ out) {
+  const int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (b >= nb) return;
+  double a[5], d[5];
+  double kmax = 1.0, gain = 1.0;
+  bool exact_only = false;
+  float* o = out + b * kFactored;
+#pragma unroll
+  for (int k = 0; k < 5; k++) {
+    const float* prm = params + b * 15 + 3 * k;
+    if (prm[1] == 0.0f) {
+      record_error(kDevErrSingular);
+      exact_only = true;
+    }
+    double F[4];
+    lu_factor(prm, F);
+    a[k] = F[0];
+    d[k] = F[3];
+    const double lam = __ddiv_rn(F[2], F[0]);
+    const double bet = __ddiv_rn(F[1], F[3]);
+    const float lam32 = __double2float_rn(lam), bet32 = __double2float_rn(bet);
+    // ratios must be finite and moderate for the fp32 butterfly to be usable
+    if (!(fabsf(lam32) <= 1.8446744e19f) || !(fabsf(bet32) <= 1.8446744e19f)) exact_only = true;
+    o[k] = lam32;
+    o[5 + k] = bet32;
+    const double mk = fmax(fmax(fabs(F[0]), fabs(F[1])), fmax(fabs(F[2]), fabs(F[3])));
+    kmax = __dmul_rn(kmax, mk);
+    gain = __dmul_rn(gain, 1.0 + fmax(fabs(double(lam32)), fabs(double(bet32))));
+  }
+  double dmax = 0.0;
+  for (int j = 0; j < 32; j++) {
+    double dj = 1.0;
+#pragma unroll
+    for (int k = 0; k < 5; k++) dj = __dmul_rn(dj, ((j >> (4 - k)) & 1) ? d[k] : a[k]);
+    const float dj32 = __double2float_rn(dj);
+    if (!(fabsf(dj32) <= 3.0e38f) || dj32 == 0.0f) exact_only = true;
+    o[10 + j] = dj32;
+    dmax = fmax(dmax, fabs(double(dj32)));
+  }
+  // upper bound of max|K| (fp64 product error is far below the 2^-20 margin)
+  const float km = __fmul_ru(__double2float_ru(kmax), 1.00000095367431640625f);
+  if (!(km <= 1.0e30f)) exact_only = true;
+  o[42] = km;
+  o[43] = exact_only ? 1.0f : 0.0f;
+  // absolute error of results that fall in the fp32 subnormal range: each of the
+  // 6 roundings on an output's path adds at most 2^-150, amplified by at most
+  // max|D| * prod_k (1 + max(|c/a|, |b/d|)); 2^-145 leaves a margin.
+  o[44] = __fmul_ru(__double2float_ru(__dmul_rn(dmax, gain)), 2.2420775429197073e-44f);
+  o[45] = o[46] = o[47] = 0.0f;
+}
+
+}  // namespace kq

@@ -1,0 +1,308 @@
+// kq_lib.cu -- C ABI of libkq (declared in include/kq.h): argument checks,
+// launch configuration and tensor-map set-up for the sm_100a kernels.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "kq.h"
+#include "kq_common.cuh"
+#include "kq_expand.cuh"
+#include "kq_misc.cuh"
+#include "kq_quant.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+cudaStream_t as_cuda(kq_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+kq_status launch_status() { return cudaGetLastError() == cudaSuccess ? KQ_OK : KQ_ERR_CUDA; }
+
+// ---- per-device facts, cached
+struct DeviceInfo {
+  std::once_flag once;
+  int sms = 0;
+  int smem_optin = 0;
+  bool ok = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+const DeviceInfo* device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  DeviceInfo& d = g_dev[dev];
+  std::call_once(d.once, [&]() {
+    d.ok = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+           cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess;
+  });
+  return d.ok ? &d : nullptr;
+}
+
+// ---- cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda)
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// ---- launch geometry of the quantizer kernels
+struct QuantGeom {
+  int W, R, threads, stages, stage_stride, smem;
+};
+
+QuantGeom quant_geometry(int nb, int smem_optin) {
+  QuantGeom g{};
+  const int ncol = (nb + 255) / 256;
+  g.W = (nb + ncol - 1) / ncol;  // <= 256 (TMA box limit)
+  int bestR = 1;
+  double bestU = -1.0;
+  for (int R = 1; R * g.W <= 256; R++) {
+    const int T = ((R * g.W + 31) / 32) * 32;
+    const double u = double(R * g.W) / double(T);
+    // prefer full warps, then CTAs near 256 threads
+    const double score = u - 0.0005 * double(T > 256 ? T - 256 : 256 - T) / 32.0;
+    if (score > bestU + 1e-12) {
+      bestU = score;
+      bestR = R;
+    }
+  }
+  g.R = bestR;
+  g.threads = ((g.R * g.W + 31) / 32) * 32;
+  const int stage_bytes = g.W * g.R * 64;
+  g.stage_stride = (stage_bytes + 1023) & ~1023;
+  int st = (96 * 1024) / g.stage_stride;
+  if (st > 6) st = 6;
+  if (st < 2) st = 2;
+  const int fixed = 1024 /*alignment slack*/ + 64 /*barriers*/;
+  while (st > 2 && st * g.stage_stride + fixed > smem_optin) st--;
+  g.stages = st;
+  g.smem = st * g.stage_stride + fixed;
+  return g;
+}
+
+template <int MODE>
+kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const float* mats, const float* factored,
+                       const float* inv_s, uint8_t* q, uint8_t* scales, cudaStream_t stream) {
+  const DeviceInfo* dev = device_info();
+  EncodeTiledFn enc = encode_tiled();
+  if (dev == nullptr || enc == nullptr) return KQ_ERR_CUDA;
+  const int nb = int(d / 32);
+  const QuantGeom g = quant_geometry(nb, dev->smem_optin);
+  if (g.smem > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
+
+  CUtensorMap tmap;
+  const cuuint64_t gdim[3] = {32, cuuint64_t(nb), cuuint64_t(M)};
+  const cuuint64_t gstride[2] = {64, cuuint64_t(ldx) * 2};
+  const cuuint32_t box[3] = {32, cuuint32_t(g.W), cuuint32_t(g.R)};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), gdim, gstride, box, estride,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return KQ_ERR_CUDA;
+
+  auto kern = kq::quant_kernel<MODE>;
+  static std::atomic<int> smem_set[kMaxDevices];
+  int devid = 0;
+  cudaGetDevice(&devid);
+  if (smem_set[devid].load() < g.smem) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev->smem_optin) != cudaSuccess)
+      return KQ_ERR_CUDA;
+    smem_set[devid].store(dev->smem_optin);
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.threads, g.smem) != cudaSuccess ||
+      per_sm < 1)
+    return KQ_ERR_CUDA;
+
+  kq::QuantParams p;
+  p.x = static_cast<const uint16_t*>(x);
+  p.ldx = ldx;
+  p.M = M;
+  p.nb = nb;
+  p.W = g.W;
+  p.R = g.R;
+  const int64_t nrt = (M + g.R - 1) / g.R;
+  if (nrt > int64_t(INT32_MAX)) return KQ_ERR_SHAPE;
+  p.n_row_tiles = int(nrt);
+  p.stages = g.stages;
+  p.stage_stride = g.stage_stride;
+  p.mats = mats;
+  p.factored = factored;
+  p.inv_s = inv_s;
+  p.q = q;
+  p.scales = scales;
+
+  const int ncol = (nb + g.W - 1) / g.W;
+  const int64_t target = int64_t(dev->sms) * per_sm;
+  int64_t gy = (target + ncol - 1) / ncol;
+  if (gy > nrt) gy = nrt;
+  if (gy > 65535) gy = 65535;
+  if (gy < 1) gy = 1;
+  kern<<<dim3(ncol, unsigned(gy)), g.threads, g.smem, stream>>>(tmap, p);
+  return launch_status();
+}
+
+kq_status check_x(const void* x, int64_t M, int64_t d, int64_t ldx) {
+  if (M < 0 || d < 0) return KQ_ERR_INVALID_ARG;
+  if (d % 32 != 0 || ldx < d) return KQ_ERR_SHAPE;
+  if (d / 32 > int64_t(INT32_MAX) / 2 || M > (int64_t(1) << 40)) return KQ_ERR_SHAPE;
+  if (x == nullptr) return KQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || ldx % 8 != 0) return KQ_ERR_ALIGN;
+  return KQ_OK;
+}
+
+kq_status check_out(const uint8_t* q, const uint8_t* scales) {
+  if (q == nullptr || scales == nullptr) return KQ_ERR_INVALID_ARG;
+  if (!aligned(q, 16)) return KQ_ERR_ALIGN;
+  return KQ_OK;
+}
+
+int grid_for(int64_t work, int threads) {
+  const DeviceInfo* dev = device_info();
+  const int64_t cap = dev ? int64_t(dev->sms) * 8 : 1184;
+  int64_t g = (work + threads - 1) / threads;
+  if (g > cap) g = cap;
+  return g < 1 ? 1 : int(g);
+}
+
+}  // namespace
+
+extern "C" {
+
+int kq_abi_version(void) { return 100; }
+
+const char* kq_status_string(kq_status s) {
+  switch (s) {
+    case KQ_OK: return "KQ_OK";
+    case KQ_ERR_INVALID_ARG: return "KQ_ERR_INVALID_ARG: null pointer, bad enum or negative size";
+    case KQ_ERR_SHAPE: return "KQ_ERR_SHAPE: d must be a multiple of 32 and ldx >= d";
+    case KQ_ERR_ALIGN: return "KQ_ERR_ALIGN: pointer or row stride not aligned as required";
+    case KQ_ERR_SINGULAR: return "KQ_ERR_SINGULAR: an LU factor has u == 0";
+    case KQ_ERR_UNSUPPORTED: return "KQ_ERR_UNSUPPORTED: variant/dtype combination not provided";
+    case KQ_ERR_CUDA: return "KQ_ERR_CUDA: a CUDA call failed";
+    case KQ_ERR_DEVICE_TIMEOUT: return "KQ_ERR_DEVICE_TIMEOUT: a kernel gave up a bounded wait";
+  }
+  return "unknown kq_status";
+}
+
+kq_status kq_expand_blocks(const float* params, int64_t nb, int inverse, kq_dtype out_dtype, void* mats,
+                           kq_stream_t stream) {
+  if (nb < 0 || (out_dtype != KQ_F32 && out_dtype != KQ_BF16)) return KQ_ERR_INVALID_ARG;
+  if (nb == 0) return KQ_OK;
+  if (params == nullptr || mats == nullptr) return KQ_ERR_INVALID_ARG;
+  if (!aligned(params, 4) || !aligned(mats, 4)) return KQ_ERR_ALIGN;
+  if (nb > (int64_t(1) << 30)) return KQ_ERR_SHAPE;
+  const int64_t n = nb * 1024;
+  kq::expand_kernel<<<unsigned((n + 255) / 256), 256, 0, as_cuda(stream)>>>(params, nb, inverse ? 1 : 0,
+                                                                           out_dtype == KQ_BF16 ? 1 : 0, mats);
+  return launch_status();
+}
+
+kq_status kq_expand_factored(const float* params, int64_t nb, float* factored, kq_stream_t stream) {
+  if (nb < 0) return KQ_ERR_INVALID_ARG;
+  if (nb == 0) return KQ_OK;
+  if (params == nullptr || factored == nullptr) return KQ_ERR_INVALID_ARG;
+  if (!aligned(params, 4) || !aligned(factored, 16)) return KQ_ERR_ALIGN;
+  if (nb > (int64_t(1) << 30)) return KQ_ERR_SHAPE;
+  kq::expand_factored_kernel<<<unsigned((nb + 127) / 128), 128, 0, as_cuda(stream)>>>(params, nb, factored);
+  return launch_status();
+}
+
+kq_status kq_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const void* mats, kq_dtype mat_dtype,
+                      const float* factored, uint8_t* q, uint8_t* scales, kq_variant variant,
+                      kq_stream_t stream) {
+  if (variant != KQ_VAR_AUTO && variant != KQ_VAR_MMA && variant != KQ_VAR_BUTTERFLY) return KQ_ERR_INVALID_ARG;
+  if (mat_dtype != KQ_F32 && mat_dtype != KQ_BF16) return KQ_ERR_INVALID_ARG;
+  kq_status st = check_x(x, M, d, ldx);
+  if (st != KQ_OK) return st;
+  if (M == 0 || d == 0) return KQ_OK;
+  st = check_out(q, scales);
+  if (st != KQ_OK) return st;
+  if (mats == nullptr) return KQ_ERR_INVALID_ARG;
+  if (!aligned(mats, 16)) return KQ_ERR_ALIGN;
+  if (variant == KQ_VAR_MMA || mat_dtype == KQ_BF16) return KQ_ERR_UNSUPPORTED;
+  if (factored == nullptr) return KQ_ERR_INVALID_ARG;
+  if (!aligned(factored, 16)) return KQ_ERR_ALIGN;
+  return launch_quant<kq::MODE_KRON>(x, M, d, ldx, static_cast<const float*>(mats), factored, nullptr, q, scales,
+                                     as_cuda(stream));
+}
+
+kq_status kq_ref_smooth_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const float* inv_s,
+                                 uint8_t* q, uint8_t* scales, kq_stream_t stream) {
+  kq_status st = check_x(x, M, d, ldx);
+  if (st != KQ_OK) return st;
+  if (M == 0 || d == 0) return KQ_OK;
+  st = check_out(q, scales);
+  if (st != KQ_OK) return st;
+  if (inv_s == nullptr) return KQ_ERR_INVALID_ARG;
+  if (!aligned(inv_s, 16)) return KQ_ERR_ALIGN;
+  return launch_quant<kq::MODE_SMOOTH>(x, M, d, ldx, nullptr, nullptr, inv_s, q, scales, as_cuda(stream));
+}
+
+kq_status kq_ref_fwht_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, uint8_t* q, uint8_t* scales,
+                               kq_stream_t stream) {
+  kq_status st = check_x(x, M, d, ldx);
+  if (st != KQ_OK) return st;
+  if (M == 0 || d == 0) return KQ_OK;
+  st = check_out(q, scales);
+  if (st != KQ_OK) return st;
+  return launch_quant<kq::MODE_FWHT>(x, M, d, ldx, nullptr, nullptr, nullptr, q, scales, as_cuda(stream));
+}
+
+kq_status kq_dequantize(const uint8_t* q, const uint8_t* scales, int64_t M, int64_t d, const void* inv_mats,
+                        kq_dtype mat_dtype, void* out, kq_dtype out_dtype, kq_stream_t stream) {
+  if (M < 0 || d < 0) return KQ_ERR_INVALID_ARG;
+  if ((mat_dtype != KQ_F32 && mat_dtype != KQ_BF16) || (out_dtype != KQ_F32 && out_dtype != KQ_BF16))
+    return KQ_ERR_INVALID_ARG;
+  if (d % 32 != 0) return KQ_ERR_SHAPE;
+  if (M == 0 || d == 0) return KQ_OK;
+  if (q == nullptr || scales == nullptr || out == nullptr) return KQ_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16) || (inv_mats != nullptr && !aligned(inv_mats, 4))) return KQ_ERR_ALIGN;
+  const int64_t nb = d / 32;
+  if (nb > int64_t(INT32_MAX)) return KQ_ERR_SHAPE;
+  kq::dequant_kernel<<<grid_for(M * nb, 256), 256, 0, as_cuda(stream)>>>(
+      q, scales, M, int(nb), inv_mats, mat_dtype == KQ_BF16 ? 1 : 0, out, out_dtype == KQ_BF16 ? 1 : 0);
+  return launch_status();
+}
+
+kq_status kq_e2m1_pack(const float* v, int64_t n, uint8_t* out, kq_stream_t stream) {
+  if (n < 0) return KQ_ERR_INVALID_ARG;
+  if (n % 2 != 0) return KQ_ERR_SHAPE;
+  if (n == 0) return KQ_OK;
+  if (v == nullptr || out == nullptr) return KQ_ERR_INVALID_ARG;
+  if (!aligned(v, 16) || !aligned(out, 4)) return KQ_ERR_ALIGN;
+  kq::e2m1_pack_kernel<<<grid_for(n / 8 + 1, 256), 256, 0, as_cuda(stream)>>>(v, n, out);
+  return launch_status();
+}
+
+kq_status kq_get_device_error(int clear) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return KQ_ERR_CUDA;
+  unsigned int flags = 0;
+  if (cudaMemcpyFromSymbol(&flags, kq::g_dev_error, sizeof(flags)) != cudaSuccess) return KQ_ERR_CUDA;
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(kq::g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return KQ_ERR_CUDA;
+  }
+  if (flags & kq::kDevErrTimeout) return KQ_ERR_DEVICE_TIMEOUT;
+  if (flags & kq::kDevErrSingular) return KQ_ERR_SINGULAR;
+  return KQ_OK;
+}
+
+}  // extern "C"

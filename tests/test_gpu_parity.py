@@ -1,0 +1,341 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  Integer outputs (codes, scales, expanded bf16/fp32 matrix
+bits) are compared exactly; the tolerance of the quantizer's stated criterion is
+checked by tests/parity.py and, because the kernels certify every scale and
+code, the tests also require exact equality."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+from mxfp4_activations_b200 import inputs  # noqa: E402
+
+from .parity import compare, unpack  # noqa: E402
+
+pytestmark = [
+    pytest.mark.gpu,
+    pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device"),
+]
+
+
+@pytest.fixture(scope="module")
+def kq():
+    from mxfp4_activations_b200 import build
+
+    build.build()
+    import mxfp4_activations_b200 as m
+
+    m.load()
+    assert m.kq_get_device_error(clear=True) == 0
+    return m
+
+
+def dev_bf16(x_bits: np.ndarray) -> "torch.Tensor":
+    return torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def dev_f32(a: np.ndarray) -> "torch.Tensor":
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()
+
+
+def host(t: "torch.Tensor") -> np.ndarray:
+    torch.cuda.synchronize()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).cpu().numpy().view(np.uint16)
+    return t.cpu().numpy()
+
+
+def gpu_quantize(kq, x_bits, params, x_dev=None):
+    p = dev_f32(params)
+    mats = kq.kq_expand_blocks(p)
+    fac = kq.kq_expand_factored(p)
+    x = dev_bf16(x_bits) if x_dev is None else x_dev
+    qd, sd = kq.kq_quantize(x, mats, fac, variant="butterfly")
+    return host(qd), host(sd)
+
+
+def check(q, s, qr, sr, yr=None, exact=True):
+    rep = compare(q, s, qr, sr, yr)
+    assert rep["ok"], rep
+    if exact:
+        assert rep["scale_mismatch"] == 0 and rep["code_mismatch"] == 0, rep
+    return rep
+
+
+# ---------------------------------------------------------------- set-up kernels
+
+def special_params():
+    p = inputs.lu_params(40, seed=77, noise=0.5)
+    p[0] = inputs.identity_params(1)[0]
+    p[1] = inputs.hadamard_params(1)[0]
+    p[2, :, 0] = -0.0          # signed-zero l
+    p[3, :, 2] = -0.0          # signed-zero v
+    p[4, :, 1] = 1e-3          # large 1/u
+    p[5, :, 1] = 3e3
+    p[6, 2] = (-1.0, 1.0, 1.0)  # d = l v + 1/u = 0: butterfly ratio undefined
+    return p
+
+
+@pytest.mark.parametrize("inverse", [False, True])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_expand_bit_exact(kq, orc, inverse, dtype):
+    params = special_params()
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    got = host(kq.kq_expand_blocks(dev_f32(params), inverse=inverse, dtype=tdt))
+    want = orc.expand(params, dtype=orc.F32 if dtype == "f32" else orc.BF16, inverse=inverse)
+    if dtype == "f32":
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    else:
+        assert np.array_equal(got, want)
+
+
+def test_expand_factored_reproduces_matrix(kq, orc):
+    params = special_params()
+    fac = host(kq.kq_expand_factored(dev_f32(params))).astype(np.float64)
+    K = orc.expand_f64(params)
+    for b in range(params.shape[0]):
+        lam, bet, D, kmax, flag = fac[b, :5], fac[b, 5:10], fac[b, 10:42], fac[b, 42], fac[b, 43]
+        assert kmax >= np.abs(K[b]).max()
+        if flag:
+            continue
+        Mk = np.ones((1, 1))
+        for k in range(5):
+            Mk = np.kron(Mk, np.array([[1.0, bet[k]], [lam[k], 1.0]]))
+        Kf = Mk * D[None, :]
+        assert np.all(np.abs(Kf - K[b]) <= 1e-6 * np.abs(K[b]) + 1e-30)
+    assert fac[6, 43] == 1.0  # d = 0 factor is routed to the exact path
+
+
+def test_singular_factor_sets_device_flag(kq):
+    p = inputs.lu_params(2, seed=1)
+    p[1, 3, 1] = 0.0
+    kq.kq_expand_blocks(dev_f32(p))
+    assert kq.kq_get_device_error(clear=True) == 4
+    assert kq.kq_get_device_error(clear=True) == 0
+
+
+# ---------------------------------------------------------------- element step
+
+def test_e2m1_pack_core_binades_exhaustive(kq, orc):
+    lo = int(np.float32(0.125).view(np.uint32))
+    hi = int(np.float32(8.0).view(np.uint32))
+    pos = np.arange(lo, hi, dtype=np.uint32)
+    for bits in (pos, pos | np.uint32(0x80000000)):
+        v = bits.view(np.float32)
+        got = host(kq.kq_e2m1_pack(dev_f32(v)))
+        want = orc.e2m1_pack(v)
+        assert np.array_equal(got, want)
+
+
+def test_e2m1_pack_random_and_specials(kq, orc):
+    rng = np.random.default_rng(5)
+    v = rng.integers(0, 2**32, 1 << 22, dtype=np.uint64).astype(np.uint32).view(np.float32)
+    v = v[~np.isnan(v)]
+    v = np.concatenate([v, np.array([0.0, -0.0, np.inf, -np.inf, 1e-45, -1e-45, 6.0, 7.0, 5.0, 0.25, 0.75],
+                                    np.float32)])
+    v = v[: (v.size // 2) * 2].astype(np.float32)
+    for n in (v.size, 2, 6, 10, 18):  # also tails shorter than 8 values
+        got = host(kq.kq_e2m1_pack(dev_f32(v[:n])))
+        assert np.array_equal(got, orc.e2m1_pack(v[:n]))
+
+
+# ---------------------------------------------------------------- quantizer vs oracle
+
+def test_quantize_cfg0_full(kq, orc):
+    x, params = inputs.config_case("cfg0", 1152)
+    q, s = gpu_quantize(kq, x, params)
+    K = orc.expand(params)
+    qr, sr = orc.quantize(x, K)
+    check(q, s, qr, sr, orc.transform(x, K))
+
+
+@pytest.mark.parametrize("M,d", [(1, 32), (3, 96), (65, 1152), (7, 5600), (130, 2240), (33, 12288), (257, 3072),
+                                 (300, 4608)])
+def test_quantize_ragged_shapes(kq, orc, M, d):
+    x = inputs.activations(M, d, "t3", seed=[M, d], outlier_frac=0.01, outlier_scale=(20.0, 100.0))
+    params = inputs.lu_params(d // 32, seed=[M, d, 9])
+    q, s = gpu_quantize(kq, x, params)
+    K = orc.expand(params)
+    qr, sr = orc.quantize(x, K)
+    check(q, s, qr, sr, orc.transform(x, K))
+
+
+def test_quantize_strided_rows(kq, orc):
+    M, d, ldx = 50, 2240, 2240 + 136
+    full = inputs.activations(M, ldx, "normal", seed=3, outlier_frac=0.01, outlier_scale=(50.0, 50.0))
+    params = inputs.lu_params(d // 32, seed=4)
+    xd = dev_bf16(full)[:, :d]
+    assert xd.stride(0) == ldx
+    q, s = gpu_quantize(kq, None, params, x_dev=xd)
+    qr, sr = orc.quantize(np.ascontiguousarray(full[:, :d]), orc.expand(params))
+    check(q, s, qr, sr)
+
+
+def test_quantize_degenerate_blocks(kq, orc):
+    rng = np.random.default_rng(8)
+    M, d = 24, 256
+    a = rng.standard_normal((M, d)).astype(np.float32)
+    a[0] = 0.0                                   # all-zero row
+    a[1, 32:64] = 0.0                            # one all-zero block
+    a[2, 64:96] = -0.0                           # negative zeros
+    a[3, 5] = np.inf                             # non-finite inputs
+    a[4, 40] = np.nan
+    a[5, 100] = -np.inf
+    a[6] *= 1e37                                 # near fp32 overflow after the transform
+    a[7] *= 1e-39                                # bf16 subnormals
+    a[8, 0:32] = 0.0
+    a[8, 3] = 1e-40                              # a single tiny value in a zero block
+    a[9, 0:32] = 3.0                             # constant block (exact cancellations)
+    a[10] = 3.4e38                               # overflow of the fp32 transform
+    x = inputs.f32_to_bf16_bits(a)
+    params = inputs.lu_params(d // 32, seed=9)
+    q, s = gpu_quantize(kq, x, params)
+    K = orc.expand(params)
+    qr, sr = orc.quantize(x, K)
+    check(q, s, qr, sr)
+
+
+def test_quantize_identity_all_bf16_patterns(kq, orc):
+    """K = I: every bf16 bit pattern (NaN/Inf included) goes through the scale and
+    element steps as its own value; 2048 blocks of 32 consecutive patterns, plus a
+    shuffled copy so that each block mixes magnitudes."""
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    rng = np.random.default_rng(10)
+    x = np.concatenate([pats, rng.permutation(pats)]).reshape(-1, 1024)
+    params = inputs.identity_params(1024 // 32)
+    q, s = gpu_quantize(kq, x, params)
+    qr, sr = orc.quantize(x, orc.expand(params))
+    check(q, s, qr, sr)
+
+
+def test_quantize_exact_ties_identity(kq, orc):
+    """Blocks whose elements sit exactly on E2M1 midpoints (and one bf16 step
+    away) under K = I, so the certified path must resolve every one of them."""
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    rows = []
+    for e in (-3, 0, 5):
+        blk = np.zeros(32, np.float32)
+        blk[0] = 4.0 * 2.0 ** e  # fixes the scale to 2^e
+        vals = np.concatenate([mids, -mids, mids * (1 + 2 ** -7), mids * (1 - 2 ** -8)])
+        blk[1:1 + len(vals[:31])] = vals[:31] * 2.0 ** e
+        rows.append(blk)
+    x = inputs.f32_to_bf16_bits(np.stack(rows).reshape(1, -1))
+    params = inputs.identity_params(x.shape[1] // 32)
+    q, s = gpu_quantize(kq, x, params)
+    qr, sr = orc.quantize(x, orc.expand(params))
+    check(q, s, qr, sr)
+
+
+def test_quantize_hadamard_init_onehot(kq, orc):
+    x = np.zeros((32, 32), np.float32)
+    for c in range(32):
+        x[c, c] = 32.0
+    xb = inputs.f32_to_bf16_bits(x)
+    params = inputs.hadamard_params(1)
+    q, s = gpu_quantize(kq, xb, params)
+    qr, sr = orc.quantize(xb, orc.expand(params))
+    check(q, s, qr, sr)
+    assert np.all(s == 127) and np.all((unpack(q) & 7) == 7)
+
+
+def sampled_rows(M: int, n: int, seed: int) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    rows = set([0, M - 1, M // 2]) | set(rng.choice(M, size=min(n, M), replace=False).tolist())
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("name,d", [("pixart", 1152), ("pixart", 4608), ("sana", 2240), ("sana", 5600),
+                                    ("flux", 3072), ("flux", 12288)])
+def test_quantize_full_config_sampled(kq, orc, name, d):
+    x, params = inputs.config_case(name, d)
+    q, s = gpu_quantize(kq, x, params)
+    rows = sampled_rows(x.shape[0], 40, seed=d)
+    K = orc.expand(params)
+    xs = np.ascontiguousarray(x[rows])
+    qr, sr = orc.quantize(xs, K)
+    check(q[rows], s[rows], qr, sr, orc.transform(xs, K))
+
+
+@pytest.mark.parametrize("M", inputs.SWEEP_M)
+def test_quantize_sweep_shapes_sampled(kq, orc, M):
+    for d in inputs.SWEEP_D:
+        if M * d > 2**28 and d != inputs.SWEEP_D[0]:
+            # largest shapes: only the first d runs here; the bench sweep covers the rest
+            continue
+        x, params = inputs.sweep_case(M, d)
+        q, s = gpu_quantize(kq, x, params)
+        rows = sampled_rows(M, 12, seed=M + d)
+        K = orc.expand(params)
+        qr, sr = orc.quantize(np.ascontiguousarray(x[rows]), K)
+        check(q[rows], s[rows], qr, sr)
+
+
+# ---------------------------------------------------------------- comparison kernels
+
+@pytest.mark.parametrize("M,d", [(64, 1152), (7, 5600), (1, 32), (300, 3072)])
+def test_smooth_parity(kq, orc, M, d):
+    x = inputs.activations(M, d, "t4", seed=[M, d, 2], outlier_frac=0.01, outlier_scale=(20.0, 100.0))
+    inv_s = inputs.smooth_inv_scale(x)
+    qd, sd = kq.kq_ref_smooth_quantize(dev_bf16(x), dev_f32(inv_s))
+    qr, sr = orc.smooth_quantize(x, inv_s)
+    check(host(qd), host(sd), qr, sr)
+
+
+@pytest.mark.parametrize("M,d", [(64, 1152), (7, 5600), (1, 32), (300, 3072)])
+def test_fwht_parity(kq, orc, M, d):
+    x = inputs.activations(M, d, "t3", seed=[M, d, 3], outlier_frac=0.01, outlier_scale=(20.0, 100.0))
+    qd, sd = kq.kq_ref_fwht_quantize(dev_bf16(x))
+    qr, sr = orc.fwht_quantize(x)
+    check(host(qd), host(sd), qr, sr)
+
+
+def test_fwht_degenerate_blocks(kq, orc):
+    a = np.random.default_rng(12).standard_normal((6, 96)).astype(np.float32)
+    a[0] = 0.0
+    a[1, :32] = 1.0    # exact cancellations: every output but one is zero
+    a[2, 3] = np.nan
+    a[3] *= 3e37
+    x = inputs.f32_to_bf16_bits(a)
+    qd, sd = kq.kq_ref_fwht_quantize(dev_bf16(x))
+    qr, sr = orc.fwht_quantize(x)
+    check(host(qd), host(sd), qr, sr)
+
+
+# ---------------------------------------------------------------- dequantize
+
+def test_dequantize_exact_without_transform(kq, orc):
+    x, params = inputs.config_case("cfg0", 1152)
+    p = dev_f32(params)
+    qd, sd = kq.kq_quantize(dev_bf16(x), kq.kq_expand_blocks(p), kq.kq_expand_factored(p))
+    got = host(kq.kq_dequantize(qd, sd))
+    want = orc.dequantize(host(qd), host(sd)).astype(np.float32)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    gotb = host(kq.kq_dequantize(qd, sd, out_dtype=torch.bfloat16))
+    assert np.array_equal(gotb, inputs.f32_to_bf16_bits(want))
+
+
+def test_dequantize_inverse_within_fp32_bound(kq, orc):
+    x, params = inputs.config_case("cfg0", 1152)
+    p = dev_f32(params)
+    qd, sd = kq.kq_quantize(dev_bf16(x), kq.kq_expand_blocks(p), kq.kq_expand_factored(p))
+    inv = kq.kq_expand_blocks(p, inverse=True)
+    got = host(kq.kq_dequantize(qd, sd, inv)).astype(np.float64)
+    Ki = orc.expand(params, inverse=True)
+    want = orc.dequantize(host(qd), host(sd), Ki)
+    yh = orc.dequantize(host(qd), host(sd))
+    M, d = want.shape
+    bound = np.einsum("rbj,bji->rbi", np.abs(yh).reshape(M, d // 32, 32),
+                      np.abs(Ki.astype(np.float64))).reshape(M, d) * 33 * 2.0 ** -24
+    assert np.all(np.abs(got - want) <= bound + 1e-30)
+    # and the round trip reconstructs x to MXFP4 accuracy (sanity, not parity)
+    xf = inputs.bf16_bits_to_f32(x).astype(np.float64)
+    rel = np.linalg.norm(got - xf) / np.linalg.norm(xf)
+    assert rel < 0.2
+
+
+def test_no_device_error_after_suite(kq):
+    assert kq.kq_get_device_error(clear=True) == 0
