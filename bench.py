@@ -133,6 +133,33 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ---------------------------------------------------------------- ranks
+
+def rank_inputs(rank: int):
+    """The FLUX-shaped batch of one rank: rank 0 uses the configuration's own
+    seed, every other rank draws an independent batch of the same shape and law
+    (weak scaling: work per rank is fixed).  The transform parameters are the
+    layer's and are the same on every rank."""
+    xs, ps = [], []
+    for d in FLUX_DS:
+        x, p = inputs.config_case("flux", d)
+        if rank:
+            x = inputs.activations(FLUX_M, d, "t3", seed=[3, d, 0, rank], outlier_frac=0.005,
+                                   outlier_scale=(100.0, 100.0))
+        xs.append(x)
+        ps.append(p)
+    return xs, ps
+
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """Elapsed time of the job: the slowest rank's time (one scalar all-reduce)."""
+    import torch
+
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------- GPU arm
 
 class QuantStep:
@@ -253,15 +280,7 @@ def run_gpu(args) -> None:
         dist.barrier()
     kq.load()
 
-    # inputs: each rank draws its own batch (weak scaling); seeds differ by rank
-    xs, ps = [], []
-    for d in FLUX_DS:
-        x, p = inputs.config_case("flux", d)
-        if rank:
-            x = inputs.activations(FLUX_M, d, "t3", seed=[3, d, 0, rank], outlier_frac=0.005,
-                                   outlier_scale=(100.0, 100.0))
-        xs.append(x)
-        ps.append(p)
+    xs, ps = rank_inputs(rank)
     step = QuantStep(torch, kq, xs, ps, n_copies=4, device=device)
     bytes_step = step.bytes_per_step()
     resident_mb = 4 * sum(x.nbytes for x in xs) / 1e6
@@ -292,9 +311,7 @@ def run_gpu(args) -> None:
         if world > 1:
             dist.barrier()
     if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks(total_ms, dist, device)
 
     err = kq.kq_get_device_error(clear=True)
     if err != 0:

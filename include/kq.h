@@ -172,6 +172,11 @@ KQ_API kq_status kq_e2m1_pack(const float* v, int64_t n, uint8_t* out, kq_stream
  * the flags.  Returns KQ_ERR_CUDA if the device cannot be read. */
 KQ_API kq_status kq_get_device_error(int clear);
 
+/* Description of the last failing CUDA call made by this library on the calling
+ * thread (for a KQ_ERR_CUDA status); "no error" if none.  Thread-local storage,
+ * valid until the thread's next failing call. */
+KQ_API const char* kq_last_error(void);
+
 /* Static, human-readable name of a status code. */
 KQ_API const char* kq_status_string(kq_status status);
 

@@ -25,6 +25,7 @@ STATUS = {
 EXPORTED = (
     "kq_expand_blocks", "kq_expand_factored", "kq_quantize", "kq_dequantize", "kq_ref_smooth_quantize",
     "kq_ref_fwht_quantize", "kq_e2m1_pack", "kq_get_device_error", "kq_status_string", "kq_abi_version",
+    "kq_last_error",
 )
 
 
@@ -60,12 +61,14 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kq_get_device_error": [I],
         "kq_status_string": [I],
         "kq_abi_version": [],
+        "kq_last_error": [],
     }
     for name, args in sig.items():
         f = getattr(L, name)
         f.argtypes = args
         f.restype = I
     L.kq_status_string.restype = ctypes.c_char_p
+    L.kq_last_error.restype = ctypes.c_char_p
     _lib = L
     return L
 
@@ -73,6 +76,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
 def _check(fn: str, status: int):
     if status != 0:
         msg = load().kq_status_string(status).decode()
+        if status == 6:
+            msg += f" ({load().kq_last_error().decode()})"
         raise KQError(fn, status, msg)
 
 

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cstdio>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -23,7 +24,19 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 cudaStream_t as_cuda(kq_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
-kq_status launch_status() { return cudaGetLastError() == cudaSuccess ? KQ_OK : KQ_ERR_CUDA; }
+// Description of the last failing CUDA call on this thread (kq_last_error).
+thread_local char g_last_error[256] = "no error";
+
+kq_status cuda_fail(const char* what, cudaError_t e) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", what, cudaGetErrorString(e), int(e));
+  cudaGetLastError();  // do not leave a stale error for the next call
+  return KQ_ERR_CUDA;
+}
+
+kq_status launch_status(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? KQ_OK : cuda_fail(what, e);
+}
 
 // ---- per-device facts, cached
 struct DeviceInfo {
@@ -64,33 +77,36 @@ EncodeTiledFn encode_tiled() {
 
 // ---- launch geometry of the quantizer kernels
 struct QuantGeom {
-  int W, R, threads, stages, stage_stride, smem;
+  int W, R, cons_warps, threads, stages, stage_stride, smem;
 };
 
 QuantGeom quant_geometry(int nb, int smem_optin) {
   QuantGeom g{};
-  const int ncol = (nb + 255) / 256;
-  g.W = (nb + ncol - 1) / ncol;  // <= 256 (TMA box limit)
+  // at most 224 consumer threads (+1 producer warp = 256): two CTAs per SM at 128 registers
+  constexpr int kMaxCons = 224;
+  const int ncol = (nb + kMaxCons - 1) / kMaxCons;
+  g.W = (nb + ncol - 1) / ncol;  // <= 224 (TMA box limit is 256)
   int bestR = 1;
   double bestU = -1.0;
-  for (int R = 1; R * g.W <= 256; R++) {
+  for (int R = 1; R * g.W <= kMaxCons; R++) {
     const int T = ((R * g.W + 31) / 32) * 32;
     const double u = double(R * g.W) / double(T);
-    // prefer full warps, then CTAs near 256 threads
-    const double score = u - 0.0005 * double(T > 256 ? T - 256 : 256 - T) / 32.0;
+    // prefer full warps, then more threads per CTA
+    const double score = u - 0.0005 * double(kMaxCons - T) / 32.0;
     if (score > bestU + 1e-12) {
       bestU = score;
       bestR = R;
     }
   }
   g.R = bestR;
-  g.threads = ((g.R * g.W + 31) / 32) * 32;
+  g.cons_warps = (g.R * g.W + 31) / 32;
+  g.threads = (g.cons_warps + 1) * 32;
   const int stage_bytes = g.W * g.R * 64;
   g.stage_stride = (stage_bytes + 1023) & ~1023;
   int st = (96 * 1024) / g.stage_stride;
   if (st > 6) st = 6;
   if (st < 2) st = 2;
-  const int fixed = 1024 /*alignment slack*/ + 64 /*barriers*/;
+  const int fixed = 1024 /*alignment slack*/ + 128 /*barriers*/;
   while (st > 2 && st * g.stage_stride + fixed > smem_optin) st--;
   g.stages = st;
   g.smem = st * g.stage_stride + fixed;
@@ -101,8 +117,9 @@ template <int MODE>
 kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const float* mats, const float* factored,
                        const float* inv_s, uint8_t* q, uint8_t* scales, cudaStream_t stream) {
   const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return cuda_fail("device query", cudaErrorInvalidDevice);
   EncodeTiledFn enc = encode_tiled();
-  if (dev == nullptr || enc == nullptr) return KQ_ERR_CUDA;
+  if (enc == nullptr) return cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
   const int nb = int(d / 32);
   const QuantGeom g = quant_geometry(nb, dev->smem_optin);
   if (g.smem > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
@@ -115,21 +132,29 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), gdim, gstride, box, estride,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return KQ_ERR_CUDA;
+    return cuda_fail("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
 
   auto kern = kq::quant_kernel<MODE>;
-  static std::atomic<int> smem_set[kMaxDevices];
+  // dynamic shared memory limit: the opt-in maximum minus the kernel's static shared memory
+  static std::atomic<int> dyn_limit[kMaxDevices];
   int devid = 0;
   cudaGetDevice(&devid);
-  if (smem_set[devid].load() < g.smem) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev->smem_optin) != cudaSuccess)
-      return KQ_ERR_CUDA;
-    smem_set[devid].store(dev->smem_optin);
+  if (dyn_limit[devid].load() == 0) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncGetAttributes", e);
+    const int lim = dev->smem_optin - int(fa.sharedSizeBytes);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
+    dyn_limit[devid].store(lim);
   }
+  if (g.smem > dyn_limit[devid].load()) return KQ_ERR_UNSUPPORTED;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.threads, g.smem) != cudaSuccess ||
-      per_sm < 1)
-    return KQ_ERR_CUDA;
+  {
+    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.threads, g.smem);
+    if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveBlocksPerMultiprocessor", e);
+    if (per_sm < 1) return cuda_fail("occupancy: no resident CTA", cudaErrorInvalidConfiguration);
+  }
 
   kq::QuantParams p;
   p.x = static_cast<const uint16_t*>(x);
@@ -143,6 +168,7 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   p.n_row_tiles = int(nrt);
   p.stages = g.stages;
   p.stage_stride = g.stage_stride;
+  p.cons_warps = g.cons_warps;
   p.mats = mats;
   p.factored = factored;
   p.inv_s = inv_s;
@@ -156,7 +182,7 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   if (gy > 65535) gy = 65535;
   if (gy < 1) gy = 1;
   kern<<<dim3(ncol, unsigned(gy)), g.threads, g.smem, stream>>>(tmap, p);
-  return launch_status();
+  return launch_status("quant_kernel launch");
 }
 
 kq_status check_x(const void* x, int64_t M, int64_t d, int64_t ldx) {
@@ -212,7 +238,7 @@ kq_status kq_expand_blocks(const float* params, int64_t nb, int inverse, kq_dtyp
   const int64_t n = nb * 1024;
   kq::expand_kernel<<<unsigned((n + 255) / 256), 256, 0, as_cuda(stream)>>>(params, nb, inverse ? 1 : 0,
                                                                            out_dtype == KQ_BF16 ? 1 : 0, mats);
-  return launch_status();
+  return launch_status("expand_kernel launch");
 }
 
 kq_status kq_expand_factored(const float* params, int64_t nb, float* factored, kq_stream_t stream) {
@@ -222,7 +248,7 @@ kq_status kq_expand_factored(const float* params, int64_t nb, float* factored, k
   if (!aligned(params, 4) || !aligned(factored, 16)) return KQ_ERR_ALIGN;
   if (nb > (int64_t(1) << 30)) return KQ_ERR_SHAPE;
   kq::expand_factored_kernel<<<unsigned((nb + 127) / 128), 128, 0, as_cuda(stream)>>>(params, nb, factored);
-  return launch_status();
+  return launch_status("expand_factored_kernel launch");
 }
 
 kq_status kq_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const void* mats, kq_dtype mat_dtype,
@@ -279,7 +305,7 @@ kq_status kq_dequantize(const uint8_t* q, const uint8_t* scales, int64_t M, int6
   if (nb > int64_t(INT32_MAX)) return KQ_ERR_SHAPE;
   kq::dequant_kernel<<<grid_for(M * nb, 256), 256, 0, as_cuda(stream)>>>(
       q, scales, M, int(nb), inv_mats, mat_dtype == KQ_BF16 ? 1 : 0, out, out_dtype == KQ_BF16 ? 1 : 0);
-  return launch_status();
+  return launch_status("dequant_kernel launch");
 }
 
 kq_status kq_e2m1_pack(const float* v, int64_t n, uint8_t* out, kq_stream_t stream) {
@@ -289,16 +315,21 @@ kq_status kq_e2m1_pack(const float* v, int64_t n, uint8_t* out, kq_stream_t stre
   if (v == nullptr || out == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(v, 16) || !aligned(out, 4)) return KQ_ERR_ALIGN;
   kq::e2m1_pack_kernel<<<grid_for(n / 8 + 1, 256), 256, 0, as_cuda(stream)>>>(v, n, out);
-  return launch_status();
+  return launch_status("e2m1_pack_kernel launch");
 }
 
+const char* kq_last_error(void) { return g_last_error; }
+
 kq_status kq_get_device_error(int clear) {
-  if (cudaDeviceSynchronize() != cudaSuccess) return KQ_ERR_CUDA;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail("cudaDeviceSynchronize", e);
   unsigned int flags = 0;
-  if (cudaMemcpyFromSymbol(&flags, kq::g_dev_error, sizeof(flags)) != cudaSuccess) return KQ_ERR_CUDA;
+  e = cudaMemcpyFromSymbol(&flags, kq::g_dev_error, sizeof(flags));
+  if (e != cudaSuccess) return cuda_fail("cudaMemcpyFromSymbol", e);
   if (clear) {
     const unsigned int zero = 0;
-    if (cudaMemcpyToSymbol(kq::g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return KQ_ERR_CUDA;
+    e = cudaMemcpyToSymbol(kq::g_dev_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail("cudaMemcpyToSymbol", e);
   }
   if (flags & kq::kDevErrTimeout) return KQ_ERR_DEVICE_TIMEOUT;
   if (flags & kq::kDevErrSingular) return KQ_ERR_SINGULAR;

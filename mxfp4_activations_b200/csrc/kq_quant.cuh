@@ -13,14 +13,22 @@
 // Data movement: a CTA owns a column tile of W blocks and walks row tiles of R
 // rows.  Each row tile (W*R blocks of 64 B) is fetched by one 3-D TMA load
 // (box {32, W, R}, 64-byte swizzle, no multicast) into a ring of shared-memory
-// stages; thread t = r*W + c handles block c of row r.  With the 64 B swizzle
-// the 16-byte chunk k of block t sits at chunk k ^ ((t >> 1) & 3), which makes
-// the four 16-byte shared loads of a warp conflict-free.
+// stages.  The last warp of the CTA only issues those loads; a stage is refilled
+// when every consumer warp has arrived on its "empty" barrier, so consumer
+// warps never wait for each other.  Consumer thread t = r*W + c handles block c
+// of row r.  With the 64 B swizzle the 16-byte chunk k of block t sits at chunk
+// k ^ ((t >> 1) & 3), which makes the four 16-byte shared loads of a warp
+// conflict-free.  The butterfly stages on index bits 1..4 run as packed f32x2
+// FMAs on element pairs (2m, 2m+1).
 //
 // Exactness (KRON, FWHT): the fp32 result y_f differs from the definition
-// y32 = fp32(sum_i x_i K32[i][j]) by at most E = C * ||x||_1 * max|K| (C covers
-// 6 fp32 roundings of the butterfly, the fp32 rounding of the coefficients and
-// of K32, and the final rounding, with a factor-two margin).  The scale is taken
+// y32 = fp32(sum_i x_i K32[i][j]) by at most E = C * ||x||_1 * max|K|.  KRON:
+// 6 roundings on each output's path (5 FMA stages, 1 multiply by D) give 6u;
+// the fp32 coefficients (5 ratios and D_j, each rounded once) put the applied
+// matrix within 6u of K, K32 is within u of K, and y32 is one more rounding:
+// 14u in all (u = 2^-24), against C = 16u.  FWHT: 6 roundings + the final one
+// = 7u (its coefficients are exactly the entries of fp32(H32)), against 8u.
+// ||x||_1 is summed with upward rounding and max|K| is rounded up.  The scale is taken
 // from y_f only when max|y| +- E has one E8M0 exponent, and each code only when
 // the values (y_f -+ E) 2^-e round (downward / upward) to the same E2M1 code;
 // every other scale or code is recomputed in fp64 in the definition's order,
@@ -36,8 +44,8 @@ namespace kq {
 enum Mode { MODE_KRON = 0, MODE_FWHT = 1, MODE_SMOOTH = 2 };
 
 constexpr float kFwhtC = 0.17677669529663688f;      // fp32 nearest to 2^-2.5
-constexpr float kKronErrC = 1.9073486328125e-06f;   // 2^-19 = 32 u (14 u needed)
-constexpr float kFwhtErrC = 9.5367431640625e-07f;   // 2^-20 = 16 u (7 u needed)
+constexpr float kKronErrC = 9.5367431640625e-07f;   // 2^-20 = 16 u (14 u needed, see below)
+constexpr float kFwhtErrC = 4.76837158203125e-07f;  // 2^-21 = 8 u (7 u needed)
 constexpr float kErrAbs = 7.174648137343064e-43f;   // 2^-140: FWHT subnormal-range slack
 constexpr uint64_t kWaitLimitNs = 2000000000ull;    // 2 s per bounded wait
 
@@ -51,6 +59,7 @@ struct QuantParams {
   int n_row_tiles;
   int stages;
   int stage_stride;       // bytes between stages (multiple of 1024)
+  int cons_warps;         // consumer warps; one more warp issues the TMA loads
   const float* mats;      // KRON: fp32 [nb][32][32] (exact path)
   const float* factored;  // KRON: [nb][48]
   const float* inv_s;     // SMOOTH: [nb*32]
@@ -59,65 +68,94 @@ struct QuantParams {
 };
 
 // ---------------------------------------------------------------- exact fp64 path
+//
+// Only elements (or blocks) whose code (or scale) the fp32 bound cannot
+// certify come here.  Every load is issued before the arithmetic so that one
+// L2 round trip serves a whole recomputation.
 
-// y32 of one element: fp32 rounding of sum_i x_i K[i][j], accumulated in fp64 in
-// increasing i from +0 (each product is exact in fp64).
+// Exact recomputation of one whole block by the whole warp: lane j computes
+// y32_j = fp32( sum_i x_i K[i][j] ) in fp64, summing in increasing i from +0
+// (each product of a bf16 and an fp32 value is exact in fp64).  Row i of K is
+// one coalesced 128-byte load across the warp and all 32 rows are in flight
+// together; x is a broadcast load.  The block's scale then comes from the
+// exact maximum and every code from the exact value, and lane `owner` stores
+// them.  Must be called by all 32 lanes with the same arguments (taken from
+// the owner lane).
 template <int MODE>
-__device__ __noinline__ float exact_y(const uint16_t* __restrict__ xb, const float* __restrict__ Kb, int j) {
+__device__ __noinline__ void exact_block_warp(const uint16_t* __restrict__ xb, const float* __restrict__ Kb,
+                                              uint8_t* __restrict__ qb, uint8_t* __restrict__ sb, int owner) {
+  const int lane = threadIdx.x & 31;
+  float kc[kBlock];
+#pragma unroll
+  for (int i = 0; i < kBlock; i++)
+    kc[i] = (MODE == MODE_FWHT) ? ((__popc(i & lane) & 1) ? -kFwhtC : kFwhtC) : __ldg(Kb + i * kBlock + lane);
+  const uint4* px = reinterpret_cast<const uint4*>(xb);
+  uint32_t xw[16];
+#pragma unroll
+  for (int k = 0; k < 4; k++) {
+    const uint4 v = __ldg(px + k);
+    xw[4 * k] = v.x;
+    xw[4 * k + 1] = v.y;
+    xw[4 * k + 2] = v.z;
+    xw[4 * k + 3] = v.w;
+  }
   double acc = 0.0;
-#pragma unroll 4
+#pragma unroll
   for (int i = 0; i < kBlock; i++) {
-    double kij;
-    if (MODE == MODE_FWHT)
-      kij = (__popc(i & j) & 1) ? -double(kFwhtC) : double(kFwhtC);
-    else
-      kij = double(Kb[i * kBlock + j]);
-    acc = __dadd_rn(acc, __dmul_rn(double(bf16_to_f32(xb[i])), kij));
+    const float xi = (i & 1) ? bf16hi(xw[i >> 1]) : bf16lo(xw[i >> 1]);
+    acc = __dadd_rn(acc, __dmul_rn(double(xi), double(kc[i])));
   }
-  return __double2float_rn(acc);
-}
-
-// Whole block in fp64: scale from the exact maximum, then every code.
-template <int MODE>
-__device__ __noinline__ void exact_block(const uint16_t* __restrict__ xb, const float* __restrict__ Kb,
-                                         uint8_t* __restrict__ qb, uint8_t* __restrict__ sb) {
-  float y[kBlock];
-  bool finite = true;
-  float amax = 0.0f;
-  for (int j = 0; j < kBlock; j++) {
-    y[j] = exact_y<MODE>(xb, Kb, j);
-    if (!isfinite(y[j])) finite = false;
-    else amax = fmaxf(amax, fabsf(y[j]));
-  }
-  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  const float y = __double2float_rn(acc);
+  const bool finite = __all_sync(0xFFFFFFFFu, isfinite(y));
+  float m = fabsf(y);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   int byte = 0xFF;
+  uint32_t code = 0u;
   if (finite) {
-    byte = e8m0_byte(amax);
-    const float s = inv_scale_of_byte(byte);
-    for (int k = 0; k < 4; k++) {
-      const float* v = y + 8 * k;
-      w[k] = e2m1x8(__fmul_rn(v[0], s), __fmul_rn(v[1], s), __fmul_rn(v[2], s), __fmul_rn(v[3], s),
-                    __fmul_rn(v[4], s), __fmul_rn(v[5], s), __fmul_rn(v[6], s), __fmul_rn(v[7], s));
-    }
+    byte = e8m0_byte(m);
+    code = e2m1_one(__fmul_rn(y, inv_scale_of_byte(byte)));
   }
-  *reinterpret_cast<uint4*>(qb) = make_uint4(w[0], w[1], w[2], w[3]);
-  *sb = uint8_t(byte);
+  // nibble j of word j/8; OR across each group of eight lanes
+  uint32_t w = code << (4 * (lane & 7));
+  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
+  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
+  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 4);
+  const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, w, 0), w1 = __shfl_sync(0xFFFFFFFFu, w, 8);
+  const uint32_t w2 = __shfl_sync(0xFFFFFFFFu, w, 16), w3 = __shfl_sync(0xFFFFFFFFu, w, 24);
+  if (lane == owner) {
+    *reinterpret_cast<uint4*>(qb) = make_uint4(w0, w1, w2, w3);
+    *sb = uint8_t(byte);
+  }
 }
 
+// Every lane whose block needs the exact path hands it to the whole warp, one
+// block at a time.  Called by all 32 lanes.
 template <int MODE>
-__device__ __noinline__ uint32_t exact_code(const uint16_t* __restrict__ xb, const float* __restrict__ Kb, int j,
-                                            float s) {
-  return e2m1_one(__fmul_rn(exact_y<MODE>(xb, Kb, j), s));
+__device__ __forceinline__ void warp_exact_pass(bool need, const uint16_t* xb, const float* Kb, uint8_t* qb,
+                                                uint8_t* sb) {
+  uint32_t pending = __ballot_sync(0xFFFFFFFFu, need);
+  while (pending) {
+    const int src = __ffs(pending) - 1;
+    pending &= pending - 1;
+    const uint16_t* xs = reinterpret_cast<const uint16_t*>(
+        __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(xb), src));
+    const float* ks = reinterpret_cast<const float*>(
+        __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(Kb), src));
+    uint8_t* qs = reinterpret_cast<uint8_t*>(__shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(qb), src));
+    uint8_t* ss = reinterpret_cast<uint8_t*>(__shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(sb), src));
+    exact_block_warp<MODE>(xs, ks, qs, ss, src);
+  }
 }
 
 // ---------------------------------------------------------------- per-thread coefficients
 
 struct Coef {
-  float lam[5];   // c_k / a_k, k = factor index (factor k acts on index bit 4-k)
-  float bet[5];   // b_k / d_k
-  float D[32];
-  float cfac;     // C * max|K|
-  float eabs;     // absolute error allowance for subnormal-range results
+  uint64_t lam2[5];  // (c_k/a_k, c_k/a_k); factor k acts on index bit 4-k
+  uint64_t bet2[5];  // (b_k/d_k, b_k/d_k)
+  uint64_t D2[16];   // (D[2m], D[2m+1]); SMOOTH: the per-channel factors
+  float cfac;        // C * max|K|
+  float eabs;        // absolute error allowance for subnormal-range results
   bool exact_only;
 };
 
@@ -136,11 +174,11 @@ __device__ __forceinline__ void load_coef(const QuantParams& p, int b, Coef& c) 
     }
 #pragma unroll
     for (int k = 0; k < 5; k++) {
-      c.lam[k] = buf[k];
-      c.bet[k] = buf[5 + k];
+      c.lam2[k] = pk2(buf[k], buf[k]);
+      c.bet2[k] = pk2(buf[5 + k], buf[5 + k]);
     }
 #pragma unroll
-    for (int j = 0; j < 32; j++) c.D[j] = buf[10 + j];
+    for (int m = 0; m < 16; m++) c.D2[m] = pk2(buf[10 + 2 * m], buf[11 + 2 * m]);
     c.cfac = __fmul_ru(kKronErrC, buf[42]);
     c.eabs = buf[44];
     c.exact_only = buf[43] != 0.0f;
@@ -149,10 +187,8 @@ __device__ __forceinline__ void load_coef(const QuantParams& p, int b, Coef& c) 
 #pragma unroll
     for (int i = 0; i < 8; i++) {
       const float4 v = __ldg(f + i);
-      c.D[4 * i + 0] = v.x;
-      c.D[4 * i + 1] = v.y;
-      c.D[4 * i + 2] = v.z;
-      c.D[4 * i + 3] = v.w;
+      c.D2[2 * i] = pk2(v.x, v.y);
+      c.D2[2 * i + 1] = pk2(v.z, v.w);
     }
     c.cfac = 0.0f;
     c.eabs = 0.0f;
@@ -164,118 +200,159 @@ __device__ __forceinline__ void load_coef(const QuantParams& p, int b, Coef& c) 
   }
 }
 
+// max_j |y_j| with NaN propagation: for each residue r = j mod 4, the eight
+// elements r, r+4, ..., r+28 through three-input maxima, then the four results.
+__device__ __forceinline__ float block_amax(const float (&y)[kBlock]) {
+  float a[4];
+#pragma unroll
+  for (int r = 0; r < 4; r++) {
+    float m = fmax3_nan(fabsf(y[r]), fabsf(y[r + 4]), fabsf(y[r + 8]));
+    m = fmax3_nan(m, fabsf(y[r + 12]), fabsf(y[r + 16]));
+    m = fmax3_nan(m, fabsf(y[r + 20]), fabsf(y[r + 24]));
+    a[r] = fmax_nan(m, fabsf(y[r + 28]));
+  }
+  return fmax_nan(fmax3_nan(a[0], a[1], a[2]), a[3]);
+}
+
+// E2M1 codes of the 8 values held in pairs Y[4k .. 4k+3].
+__device__ __forceinline__ uint32_t codes8(const uint64_t* Y) {
+  float v[8];
+#pragma unroll
+  for (int h = 0; h < 4; h++) upk2(Y[h], v[2 * h], v[2 * h + 1]);
+  return e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+}
+
 // ---------------------------------------------------------------- one block of one row
 
 template <int MODE>
 __device__ __forceinline__ void quant_block(const QuantParams& p, const Coef& c, const uint4 (&xr)[4], int64_t row,
-                                            int b) {
+                                            int b, bool act) {
   uint8_t* qb = p.q + row * int64_t(p.nb) * 16 + int64_t(b) * 16;
   uint8_t* sb = p.scales + row * int64_t(p.nb) + b;
   const uint16_t* xb = p.x + row * p.ldx + int64_t(b) * kBlock;
   const float* Kb = (MODE == MODE_KRON) ? p.mats + int64_t(b) * kBlock * kBlock : nullptr;
 
-  float y[kBlock];
+  float x[kBlock];
 #pragma unroll
   for (int k = 0; k < 4; k++) {
     const uint32_t w[4] = {xr[k].x, xr[k].y, xr[k].z, xr[k].w};
 #pragma unroll
     for (int h = 0; h < 4; h++) {
-      y[8 * k + 2 * h] = bf16lo(w[h]);
-      y[8 * k + 2 * h + 1] = bf16hi(w[h]);
+      x[8 * k + 2 * h] = bf16lo(w[h]);
+      x[8 * k + 2 * h + 1] = bf16hi(w[h]);
     }
   }
+  uint64_t Y[16];
+  float y[kBlock];
 
   if (MODE == MODE_SMOOTH) {
-    float amax = 0.0f;
 #pragma unroll
-    for (int j = 0; j < kBlock; j++) {
-      y[j] = __fmul_rn(y[j], c.D[j]);  // exactly the definition: one fp32 rounding
-      amax = fmax_nan(amax, fabsf(y[j]));
-    }
+    for (int m = 0; m < 16; m++) Y[m] = mul2_rn(pk2(x[2 * m], x[2 * m + 1]), c.D2[m]);  // one rounding each
+#pragma unroll
+    for (int m = 0; m < 16; m++) upk2(Y[m], y[2 * m], y[2 * m + 1]);
+    const float amax = block_amax(y);
+    if (!act) return;
     if (!(amax <= FLT_MAX)) {
       *reinterpret_cast<uint4*>(qb) = make_uint4(0u, 0u, 0u, 0u);
       *sb = 0xFF;
       return;
     }
     const int byte = e8m0_byte(amax);
-    const float s = inv_scale_of_byte(byte);
-    uint32_t w[4];
+    const uint64_t S2 = pk2(inv_scale_of_byte(byte), inv_scale_of_byte(byte));
 #pragma unroll
-    for (int k = 0; k < 4; k++) {
-      const float* v = y + 8 * k;
-      w[k] = e2m1x8(__fmul_rn(v[0], s), __fmul_rn(v[1], s), __fmul_rn(v[2], s), __fmul_rn(v[3], s),
-                    __fmul_rn(v[4], s), __fmul_rn(v[5], s), __fmul_rn(v[6], s), __fmul_rn(v[7], s));
-    }
-    *reinterpret_cast<uint4*>(qb) = make_uint4(w[0], w[1], w[2], w[3]);
+    for (int m = 0; m < 16; m++) Y[m] = mul2_rn(Y[m], S2);
+    *reinterpret_cast<uint4*>(qb) = make_uint4(codes8(Y), codes8(Y + 4), codes8(Y + 8), codes8(Y + 12));
     *sb = uint8_t(byte);
     return;
   }
 
-  // ||x||_1, rounded upward so that it bounds the exact norm
-  float l1 = 0.0f;
+  // ||x||_1 rounded upward (four partial sums for ILP)
+  float l1p[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-  for (int j = 0; j < kBlock; j++) l1 = __fadd_ru(l1, fabsf(y[j]));
+  for (int j = 0; j < kBlock; j++) l1p[j & 3] = __fadd_ru(l1p[j & 3], fabsf(x[j]));
+  const float l1 = __fadd_ru(__fadd_ru(l1p[0], l1p[1]), __fadd_ru(l1p[2], l1p[3]));
 
-  // butterfly: stage on index bit pb applies factor k = 4 - pb
+  // stage on index bit 0 (factor 4), scalar: the pair partners share a register pair
+  {
+    float l4 = 1.0f, b4 = -1.0f;
+    if (MODE == MODE_KRON) {
+      float t0;
+      upk2(c.lam2[4], l4, t0);
+      upk2(c.bet2[4], b4, t0);
+    }
 #pragma unroll
-  for (int pb = 0; pb < 5; pb++) {
-    const float lam = (MODE == MODE_FWHT) ? 1.0f : c.lam[4 - pb];
-    const float bet = (MODE == MODE_FWHT) ? -1.0f : c.bet[4 - pb];
-#pragma unroll
-    for (int i = 0; i < kBlock; i++) {
-      if (i & (1 << pb)) continue;
-      const int i1 = i | (1 << pb);
-      const float x0 = y[i], x1 = y[i1];
-      y[i] = __fmaf_rn(lam, x1, x0);
-      y[i1] = __fmaf_rn(bet, x0, x1);
+    for (int m = 0; m < 16; m++) {
+      const float x0 = x[2 * m], x1 = x[2 * m + 1];
+      if (MODE == MODE_FWHT) {
+        x[2 * m] = __fadd_rn(x0, x1);
+        x[2 * m + 1] = __fsub_rn(x1, x0);
+      } else {
+        x[2 * m] = __fmaf_rn(l4, x1, x0);
+        x[2 * m + 1] = __fmaf_rn(b4, x0, x1);
+      }
     }
   }
-  float amax = 0.0f;
 #pragma unroll
-  for (int j = 0; j < kBlock; j++) {
-    const float dj = (MODE == MODE_FWHT) ? ((__popc(j) & 1) ? -kFwhtC : kFwhtC) : c.D[j];
-    y[j] = __fmul_rn(y[j], dj);
-    amax = fmax_nan(amax, fabsf(y[j]));
+  for (int m = 0; m < 16; m++) Y[m] = pk2(x[2 * m], x[2 * m + 1]);
+  // stages on index bits 1..4 (factors 3..0) on packed pairs
+#pragma unroll
+  for (int pb = 1; pb < 5; pb++) {
+#pragma unroll
+    for (int m = 0; m < 16; m++) {
+      if (m & (1 << (pb - 1))) continue;
+      const int m1 = m | (1 << (pb - 1));
+      const uint64_t y0 = Y[m], y1 = Y[m1];
+      if (MODE == MODE_FWHT) {
+        Y[m] = add2_rn(y0, y1);
+        Y[m1] = sub2_rn(y1, y0);
+      } else {
+        Y[m] = fma2_rn(c.lam2[4 - pb], y1, y0);
+        Y[m1] = fma2_rn(c.bet2[4 - pb], y0, y1);
+      }
+    }
   }
+  // diagonal: D_j (FWHT: +-2^-2.5 with the sign of (-1)^popcount(j))
+#pragma unroll
+  for (int m = 0; m < 16; m++) {
+    if (MODE == MODE_FWHT) {
+      const float sg = (__popc(m) & 1) ? -kFwhtC : kFwhtC;
+      Y[m] = mul2_rn(pk2(sg, -sg), Y[m]);
+    } else {
+      Y[m] = mul2_rn(c.D2[m], Y[m]);
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < 16; m++) upk2(Y[m], y[2 * m], y[2 * m + 1]);
+  const float amax = block_amax(y);
 
-  if (l1 == 0.0f) {  // all inputs are +-0: every y is +0 by definition
-    *reinterpret_cast<uint4*>(qb) = make_uint4(0u, 0u, 0u, 0u);
-    *sb = 0;
-    return;
-  }
+  // all inputs +-0: every y is +0 by definition (byte 0, codes 0)
+  const bool zero_block = l1 == 0.0f;
   const float E = __fmaf_ru(c.cfac, l1, c.eabs);
   bool exact = c.exact_only || !(amax <= FLT_MAX) || !(E <= FLT_MAX);
   const int byte = e8m0_byte(__fadd_ru(amax, E));
-  if (!exact && byte != e8m0_byte(fmaxf(__fsub_rd(amax, E), 0.0f))) exact = true;
-  if (exact) {
-    exact_block<MODE>(xb, Kb, qb, sb);
-    return;
-  }
-  const float s = inv_scale_of_byte(byte);
+  if (byte != e8m0_byte(fmaxf(__fsub_rd(amax, E), 0.0f))) exact = true;
+  const float s = inv_scale_of_byte(exact ? 0 : byte);
   const float eb = __fmul_ru(E, s);
+  const uint64_t S2 = pk2(s, s), NE2 = pk2(-eb, -eb), PE2 = pk2(eb, eb);
+  uint64_t V[16];
   uint32_t cm[4], cp[4];
 #pragma unroll
-  for (int k = 0; k < 4; k++) {
-    const float* v = y + 8 * k;
-    cm[k] = e2m1x8(__fmaf_rd(v[0], s, -eb), __fmaf_rd(v[1], s, -eb), __fmaf_rd(v[2], s, -eb),
-                   __fmaf_rd(v[3], s, -eb), __fmaf_rd(v[4], s, -eb), __fmaf_rd(v[5], s, -eb),
-                   __fmaf_rd(v[6], s, -eb), __fmaf_rd(v[7], s, -eb));
-    cp[k] = e2m1x8(__fmaf_ru(v[0], s, eb), __fmaf_ru(v[1], s, eb), __fmaf_ru(v[2], s, eb),
-                   __fmaf_ru(v[3], s, eb), __fmaf_ru(v[4], s, eb), __fmaf_ru(v[5], s, eb),
-                   __fmaf_ru(v[6], s, eb), __fmaf_ru(v[7], s, eb));
-  }
-  const uint32_t diff = (cm[0] ^ cp[0]) | (cm[1] ^ cp[1]) | (cm[2] ^ cp[2]) | (cm[3] ^ cp[3]);
-  if (diff != 0u) {
+  for (int m = 0; m < 16; m++) V[m] = fma2_rd(Y[m], S2, NE2);
 #pragma unroll
-    for (int k = 0; k < 4; k++) {
-      uint32_t dm = cm[k] ^ cp[k];
-      while (dm) {
-        const int nib = (__ffs(dm) - 1) >> 2;
-        const uint32_t code = exact_code<MODE>(xb, Kb, 8 * k + nib, s);
-        cm[k] = (cm[k] & ~(0xFu << (4 * nib))) | (code << (4 * nib));
-        dm &= ~(0xFu << (4 * nib));
-      }
-    }
+  for (int k = 0; k < 4; k++) cm[k] = codes8(V + 4 * k);
+#pragma unroll
+  for (int m = 0; m < 16; m++) V[m] = fma2_ru(Y[m], S2, PE2);
+#pragma unroll
+  for (int k = 0; k < 4; k++) cp[k] = codes8(V + 4 * k);
+  const uint32_t diff = (cm[0] ^ cp[0]) | (cm[1] ^ cp[1]) | (cm[2] ^ cp[2]) | (cm[3] ^ cp[3]);
+  // a block with an uncertain scale or an uncertain code is recomputed exactly
+  const bool need = act && !zero_block && (exact || diff != 0u);
+  warp_exact_pass<MODE>(need, xb, Kb, qb, sb);
+  if (!act || need) return;
+  if (zero_block) {
+    *reinterpret_cast<uint4*>(qb) = make_uint4(0u, 0u, 0u, 0u);
+    *sb = 0;
+    return;
   }
   *reinterpret_cast<uint4*>(qb) = make_uint4(cm[0], cm[1], cm[2], cm[3]);
   *sb = uint8_t(byte);
@@ -284,66 +361,66 @@ __device__ __forceinline__ void quant_block(const QuantParams& p, const Coef& c,
 // ---------------------------------------------------------------- kernel
 
 template <int MODE>
-__global__ void __launch_bounds__(256) quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
+__global__ void __launch_bounds__(256, 2) quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ int s_abort;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(base + p.stages * p.stage_stride);
+  uint64_t* empty = full + p.stages;
 
-  const int t = threadIdx.x;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const uint32_t stage_bytes = uint32_t(p.W) * uint32_t(p.R) * 64u;
+  const int my_tiles = (p.n_row_tiles - int(blockIdx.y) + int(gridDim.y) - 1) / int(gridDim.y);
+
+  if (t == 0) {
+    for (int s = 0; s < p.stages; s++) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], uint32_t(p.cons_warps));
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == p.cons_warps) {  // producer warp: one thread issues every TMA load
+    if (lane == 0) {
+      prefetch_tensormap(&tmap);
+      int it = 0;
+      for (; it < my_tiles; it++) {
+        const int s = it % p.stages;
+        if (it >= p.stages && !mbar_wait_bounded(&empty[s], uint32_t(it / p.stages - 1) & 1u, kWaitLimitNs)) break;
+        const int tile = int(blockIdx.y) + it * int(gridDim.y);
+        mbar_arrive_expect_tx(&full[s], stage_bytes);
+        tma_load_3d(base + s * p.stage_stride, &tmap, &full[s], 0, int(blockIdx.x) * p.W, tile * p.R);
+      }
+      if (it < my_tiles) {  // consumers stopped: let the loads still in flight land before exiting
+        for (int k = (it > p.stages ? it - p.stages : 0); k < it; k++)
+          mbar_wait_bounded(&full[k % p.stages], uint32_t(k / p.stages) & 1u, kWaitLimitNs / 4);
+      }
+    }
+    return;
+  }
+
   const int bb = t % p.W, rr = t / p.W;
   const int b = blockIdx.x * p.W + bb;
   const bool has_tile = rr < p.R;
   const bool active = has_tile && b < p.nb;
-  const uint32_t stage_bytes = uint32_t(p.W) * uint32_t(p.R) * 64u;
-  const int my_tiles = (p.n_row_tiles - int(blockIdx.y) + int(gridDim.y) - 1) / int(gridDim.y);
-
-  Coef c;
+  Coef c = {};
   if (active) load_coef<MODE>(p, b, c);
 
-  if (t == 0) {
-    s_abort = 0;
-    prefetch_tensormap(&tmap);
-    for (int s = 0; s < p.stages; s++) mbar_init(&full[s], 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (t == 0) {
-    const int first = my_tiles < p.stages ? my_tiles : p.stages;
-    for (int s = 0; s < first; s++) {
-      const int tile = int(blockIdx.y) + s * int(gridDim.y);
-      mbar_arrive_expect_tx(&full[s], stage_bytes);
-      tma_load_3d(base + s * p.stage_stride, &tmap, &full[s], 0, int(blockIdx.x) * p.W, tile * p.R);
-    }
-  }
-
   const int sw = (t >> 1) & 3;
-  int it = 0;
-  for (; it < my_tiles; it++) {
+  for (int it = 0; it < my_tiles; it++) {
     const int s = it % p.stages;
-    const uint32_t parity = uint32_t(it / p.stages) & 1u;
-    if (!mbar_wait_bounded(&full[s], parity, kWaitLimitNs)) s_abort = 1;
-    uint4 xr[4];
+    if (!mbar_wait_bounded(&full[s], uint32_t(it / p.stages) & 1u, kWaitLimitNs)) break;
+    uint4 xr[4] = {};
     if (has_tile) {
       const uint4* blk = reinterpret_cast<const uint4*>(base + s * p.stage_stride + t * 64);
 #pragma unroll
       for (int k = 0; k < 4; k++) xr[k] = blk[k ^ sw];
     }
-    __syncthreads();
-    if (s_abort) break;
-    if (t == 0 && it + p.stages < my_tiles) {
-      const int tile = int(blockIdx.y) + (it + p.stages) * int(gridDim.y);
-      mbar_arrive_expect_tx(&full[s], stage_bytes);
-      tma_load_3d(base + s * p.stage_stride, &tmap, &full[s], 0, int(blockIdx.x) * p.W, tile * p.R);
-    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
     const int64_t row = int64_t(int(blockIdx.y) + it * int(gridDim.y)) * p.R + rr;
-    if (active && row < p.M) quant_block<MODE>(p, c, xr, row, b);
-  }
-  if (it < my_tiles && t == 0) {
-    // a wait ran out: drain the loads still in flight (bounded) before exiting
-    const int last = (it + p.stages < my_tiles) ? it + p.stages : my_tiles;
-    for (int k = it; k < last; k++)
-      mbar_wait_bounded(&full[k % p.stages], uint32_t(k / p.stages) & 1u, kWaitLimitNs / 4);
+    // every lane takes part (the exact path is warp-cooperative); only real blocks store
+    quant_block<MODE>(p, c, xr, row, b, active && row < p.M);
   }
 }
 
