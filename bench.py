@@ -173,6 +173,7 @@ class QuantStep:
         for d, x, params in zip(FLUX_DS, xs_host, params_host):
             p = torch.from_numpy(params).to(device)
             mats = kq.kq_expand_blocks(p)
+            mats16 = kq.kq_expand_blocks(p, dtype=torch.bfloat16)
             fac = kq.kq_expand_factored(p)
             x0 = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
             copies = [x0] + [x0.clone() for _ in range(n_copies - 1)]
@@ -180,7 +181,8 @@ class QuantStep:
             qs = [torch.empty((M, d // 2), dtype=torch.uint8, device=device) for _ in range(n_copies)]
             ss = [torch.empty((M, d // 32), dtype=torch.uint8, device=device) for _ in range(n_copies)]
             inv_s = torch.from_numpy(inputs.smooth_inv_scale(x)).to(device)
-            self.items.append(dict(d=d, M=M, params=p, mats=mats, fac=fac, x=copies, q=qs, s=ss, inv_s=inv_s))
+            self.items.append(dict(d=d, M=M, params=p, mats=mats, mats16=mats16, fac=fac, x=copies, q=qs, s=ss,
+                                   inv_s=inv_s))
         self.n = n_copies
         self.stream = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
@@ -191,6 +193,12 @@ class QuantStep:
         if kind == "kroquant":
             st = self.lib.kq_quantize(x.data_ptr(), M, d, d, item["mats"].data_ptr(), 0, item["fac"].data_ptr(),
                                       q.data_ptr(), s.data_ptr(), 2, self.stream)
+        elif kind == "kroquant_mma":
+            st = self.lib.kq_quantize(x.data_ptr(), M, d, d, item["mats"].data_ptr(), 0, None,
+                                      q.data_ptr(), s.data_ptr(), 1, self.stream)
+        elif kind == "kroquant_mma_bf16":
+            st = self.lib.kq_quantize(x.data_ptr(), M, d, d, item["mats16"].data_ptr(), 1, None,
+                                      q.data_ptr(), s.data_ptr(), 1, self.stream)
         elif kind == "smooth":
             st = self.lib.kq_ref_smooth_quantize(x.data_ptr(), M, d, d, item["inv_s"].data_ptr(), q.data_ptr(),
                                                  s.data_ptr(), self.stream)
@@ -319,7 +327,7 @@ def run_gpu(args) -> None:
 
     # comparison kernels on the same inputs (after the timed region)
     comp = {}
-    for kind in ("smooth", "fwht", "kroquant"):
+    for kind in ("smooth", "fwht", "kroquant", "kroquant_mma", "kroquant_mma_bf16"):
         timed(torch, step, 20, kind, per_launch=False)
         ms, lm = timed(torch, step, max(50, args.steps), kind, per_launch=True)
         n = max(50, args.steps)

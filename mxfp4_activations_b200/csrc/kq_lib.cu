@@ -14,6 +14,7 @@
 #include "kq_common.cuh"
 #include "kq_expand.cuh"
 #include "kq_misc.cuh"
+#include "kq_mma.cuh"
 #include "kq_quant.cuh"
 
 namespace {
@@ -185,6 +186,57 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   return launch_status("quant_kernel launch");
 }
 
+// Tensor-core variant: 128-row x 4-block tiles, one CTA per column group and
+// row-tile stride, two CTAs per SM (256 tensor-memory columns each).
+kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, const void* mats, bool mats_bf16,
+                           uint8_t* q, uint8_t* scales, cudaStream_t stream) {
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return cuda_fail("device query", cudaErrorInvalidDevice);
+  EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
+  const int nb = int(d / 32);
+  CUtensorMap tmap;
+  const cuuint64_t gdim[3] = {32, cuuint64_t(M), cuuint64_t(nb)};
+  const cuuint64_t gstride[2] = {cuuint64_t(ldx) * 2, 64};
+  const cuuint32_t box[3] = {32, cuuint32_t(kq::kMmaRows), cuuint32_t(kq::kMmaWb)};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), gdim, gstride, box, estride,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cuda_fail("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
+  const int smem = 1024 + kq::kMmaStages * kq::kMmaAStageBytes + kq::kMmaWb * 3 * kq::kMmaBBytes + 256;
+  if (smem > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
+  auto kern = mats_bf16 ? kq::quant_mma_kernel<kq::KSRC_BF16> : kq::quant_mma_kernel<kq::KSRC_F32>;
+  static std::atomic<int> attr_set[2][kMaxDevices];
+  int devid = 0;
+  cudaGetDevice(&devid);
+  if (!attr_set[mats_bf16][devid].load()) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
+    attr_set[mats_bf16][devid].store(1);
+  }
+  kq::MmaParams p;
+  p.x = static_cast<const uint16_t*>(x);
+  p.ldx = ldx;
+  p.M = M;
+  p.nb = nb;
+  const int64_t nrt = (M + kq::kMmaRows - 1) / kq::kMmaRows;
+  if (nrt > int64_t(INT32_MAX) / 2) return KQ_ERR_SHAPE;
+  p.n_row_tiles = int(nrt);
+  p.nsplit = mats_bf16 ? 1 : 3;
+  p.mats = mats;
+  p.q = q;
+  p.scales = scales;
+  const int ngroups = (nb + kq::kMmaWb - 1) / kq::kMmaWb;
+  if (ngroups > 65535 * 1024) return KQ_ERR_SHAPE;
+  int64_t gy = (int64_t(dev->sms) * 2) / ngroups;
+  if (gy < 1) gy = 1;
+  if (gy > nrt) gy = nrt;
+  if (gy > 65535) gy = 65535;
+  kern<<<dim3(ngroups, unsigned(gy)), kq::kMmaThreads, smem, stream>>>(tmap, p);
+  return launch_status("quant_mma_kernel launch");
+}
+
 kq_status check_x(const void* x, int64_t M, int64_t d, int64_t ldx) {
   if (M < 0 || d < 0) return KQ_ERR_INVALID_ARG;
   if (d % 32 != 0 || ldx < d) return KQ_ERR_SHAPE;
@@ -263,7 +315,13 @@ kq_status kq_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const vo
   if (st != KQ_OK) return st;
   if (mats == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(mats, 16)) return KQ_ERR_ALIGN;
-  if (variant == KQ_VAR_MMA || mat_dtype == KQ_BF16) return KQ_ERR_UNSUPPORTED;
+  // bf16 matrices are only served by the tensor-core variant; AUTO picks the
+  // butterfly for fp32 matrices when the factored form is given
+  const bool use_mma = variant == KQ_VAR_MMA || mat_dtype == KQ_BF16 ||
+                       (variant == KQ_VAR_AUTO && factored == nullptr);
+  if (variant == KQ_VAR_BUTTERFLY && mat_dtype == KQ_BF16) return KQ_ERR_UNSUPPORTED;
+  if (use_mma)
+    return launch_quant_mma(x, M, d, ldx, mats, mat_dtype == KQ_BF16, q, scales, as_cuda(stream));
   if (factored == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(factored, 16)) return KQ_ERR_ALIGN;
   return launch_quant<kq::MODE_KRON>(x, M, d, ldx, static_cast<const float*>(mats), factored, nullptr, q, scales,

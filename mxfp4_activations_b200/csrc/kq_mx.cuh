@@ -1,0 +1,178 @@
+// kq_mx.cuh -- the MXFP4 step shared by the quantizer kernels: block maximum,
+// E2M1 codes, and the certified selection between the fast fp32 result and an
+// exact fp64 recomputation.
+//
+// MXFP4 ("W4A4 (MXFP4e2)" in the KroQuant abstract): one E8M0 scale 2^e per 32
+// elements with e = floor(log2 max|y|) - 2 (OCP MX rule for E2M1), clamped to
+// [-127, 127]; each element v = y 2^-e is rounded to E2M1 (nearest, ties to
+// even, saturating at 6, sign kept).  A block with a non-finite y gets scale
+// byte 0xFF and zero codes; an all-zero input block is +0 everywhere.
+#pragma once
+
+#include <float.h>
+
+#include "kq_common.cuh"
+
+namespace kq {
+
+constexpr float kFwhtC = 0.17677669529663688f;    // fp32 nearest to 2^-2.5
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per bounded wait
+
+// Where the exact path reads K[i][j] from.
+enum KSource { KSRC_F32 = 0, KSRC_BF16 = 1, KSRC_FWHT = 2 };
+
+template <int KSRC>
+__device__ __forceinline__ float k_entry(const void* __restrict__ Kb, int i, int j) {
+  if (KSRC == KSRC_FWHT) return (__popc(i & j) & 1) ? -kFwhtC : kFwhtC;
+  if (KSRC == KSRC_BF16) return bf16_to_f32(__ldg(static_cast<const unsigned short*>(Kb) + i * kBlock + j));
+  return __ldg(static_cast<const float*>(Kb) + i * kBlock + j);
+}
+
+// max_j |y_j| with NaN propagation: for each residue r = j mod 4, the eight
+// elements r, r+4, ..., r+28 through three-input maxima, then the four results.
+__device__ __forceinline__ float block_amax(const float (&y)[kBlock]) {
+  float a[4];
+#pragma unroll
+  for (int r = 0; r < 4; r++) {
+    float m = fmax3_nan(fabsf(y[r]), fabsf(y[r + 4]), fabsf(y[r + 8]));
+    m = fmax3_nan(m, fabsf(y[r + 12]), fabsf(y[r + 16]));
+    m = fmax3_nan(m, fabsf(y[r + 20]), fabsf(y[r + 24]));
+    a[r] = fmax_nan(m, fabsf(y[r + 28]));
+  }
+  return fmax_nan(fmax3_nan(a[0], a[1], a[2]), a[3]);
+}
+
+// E2M1 codes of the 8 values held in pairs Y[4k .. 4k+3].
+__device__ __forceinline__ uint32_t codes8(const uint64_t* Y) {
+  float v[8];
+#pragma unroll
+  for (int h = 0; h < 4; h++) upk2(Y[h], v[2 * h], v[2 * h + 1]);
+  return e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+}
+
+// ---------------------------------------------------------------- exact fp64 path
+//
+// Only elements (or blocks) whose code (or scale) the fp32 bound cannot
+// certify come here.  Every load is issued before the arithmetic so that one
+// L2 round trip serves a whole recomputation.
+
+// Exact recomputation of one whole block by the whole warp: lane j computes
+// y32_j = fp32( sum_i x_i K[i][j] ) in fp64, summing in increasing i from +0
+// (each product of a bf16 and an fp32 or bf16 value is exact in fp64).  Row i of K is
+// one coalesced 128-byte load across the warp and all 32 rows are in flight
+// together; x is a broadcast load.  The block's scale then comes from the
+// exact maximum and every code from the exact value, and lane `owner` stores
+// them.  Must be called by all 32 lanes with the same arguments (taken from
+// the owner lane).
+template <int KSRC>
+__device__ __noinline__ void exact_block_warp(const uint16_t* __restrict__ xb, const void* __restrict__ Kb,
+                                              uint8_t* __restrict__ qb, uint8_t* __restrict__ sb, int owner) {
+  const int lane = threadIdx.x & 31;
+  float kc[kBlock];
+#pragma unroll
+  for (int i = 0; i < kBlock; i++)
+    kc[i] = k_entry<KSRC>(Kb, i, lane);
+  const uint4* px = reinterpret_cast<const uint4*>(xb);
+  uint32_t xw[16];
+#pragma unroll
+  for (int k = 0; k < 4; k++) {
+    const uint4 v = __ldg(px + k);
+    xw[4 * k] = v.x;
+    xw[4 * k + 1] = v.y;
+    xw[4 * k + 2] = v.z;
+    xw[4 * k + 3] = v.w;
+  }
+  double acc = 0.0;
+#pragma unroll
+  for (int i = 0; i < kBlock; i++) {
+    const float xi = (i & 1) ? bf16hi(xw[i >> 1]) : bf16lo(xw[i >> 1]);
+    acc = __dadd_rn(acc, __dmul_rn(double(xi), double(kc[i])));
+  }
+  const float y = __double2float_rn(acc);
+  const bool finite = __all_sync(0xFFFFFFFFu, isfinite(y));
+  float m = fabsf(y);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  int byte = 0xFF;
+  uint32_t code = 0u;
+  if (finite) {
+    byte = e8m0_byte(m);
+    code = e2m1_one(__fmul_rn(y, inv_scale_of_byte(byte)));
+  }
+  // nibble j of word j/8; OR across each group of eight lanes
+  uint32_t w = code << (4 * (lane & 7));
+  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
+  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
+  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 4);
+  const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, w, 0), w1 = __shfl_sync(0xFFFFFFFFu, w, 8);
+  const uint32_t w2 = __shfl_sync(0xFFFFFFFFu, w, 16), w3 = __shfl_sync(0xFFFFFFFFu, w, 24);
+  if (lane == owner) {
+    *reinterpret_cast<uint4*>(qb) = make_uint4(w0, w1, w2, w3);
+    *sb = uint8_t(byte);
+  }
+}
+
+// Every lane whose block needs the exact path hands it to the whole warp, one
+// block at a time.  Called by all 32 lanes.
+template <int KSRC>
+__device__ __forceinline__ void warp_exact_pass(bool need, const uint16_t* xb, const void* Kb, uint8_t* qb,
+                                                uint8_t* sb) {
+  uint32_t pending = __ballot_sync(0xFFFFFFFFu, need);
+  while (pending) {
+    const int src = __ffs(pending) - 1;
+    pending &= pending - 1;
+    const uint16_t* xs = reinterpret_cast<const uint16_t*>(
+        __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(xb), src));
+    const void* ks = reinterpret_cast<const void*>(
+        __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(Kb), src));
+    uint8_t* qs = reinterpret_cast<uint8_t*>(__shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(qb), src));
+    uint8_t* ss = reinterpret_cast<uint8_t*>(__shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(sb), src));
+    exact_block_warp<KSRC>(xs, ks, qs, ss, src);
+  }
+}
+
+// The certified MXFP4 step of one block.  Y holds the fast fp32 y as pairs,
+// amax = max|y| (NaN-propagating), and E = cfac * l1 + eabs bounds |y - y32|
+// for every element, y32 being the definition's value.  The scale is taken from
+// amax only when amax - E and amax + E (directed rounding) give the same E8M0
+// byte; each code only when (y - E) 2^-e rounded down and (y + E) 2^-e rounded
+// up give the same E2M1 code.  Any block that fails either test is recomputed
+// exactly by the warp.  Must be called by all 32 lanes; act marks real blocks.
+template <int KSRC>
+__device__ __forceinline__ void certify_store(const uint64_t (&Y)[16], float amax, float l1, float cfac, float eabs,
+                                              bool exact_only, bool act, const uint16_t* xb, const void* Kb,
+                                              uint8_t* qb, uint8_t* sb) {
+  // all inputs +-0: every y is +0 by definition (byte 0, codes 0)
+  const bool zero_block = l1 == 0.0f;
+  const float E = __fmaf_ru(cfac, l1, eabs);
+  bool exact = exact_only || !(amax <= FLT_MAX) || !(E <= FLT_MAX);
+  const int byte = e8m0_byte(__fadd_ru(amax, E));
+  if (byte != e8m0_byte(fmaxf(__fsub_rd(amax, E), 0.0f))) exact = true;
+  const float s = inv_scale_of_byte(exact ? 0 : byte);
+  const float eb = __fmul_ru(E, s);
+  const uint64_t S2 = pk2(s, s), NE2 = pk2(-eb, -eb), PE2 = pk2(eb, eb);
+  uint64_t V[16];
+  uint32_t cm[4], cp[4];
+#pragma unroll
+  for (int m = 0; m < 16; m++) V[m] = fma2_rd(Y[m], S2, NE2);
+#pragma unroll
+  for (int k = 0; k < 4; k++) cm[k] = codes8(V + 4 * k);
+#pragma unroll
+  for (int m = 0; m < 16; m++) V[m] = fma2_ru(Y[m], S2, PE2);
+#pragma unroll
+  for (int k = 0; k < 4; k++) cp[k] = codes8(V + 4 * k);
+  const uint32_t diff = (cm[0] ^ cp[0]) | (cm[1] ^ cp[1]) | (cm[2] ^ cp[2]) | (cm[3] ^ cp[3]);
+  // a block with an uncertain scale or an uncertain code is recomputed exactly
+  const bool need = act && !zero_block && (exact || diff != 0u);
+  warp_exact_pass<KSRC>(need, xb, Kb, qb, sb);
+  if (!act || need) return;
+  if (zero_block) {
+    *reinterpret_cast<uint4*>(qb) = make_uint4(0u, 0u, 0u, 0u);
+    *sb = 0;
+    return;
+  }
+  *reinterpret_cast<uint4*>(qb) = make_uint4(cm[0], cm[1], cm[2], cm[3]);
+  *sb = uint8_t(byte);
+}
+
+}  // namespace kq

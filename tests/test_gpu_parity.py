@@ -49,13 +49,22 @@ def host(t: "torch.Tensor") -> np.ndarray:
     return t.cpu().numpy()
 
 
-def gpu_quantize(kq, x_bits, params, x_dev=None):
+# (variant, matrix dtype): the butterfly serves fp32 matrices; the tensor-core
+# variant serves fp32 (three exact bf16 parts) and bf16 matrices.
+VARIANTS = [("butterfly", "f32"), ("mma", "f32"), ("mma", "bf16")]
+
+
+def gpu_quantize(kq, x_bits, params, x_dev=None, variant="butterfly", mdt="f32"):
     p = dev_f32(params)
-    mats = kq.kq_expand_blocks(p)
-    fac = kq.kq_expand_factored(p)
+    mats = kq.kq_expand_blocks(p, dtype=torch.float32 if mdt == "f32" else torch.bfloat16)
+    fac = kq.kq_expand_factored(p) if variant == "butterfly" else None
     x = dev_bf16(x_bits) if x_dev is None else x_dev
-    qd, sd = kq.kq_quantize(x, mats, fac, variant="butterfly")
+    qd, sd = kq.kq_quantize(x, mats, fac, variant=variant)
     return host(qd), host(sd)
+
+
+def oracle_mats(orc, params, mdt):
+    return orc.expand(params, dtype=orc.F32 if mdt == "f32" else orc.BF16)
 
 
 def check(q, s, qr, sr, yr=None, exact=True):
@@ -145,37 +154,41 @@ def test_e2m1_pack_random_and_specials(kq, orc):
 
 # ---------------------------------------------------------------- quantizer vs oracle
 
-def test_quantize_cfg0_full(kq, orc):
+@pytest.mark.parametrize("variant,mdt", VARIANTS)
+def test_quantize_cfg0_full(kq, orc, variant, mdt):
     x, params = inputs.config_case("cfg0", 1152)
-    q, s = gpu_quantize(kq, x, params)
-    K = orc.expand(params)
+    q, s = gpu_quantize(kq, x, params, variant=variant, mdt=mdt)
+    K = oracle_mats(orc, params, mdt)
     qr, sr = orc.quantize(x, K)
     check(q, s, qr, sr, orc.transform(x, K))
 
 
+@pytest.mark.parametrize("variant,mdt", VARIANTS)
 @pytest.mark.parametrize("M,d", [(1, 32), (3, 96), (65, 1152), (7, 5600), (130, 2240), (33, 12288), (257, 3072),
                                  (300, 4608)])
-def test_quantize_ragged_shapes(kq, orc, M, d):
+def test_quantize_ragged_shapes(kq, orc, M, d, variant, mdt):
     x = inputs.activations(M, d, "t3", seed=[M, d], outlier_frac=0.01, outlier_scale=(20.0, 100.0))
     params = inputs.lu_params(d // 32, seed=[M, d, 9])
-    q, s = gpu_quantize(kq, x, params)
-    K = orc.expand(params)
+    q, s = gpu_quantize(kq, x, params, variant=variant, mdt=mdt)
+    K = oracle_mats(orc, params, mdt)
     qr, sr = orc.quantize(x, K)
     check(q, s, qr, sr, orc.transform(x, K))
 
 
-def test_quantize_strided_rows(kq, orc):
+@pytest.mark.parametrize("variant,mdt", VARIANTS)
+def test_quantize_strided_rows(kq, orc, variant, mdt):
     M, d, ldx = 50, 2240, 2240 + 136
     full = inputs.activations(M, ldx, "normal", seed=3, outlier_frac=0.01, outlier_scale=(50.0, 50.0))
     params = inputs.lu_params(d // 32, seed=4)
     xd = dev_bf16(full)[:, :d]
     assert xd.stride(0) == ldx
-    q, s = gpu_quantize(kq, None, params, x_dev=xd)
-    qr, sr = orc.quantize(np.ascontiguousarray(full[:, :d]), orc.expand(params))
+    q, s = gpu_quantize(kq, None, params, x_dev=xd, variant=variant, mdt=mdt)
+    qr, sr = orc.quantize(np.ascontiguousarray(full[:, :d]), oracle_mats(orc, params, mdt))
     check(q, s, qr, sr)
 
 
-def test_quantize_degenerate_blocks(kq, orc):
+@pytest.mark.parametrize("variant,mdt", VARIANTS)
+def test_quantize_degenerate_blocks(kq, orc, variant, mdt):
     rng = np.random.default_rng(8)
     M, d = 24, 256
     a = rng.standard_normal((M, d)).astype(np.float32)
@@ -193,13 +206,14 @@ def test_quantize_degenerate_blocks(kq, orc):
     a[10] = 3.4e38                               # overflow of the fp32 transform
     x = inputs.f32_to_bf16_bits(a)
     params = inputs.lu_params(d // 32, seed=9)
-    q, s = gpu_quantize(kq, x, params)
-    K = orc.expand(params)
+    q, s = gpu_quantize(kq, x, params, variant=variant, mdt=mdt)
+    K = oracle_mats(orc, params, mdt)
     qr, sr = orc.quantize(x, K)
     check(q, s, qr, sr)
 
 
-def test_quantize_identity_all_bf16_patterns(kq, orc):
+@pytest.mark.parametrize("variant,mdt", VARIANTS)
+def test_quantize_identity_all_bf16_patterns(kq, orc, variant, mdt):
     """K = I: every bf16 bit pattern (NaN/Inf included) goes through the scale and
     element steps as its own value; 2048 blocks of 32 consecutive patterns, plus a
     shuffled copy so that each block mixes magnitudes."""
@@ -207,12 +221,13 @@ def test_quantize_identity_all_bf16_patterns(kq, orc):
     rng = np.random.default_rng(10)
     x = np.concatenate([pats, rng.permutation(pats)]).reshape(-1, 1024)
     params = inputs.identity_params(1024 // 32)
-    q, s = gpu_quantize(kq, x, params)
-    qr, sr = orc.quantize(x, orc.expand(params))
+    q, s = gpu_quantize(kq, x, params, variant=variant, mdt=mdt)
+    qr, sr = orc.quantize(x, oracle_mats(orc, params, mdt))
     check(q, s, qr, sr)
 
 
-def test_quantize_exact_ties_identity(kq, orc):
+@pytest.mark.parametrize("variant,mdt", VARIANTS)
+def test_quantize_exact_ties_identity(kq, orc, variant, mdt):
     """Blocks whose elements sit exactly on E2M1 midpoints (and one bf16 step
     away) under K = I, so the certified path must resolve every one of them."""
     mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
@@ -225,19 +240,20 @@ def test_quantize_exact_ties_identity(kq, orc):
         rows.append(blk)
     x = inputs.f32_to_bf16_bits(np.stack(rows).reshape(1, -1))
     params = inputs.identity_params(x.shape[1] // 32)
-    q, s = gpu_quantize(kq, x, params)
-    qr, sr = orc.quantize(x, orc.expand(params))
+    q, s = gpu_quantize(kq, x, params, variant=variant, mdt=mdt)
+    qr, sr = orc.quantize(x, oracle_mats(orc, params, mdt))
     check(q, s, qr, sr)
 
 
-def test_quantize_hadamard_init_onehot(kq, orc):
+@pytest.mark.parametrize("variant,mdt", VARIANTS)
+def test_quantize_hadamard_init_onehot(kq, orc, variant, mdt):
     x = np.zeros((32, 32), np.float32)
     for c in range(32):
         x[c, c] = 32.0
     xb = inputs.f32_to_bf16_bits(x)
     params = inputs.hadamard_params(1)
-    q, s = gpu_quantize(kq, xb, params)
-    qr, sr = orc.quantize(xb, orc.expand(params))
+    q, s = gpu_quantize(kq, xb, params, variant=variant, mdt=mdt)
+    qr, sr = orc.quantize(xb, oracle_mats(orc, params, mdt))
     check(q, s, qr, sr)
     assert np.all(s == 127) and np.all((unpack(q) & 7) == 7)
 
@@ -248,28 +264,30 @@ def sampled_rows(M: int, n: int, seed: int) -> np.ndarray:
     return np.array(sorted(rows))
 
 
+@pytest.mark.parametrize("variant,mdt", VARIANTS)
 @pytest.mark.parametrize("name,d", [("pixart", 1152), ("pixart", 4608), ("sana", 2240), ("sana", 5600),
                                     ("flux", 3072), ("flux", 12288)])
-def test_quantize_full_config_sampled(kq, orc, name, d):
+def test_quantize_full_config_sampled(kq, orc, name, d, variant, mdt):
     x, params = inputs.config_case(name, d)
-    q, s = gpu_quantize(kq, x, params)
+    q, s = gpu_quantize(kq, x, params, variant=variant, mdt=mdt)
     rows = sampled_rows(x.shape[0], 40, seed=d)
-    K = orc.expand(params)
+    K = oracle_mats(orc, params, mdt)
     xs = np.ascontiguousarray(x[rows])
     qr, sr = orc.quantize(xs, K)
     check(q[rows], s[rows], qr, sr, orc.transform(xs, K))
 
 
+@pytest.mark.parametrize("variant,mdt", VARIANTS)
 @pytest.mark.parametrize("M", inputs.SWEEP_M)
-def test_quantize_sweep_shapes_sampled(kq, orc, M):
+def test_quantize_sweep_shapes_sampled(kq, orc, M, variant, mdt):
     for d in inputs.SWEEP_D:
         if M * d > 2**28 and d != inputs.SWEEP_D[0]:
             # largest shapes: only the first d runs here; the bench sweep covers the rest
             continue
         x, params = inputs.sweep_case(M, d)
-        q, s = gpu_quantize(kq, x, params)
+        q, s = gpu_quantize(kq, x, params, variant=variant, mdt=mdt)
         rows = sampled_rows(M, 12, seed=M + d)
-        K = orc.expand(params)
+        K = oracle_mats(orc, params, mdt)
         qr, sr = orc.quantize(np.ascontiguousarray(x[rows]), K)
         check(q[rows], s[rows], qr, sr)
 
