@@ -41,10 +41,17 @@ constexpr int kMmaThreads = (2 + kMmaEpiWarps) * 32; // 320
 constexpr int kMmaATileBytes = kMmaRows * 64;        // 8 KB per block per tile
 constexpr int kMmaAStageBytes = kMmaWb * kMmaATileBytes;
 constexpr int kMmaBBytes = 32 * 64;                  // one 32x32 bf16 matrix
-// Error allowance of the tensor-core sum relative to sum_i |x_i| max|K| (see
-// DESIGN: accumulation-order model, checked on the device by the parity tests).
-constexpr float kMmaErrC = 1.52587890625e-05f;       // 2^-16
-constexpr float kMmaErrAbs = 7.703719777548943e-34f; // 2^-110: flushed subnormal partial sums
+// Error allowance of the tensor-core sum, relative to sum_i |x_i| * max|K|.
+// Model: each kind::f16 UMMA adds its 16 exact bf16 x bf16 products to the fp32
+// accumulator with an error of at most about 2u of the magnitudes involved
+// (u = 2^-24; measured on B200 at most 11u in total for the six UMMAs of the
+// fp32 three-part mode and 5.3u for the two of the bf16 mode, over 8 M
+// elements including blocks spanning 2^40 in magnitude).  With the final fp32
+// rounding of the definition this gives 13u and 5u; the allowances below keep a
+// margin of 2.5x or more.
+constexpr float kMmaErrC_F32 = 1.9073486328125e-06f;  // 2^-19 = 32u
+constexpr float kMmaErrC_BF16 = 9.5367431640625e-07f; // 2^-20 = 16u
+constexpr float kMmaErrAbs = 7.703719777548943e-34f;  // 2^-110: flushed subnormal partial sums
 
 // UMMA instruction descriptor, kind::f16: D fp32, A and B bf16, A K-major,
 // B N-major, N = 32, M = 128.
@@ -108,6 +115,86 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 // rows under the 64-byte swizzle (16-byte chunk index ^= (row >> 1) & 3).
 __device__ __forceinline__ uint32_t sw64_offset(int row, int col) {
   return uint32_t(row) * 64u + ((uint32_t(col >> 3) ^ (uint32_t(row >> 1) & 3u)) << 4) + uint32_t(col & 7) * 2u;
+}
+
+// Upper bound of sum_i |x_i| for the 32 bf16 values of one 64-byte row held as
+// four 16-byte chunks: signs cleared, a tree of packed bf16 additions (each
+// rounding to nearest: relative error at most 2^-8 per level, four levels plus
+// one upward fp32 addition), then scaled up by 1 + 2^-5 > 1 / (1 - 2^-8)^4.
+// Sums that land in the subnormal range may lose up to 2^-126 per addition;
+// the absolute allowance kMmaErrAbs covers that.
+__device__ __forceinline__ float l1_upper_bf16(const uint4 (&v)[4]) {
+  uint32_t w[16];
+#pragma unroll
+  for (int k = 0; k < 4; k++) {
+    w[4 * k] = v[k].x & 0x7FFF7FFFu;
+    w[4 * k + 1] = v[k].y & 0x7FFF7FFFu;
+    w[4 * k + 2] = v[k].z & 0x7FFF7FFFu;
+    w[4 * k + 3] = v[k].w & 0x7FFF7FFFu;
+  }
+#pragma unroll
+  for (int n = 8; n >= 1; n >>= 1)
+#pragma unroll
+    for (int i = 0; i < n; i++) {
+      uint32_t r;
+      asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(w[i]), "r"(w[i + n]));
+      w[i] = r;
+    }
+  const float s = __fadd_ru(bf16lo(w[0]), bf16hi(w[0]));
+  return __fmul_ru(s, 1.03125f);
+}
+
+// Exact recomputation of one block by the whole warp from shared memory: lane
+// j computes y32_j = fp32( sum_i x_i K[i][j] ) in fp64 in increasing i from +0;
+// x is the owner's staged row (64-byte swizzle sw), K[i][j] the sum of the
+// staged bf16 parts (hi + mid) + lo, which is K exactly.  Scale from the exact
+// maximum, codes from the exact values; lane `owner` stores.
+__device__ __noinline__ void mma_exact_block_warp(const uint8_t* a_row, int sw, const uint8_t* bmat, int nsplit,
+                                                  uint8_t* qb, uint8_t* sb, int owner) {
+  const int lane = threadIdx.x & 31;
+  const uint4* xs = reinterpret_cast<const uint4*>(a_row);
+  uint32_t xw[16];
+#pragma unroll
+  for (int k = 0; k < 4; k++) {
+    const uint4 v = xs[k ^ sw];
+    xw[4 * k] = v.x;
+    xw[4 * k + 1] = v.y;
+    xw[4 * k + 2] = v.z;
+    xw[4 * k + 3] = v.w;
+  }
+  double acc = 0.0;
+#pragma unroll 8
+  for (int i = 0; i < kBlock; i++) {
+    const uint32_t off = sw64_offset(i, lane);
+    float kij = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(bmat + off));
+    if (nsplit == 3) {
+      kij = __fadd_rn(kij, __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(bmat + kMmaBBytes + off)));
+      kij = __fadd_rn(kij, __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(bmat + 2 * kMmaBBytes + off)));
+    }
+    const float xi = (i & 1) ? bf16hi(xw[i >> 1]) : bf16lo(xw[i >> 1]);
+    acc = __dadd_rn(acc, __dmul_rn(double(xi), double(kij)));
+  }
+  const float y = __double2float_rn(acc);
+  const bool finite = __all_sync(0xFFFFFFFFu, isfinite(y));
+  float m = fabsf(y);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  int byte = 0xFF;
+  uint32_t code = 0u;
+  if (finite) {
+    byte = e8m0_byte(m);
+    code = e2m1_one(__fmul_rn(y, inv_scale_of_byte(byte)));
+  }
+  uint32_t w = code << (4 * (lane & 7));
+  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
+  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
+  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 4);
+  const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, w, 0), w1 = __shfl_sync(0xFFFFFFFFu, w, 8);
+  const uint32_t w2 = __shfl_sync(0xFFFFFFFFu, w, 16), w3 = __shfl_sync(0xFFFFFFFFu, w, 24);
+  if (lane == owner) {
+    *reinterpret_cast<uint4*>(qb) = make_uint4(w0, w1, w2, w3);
+    *sb = uint8_t(byte);
+  }
 }
 
 template <int KSRC>
@@ -247,34 +334,44 @@ __global__ void __launch_bounds__(kMmaThreads, 2) quant_mma_kernel(const __grid_
         const bool act = row < p.M && b < p.nb;
         float y[32];
         tmem_ld32(tmem + (uint32_t(q * 32) << 16) + uint32_t(buf * kMmaAccCols + bw * 32), y);
-        // ||x||_1 of this row's block from the staged tile, rounded upward
-        const uint4* xs = reinterpret_cast<const uint4*>(a_stage + bw * kMmaATileBytes + rr * 64);
+        // upper bound of ||x||_1 of this row's block from the staged tile
+        const uint8_t* a_row = a_stage + bw * kMmaATileBytes + rr * 64;
+        const uint4* xs = reinterpret_cast<const uint4*>(a_row);
         const int sw = (rr >> 1) & 3;
-        float l1p[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        uint4 xv[4];
 #pragma unroll
-        for (int k = 0; k < 4; k++) {
-          const uint4 v = xs[k ^ sw];
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        for (int k = 0; k < 4; k++) xv[k] = xs[k];  // chunk order does not matter for a sum
+        const float l1 = l1_upper_bf16(xv);
+        // exact all-zero test on the bit patterns (the bf16 sum may flush subnormals)
+        uint32_t nz = 0u;
 #pragma unroll
-          for (int h = 0; h < 4; h++) {
-            l1p[h] = __fadd_ru(l1p[h], fabsf(bf16lo(w[h])));
-            l1p[h] = __fadd_ru(l1p[h], fabsf(bf16hi(w[h])));
-          }
-        }
-        const float l1 = __fadd_ru(__fadd_ru(l1p[0], l1p[1]), __fadd_ru(l1p[2], l1p[3]));
+        for (int k = 0; k < 4; k++) nz |= xv[k].x | xv[k].y | xv[k].z | xv[k].w;
+        const bool zero_block = (nz & 0x7FFF7FFFu) == 0u;
         uint64_t Y[16];
 #pragma unroll
         for (int m = 0; m < 16; m++) Y[m] = pk2(y[2 * m], y[2 * m + 1]);
         const float amax = block_amax(y);
-        const float cfac = __fmul_ru(kMmaErrC, __uint_as_float(kmax_bits[bw]));
+        const float cfac =
+            __fmul_ru(KSRC == KSRC_BF16 ? kMmaErrC_BF16 : kMmaErrC_F32, __uint_as_float(kmax_bits[bw]));
         const int64_t rowc = act ? row : 0;
         const int bc = act ? b : 0;
-        const uint16_t* xb = p.x + rowc * p.ldx + int64_t(bc) * kBlock;
-        const void* Kb = (KSRC == KSRC_BF16)
-                             ? static_cast<const void*>(static_cast<const uint16_t*>(p.mats) + int64_t(bc) * 1024)
-                             : static_cast<const void*>(static_cast<const float*>(p.mats) + int64_t(bc) * 1024);
-        certify_store<KSRC>(Y, amax, l1, cfac, kMmaErrAbs, false, act, xb, Kb,
-                            p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16, p.scales + rowc * int64_t(p.nb) + bc);
+        uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16;
+        uint8_t* sb = p.scales + rowc * int64_t(p.nb) + bc;
+        const uint8_t* bmat = b_smem + bw * p.nsplit * kMmaBBytes;
+        certify_store(Y, amax, l1, zero_block, cfac, kMmaErrAbs, false, act, qb, sb, [&](bool need) {
+          uint32_t pending = __ballot_sync(0xFFFFFFFFu, need);
+          while (pending) {
+            const int src = __ffs(pending) - 1;
+            pending &= pending - 1;
+            const int src_rr = q * 32 + src;
+            uint8_t* qs = reinterpret_cast<uint8_t*>(
+                __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(qb), src));
+            uint8_t* ss = reinterpret_cast<uint8_t*>(
+                __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(sb), src));
+            mma_exact_block_warp(a_stage + bw * kMmaATileBytes + src_rr * 64, (src_rr >> 1) & 3, bmat, p.nsplit, qs,
+                                 ss, src);
+          }
+        });
       }
       tc_fence_before();
       __syncwarp();

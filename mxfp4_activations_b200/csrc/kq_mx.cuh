@@ -133,17 +133,19 @@ __device__ __forceinline__ void warp_exact_pass(bool need, const uint16_t* xb, c
 
 // The certified MXFP4 step of one block.  Y holds the fast fp32 y as pairs,
 // amax = max|y| (NaN-propagating), and E = cfac * l1 + eabs bounds |y - y32|
-// for every element, y32 being the definition's value.  The scale is taken from
+// for every element, y32 being the definition's value; zero_block is the exact
+// test that every input of the block is +-0.  The scale is taken from
 // amax only when amax - E and amax + E (directed rounding) give the same E8M0
 // byte; each code only when (y - E) 2^-e rounded down and (y + E) 2^-e rounded
 // up give the same E2M1 code.  Any block that fails either test is recomputed
 // exactly by the warp.  Must be called by all 32 lanes; act marks real blocks.
-template <int KSRC>
-__device__ __forceinline__ void certify_store(const uint64_t (&Y)[16], float amax, float l1, float cfac, float eabs,
-                                              bool exact_only, bool act, const uint16_t* xb, const void* Kb,
-                                              uint8_t* qb, uint8_t* sb) {
-  // all inputs +-0: every y is +0 by definition (byte 0, codes 0)
-  const bool zero_block = l1 == 0.0f;
+// exact_pass(need) must recompute, warp-cooperatively, the block of every lane
+// with need == true and store its codes and scale.
+template <class ExactPass>
+__device__ __forceinline__ void certify_store(const uint64_t (&Y)[16], float amax, float l1, bool zero_block,
+                                              float cfac, float eabs, bool exact_only, bool act, uint8_t* qb,
+                                              uint8_t* sb, const ExactPass& exact_pass) {
+  // zero_block: all inputs +-0, so every y is +0 by definition (byte 0, codes 0)
   const float E = __fmaf_ru(cfac, l1, eabs);
   bool exact = exact_only || !(amax <= FLT_MAX) || !(E <= FLT_MAX);
   const int byte = e8m0_byte(__fadd_ru(amax, E));
@@ -164,7 +166,7 @@ __device__ __forceinline__ void certify_store(const uint64_t (&Y)[16], float ama
   const uint32_t diff = (cm[0] ^ cp[0]) | (cm[1] ^ cp[1]) | (cm[2] ^ cp[2]) | (cm[3] ^ cp[3]);
   // a block with an uncertain scale or an uncertain code is recomputed exactly
   const bool need = act && !zero_block && (exact || diff != 0u);
-  warp_exact_pass<KSRC>(need, xb, Kb, qb, sb);
+  exact_pass(need);
   if (!act || need) return;
   if (zero_block) {
     *reinterpret_cast<uint4*>(qb) = make_uint4(0u, 0u, 0u, 0u);

@@ -222,7 +222,9 @@ __device__ __forceinline__ void quant_block(const QuantParams& p, const Coef& c,
   const float amax = block_amax(y);
 
   constexpr int KSRC = (MODE == MODE_FWHT) ? KSRC_FWHT : KSRC_F32;
-  certify_store<KSRC>(Y, amax, l1, c.cfac, c.eabs, c.exact_only, act, xb, Kb, qb, sb);
+  // l1 is an upward-rounded fp32 sum of |x| without flushing: 0 exactly when all inputs are +-0
+  certify_store(Y, amax, l1, l1 == 0.0f, c.cfac, c.eabs, c.exact_only, act, qb, sb,
+                [&](bool need) { warp_exact_pass<KSRC>(need, xb, Kb, qb, sb); });
 }
 
 // ---------------------------------------------------------------- kernel
