@@ -186,8 +186,8 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   return launch_status("quant_kernel launch");
 }
 
-// Tensor-core variant: 128-row x 4-block tiles, one CTA per column group and
-// row-tile stride, two CTAs per SM (256 tensor-memory columns each).
+// Tensor-core variant: 128-row x 1-block tiles, one CTA per block column and
+// row-tile stride, up to four CTAs per SM (128 tensor-memory columns each).
 kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, const void* mats, bool mats_bf16,
                            uint8_t* q, uint8_t* scales, cudaStream_t stream) {
   const DeviceInfo* dev = device_info();
@@ -198,13 +198,13 @@ kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, con
   CUtensorMap tmap;
   const cuuint64_t gdim[3] = {32, cuuint64_t(M), cuuint64_t(nb)};
   const cuuint64_t gstride[2] = {cuuint64_t(ldx) * 2, 64};
-  const cuuint32_t box[3] = {32, cuuint32_t(kq::kMmaRows), cuuint32_t(kq::kMmaWb)};
+  const cuuint32_t box[3] = {32, cuuint32_t(kq::kMmaRows), 1};
   const cuuint32_t estride[3] = {1, 1, 1};
   if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), gdim, gstride, box, estride,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cuda_fail("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
-  const int smem = 1024 + kq::kMmaStages * kq::kMmaAStageBytes + kq::kMmaWb * 3 * kq::kMmaBBytes + 256;
+  const int smem = 1024 + kq::kMmaStages * kq::kMmaATileBytes + 3 * kq::kMmaBBytes + 256;
   if (smem > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
   auto kern = mats_bf16 ? kq::quant_mma_kernel<kq::KSRC_BF16> : kq::quant_mma_kernel<kq::KSRC_F32>;
   static std::atomic<int> attr_set[2][kMaxDevices];
@@ -221,19 +221,20 @@ kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, con
   p.M = M;
   p.nb = nb;
   const int64_t nrt = (M + kq::kMmaRows - 1) / kq::kMmaRows;
-  if (nrt > int64_t(INT32_MAX) / 2) return KQ_ERR_SHAPE;
+  if (nrt > int64_t(INT32_MAX) / 2 || nb > 2147483647) return KQ_ERR_SHAPE;
   p.n_row_tiles = int(nrt);
   p.nsplit = mats_bf16 ? 1 : 3;
   p.mats = mats;
   p.q = q;
   p.scales = scales;
-  const int ngroups = (nb + kq::kMmaWb - 1) / kq::kMmaWb;
-  if (ngroups > 65535 * 1024) return KQ_ERR_SHAPE;
-  int64_t gy = (int64_t(dev->sms) * 2) / ngroups;
+  // about two waves of four CTAs per SM, at least two row tiles per CTA when possible
+  const int64_t slots = int64_t(dev->sms) * 4;
+  int64_t gy = (2 * slots + nb - 1) / nb;
+  const int64_t gy_cap = (nrt + 1) / 2;
+  if (gy > gy_cap) gy = gy_cap;
   if (gy < 1) gy = 1;
-  if (gy > nrt) gy = nrt;
   if (gy > 65535) gy = 65535;
-  kern<<<dim3(ngroups, unsigned(gy)), kq::kMmaThreads, smem, stream>>>(tmap, p);
+  kern<<<dim3(unsigned(nb), unsigned(gy)), kq::kMmaThreads, smem, stream>>>(tmap, p);
   return launch_status("quant_mma_kernel launch");
 }
 

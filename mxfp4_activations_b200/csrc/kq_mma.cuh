@@ -11,17 +11,19 @@
 // accumulate in the same tensor-memory columns, so the tensor core sees K32
 // exactly; for bf16 matrices one part.
 //
-// CTA roles (one CTA per 128-row tile x 4-block column group at a time):
-//   warp 0     TMA producer: one 3-D load per tile (box {32, 128, 4}), no multicast
-//   warp 1     allocates 256 tensor-memory columns, one lane issues the UMMAs
-//              (2 or 6 per block) and commits them to an mbarrier
-//   warps 2-9  epilogue: tcgen05.ld of 32 fp32 columns per row, the row's L1
-//              norm from the staged tile, then the certified MXFP4 step shared
-//              with the butterfly kernel (kq_mx.cuh).  Warp w reads tensor-memory
-//              lanes 32*(w%4)..+31; warps w and w+4 take alternate blocks.
-// Two A-tile stages and two accumulator buffers overlap load, MMA and epilogue.
-// Every wait is bounded; on a timeout the CTA drains what it issued, frees its
-// tensor memory and exits with the device error flag set.
+// CTA roles (a CTA owns one 32-element block column and a stride of 128-row tiles):
+//   warp 0     TMA producer: one 3-D load per tile (box {32, 128, 1}), no multicast
+//   warp 1     allocates 128 tensor-memory columns, one lane issues the UMMAs
+//              (2 or 6 per tile) and commits them to an mbarrier
+//   warps 2-5  epilogue: tcgen05.ld of 32 fp32 columns per row (warp w reads
+//              tensor-memory lanes 32*(w%4)..+31), the row's L1 bound from the staged
+//              tile, then release of the accumulator buffer and the tile stage before
+//              the certified MXFP4 step shared with the butterfly kernel (kq_mx.cuh);
+//              its rare exact recomputation re-reads x and K from global memory.
+// Six tile stages and four accumulator buffers keep load, MMA and epilogue
+// overlapped; up to four CTAs share an SM.  Every wait is bounded; on a timeout
+// the CTA drains what it issued, frees its tensor memory and exits with the
+// device error flag set.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -32,14 +34,12 @@
 namespace kq {
 
 constexpr int kMmaRows = 128;                        // UMMA M (rows per tile)
-constexpr int kMmaWb = 4;                            // blocks per tile
-constexpr int kMmaStages = 2;                        // A-tile stages
-constexpr int kMmaAccCols = kMmaWb * 32;             // tensor-memory columns per accumulator buffer
-constexpr int kMmaTmemCols = 2 * kMmaAccCols;        // two buffers: 256 columns
-constexpr int kMmaEpiWarps = 8;
-constexpr int kMmaThreads = (2 + kMmaEpiWarps) * 32; // 320
-constexpr int kMmaATileBytes = kMmaRows * 64;        // 8 KB per block per tile
-constexpr int kMmaAStageBytes = kMmaWb * kMmaATileBytes;
+constexpr int kMmaStages = 6;                        // tile stages
+constexpr int kMmaAccBufs = 4;                       // accumulator buffers of 32 columns
+constexpr int kMmaTmemCols = kMmaAccBufs * 32;       // 128 columns
+constexpr int kMmaEpiWarps = 4;
+constexpr int kMmaThreads = (2 + kMmaEpiWarps) * 32; // 192
+constexpr int kMmaATileBytes = kMmaRows * 64;        // 8 KB per tile
 constexpr int kMmaBBytes = 32 * 64;                  // one 32x32 bf16 matrix
 // Error allowance of the tensor-core sum, relative to sum_i |x_i| * max|K|.
 // Model: each kind::f16 UMMA adds its 16 exact bf16 x bf16 products to the fp32
@@ -144,76 +144,23 @@ __device__ __forceinline__ float l1_upper_bf16(const uint4 (&v)[4]) {
   return __fmul_ru(s, 1.03125f);
 }
 
-// Exact recomputation of one block by the whole warp from shared memory: lane
-// j computes y32_j = fp32( sum_i x_i K[i][j] ) in fp64 in increasing i from +0;
-// x is the owner's staged row (64-byte swizzle sw), K[i][j] the sum of the
-// staged bf16 parts (hi + mid) + lo, which is K exactly.  Scale from the exact
-// maximum, codes from the exact values; lane `owner` stores.
-__device__ __noinline__ void mma_exact_block_warp(const uint8_t* a_row, int sw, const uint8_t* bmat, int nsplit,
-                                                  uint8_t* qb, uint8_t* sb, int owner) {
-  const int lane = threadIdx.x & 31;
-  const uint4* xs = reinterpret_cast<const uint4*>(a_row);
-  uint32_t xw[16];
-#pragma unroll
-  for (int k = 0; k < 4; k++) {
-    const uint4 v = xs[k ^ sw];
-    xw[4 * k] = v.x;
-    xw[4 * k + 1] = v.y;
-    xw[4 * k + 2] = v.z;
-    xw[4 * k + 3] = v.w;
-  }
-  double acc = 0.0;
-#pragma unroll 8
-  for (int i = 0; i < kBlock; i++) {
-    const uint32_t off = sw64_offset(i, lane);
-    float kij = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(bmat + off));
-    if (nsplit == 3) {
-      kij = __fadd_rn(kij, __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(bmat + kMmaBBytes + off)));
-      kij = __fadd_rn(kij, __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(bmat + 2 * kMmaBBytes + off)));
-    }
-    const float xi = (i & 1) ? bf16hi(xw[i >> 1]) : bf16lo(xw[i >> 1]);
-    acc = __dadd_rn(acc, __dmul_rn(double(xi), double(kij)));
-  }
-  const float y = __double2float_rn(acc);
-  const bool finite = __all_sync(0xFFFFFFFFu, isfinite(y));
-  float m = fabsf(y);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  int byte = 0xFF;
-  uint32_t code = 0u;
-  if (finite) {
-    byte = e8m0_byte(m);
-    code = e2m1_one(__fmul_rn(y, inv_scale_of_byte(byte)));
-  }
-  uint32_t w = code << (4 * (lane & 7));
-  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
-  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
-  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 4);
-  const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, w, 0), w1 = __shfl_sync(0xFFFFFFFFu, w, 8);
-  const uint32_t w2 = __shfl_sync(0xFFFFFFFFu, w, 16), w3 = __shfl_sync(0xFFFFFFFFu, w, 24);
-  if (lane == owner) {
-    *reinterpret_cast<uint4*>(qb) = make_uint4(w0, w1, w2, w3);
-    *sb = uint8_t(byte);
-  }
-}
-
 template <int KSRC>
-__global__ void __launch_bounds__(kMmaThreads, 2) quant_mma_kernel(const __grid_constant__ CUtensorMap tmap,
+__global__ void __launch_bounds__(kMmaThreads, 4) quant_mma_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                    const MmaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* a_smem = base;                                            // [stages][Wb][128][64 B]
-  uint8_t* b_smem = base + kMmaStages * kMmaAStageBytes;             // [Wb][nsplit][32][64 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(b_smem + kMmaWb * 3 * kMmaBBytes);
-  uint64_t* full_a = bars;                   // [stages]  TMA landed
-  uint64_t* empty_a = bars + kMmaStages;     // [stages]  epilogue done with the tile
-  uint64_t* mma_full = bars + 2 * kMmaStages;       // [2] accumulators ready
-  uint64_t* tmem_empty = bars + 2 * kMmaStages + 2; // [2] accumulators read
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kMmaStages + 4);
-  uint32_t* kmax_bits = tmem_slot + 1;       // [Wb] max |K| per block, as fp32 bits
+  uint8_t* a_smem = base;                                   // [stages][128][64 B]
+  uint8_t* b_smem = base + kMmaStages * kMmaATileBytes;     // [nsplit][32][64 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(b_smem + 3 * kMmaBBytes);
+  uint64_t* full_a = bars;                                  // [stages]  TMA landed
+  uint64_t* empty_a = bars + kMmaStages;                    // [stages]  epilogue read the tile
+  uint64_t* mma_full = bars + 2 * kMmaStages;               // [bufs]    accumulators ready
+  uint64_t* tmem_empty = bars + 2 * kMmaStages + kMmaAccBufs;  // [bufs] accumulators read
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kMmaStages + 2 * kMmaAccBufs);
+  uint32_t* kmax_bits = tmem_slot + 1;                      // max |K| of the block, as fp32 bits
 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int group = blockIdx.x;
+  const int b = blockIdx.x;  // the block column of this CTA
   const int my_tiles = (p.n_row_tiles - int(blockIdx.y) + int(gridDim.y) - 1) / int(gridDim.y);
 
   if (t == 0) {
@@ -221,39 +168,33 @@ __global__ void __launch_bounds__(kMmaThreads, 2) quant_mma_kernel(const __grid_
       mbar_init(&full_a[s], 1);
       mbar_init(&empty_a[s], kMmaEpiWarps);
     }
-    for (int b = 0; b < 2; b++) {
-      mbar_init(&mma_full[b], 1);
-      mbar_init(&tmem_empty[b], kMmaEpiWarps);
+    for (int i = 0; i < kMmaAccBufs; i++) {
+      mbar_init(&mma_full[i], 1);
+      mbar_init(&tmem_empty[i], kMmaEpiWarps);
     }
     fence_mbar_init();
+    *kmax_bits = 0u;
   }
-  if (t < kMmaWb) kmax_bits[t] = 0u;
   __syncthreads();
 
-  // B operands: this group's matrices, split into bf16 parts, written in the
-  // 64-byte-swizzled N-major layout the descriptors describe.
-  for (int e = t; e < kMmaWb * 1024; e += kMmaThreads) {
-    const int bw = e >> 10, i = (e >> 5) & 31, j = e & 31;
-    const int b = group * kMmaWb + bw;
-    float kf = 0.0f;
-    if (b < p.nb) {
-      const int64_t idx = int64_t(b) * 1024 + (e & 1023);
-      kf = (KSRC == KSRC_BF16) ? bf16_to_f32(static_cast<const uint16_t*>(p.mats)[idx])
-                               : static_cast<const float*>(p.mats)[idx];
-    }
-    atomicMax(&kmax_bits[bw], __float_as_uint(fabsf(kf)) & 0x7FFFFFFFu);
+  // B operand: K_b split into bf16 parts, 64-byte-swizzled N-major layout.
+  for (int e = t; e < 1024; e += kMmaThreads) {
+    const int i = e >> 5, j = e & 31;
+    const int64_t idx = int64_t(b) * 1024 + e;
+    const float kf = (KSRC == KSRC_BF16) ? bf16_to_f32(static_cast<const uint16_t*>(p.mats)[idx])
+                                         : static_cast<const float*>(p.mats)[idx];
+    atomicMax(kmax_bits, __float_as_uint(fabsf(kf)) & 0x7FFFFFFFu);
     const uint32_t off = sw64_offset(i, j);
-    uint8_t* mb = b_smem + bw * p.nsplit * kMmaBBytes;
     if (p.nsplit == 1) {
-      *reinterpret_cast<__nv_bfloat16*>(mb + off) = __float2bfloat16_rn(kf);
+      *reinterpret_cast<__nv_bfloat16*>(b_smem + off) = __float2bfloat16_rn(kf);
     } else {
       const __nv_bfloat16 hi = __float2bfloat16_rn(kf);
       const float r1 = __fsub_rn(kf, __bfloat162float(hi));
       const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
       const float r2 = __fsub_rn(r1, __bfloat162float(mid));
-      *reinterpret_cast<__nv_bfloat16*>(mb + off) = hi;
-      *reinterpret_cast<__nv_bfloat16*>(mb + kMmaBBytes + off) = mid;
-      *reinterpret_cast<__nv_bfloat16*>(mb + 2 * kMmaBBytes + off) = __float2bfloat16_rn(r2);
+      *reinterpret_cast<__nv_bfloat16*>(b_smem + off) = hi;
+      *reinterpret_cast<__nv_bfloat16*>(b_smem + kMmaBBytes + off) = mid;
+      *reinterpret_cast<__nv_bfloat16*>(b_smem + 2 * kMmaBBytes + off) = __float2bfloat16_rn(r2);
     }
   }
   if (warp == 1) {
@@ -279,8 +220,8 @@ __global__ void __launch_bounds__(kMmaThreads, 2) quant_mma_kernel(const __grid_
             !mbar_wait_bounded(&empty_a[s], uint32_t(it / kMmaStages - 1) & 1u, kWaitLimitNs))
           break;
         const int tile = int(blockIdx.y) + it * int(gridDim.y);
-        mbar_arrive_expect_tx(&full_a[s], uint32_t(kMmaAStageBytes));
-        tma_load_3d(a_smem + s * kMmaAStageBytes, &tmap, &full_a[s], 0, tile * kMmaRows, group * kMmaWb);
+        mbar_arrive_expect_tx(&full_a[s], uint32_t(kMmaATileBytes));
+        tma_load_3d(a_smem + s * kMmaATileBytes, &tmap, &full_a[s], 0, tile * kMmaRows, b);
       }
       if (it < my_tiles) {
         for (int k = (it > kMmaStages ? it - kMmaStages : 0); k < it; k++)
@@ -290,95 +231,76 @@ __global__ void __launch_bounds__(kMmaThreads, 2) quant_mma_kernel(const __grid_
   } else if (warp == 1) {
     // ------------------------------------------------ UMMA issuer
     if (lane == 0) {
+      const uint32_t b_base = smem_addr(b_smem);
       int it = 0;
       for (; it < my_tiles; it++) {
-        const int s = it % kMmaStages, buf = it & 1;
+        const int s = it % kMmaStages, buf = it % kMmaAccBufs;
         if (!mbar_wait_bounded(&full_a[s], uint32_t(it / kMmaStages) & 1u, kWaitLimitNs)) break;
-        if (it >= 2 && !mbar_wait_bounded(&tmem_empty[buf], uint32_t(it / 2 - 1) & 1u, kWaitLimitNs)) break;
+        if (it >= kMmaAccBufs &&
+            !mbar_wait_bounded(&tmem_empty[buf], uint32_t(it / kMmaAccBufs - 1) & 1u, kWaitLimitNs))
+          break;
         tc_fence_after();
-        const uint32_t a_base = smem_addr(a_smem + s * kMmaAStageBytes);
-        const uint32_t b_base = smem_addr(b_smem);
+        const uint32_t a_base = smem_addr(a_smem + s * kMmaATileBytes);
+        const uint32_t d = tmem + uint32_t(buf * 32);
+        for (int sp = 0; sp < p.nsplit; sp++) {
 #pragma unroll
-        for (int bw = 0; bw < kMmaWb; bw++) {
-          const uint32_t d = tmem + uint32_t(buf * kMmaAccCols + bw * 32);
-          for (int sp = 0; sp < p.nsplit; sp++) {
-#pragma unroll
-            for (int kh = 0; kh < 2; kh++) {
-              const uint64_t ad = umma_desc(a_base + bw * kMmaATileBytes + kh * 32, 16, 512);
-              const uint64_t bd = umma_desc(b_base + (bw * p.nsplit + sp) * kMmaBBytes + kh * 1024, 2048, 512);
-              umma_bf16(d, ad, bd, (sp | kh) != 0 ? 1u : 0u);
-            }
+          for (int kh = 0; kh < 2; kh++) {
+            const uint64_t ad = umma_desc(a_base + kh * 32, 16, 512);
+            const uint64_t bd = umma_desc(b_base + sp * kMmaBBytes + kh * 1024, 2048, 512);
+            umma_bf16(d, ad, bd, (sp | kh) != 0 ? 1u : 0u);
           }
         }
         umma_commit(&mma_full[buf]);
       }
       if (it > 0) {  // the last commit must have landed before tensor memory is freed
         const int k = it - 1;
-        mbar_wait_bounded(&mma_full[k & 1], uint32_t(k / 2) & 1u, kWaitLimitNs / 4);
+        mbar_wait_bounded(&mma_full[k % kMmaAccBufs], uint32_t(k / kMmaAccBufs) & 1u, kWaitLimitNs / 4);
       }
     }
   } else {
     // ------------------------------------------------ epilogue
-    const int q = warp & 3;                 // tensor-memory lane quarter
-    const int half = (warp - 2) >> 2;       // which alternate blocks
-    const int rr = q * 32 + lane;           // row inside the tile
+    const int q = warp & 3;        // tensor-memory lane quarter
+    const int rr = q * 32 + lane;  // row inside the tile
+    const int sw = (rr >> 1) & 3;
+    const float cfac = __fmul_ru(KSRC == KSRC_BF16 ? kMmaErrC_BF16 : kMmaErrC_F32, __uint_as_float(*kmax_bits));
+    const void* Kb = (KSRC == KSRC_BF16)
+                         ? static_cast<const void*>(static_cast<const uint16_t*>(p.mats) + int64_t(b) * 1024)
+                         : static_cast<const void*>(static_cast<const float*>(p.mats) + int64_t(b) * 1024);
     for (int it = 0; it < my_tiles; it++) {
-      const int s = it % kMmaStages, buf = it & 1;
-      if (!mbar_wait_bounded(&mma_full[buf], uint32_t(it / 2) & 1u, kWaitLimitNs)) break;
+      const int s = it % kMmaStages, buf = it % kMmaAccBufs;
+      if (!mbar_wait_bounded(&mma_full[buf], uint32_t(it / kMmaAccBufs) & 1u, kWaitLimitNs)) break;
       tc_fence_after();
-      const int64_t row = int64_t(int(blockIdx.y) + it * int(gridDim.y)) * kMmaRows + rr;
-      const uint8_t* a_stage = a_smem + s * kMmaAStageBytes;
-#pragma unroll 1
-      for (int bw = half; bw < kMmaWb; bw += 2) {
-        const int b = group * kMmaWb + bw;
-        const bool act = row < p.M && b < p.nb;
-        float y[32];
-        tmem_ld32(tmem + (uint32_t(q * 32) << 16) + uint32_t(buf * kMmaAccCols + bw * 32), y);
-        // upper bound of ||x||_1 of this row's block from the staged tile
-        const uint8_t* a_row = a_stage + bw * kMmaATileBytes + rr * 64;
-        const uint4* xs = reinterpret_cast<const uint4*>(a_row);
-        const int sw = (rr >> 1) & 3;
-        uint4 xv[4];
+      float y[32];
+      tmem_ld32(tmem + (uint32_t(q * 32) << 16) + uint32_t(buf * 32), y);
+      // this row's inputs from the staged tile: L1 upper bound and exact zero test
+      const uint4* xs = reinterpret_cast<const uint4*>(a_smem + s * kMmaATileBytes + rr * 64);
+      uint4 xv[4];
 #pragma unroll
-        for (int k = 0; k < 4; k++) xv[k] = xs[k];  // chunk order does not matter for a sum
-        const float l1 = l1_upper_bf16(xv);
-        // exact all-zero test on the bit patterns (the bf16 sum may flush subnormals)
-        uint32_t nz = 0u;
-#pragma unroll
-        for (int k = 0; k < 4; k++) nz |= xv[k].x | xv[k].y | xv[k].z | xv[k].w;
-        const bool zero_block = (nz & 0x7FFF7FFFu) == 0u;
-        uint64_t Y[16];
-#pragma unroll
-        for (int m = 0; m < 16; m++) Y[m] = pk2(y[2 * m], y[2 * m + 1]);
-        const float amax = block_amax(y);
-        const float cfac =
-            __fmul_ru(KSRC == KSRC_BF16 ? kMmaErrC_BF16 : kMmaErrC_F32, __uint_as_float(kmax_bits[bw]));
-        const int64_t rowc = act ? row : 0;
-        const int bc = act ? b : 0;
-        uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16;
-        uint8_t* sb = p.scales + rowc * int64_t(p.nb) + bc;
-        const uint8_t* bmat = b_smem + bw * p.nsplit * kMmaBBytes;
-        certify_store(Y, amax, l1, zero_block, cfac, kMmaErrAbs, false, act, qb, sb, [&](bool need) {
-          uint32_t pending = __ballot_sync(0xFFFFFFFFu, need);
-          while (pending) {
-            const int src = __ffs(pending) - 1;
-            pending &= pending - 1;
-            const int src_rr = q * 32 + src;
-            uint8_t* qs = reinterpret_cast<uint8_t*>(
-                __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(qb), src));
-            uint8_t* ss = reinterpret_cast<uint8_t*>(
-                __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(sb), src));
-            mma_exact_block_warp(a_stage + bw * kMmaATileBytes + src_rr * 64, (src_rr >> 1) & 3, bmat, p.nsplit, qs,
-                                 ss, src);
-          }
-        });
-      }
+      for (int k = 0; k < 4; k++) xv[k] = xs[k ^ sw];
+      // accumulators and tile are no longer needed: release them before the math
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&tmem_empty[buf]);
         mbar_arrive(&empty_a[s]);
       }
+      const float l1 = l1_upper_bf16(xv);
+      uint32_t nz = 0u;
+#pragma unroll
+      for (int k = 0; k < 4; k++) nz |= xv[k].x | xv[k].y | xv[k].z | xv[k].w;
+      const bool zero_block = (nz & 0x7FFF7FFFu) == 0u;
+      const int64_t row = int64_t(int(blockIdx.y) + it * int(gridDim.y)) * kMmaRows + rr;
+      const bool act = row < p.M;
+      const int64_t rowc = act ? row : 0;
+      uint64_t Y[16];
+#pragma unroll
+      for (int m2 = 0; m2 < 16; m2++) Y[m2] = pk2(y[2 * m2], y[2 * m2 + 1]);
+      const float amax = block_amax(y);
+      uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(b) * 16;
+      uint8_t* sb = p.scales + rowc * int64_t(p.nb) + b;
+      const uint16_t* xb = p.x + rowc * p.ldx + int64_t(b) * kBlock;
+      certify_store(Y, amax, l1, zero_block, cfac, kMmaErrAbs, false, act, qb, sb,
+                    [&](bool need) { warp_exact_pass<KSRC>(need, xb, Kb, qb, sb); });
     }
   }
   tc_fence_before();
