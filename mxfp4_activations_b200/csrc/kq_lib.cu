@@ -186,8 +186,8 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   return launch_status("quant_kernel launch");
 }
 
-// Tensor-core variant: 128-row x 1-block tiles, one CTA per block column and
-// row-tile stride, up to four CTAs per SM (128 tensor-memory columns each).
+// Tensor-core variant: 128-row x 4-block tiles, one CTA per 4-block column group
+// and row-tile stride, one CTA per SM (it holds all 512 tensor-memory columns).
 kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, const void* mats, bool mats_bf16,
                            uint8_t* q, uint8_t* scales, cudaStream_t stream) {
   const DeviceInfo* dev = device_info();
@@ -198,13 +198,13 @@ kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, con
   CUtensorMap tmap;
   const cuuint64_t gdim[3] = {32, cuuint64_t(M), cuuint64_t(nb)};
   const cuuint64_t gstride[2] = {cuuint64_t(ldx) * 2, 64};
-  const cuuint32_t box[3] = {32, cuuint32_t(kq::kMmaRows), 1};
+  const cuuint32_t box[3] = {32, cuuint32_t(kq::kMmaRows), cuuint32_t(kq::kMmaWb)};
   const cuuint32_t estride[3] = {1, 1, 1};
   if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), gdim, gstride, box, estride,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cuda_fail("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
-  const int smem = 1024 + kq::kMmaStages * kq::kMmaATileBytes + 3 * kq::kMmaBBytes + 256;
+  const int smem = 1024 + kq::kMmaStages * kq::kMmaAStageBytes + kq::kMmaWb * 3 * kq::kMmaBBytes + 256;
   if (smem > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
   auto kern = mats_bf16 ? kq::quant_mma_kernel<kq::KSRC_BF16> : kq::quant_mma_kernel<kq::KSRC_F32>;
   static std::atomic<int> attr_set[2][kMaxDevices];
@@ -227,14 +227,19 @@ kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, con
   p.mats = mats;
   p.q = q;
   p.scales = scales;
-  // about two waves of four CTAs per SM, at least two row tiles per CTA when possible
-  const int64_t slots = int64_t(dev->sms) * 4;
-  int64_t gy = (2 * slots + nb - 1) / nb;
-  const int64_t gy_cap = (nrt + 1) / 2;
-  if (gy > gy_cap) gy = gy_cap;
-  if (gy < 1) gy = 1;
-  if (gy > 65535) gy = 65535;
-  kern<<<dim3(unsigned(nb), unsigned(gy)), kq::kMmaThreads, smem, stream>>>(tmap, p);
+  // one CTA per SM: pick the row-tile stride that minimises the estimated
+  // makespan (waves of CTAs x row tiles per CTA)
+  const int64_t ngroups = (nb + kq::kMmaWb - 1) / kq::kMmaWb;
+  int64_t gy = 1, best = INT64_MAX;
+  for (int64_t g = 1; g <= nrt && g <= 65535; g++) {
+    const int64_t waves = (ngroups * g + dev->sms - 1) / dev->sms;
+    const int64_t cost = waves * ((nrt + g - 1) / g);
+    if (cost < best) {
+      best = cost;
+      gy = g;
+    }
+  }
+  kern<<<dim3(unsigned(ngroups), unsigned(gy)), kq::kMmaThreads, smem, stream>>>(tmap, p);
   return launch_status("quant_mma_kernel launch");
 }
 

@@ -11,19 +11,21 @@
 // accumulate in the same tensor-memory columns, so the tensor core sees K32
 // exactly; for bf16 matrices one part.
 //
-// CTA roles (a CTA owns one 32-element block column and a stride of 128-row tiles):
-//   warp 0     TMA producer: one 3-D load per tile (box {32, 128, 1}), no multicast
-//   warp 1     allocates 128 tensor-memory columns, one lane issues the UMMAs
-//              (2 or 6 per tile) and commits them to an mbarrier
-//   warps 2-5  epilogue: tcgen05.ld of 32 fp32 columns per row (warp w reads
-//              tensor-memory lanes 32*(w%4)..+31), the row's L1 bound from the staged
-//              tile, then release of the accumulator buffer and the tile stage before
-//              the certified MXFP4 step shared with the butterfly kernel (kq_mx.cuh);
-//              its rare exact recomputation re-reads x and K from global memory.
-// Six tile stages and four accumulator buffers keep load, MMA and epilogue
-// overlapped; up to four CTAs share an SM.  Every wait is bounded; on a timeout
-// the CTA drains what it issued, frees its tensor memory and exits with the
-// device error flag set.
+// CTA roles (a CTA owns a group of four 32-element block columns and a stride of
+// 128-row tiles; one CTA per SM holds all 512 tensor-memory columns):
+//   warp 0      TMA producer: one 3-D load per tile (box {32, 128, 4}: each row
+//               reads 256 contiguous bytes), no multicast
+//   warp 1      allocates the tensor memory; one lane issues the UMMAs (2 or 6 per
+//               block) and commits each tile to an mbarrier
+//   warps 2-17  epilogue: warp w handles block (w-2)/4 of the tile for tensor-memory
+//               lanes 32*(w%4)..+31: tcgen05.ld of 32 fp32 columns per row, the row's
+//               L1 bound and zero test from the staged tile, release of the
+//               accumulator buffer and the tile stage, then the certified MXFP4 step
+//               shared with the butterfly kernel (kq_mx.cuh); its rare exact
+//               recomputation re-reads x and K from global memory.
+// Four tile stages and four accumulator buffers keep load, MMA and epilogue
+// overlapped.  Every wait is bounded; on a timeout the CTA drains what it issued,
+// frees its tensor memory and exits with the device error flag set.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -34,12 +36,15 @@
 namespace kq {
 
 constexpr int kMmaRows = 128;                        // UMMA M (rows per tile)
-constexpr int kMmaStages = 6;                        // tile stages
-constexpr int kMmaAccBufs = 4;                       // accumulator buffers of 32 columns
-constexpr int kMmaTmemCols = kMmaAccBufs * 32;       // 128 columns
-constexpr int kMmaEpiWarps = 4;
-constexpr int kMmaThreads = (2 + kMmaEpiWarps) * 32; // 192
-constexpr int kMmaATileBytes = kMmaRows * 64;        // 8 KB per tile
+constexpr int kMmaWb = 4;                            // blocks per tile
+constexpr int kMmaStages = 4;                        // tile stages
+constexpr int kMmaAccBufs = 4;                       // accumulator buffers
+constexpr int kMmaAccCols = kMmaWb * 32;             // columns per buffer
+constexpr int kMmaTmemCols = kMmaAccBufs * kMmaAccCols;  // 512: the whole tensor memory
+constexpr int kMmaEpiWarps = 4 * kMmaWb;             // one warp per (block, lane quarter)
+constexpr int kMmaThreads = (2 + kMmaEpiWarps) * 32; // 576
+constexpr int kMmaATileBytes = kMmaRows * 64;        // 8 KB per block of a tile
+constexpr int kMmaAStageBytes = kMmaWb * kMmaATileBytes;  // 32 KB per tile
 constexpr int kMmaBBytes = 32 * 64;                  // one 32x32 bf16 matrix
 // Error allowance of the tensor-core sum, relative to sum_i |x_i| * max|K|.
 // Model: each kind::f16 UMMA adds its 16 exact bf16 x bf16 products to the fp32
@@ -145,22 +150,22 @@ __device__ __forceinline__ float l1_upper_bf16(const uint4 (&v)[4]) {
 }
 
 template <int KSRC>
-__global__ void __launch_bounds__(kMmaThreads, 4) quant_mma_kernel(const __grid_constant__ CUtensorMap tmap,
+__global__ void __launch_bounds__(kMmaThreads, 1) quant_mma_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                    const MmaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* a_smem = base;                                   // [stages][128][64 B]
-  uint8_t* b_smem = base + kMmaStages * kMmaATileBytes;     // [nsplit][32][64 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(b_smem + 3 * kMmaBBytes);
+  uint8_t* a_smem = base;                                   // [stages][Wb][128][64 B]
+  uint8_t* b_smem = base + kMmaStages * kMmaAStageBytes;    // [Wb][nsplit][32][64 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(b_smem + kMmaWb * 3 * kMmaBBytes);
   uint64_t* full_a = bars;                                  // [stages]  TMA landed
   uint64_t* empty_a = bars + kMmaStages;                    // [stages]  epilogue read the tile
   uint64_t* mma_full = bars + 2 * kMmaStages;               // [bufs]    accumulators ready
   uint64_t* tmem_empty = bars + 2 * kMmaStages + kMmaAccBufs;  // [bufs] accumulators read
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kMmaStages + 2 * kMmaAccBufs);
-  uint32_t* kmax_bits = tmem_slot + 1;                      // max |K| of the block, as fp32 bits
+  uint32_t* kmax_bits = tmem_slot + 1;                      // [Wb] max |K| per block, as fp32 bits
 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int b = blockIdx.x;  // the block column of this CTA
+  const int group = blockIdx.x;
   const int my_tiles = (p.n_row_tiles - int(blockIdx.y) + int(gridDim.y) - 1) / int(gridDim.y);
 
   if (t == 0) {
@@ -173,28 +178,44 @@ __global__ void __launch_bounds__(kMmaThreads, 4) quant_mma_kernel(const __grid_
       mbar_init(&tmem_empty[i], kMmaEpiWarps);
     }
     fence_mbar_init();
-    *kmax_bits = 0u;
   }
+  if (t < kMmaWb) kmax_bits[t] = 0u;
   __syncthreads();
 
-  // B operand: K_b split into bf16 parts, 64-byte-swizzled N-major layout.
-  for (int e = t; e < 1024; e += kMmaThreads) {
-    const int i = e >> 5, j = e & 31;
-    const int64_t idx = int64_t(b) * 1024 + e;
-    const float kf = (KSRC == KSRC_BF16) ? bf16_to_f32(static_cast<const uint16_t*>(p.mats)[idx])
-                                         : static_cast<const float*>(p.mats)[idx];
-    atomicMax(kmax_bits, __float_as_uint(fabsf(kf)) & 0x7FFFFFFFu);
-    const uint32_t off = sw64_offset(i, j);
-    if (p.nsplit == 1) {
-      *reinterpret_cast<__nv_bfloat16*>(b_smem + off) = __float2bfloat16_rn(kf);
-    } else {
-      const __nv_bfloat16 hi = __float2bfloat16_rn(kf);
-      const float r1 = __fsub_rn(kf, __bfloat162float(hi));
-      const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-      const float r2 = __fsub_rn(r1, __bfloat162float(mid));
-      *reinterpret_cast<__nv_bfloat16*>(b_smem + off) = hi;
-      *reinterpret_cast<__nv_bfloat16*>(b_smem + kMmaBBytes + off) = mid;
-      *reinterpret_cast<__nv_bfloat16*>(b_smem + 2 * kMmaBBytes + off) = __float2bfloat16_rn(r2);
+  // B operands: this group's matrices split into bf16 parts, 64-byte-swizzled
+  // N-major layout; max |K| per block reduced per warp, then one atomic.
+  {
+    uint32_t kloc[kMmaWb] = {};
+    for (int e = t; e < kMmaWb * 1024; e += kMmaThreads) {
+      const int bw = e >> 10, i = (e >> 5) & 31, j = e & 31;
+      const int b = group * kMmaWb + bw;
+      float kf = 0.0f;
+      if (b < p.nb) {
+        const int64_t idx = int64_t(b) * 1024 + (e & 1023);
+        kf = (KSRC == KSRC_BF16) ? bf16_to_f32(static_cast<const uint16_t*>(p.mats)[idx])
+                                 : static_cast<const float*>(p.mats)[idx];
+      }
+#pragma unroll
+      for (int k = 0; k < kMmaWb; k++)
+        if (k == bw) kloc[k] = max(kloc[k], __float_as_uint(fabsf(kf)) & 0x7FFFFFFFu);
+      const uint32_t off = sw64_offset(i, j);
+      uint8_t* mb = b_smem + bw * p.nsplit * kMmaBBytes;
+      if (p.nsplit == 1) {
+        *reinterpret_cast<__nv_bfloat16*>(mb + off) = __float2bfloat16_rn(kf);
+      } else {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(kf);
+        const float r1 = __fsub_rn(kf, __bfloat162float(hi));
+        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+        const float r2 = __fsub_rn(r1, __bfloat162float(mid));
+        *reinterpret_cast<__nv_bfloat16*>(mb + off) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(mb + kMmaBBytes + off) = mid;
+        *reinterpret_cast<__nv_bfloat16*>(mb + 2 * kMmaBBytes + off) = __float2bfloat16_rn(r2);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kMmaWb; k++) {
+      const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, kloc[k]);
+      if (lane == 0 && m != 0u) atomicMax(&kmax_bits[k], m);
     }
   }
   if (warp == 1) {
@@ -220,8 +241,8 @@ __global__ void __launch_bounds__(kMmaThreads, 4) quant_mma_kernel(const __grid_
             !mbar_wait_bounded(&empty_a[s], uint32_t(it / kMmaStages - 1) & 1u, kWaitLimitNs))
           break;
         const int tile = int(blockIdx.y) + it * int(gridDim.y);
-        mbar_arrive_expect_tx(&full_a[s], uint32_t(kMmaATileBytes));
-        tma_load_3d(a_smem + s * kMmaATileBytes, &tmap, &full_a[s], 0, tile * kMmaRows, b);
+        mbar_arrive_expect_tx(&full_a[s], uint32_t(kMmaAStageBytes));
+        tma_load_3d(a_smem + s * kMmaAStageBytes, &tmap, &full_a[s], 0, tile * kMmaRows, group * kMmaWb);
       }
       if (it < my_tiles) {
         for (int k = (it > kMmaStages ? it - kMmaStages : 0); k < it; k++)
@@ -240,14 +261,17 @@ __global__ void __launch_bounds__(kMmaThreads, 4) quant_mma_kernel(const __grid_
             !mbar_wait_bounded(&tmem_empty[buf], uint32_t(it / kMmaAccBufs - 1) & 1u, kWaitLimitNs))
           break;
         tc_fence_after();
-        const uint32_t a_base = smem_addr(a_smem + s * kMmaATileBytes);
-        const uint32_t d = tmem + uint32_t(buf * 32);
-        for (int sp = 0; sp < p.nsplit; sp++) {
+        const uint32_t a_base = smem_addr(a_smem + s * kMmaAStageBytes);
 #pragma unroll
-          for (int kh = 0; kh < 2; kh++) {
-            const uint64_t ad = umma_desc(a_base + kh * 32, 16, 512);
-            const uint64_t bd = umma_desc(b_base + sp * kMmaBBytes + kh * 1024, 2048, 512);
-            umma_bf16(d, ad, bd, (sp | kh) != 0 ? 1u : 0u);
+        for (int bw = 0; bw < kMmaWb; bw++) {
+          const uint32_t d = tmem + uint32_t(buf * kMmaAccCols + bw * 32);
+          for (int sp = 0; sp < p.nsplit; sp++) {
+#pragma unroll
+            for (int kh = 0; kh < 2; kh++) {
+              const uint64_t ad = umma_desc(a_base + bw * kMmaATileBytes + kh * 32, 16, 512);
+              const uint64_t bd = umma_desc(b_base + (bw * p.nsplit + sp) * kMmaBBytes + kh * 1024, 2048, 512);
+              umma_bf16(d, ad, bd, (sp | kh) != 0 ? 1u : 0u);
+            }
           }
         }
         umma_commit(&mma_full[buf]);
@@ -259,21 +283,25 @@ __global__ void __launch_bounds__(kMmaThreads, 4) quant_mma_kernel(const __grid_
     }
   } else {
     // ------------------------------------------------ epilogue
-    const int q = warp & 3;        // tensor-memory lane quarter
-    const int rr = q * 32 + lane;  // row inside the tile
+    const int q = warp & 3;            // tensor-memory lane quarter
+    const int bw = (warp - 2) >> 2;    // block of the tile
+    const int rr = q * 32 + lane;      // row inside the tile
     const int sw = (rr >> 1) & 3;
-    const float cfac = __fmul_ru(KSRC == KSRC_BF16 ? kMmaErrC_BF16 : kMmaErrC_F32, __uint_as_float(*kmax_bits));
+    const int b = group * kMmaWb + bw;
+    const bool col_ok = b < p.nb;
+    const int bc = col_ok ? b : 0;
+    const float cfac = __fmul_ru(KSRC == KSRC_BF16 ? kMmaErrC_BF16 : kMmaErrC_F32, __uint_as_float(kmax_bits[bw]));
     const void* Kb = (KSRC == KSRC_BF16)
-                         ? static_cast<const void*>(static_cast<const uint16_t*>(p.mats) + int64_t(b) * 1024)
-                         : static_cast<const void*>(static_cast<const float*>(p.mats) + int64_t(b) * 1024);
+                         ? static_cast<const void*>(static_cast<const uint16_t*>(p.mats) + int64_t(bc) * 1024)
+                         : static_cast<const void*>(static_cast<const float*>(p.mats) + int64_t(bc) * 1024);
     for (int it = 0; it < my_tiles; it++) {
       const int s = it % kMmaStages, buf = it % kMmaAccBufs;
       if (!mbar_wait_bounded(&mma_full[buf], uint32_t(it / kMmaAccBufs) & 1u, kWaitLimitNs)) break;
       tc_fence_after();
       float y[32];
-      tmem_ld32(tmem + (uint32_t(q * 32) << 16) + uint32_t(buf * 32), y);
+      tmem_ld32(tmem + (uint32_t(q * 32) << 16) + uint32_t(buf * kMmaAccCols + bw * 32), y);
       // this row's inputs from the staged tile: L1 upper bound and exact zero test
-      const uint4* xs = reinterpret_cast<const uint4*>(a_smem + s * kMmaATileBytes + rr * 64);
+      const uint4* xs = reinterpret_cast<const uint4*>(a_smem + s * kMmaAStageBytes + bw * kMmaATileBytes + rr * 64);
       uint4 xv[4];
 #pragma unroll
       for (int k = 0; k < 4; k++) xv[k] = xs[k ^ sw];
@@ -290,15 +318,15 @@ __global__ void __launch_bounds__(kMmaThreads, 4) quant_mma_kernel(const __grid_
       for (int k = 0; k < 4; k++) nz |= xv[k].x | xv[k].y | xv[k].z | xv[k].w;
       const bool zero_block = (nz & 0x7FFF7FFFu) == 0u;
       const int64_t row = int64_t(int(blockIdx.y) + it * int(gridDim.y)) * kMmaRows + rr;
-      const bool act = row < p.M;
+      const bool act = col_ok && row < p.M;
       const int64_t rowc = act ? row : 0;
       uint64_t Y[16];
 #pragma unroll
       for (int m2 = 0; m2 < 16; m2++) Y[m2] = pk2(y[2 * m2], y[2 * m2 + 1]);
       const float amax = block_amax(y);
-      uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(b) * 16;
-      uint8_t* sb = p.scales + rowc * int64_t(p.nb) + b;
-      const uint16_t* xb = p.x + rowc * p.ldx + int64_t(b) * kBlock;
+      uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16;
+      uint8_t* sb = p.scales + rowc * int64_t(p.nb) + bc;
+      const uint16_t* xb = p.x + rowc * p.ldx + int64_t(bc) * kBlock;
       certify_store(Y, amax, l1, zero_block, cfac, kMmaErrAbs, false, act, qb, sb,
                     [&](bool need) { warp_exact_pass<KSRC>(need, xb, Kb, qb, sb); });
     }
