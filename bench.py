@@ -496,7 +496,8 @@ def run_sweep(args) -> None:
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     cases = [(name, M, d) for name, c in inputs.CONFIGS.items() for d in c["ds"] for M in [c["M"]]]
     cases += [("sweep", M, d) for M in inputs.SWEEP_M for d in inputs.SWEEP_D]
-    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    # clean-L2 flush: reading a buffer larger than L2 leaves no dirty lines behind
+    flush = torch.ones(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
     for name, M, d in cases:
         x, p = inputs.sweep_case(M, d) if name == "sweep" else inputs.config_case(name, d)
         xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
@@ -505,9 +506,14 @@ def run_sweep(args) -> None:
         inv_s = torch.from_numpy(inputs.smooth_inv_scale(x)).cuda()
         q = torch.empty((M, d // 2), dtype=torch.uint8, device="cuda")
         s = torch.empty((M, d // 32), dtype=torch.uint8, device="cuda")
+        mats16 = kq.kq_expand_blocks(pd, dtype=torch.bfloat16)
         calls = {
             "kroquant": lambda: lib.kq_quantize(xd.data_ptr(), M, d, d, mats.data_ptr(), 0, fac.data_ptr(),
                                                 q.data_ptr(), s.data_ptr(), 2, stream),
+            "kroquant_mma": lambda: lib.kq_quantize(xd.data_ptr(), M, d, d, mats.data_ptr(), 0, None,
+                                                    q.data_ptr(), s.data_ptr(), 1, stream),
+            "kroquant_mma_bf16": lambda: lib.kq_quantize(xd.data_ptr(), M, d, d, mats16.data_ptr(), 1, None,
+                                                         q.data_ptr(), s.data_ptr(), 1, stream),
             "smooth": lambda: lib.kq_ref_smooth_quantize(xd.data_ptr(), M, d, d, inv_s.data_ptr(), q.data_ptr(),
                                                          s.data_ptr(), stream),
             "fwht": lambda: lib.kq_ref_fwht_quantize(xd.data_ptr(), M, d, d, q.data_ptr(), s.data_ptr(), stream),
@@ -519,7 +525,7 @@ def run_sweep(args) -> None:
                 assert fn() == 0
             times = []
             for _ in range(reps):
-                flush.fill_(1.0)  # evict L2 between launches
+                flush.sum()  # evict L2 between launches
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record()
                 assert fn() == 0
@@ -529,9 +535,10 @@ def run_sweep(args) -> None:
             med = statistics.median(times)
             res[kind] = {"us_median": round(med, 3), "us_best": round(min(times), 3),
                          "gbs_median": round(algo_bytes(M, d) / (med * 1e-6) / 1e9, 1)}
-        line = {"sweep": name, "M": M, "d": d, "bytes": algo_bytes(M, d), **res,
-                "kroquant_vs_smooth_speed": round(res["smooth"]["us_median"] / res["kroquant"]["us_median"], 3),
-                "kroquant_vs_fwht_speed": round(res["fwht"]["us_median"] / res["kroquant"]["us_median"], 3)}
+        best_f32 = min(("kroquant", "kroquant_mma"), key=lambda k: res[k]["us_median"])
+        line = {"sweep": name, "M": M, "d": d, "bytes": algo_bytes(M, d), **res, "best_f32_variant": best_f32,
+                "kroquant_vs_smooth_speed": round(res["smooth"]["us_median"] / res[best_f32]["us_median"], 3),
+                "kroquant_vs_fwht_speed": round(res["fwht"]["us_median"] / res[best_f32]["us_median"], 3)}
         print(json.dumps(line), flush=True)
         del xd, q, s
     assert kq.kq_get_device_error(clear=True) == 0

@@ -76,42 +76,20 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// ---- launch geometry of the quantizer kernels
-struct QuantGeom {
-  int W, R, cons_warps, threads, stages, stage_stride, smem;
-};
+// ---- launch of the quantizer kernels (tile: 8 block columns x 32 rows)
 
-QuantGeom quant_geometry(int nb, int smem_optin) {
-  QuantGeom g{};
-  // at most 224 consumer threads (+1 producer warp = 256): two CTAs per SM at 128 registers
-  constexpr int kMaxCons = 224;
-  const int ncol = (nb + kMaxCons - 1) / kMaxCons;
-  g.W = (nb + ncol - 1) / ncol;  // <= 224 (TMA box limit is 256)
-  int bestR = 1;
-  double bestU = -1.0;
-  for (int R = 1; R * g.W <= kMaxCons; R++) {
-    const int T = ((R * g.W + 31) / 32) * 32;
-    const double u = double(R * g.W) / double(T);
-    // prefer full warps, then more threads per CTA
-    const double score = u - 0.0005 * double(kMaxCons - T) / 32.0;
-    if (score > bestU + 1e-12) {
-      bestU = score;
-      bestR = R;
-    }
-  }
-  g.R = bestR;
-  g.cons_warps = (g.R * g.W + 31) / 32;
-  g.threads = (g.cons_warps + 1) * 32;
-  const int stage_bytes = g.W * g.R * 64;
-  g.stage_stride = (stage_bytes + 1023) & ~1023;
-  int st = (96 * 1024) / g.stage_stride;
-  if (st > 6) st = 6;
-  if (st < 2) st = 2;
-  const int fixed = 1024 /*alignment slack*/ + 128 /*barriers*/;
-  while (st > 2 && st * g.stage_stride + fixed > smem_optin) st--;
-  g.stages = st;
-  g.smem = st * g.stage_stride + fixed;
-  return g;
+// Row-tile stride for a grid of ncol column groups on sms SMs holding per_sm
+// CTAs each: fill the resident slots once, then balance the row tiles.
+int64_t row_stride(int64_t ncol, int64_t nrt, int sms, int per_sm) {
+  const int64_t slots = int64_t(sms) * per_sm;
+  int64_t gy = slots / ncol;
+  if (gy < 1) gy = 1;
+  if (gy > nrt) gy = nrt;
+  // same makespan (row tiles per CTA) with fewer CTAs: drop the surplus
+  const int64_t per = (nrt + gy - 1) / gy;
+  gy = (nrt + per - 1) / per;
+  if (gy > 65535) gy = 65535;
+  return gy;
 }
 
 template <int MODE>
@@ -122,13 +100,15 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   EncodeTiledFn enc = encode_tiled();
   if (enc == nullptr) return cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
   const int nb = int(d / 32);
-  const QuantGeom g = quant_geometry(nb, dev->smem_optin);
-  if (g.smem > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
+  const int stages = kq::kQMaxStages;
+  const int smem = 1024 /*alignment slack*/ + stages * kq::kQStageBytes + kq::kQCols * kq::kQCoef * 4 +
+                   2 * kq::kQMaxStages * 8;
+  if (smem > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
 
   CUtensorMap tmap;
-  const cuuint64_t gdim[3] = {32, cuuint64_t(nb), cuuint64_t(M)};
-  const cuuint64_t gstride[2] = {64, cuuint64_t(ldx) * 2};
-  const cuuint32_t box[3] = {32, cuuint32_t(g.W), cuuint32_t(g.R)};
+  const cuuint64_t gdim[3] = {32, cuuint64_t(M), cuuint64_t(nb)};
+  const cuuint64_t gstride[2] = {cuuint64_t(ldx) * 2, 64};
+  const cuuint32_t box[3] = {32, cuuint32_t(kq::kQRows), cuuint32_t(kq::kQCols)};
   const cuuint32_t estride[3] = {1, 1, 1};
   if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), gdim, gstride, box, estride,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -136,25 +116,21 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
     return cuda_fail("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
 
   auto kern = kq::quant_kernel<MODE>;
-  // dynamic shared memory limit: the opt-in maximum minus the kernel's static shared memory
-  static std::atomic<int> dyn_limit[kMaxDevices];
+  static std::atomic<int> attr_set[kMaxDevices];
   int devid = 0;
   cudaGetDevice(&devid);
-  if (dyn_limit[devid].load() == 0) {
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
-    if (e != cudaSuccess) return cuda_fail("cudaFuncGetAttributes", e);
-    const int lim = dev->smem_optin - int(fa.sharedSizeBytes);
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+  if (!attr_set[devid].load()) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
-    dyn_limit[devid].store(lim);
+    attr_set[devid].store(1);
   }
-  if (g.smem > dyn_limit[devid].load()) return KQ_ERR_UNSUPPORTED;
-  int per_sm = 0;
-  {
-    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.threads, g.smem);
+  static std::atomic<int> occ[kMaxDevices];
+  int per_sm = occ[devid].load();
+  if (per_sm == 0) {
+    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kq::kQThreads, smem);
     if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveBlocksPerMultiprocessor", e);
     if (per_sm < 1) return cuda_fail("occupancy: no resident CTA", cudaErrorInvalidConfiguration);
+    occ[devid].store(per_sm);
   }
 
   kq::QuantParams p;
@@ -162,27 +138,20 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   p.ldx = ldx;
   p.M = M;
   p.nb = nb;
-  p.W = g.W;
-  p.R = g.R;
-  const int64_t nrt = (M + g.R - 1) / g.R;
-  if (nrt > int64_t(INT32_MAX)) return KQ_ERR_SHAPE;
+  const int64_t nrt = (M + kq::kQRows - 1) / kq::kQRows;
+  if (nrt > int64_t(INT32_MAX) / kq::kQRows) return KQ_ERR_SHAPE;  // TMA row coordinates are int32
   p.n_row_tiles = int(nrt);
-  p.stages = g.stages;
-  p.stage_stride = g.stage_stride;
-  p.cons_warps = g.cons_warps;
+  p.stages = stages;
   p.mats = mats;
   p.factored = factored;
   p.inv_s = inv_s;
   p.q = q;
   p.scales = scales;
 
-  const int ncol = (nb + g.W - 1) / g.W;
-  const int64_t target = int64_t(dev->sms) * per_sm;
-  int64_t gy = (target + ncol - 1) / ncol;
-  if (gy > nrt) gy = nrt;
-  if (gy > 65535) gy = 65535;
-  if (gy < 1) gy = 1;
-  kern<<<dim3(ncol, unsigned(gy)), g.threads, g.smem, stream>>>(tmap, p);
+  const int64_t ncol = (nb + kq::kQCols - 1) / kq::kQCols;
+  if (ncol > int64_t(INT32_MAX)) return KQ_ERR_SHAPE;
+  const int64_t gy = row_stride(ncol, nrt, dev->sms, per_sm);
+  kern<<<dim3(unsigned(ncol), unsigned(gy)), kq::kQThreads, smem, stream>>>(tmap, p);
   return launch_status("quant_kernel launch");
 }
 

@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) quant_mma_kernel(const __grid_
       uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16;
       uint8_t* sb = p.scales + rowc * int64_t(p.nb) + bc;
       const uint16_t* xb = p.x + rowc * p.ldx + int64_t(bc) * kBlock;
-      certify_store(Y, amax, l1, zero_block, cfac, kMmaErrAbs, false, act, qb, sb,
+      certify_store(Y, amax, l1, zero_block, cfac, kMmaErrAbs, !(cfac <= FLT_MAX), act, qb, sb,
                     [&](bool need) { warp_exact_pass<KSRC>(need, xb, Kb, qb, sb); });
     }
   }

@@ -134,7 +134,8 @@ __device__ __forceinline__ void warp_exact_pass(bool need, const uint16_t* xb, c
 // The certified MXFP4 step of one block.  Y holds the fast fp32 y as pairs,
 // amax = max|y| (NaN-propagating), and E = cfac * l1 + eabs bounds |y - y32|
 // for every element, y32 being the definition's value; zero_block is the exact
-// test that every input of the block is +-0.  The scale is taken from
+// test that every input of the block is +-0 (then y = +0 when every matrix entry
+// is finite).  exact_only sends every block, zero or not, to the exact path.  The scale is taken from
 // amax only when amax - E and amax + E (directed rounding) give the same E8M0
 // byte; each code only when (y - E) 2^-e rounded down and (y + E) 2^-e rounded
 // up give the same E2M1 code.  Any block that fails either test is recomputed
@@ -164,8 +165,9 @@ __device__ __forceinline__ void certify_store(const uint64_t (&Y)[16], float ama
 #pragma unroll
   for (int k = 0; k < 4; k++) cp[k] = codes8(V + 4 * k);
   const uint32_t diff = (cm[0] ^ cp[0]) | (cm[1] ^ cp[1]) | (cm[2] ^ cp[2]) | (cm[3] ^ cp[3]);
-  // a block with an uncertain scale or an uncertain code is recomputed exactly
-  const bool need = act && !zero_block && (exact || diff != 0u);
+  // a block with an uncertain scale or an uncertain code is recomputed exactly;
+  // with exact_only (matrix entries possibly non-finite) so is an all-zero block
+  const bool need = act && (exact_only || (!zero_block && (exact || diff != 0u)));
   exact_pass(need);
   if (!act || need) return;
   if (zero_block) {

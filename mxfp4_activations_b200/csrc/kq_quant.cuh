@@ -10,16 +10,22 @@
 //               form (c/a = 1, b/d = -1, D_j = +-2^-2.5): the FWHT comparison point.
 //   MODE_SMOOTH per-channel scaling y_j = x_j s_j: the SmoothQuant comparison point.
 //
-// Data movement: a CTA owns a column tile of W blocks and walks row tiles of R
-// rows.  Each row tile (W*R blocks of 64 B) is fetched by one 3-D TMA load
-// (box {32, W, R}, 64-byte swizzle, no multicast) into a ring of shared-memory
-// stages.  The last warp of the CTA only issues those loads; a stage is refilled
-// when every consumer warp has arrived on its "empty" barrier, so consumer
-// warps never wait for each other.  Consumer thread t = r*W + c handles block c
-// of row r.  With the 64 B swizzle the 16-byte chunk k of block t sits at chunk
-// k ^ ((t >> 1) & 3), which makes the four 16-byte shared loads of a warp
-// conflict-free.  The butterfly stages on index bits 1..4 run as packed f32x2
-// FMAs on element pairs (2m, 2m+1).
+// Data movement: a tile is 8 block columns x 32 rows (16 KB of bf16), fetched by
+// one 3-D TMA load (box {32 elements, 32 rows, 8 blocks}, 64-byte swizzle, no
+// multicast) into a ring of shared-memory stages; in shared memory the tile is
+// [block column][row][64 B].  A CTA owns one group of 8 block columns and walks
+// a stride of row tiles.  Its last warp only issues the loads; a stage is
+// refilled when every consumer warp has arrived on its "empty" barrier, so
+// consumer warps never wait for each other.  Consumer warp w holds block
+// columns 4(w&1)..4(w&1)+3 and rows 8(w>>1)..8(w>>1)+7 of each tile: lane l
+// takes column 4(w&1) + l/8 and row 8(w>>1) + l%8.  Eight lanes share a column,
+// so the per-column coefficients are read from a shared table by broadcast loads
+// (four distinct addresses per warp, in distinct banks) instead of living in
+// registers, and the four 16-byte shared loads of a block stay conflict-free
+// under the swizzle (chunk k of 64-byte row t sits at chunk k ^ ((t >> 1) & 3)).
+// Each row's four blocks give 64 contiguous bytes of codes per warp store.
+// The butterfly stages on index bits 1..4 run as packed f32x2 FMAs on element
+// pairs (2m, 2m+1).
 //
 // Exactness (KRON, FWHT): the fp32 result y_f differs from the definition
 // y32 = fp32(sum_i x_i K32[i][j]) by at most E = C * ||x||_1 * max|K|.  KRON:
@@ -48,17 +54,27 @@ constexpr float kKronErrC = 9.5367431640625e-07f;   // 2^-20 = 16 u (14 u needed
 constexpr float kFwhtErrC = 4.76837158203125e-07f;  // 2^-21 = 8 u (7 u needed)
 constexpr float kErrAbs = 7.174648137343064e-43f;   // 2^-140: FWHT subnormal-range slack
 
+// Tile geometry (see "Data movement" above).
+constexpr int kQCols = 8;                        // block columns per tile
+constexpr int kQRows = 32;                       // rows per tile
+constexpr int kQConsWarps = 8;                   // consumer warps (4 columns x 8 rows each)
+constexpr int kQThreads = (kQConsWarps + 1) * 32;  // + the TMA producer warp
+constexpr int kQStageBytes = kQCols * kQRows * 64;  // 16 KB
+constexpr int kQMaxStages = 4;
+// Shared coefficient table, one record of kQCoef floats per block column:
+//   [4s .. 4s+3]  (lam, lam, bet, bet) of the stage on index bit s+1 (factor 3-s), s = 0..3
+//   [16 .. 47]    D_0 .. D_31 (SMOOTH: the 32 per-channel factors)
+//   [48 .. 51]    lam and bet of factor 4 (index bit 0), C * max|K| (+inf: exact path
+//                 only), absolute allowance
+constexpr int kQCoef = 56;
+
 struct QuantParams {
   const uint16_t* x;      // bf16 bits [M][ldx] (exact path re-reads rows from here)
   int64_t ldx;
   int64_t M;
   int nb;                 // blocks per row (d / 32)
-  int W;                  // blocks per column tile
-  int R;                  // rows per row tile
-  int n_row_tiles;
-  int stages;
-  int stage_stride;       // bytes between stages (multiple of 1024)
-  int cons_warps;         // consumer warps; one more warp issues the TMA loads
+  int n_row_tiles;        // ceil(M / 32)
+  int stages;             // shared-memory stages (<= kQMaxStages)
   const float* mats;      // KRON: fp32 [nb][32][32] (exact path)
   const float* factored;  // KRON: [nb][48]
   const float* inv_s;     // SMOOTH: [nb*32]
@@ -66,68 +82,33 @@ struct QuantParams {
   uint8_t* scales;        // [M][nb]
 };
 
-// ---------------------------------------------------------------- per-thread coefficients
-
-struct Coef {
-  uint64_t lam2[5];  // (c_k/a_k, c_k/a_k); factor k acts on index bit 4-k
-  uint64_t bet2[5];  // (b_k/d_k, b_k/d_k)
-  uint64_t D2[16];   // (D[2m], D[2m+1]); SMOOTH: the per-channel factors
-  float cfac;        // C * max|K|
-  float eabs;        // absolute error allowance for subnormal-range results
-  bool exact_only;
-};
-
+// Entry f of the coefficient record of block column b (fp32 bits as read by
+// the consumer warps).
 template <int MODE>
-__device__ __forceinline__ void load_coef(const QuantParams& p, int b, Coef& c) {
+__device__ __forceinline__ float coef_entry(const QuantParams& p, int b, int f) {
   if (MODE == MODE_KRON) {
-    const float4* f = reinterpret_cast<const float4*>(p.factored + int64_t(b) * kFactored);
-    float buf[kFactored];
-#pragma unroll
-    for (int i = 0; i < kFactored / 4; i++) {
-      const float4 v = __ldg(f + i);
-      buf[4 * i + 0] = v.x;
-      buf[4 * i + 1] = v.y;
-      buf[4 * i + 2] = v.z;
-      buf[4 * i + 3] = v.w;
+    const float* fb = p.factored + int64_t(b) * kFactored;
+    if (f < 16) {
+      const int k = 3 - (f >> 2);                  // factor of this stage
+      return __ldg(fb + ((f & 2) ? 5 + k : k));    // bet_k = b/d, lam_k = c/a
     }
-#pragma unroll
-    for (int k = 0; k < 5; k++) {
-      c.lam2[k] = pk2(buf[k], buf[k]);
-      c.bet2[k] = pk2(buf[5 + k], buf[5 + k]);
-    }
-#pragma unroll
-    for (int m = 0; m < 16; m++) c.D2[m] = pk2(buf[10 + 2 * m], buf[11 + 2 * m]);
-    c.cfac = __fmul_ru(kKronErrC, buf[42]);
-    c.eabs = buf[44];
-    c.exact_only = buf[43] != 0.0f;
-  } else if (MODE == MODE_SMOOTH) {
-    const float4* f = reinterpret_cast<const float4*>(p.inv_s + int64_t(b) * kBlock);
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-      const float4 v = __ldg(f + i);
-      c.D2[2 * i] = pk2(v.x, v.y);
-      c.D2[2 * i + 1] = pk2(v.z, v.w);
-    }
-    c.cfac = 0.0f;
-    c.eabs = 0.0f;
-    c.exact_only = false;
-  } else {
-    c.cfac = kFwhtErrC * kFwhtC;
-    c.eabs = kErrAbs;
-    c.exact_only = false;
+    if (f < 48) return __ldg(fb + 10 + (f - 16));  // D
+    if (f == 48) return __ldg(fb + 4);
+    if (f == 49) return __ldg(fb + 9);
+    if (f == 50) return __ldg(fb + 43) != 0.0f ? __int_as_float(0x7F800000) : __fmul_ru(kKronErrC, __ldg(fb + 42));
+    if (f == 51) return __ldg(fb + 44);
+    return 0.0f;
   }
+  if (MODE == MODE_SMOOTH) return (f >= 16 && f < 48) ? __ldg(p.inv_s + int64_t(b) * kBlock + (f - 16)) : 0.0f;
+  return 0.0f;
 }
 
 // ---------------------------------------------------------------- one block of one row
-
+//
+// cf: shared-memory address of this block column's coefficient record.
 template <int MODE>
-__device__ __forceinline__ void quant_block(const QuantParams& p, const Coef& c, const uint4 (&xr)[4], int64_t row,
-                                            int b, bool act) {
-  uint8_t* qb = p.q + row * int64_t(p.nb) * 16 + int64_t(b) * 16;
-  uint8_t* sb = p.scales + row * int64_t(p.nb) + b;
-  const uint16_t* xb = p.x + row * p.ldx + int64_t(b) * kBlock;
-  const float* Kb = (MODE == MODE_KRON) ? p.mats + int64_t(b) * kBlock * kBlock : nullptr;
-
+__device__ __forceinline__ void quant_block(uint32_t cf, const uint4 (&xr)[4], bool act, uint8_t* qb, uint8_t* sb,
+                                            const uint16_t* xb, const float* Kb) {
   float x[kBlock];
 #pragma unroll
   for (int k = 0; k < 4; k++) {
@@ -143,7 +124,11 @@ __device__ __forceinline__ void quant_block(const QuantParams& p, const Coef& c,
 
   if (MODE == MODE_SMOOTH) {
 #pragma unroll
-    for (int m = 0; m < 16; m++) Y[m] = mul2_rn(pk2(x[2 * m], x[2 * m + 1]), c.D2[m]);  // one rounding each
+    for (int i = 0; i < 8; i++) {
+      const uint4 dv = lds128(cf + 64 + 16 * i);
+      Y[2 * i] = mul2_rn(pk2(x[4 * i], x[4 * i + 1]), pk2(__uint_as_float(dv.x), __uint_as_float(dv.y)));
+      Y[2 * i + 1] = mul2_rn(pk2(x[4 * i + 2], x[4 * i + 3]), pk2(__uint_as_float(dv.z), __uint_as_float(dv.w)));
+    }
 #pragma unroll
     for (int m = 0; m < 16; m++) upk2(Y[m], y[2 * m], y[2 * m + 1]);
     const float amax = block_amax(y);
@@ -168,13 +153,19 @@ __device__ __forceinline__ void quant_block(const QuantParams& p, const Coef& c,
   for (int j = 0; j < kBlock; j++) l1p[j & 3] = __fadd_ru(l1p[j & 3], fabsf(x[j]));
   const float l1 = __fadd_ru(__fadd_ru(l1p[0], l1p[1]), __fadd_ru(l1p[2], l1p[3]));
 
+  float cfac, eabs;
   // stage on index bit 0 (factor 4), scalar: the pair partners share a register pair
   {
     float l4 = 1.0f, b4 = -1.0f;
     if (MODE == MODE_KRON) {
-      float t0;
-      upk2(c.lam2[4], l4, t0);
-      upk2(c.bet2[4], b4, t0);
+      const uint4 s0 = lds128(cf + 192);
+      l4 = __uint_as_float(s0.x);
+      b4 = __uint_as_float(s0.y);
+      cfac = __uint_as_float(s0.z);
+      eabs = __uint_as_float(s0.w);
+    } else {
+      cfac = kFwhtErrC * kFwhtC;
+      eabs = kErrAbs;
     }
 #pragma unroll
     for (int m = 0; m < 16; m++) {
@@ -193,6 +184,12 @@ __device__ __forceinline__ void quant_block(const QuantParams& p, const Coef& c,
   // stages on index bits 1..4 (factors 3..0) on packed pairs
 #pragma unroll
   for (int pb = 1; pb < 5; pb++) {
+    uint64_t L2 = 0, B2 = 0;
+    if (MODE == MODE_KRON) {
+      const uint4 c = lds128(cf + 16 * (pb - 1));
+      L2 = pk2(__uint_as_float(c.x), __uint_as_float(c.y));
+      B2 = pk2(__uint_as_float(c.z), __uint_as_float(c.w));
+    }
 #pragma unroll
     for (int m = 0; m < 16; m++) {
       if (m & (1 << (pb - 1))) continue;
@@ -202,19 +199,24 @@ __device__ __forceinline__ void quant_block(const QuantParams& p, const Coef& c,
         Y[m] = add2_rn(y0, y1);
         Y[m1] = sub2_rn(y1, y0);
       } else {
-        Y[m] = fma2_rn(c.lam2[4 - pb], y1, y0);
-        Y[m1] = fma2_rn(c.bet2[4 - pb], y0, y1);
+        Y[m] = fma2_rn(L2, y1, y0);
+        Y[m1] = fma2_rn(B2, y0, y1);
       }
     }
   }
   // diagonal: D_j (FWHT: +-2^-2.5 with the sign of (-1)^popcount(j))
+  if (MODE == MODE_FWHT) {
 #pragma unroll
-  for (int m = 0; m < 16; m++) {
-    if (MODE == MODE_FWHT) {
+    for (int m = 0; m < 16; m++) {
       const float sg = (__popc(m) & 1) ? -kFwhtC : kFwhtC;
       Y[m] = mul2_rn(pk2(sg, -sg), Y[m]);
-    } else {
-      Y[m] = mul2_rn(c.D2[m], Y[m]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const uint4 dv = lds128(cf + 64 + 16 * i);
+      Y[2 * i] = mul2_rn(pk2(__uint_as_float(dv.x), __uint_as_float(dv.y)), Y[2 * i]);
+      Y[2 * i + 1] = mul2_rn(pk2(__uint_as_float(dv.z), __uint_as_float(dv.w)), Y[2 * i + 1]);
     }
   }
 #pragma unroll
@@ -223,33 +225,35 @@ __device__ __forceinline__ void quant_block(const QuantParams& p, const Coef& c,
 
   constexpr int KSRC = (MODE == MODE_FWHT) ? KSRC_FWHT : KSRC_F32;
   // l1 is an upward-rounded fp32 sum of |x| without flushing: 0 exactly when all inputs are +-0
-  certify_store(Y, amax, l1, l1 == 0.0f, c.cfac, c.eabs, c.exact_only, act, qb, sb,
+  // cfac = +inf marks a column whose butterfly form is unusable: every block exact
+  certify_store(Y, amax, l1, l1 == 0.0f, cfac, eabs, !(cfac <= FLT_MAX), act, qb, sb,
                 [&](bool need) { warp_exact_pass<KSRC>(need, xb, Kb, qb, sb); });
 }
 
 // ---------------------------------------------------------------- kernel
 
 template <int MODE>
-__global__ void __launch_bounds__(256, 2) quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
+__global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + p.stages * p.stage_stride);
-  uint64_t* empty = full + p.stages;
+  float* coef = reinterpret_cast<float*>(base + p.stages * kQStageBytes);  // [kQCols][kQCoef]
+  uint64_t* full = reinterpret_cast<uint64_t*>(coef + kQCols * kQCoef);
+  uint64_t* empty = full + kQMaxStages;
 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const uint32_t stage_bytes = uint32_t(p.W) * uint32_t(p.R) * 64u;
+  const int col0 = int(blockIdx.x) * kQCols;
   const int my_tiles = (p.n_row_tiles - int(blockIdx.y) + int(gridDim.y) - 1) / int(gridDim.y);
 
   if (t == 0) {
     for (int s = 0; s < p.stages; s++) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], uint32_t(p.cons_warps));
+      mbar_init(&empty[s], uint32_t(kQConsWarps));
     }
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == p.cons_warps) {  // producer warp: one thread issues every TMA load
+  if (warp == kQConsWarps) {  // producer warp: one thread issues every TMA load
     if (lane == 0) {
       prefetch_tensormap(&tmap);
       int it = 0;
@@ -257,8 +261,8 @@ __global__ void __launch_bounds__(256, 2) quant_kernel(const __grid_constant__ C
         const int s = it % p.stages;
         if (it >= p.stages && !mbar_wait_bounded(&empty[s], uint32_t(it / p.stages - 1) & 1u, kWaitLimitNs)) break;
         const int tile = int(blockIdx.y) + it * int(gridDim.y);
-        mbar_arrive_expect_tx(&full[s], stage_bytes);
-        tma_load_3d(base + s * p.stage_stride, &tmap, &full[s], 0, int(blockIdx.x) * p.W, tile * p.R);
+        mbar_arrive_expect_tx(&full[s], uint32_t(kQStageBytes));
+        tma_load_3d(base + s * kQStageBytes, &tmap, &full[s], 0, tile * kQRows, col0);
       }
       if (it < my_tiles) {  // consumers stopped: let the loads still in flight land before exiting
         for (int k = (it > p.stages ? it - p.stages : 0); k < it; k++)
@@ -268,28 +272,56 @@ __global__ void __launch_bounds__(256, 2) quant_kernel(const __grid_constant__ C
     return;
   }
 
-  const int bb = t % p.W, rr = t / p.W;
-  const int b = blockIdx.x * p.W + bb;
-  const bool has_tile = rr < p.R;
-  const bool active = has_tile && b < p.nb;
-  Coef c = {};
-  if (active) load_coef<MODE>(p, b, c);
+  // coefficient table of this CTA's columns (consumer warps only; the producer
+  // is already streaming the first tiles)
+  if (MODE != MODE_FWHT) {
+    constexpr int kN = kQCols * kQCoef;
+    constexpr int kPer = (kN + kQConsWarps * 32 - 1) / (kQConsWarps * 32);
+    float v[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; i++) {
+      const int e = t + i * kQConsWarps * 32;
+      const int c = e / kQCoef;
+      v[i] = (e < kN && col0 + c < p.nb) ? coef_entry<MODE>(p, col0 + c, e - c * kQCoef) : 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; i++) {
+      const int e = t + i * kQConsWarps * 32;
+      if (e < kN) coef[e] = v[i];
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(kQConsWarps * 32) : "memory");
+  }
 
-  const int sw = (t >> 1) & 3;
-  for (int it = 0; it < my_tiles; it++) {
+  const int cl = (warp & 1) * 4 + (lane >> 3);  // block column inside the tile
+  const int rl = (warp >> 1) * 8 + (lane & 7);  // row inside the tile
+  const int b = col0 + cl;
+  const bool col_ok = b < p.nb;
+  const int bc = col_ok ? b : 0;
+  const uint32_t cf = smem_addr(coef + cl * kQCoef);
+  const uint32_t xoff = uint32_t(cl * kQRows + rl) * 64u;
+  const int sw = (rl >> 1) & 3;
+  const uint32_t sbase = smem_addr(base);
+  const float* Kb = (MODE == MODE_KRON) ? p.mats + int64_t(bc) * kBlock * kBlock : nullptr;
+  // per-tile pointer steps: gridDim.y row tiles of kQRows rows
+  const int64_t row_step = int64_t(gridDim.y) * kQRows;
+  int64_t row = int64_t(blockIdx.y) * kQRows + rl;
+
+  for (int it = 0; it < my_tiles; it++, row += row_step) {
     const int s = it % p.stages;
     if (!mbar_wait_bounded(&full[s], uint32_t(it / p.stages) & 1u, kWaitLimitNs)) break;
-    uint4 xr[4] = {};
-    if (has_tile) {
-      const uint4* blk = reinterpret_cast<const uint4*>(base + s * p.stage_stride + t * 64);
+    uint4 xr[4];
+    const uint32_t blk = sbase + uint32_t(s) * kQStageBytes + xoff;
 #pragma unroll
-      for (int k = 0; k < 4; k++) xr[k] = blk[k ^ sw];
-    }
+    for (int k = 0; k < 4; k++) xr[k] = lds128(blk + uint32_t((k ^ sw) << 4));
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
-    const int64_t row = int64_t(int(blockIdx.y) + it * int(gridDim.y)) * p.R + rr;
+    const bool act = col_ok && row < p.M;
+    const int64_t rowc = act ? row : 0;
+    uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16;
+    uint8_t* sb = p.scales + rowc * int64_t(p.nb) + bc;
+    const uint16_t* xb = p.x + rowc * p.ldx + int64_t(bc) * kBlock;
     // every lane takes part (the exact path is warp-cooperative); only real blocks store
-    quant_block<MODE>(p, c, xr, row, b, active && row < p.M);
+    quant_block<MODE>(cf, xr, act, qb, sb, xb, Kb);
   }
 }
 
