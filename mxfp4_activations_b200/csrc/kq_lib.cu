@@ -44,6 +44,7 @@ struct DeviceInfo {
   std::once_flag once;
   int sms = 0;
   int smem_optin = 0;
+  int smem_per_sm = 0;
   bool ok = false;
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -54,7 +55,8 @@ const DeviceInfo* device_info() {
   DeviceInfo& d = g_dev[dev];
   std::call_once(d.once, [&]() {
     d.ok = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
-           cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess;
+           cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess &&
+           cudaDeviceGetAttribute(&d.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) == cudaSuccess;
   });
   return d.ok ? &d : nullptr;
 }
@@ -156,7 +158,7 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
 }
 
 // Tensor-core variant: 128-row x 4-block tiles, one CTA per 4-block column group
-// and row-tile stride, one CTA per SM (it holds all 512 tensor-memory columns).
+// and row-tile stride, two CTAs per SM (256 tensor-memory columns each).
 kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, const void* mats, bool mats_bf16,
                            uint8_t* q, uint8_t* scales, cudaStream_t stream) {
   const DeviceInfo* dev = device_info();
@@ -196,18 +198,14 @@ kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, con
   p.mats = mats;
   p.q = q;
   p.scales = scales;
-  // one CTA per SM: pick the row-tile stride that minimises the estimated
-  // makespan (waves of CTAs x row tiles per CTA)
+  // Resident CTAs per SM.  The runtime's occupancy query reports one CTA per SM
+  // for any kernel that touches tensor memory (it cannot know how many columns
+  // the kernel allocates), so the count comes from the kernel's own budget:
+  // kMmaCtasPerSm x 128 tensor-memory columns <= 512, registers capped by the
+  // launch bound, and the shared memory checked here.
+  const int per_sm = (smem + 1024) * kq::kMmaCtasPerSm <= dev->smem_per_sm ? kq::kMmaCtasPerSm : 1;
   const int64_t ngroups = (nb + kq::kMmaWb - 1) / kq::kMmaWb;
-  int64_t gy = 1, best = INT64_MAX;
-  for (int64_t g = 1; g <= nrt && g <= 65535; g++) {
-    const int64_t waves = (ngroups * g + dev->sms - 1) / dev->sms;
-    const int64_t cost = waves * ((nrt + g - 1) / g);
-    if (cost < best) {
-      best = cost;
-      gy = g;
-    }
-  }
+  const int64_t gy = row_stride(ngroups, nrt, dev->sms, per_sm);
   kern<<<dim3(unsigned(ngroups), unsigned(gy)), kq::kMmaThreads, smem, stream>>>(tmap, p);
   return launch_status("quant_mma_kernel launch");
 }

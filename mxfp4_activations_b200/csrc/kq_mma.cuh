@@ -11,20 +11,22 @@
 // accumulate in the same tensor-memory columns, so the tensor core sees K32
 // exactly; for bf16 matrices one part.
 //
-// CTA roles (a CTA owns a group of four 32-element block columns and a stride of
-// 128-row tiles; one CTA per SM holds all 512 tensor-memory columns):
-//   warp 0      TMA producer: one 3-D load per tile (box {32, 128, 4}: each row
-//               reads 256 contiguous bytes), no multicast
+// CTA roles (a CTA owns a group of two 32-element block columns and a stride of
+// 128-row tiles; three CTAs share an SM, 128 tensor-memory columns each; ten
+// warps per CTA keep every SM sub-partition's register file within bounds):
+//   warp 0      TMA producer: one 3-D load per tile (box {32, 128, 2}: each row
+//               reads 128 contiguous bytes), no multicast; it starts streaming
+//               while the other warps build the B operands
 //   warp 1      allocates the tensor memory; one lane issues the UMMAs (2 or 6 per
 //               block) and commits each tile to an mbarrier
-//   warps 2-17  epilogue: warp w handles block (w-2)/4 of the tile for tensor-memory
+//   warps 2-9   epilogue: warp w handles block (w-2)/4 of the tile for tensor-memory
 //               lanes 32*(w%4)..+31: tcgen05.ld of 32 fp32 columns per row, the row's
 //               L1 bound and zero test from the staged tile, release of the
 //               accumulator buffer and the tile stage, then the certified MXFP4 step
 //               shared with the butterfly kernel (kq_mx.cuh); its rare exact
 //               recomputation re-reads x and K from global memory.
-// Four tile stages and four accumulator buffers keep load, MMA and epilogue
-// overlapped.  Every wait is bounded; on a timeout the CTA drains what it issued,
+// Three tile stages and two accumulator buffers per CTA keep load, MMA and
+// epilogue overlapped.  Every wait is bounded; on a timeout the CTA drains what it issued,
 // frees its tensor memory and exits with the device error flag set.
 #pragma once
 
@@ -36,15 +38,18 @@
 namespace kq {
 
 constexpr int kMmaRows = 128;                        // UMMA M (rows per tile)
-constexpr int kMmaWb = 4;                            // blocks per tile
-constexpr int kMmaStages = 4;                        // tile stages
-constexpr int kMmaAccBufs = 4;                       // accumulator buffers
+constexpr int kMmaWb = 2;                            // blocks per tile
+constexpr int kMmaStages = 3;                        // tile stages
+constexpr int kMmaAccBufs = 2;                       // accumulator buffers
 constexpr int kMmaAccCols = kMmaWb * 32;             // columns per buffer
-constexpr int kMmaTmemCols = kMmaAccBufs * kMmaAccCols;  // 512: the whole tensor memory
+constexpr int kMmaTmemCols = kMmaAccBufs * kMmaAccCols;  // 128 of the SM's 512
+constexpr int kMmaCtasPerSm = 3;
+static_assert(kMmaTmemCols * kMmaCtasPerSm <= 512, "co-resident CTAs must fit the tensor memory");
+static_assert((kMmaTmemCols & (kMmaTmemCols - 1)) == 0 && kMmaTmemCols >= 32, "tcgen05.alloc takes a power of 2 >= 32");
 constexpr int kMmaEpiWarps = 4 * kMmaWb;             // one warp per (block, lane quarter)
 constexpr int kMmaThreads = (2 + kMmaEpiWarps) * 32; // 576
 constexpr int kMmaATileBytes = kMmaRows * 64;        // 8 KB per block of a tile
-constexpr int kMmaAStageBytes = kMmaWb * kMmaATileBytes;  // 32 KB per tile
+constexpr int kMmaAStageBytes = kMmaWb * kMmaATileBytes;  // 16 KB per tile
 constexpr int kMmaBBytes = 32 * 64;                  // one 32x32 bf16 matrix
 // Error allowance of the tensor-core sum, relative to sum_i |x_i| * max|K|.
 // Model: each kind::f16 UMMA adds its 16 exact bf16 x bf16 products to the fp32
@@ -150,7 +155,7 @@ __device__ __forceinline__ float l1_upper_bf16(const uint4 (&v)[4]) {
 }
 
 template <int KSRC>
-__global__ void __launch_bounds__(kMmaThreads, 1) quant_mma_kernel(const __grid_constant__ CUtensorMap tmap,
+__global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                    const MmaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -182,23 +187,37 @@ __global__ void __launch_bounds__(kMmaThreads, 1) quant_mma_kernel(const __grid_
   if (t < kMmaWb) kmax_bits[t] = 0u;
   __syncthreads();
 
-  // B operands: this group's matrices split into bf16 parts, 64-byte-swizzled
-  // N-major layout; max |K| per block reduced per warp, then one atomic.
-  {
-    uint32_t kloc[kMmaWb] = {};
-    for (int e = t; e < kMmaWb * 1024; e += kMmaThreads) {
-      const int bw = e >> 10, i = (e >> 5) & 31, j = e & 31;
-      const int b = group * kMmaWb + bw;
-      float kf = 0.0f;
-      if (b < p.nb) {
+  if (warp >= 1) {
+    // B operands, built by the MMA and epilogue warps while the producer streams
+    // A: this group's matrices split into bf16 parts in the 64-byte-swizzled
+    // N-major layout; every load is issued before the first store.  max |K| per
+    // block is reduced per warp, then one shared atomic.
+    constexpr int kSetupThreads = kMmaThreads - 32;
+    constexpr int kPer = (kMmaWb * 1024 + kSetupThreads - 1) / kSetupThreads;
+    const int tt = t - 32;
+    float kv[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; i++) {
+      const int e = tt + i * kSetupThreads;
+      const int b = group * kMmaWb + (e >> 10);
+      kv[i] = 0.0f;
+      if (e < kMmaWb * 1024 && b < p.nb) {
         const int64_t idx = int64_t(b) * 1024 + (e & 1023);
-        kf = (KSRC == KSRC_BF16) ? bf16_to_f32(static_cast<const uint16_t*>(p.mats)[idx])
-                                 : static_cast<const float*>(p.mats)[idx];
+        kv[i] = (KSRC == KSRC_BF16) ? bf16_to_f32(__ldg(static_cast<const unsigned short*>(p.mats) + idx))
+                                    : __ldg(static_cast<const float*>(p.mats) + idx);
       }
+    }
+    uint32_t kloc[kMmaWb] = {};
+#pragma unroll
+    for (int i = 0; i < kPer; i++) {
+      const int e = tt + i * kSetupThreads;
+      if (e >= kMmaWb * 1024) continue;
+      const int bw = e >> 10, r = (e >> 5) & 31, c = e & 31;
+      const float kf = kv[i];
 #pragma unroll
       for (int k = 0; k < kMmaWb; k++)
-        if (k == bw) kloc[k] = max(kloc[k], __float_as_uint(fabsf(kf)) & 0x7FFFFFFFu);
-      const uint32_t off = sw64_offset(i, j);
+        if (k == bw) kloc[k] = max(kloc[k], __float_as_uint(kf) & 0x7FFFFFFFu);
+      const uint32_t off = sw64_offset(r, c);
       uint8_t* mb = b_smem + bw * p.nsplit * kMmaBBytes;
       if (p.nsplit == 1) {
         *reinterpret_cast<__nv_bfloat16*>(mb + off) = __float2bfloat16_rn(kf);
@@ -217,18 +236,18 @@ __global__ void __launch_bounds__(kMmaThreads, 1) quant_mma_kernel(const __grid_
       const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, kloc[k]);
       if (lane == 0 && m != 0u) atomicMax(&kmax_bits[k], m);
     }
+    if (warp == 1) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                   "r"(uint32_t(kMmaTmemCols))
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // B writes -> tensor core
+    tc_fence_before();
+    asm volatile("bar.sync 1, %0;" ::"r"(kSetupThreads) : "memory");
+    tc_fence_after();
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
-                 "r"(uint32_t(kMmaTmemCols))
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // B writes -> tensor core
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = warp >= 1 ? *tmem_slot : 0u;
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
@@ -298,13 +317,23 @@ __global__ void __launch_bounds__(kMmaThreads, 1) quant_mma_kernel(const __grid_
       const int s = it % kMmaStages, buf = it % kMmaAccBufs;
       if (!mbar_wait_bounded(&mma_full[buf], uint32_t(it / kMmaAccBufs) & 1u, kWaitLimitNs)) break;
       tc_fence_after();
+      // this row's inputs from the staged tile first (their registers die before
+      // the accumulators arrive): L1 upper bound and exact zero test
+      const uint4* xs = reinterpret_cast<const uint4*>(a_smem + s * kMmaAStageBytes + bw * kMmaATileBytes + rr * 64);
+      float l1;
+      bool zero_block;
+      {
+        uint4 xv[4];
+#pragma unroll
+        for (int k = 0; k < 4; k++) xv[k] = xs[k ^ sw];
+        l1 = l1_upper_bf16(xv);
+        uint32_t nz = 0u;
+#pragma unroll
+        for (int k = 0; k < 4; k++) nz |= xv[k].x | xv[k].y | xv[k].z | xv[k].w;
+        zero_block = (nz & 0x7FFF7FFFu) == 0u;
+      }
       float y[32];
       tmem_ld32(tmem + (uint32_t(q * 32) << 16) + uint32_t(buf * kMmaAccCols + bw * 32), y);
-      // this row's inputs from the staged tile: L1 upper bound and exact zero test
-      const uint4* xs = reinterpret_cast<const uint4*>(a_smem + s * kMmaAStageBytes + bw * kMmaATileBytes + rr * 64);
-      uint4 xv[4];
-#pragma unroll
-      for (int k = 0; k < 4; k++) xv[k] = xs[k ^ sw];
       // accumulators and tile are no longer needed: release them before the math
       tc_fence_before();
       __syncwarp();
@@ -312,11 +341,6 @@ __global__ void __launch_bounds__(kMmaThreads, 1) quant_mma_kernel(const __grid_
         mbar_arrive(&tmem_empty[buf]);
         mbar_arrive(&empty_a[s]);
       }
-      const float l1 = l1_upper_bf16(xv);
-      uint32_t nz = 0u;
-#pragma unroll
-      for (int k = 0; k < 4; k++) nz |= xv[k].x | xv[k].y | xv[k].z | xv[k].w;
-      const bool zero_block = (nz & 0x7FFF7FFFu) == 0u;
       const int64_t row = int64_t(int(blockIdx.y) + it * int(gridDim.y)) * kMmaRows + rr;
       const bool act = col_ok && row < p.M;
       const int64_t rowc = act ? row : 0;
