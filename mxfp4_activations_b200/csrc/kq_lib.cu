@@ -102,9 +102,8 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   EncodeTiledFn enc = encode_tiled();
   if (enc == nullptr) return cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
   const int nb = int(d / 32);
-  const int stages = kq::kQMaxStages;
-  const int smem = 1024 /*alignment slack*/ + stages * kq::kQStageBytes + kq::kQCols * kq::kQCoef * 4 +
-                   2 * kq::kQMaxStages * 8;
+  const int smem = 1024 /*alignment slack*/ + kq::kQStages * kq::kQStageBytes + kq::kQCols * kq::kQCoef * 4 +
+                   2 * kq::kQStages * 8;
   if (smem > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
 
   CUtensorMap tmap;
@@ -143,7 +142,7 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   const int64_t nrt = (M + kq::kQRows - 1) / kq::kQRows;
   if (nrt > int64_t(INT32_MAX) / kq::kQRows) return KQ_ERR_SHAPE;  // TMA row coordinates are int32
   p.n_row_tiles = int(nrt);
-  p.stages = stages;
+  p.coef_offset = kq::kQStages * kq::kQStageBytes;
   p.mats = mats;
   p.factored = factored;
   p.inv_s = inv_s;

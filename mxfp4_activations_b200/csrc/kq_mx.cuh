@@ -154,16 +154,19 @@ __device__ __forceinline__ void certify_store(const uint64_t (&Y)[16], float ama
   const float s = inv_scale_of_byte(exact ? 0 : byte);
   const float eb = __fmul_ru(E, s);
   const uint64_t S2 = pk2(s, s), NE2 = pk2(-eb, -eb), PE2 = pk2(eb, eb);
-  uint64_t V[16];
+  // eight elements at a time: the lower and upper bounds of each group are
+  // converted while the other groups' pairs stay in registers
   uint32_t cm[4], cp[4];
 #pragma unroll
-  for (int m = 0; m < 16; m++) V[m] = fma2_rd(Y[m], S2, NE2);
+  for (int k = 0; k < 4; k++) {
+    uint64_t V[4];
 #pragma unroll
-  for (int k = 0; k < 4; k++) cm[k] = codes8(V + 4 * k);
+    for (int m = 0; m < 4; m++) V[m] = fma2_rd(Y[4 * k + m], S2, NE2);
+    cm[k] = codes8(V);
 #pragma unroll
-  for (int m = 0; m < 16; m++) V[m] = fma2_ru(Y[m], S2, PE2);
-#pragma unroll
-  for (int k = 0; k < 4; k++) cp[k] = codes8(V + 4 * k);
+    for (int m = 0; m < 4; m++) V[m] = fma2_ru(Y[4 * k + m], S2, PE2);
+    cp[k] = codes8(V);
+  }
   const uint32_t diff = (cm[0] ^ cp[0]) | (cm[1] ^ cp[1]) | (cm[2] ^ cp[2]) | (cm[3] ^ cp[3]);
   // a block with an uncertain scale or an uncertain code is recomputed exactly;
   // with exact_only (matrix entries possibly non-finite) so is an all-zero block

@@ -60,7 +60,7 @@ constexpr int kQRows = 32;                       // rows per tile
 constexpr int kQConsWarps = 8;                   // consumer warps (4 columns x 8 rows each)
 constexpr int kQThreads = (kQConsWarps + 1) * 32;  // + the TMA producer warp
 constexpr int kQStageBytes = kQCols * kQRows * 64;  // 16 KB
-constexpr int kQMaxStages = 4;
+constexpr int kQStages = 4;
 // Shared coefficient table, one record of kQCoef floats per block column:
 //   [4s .. 4s+3]  (lam, lam, bet, bet) of the stage on index bit s+1 (factor 3-s), s = 0..3
 //   [16 .. 47]    D_0 .. D_31 (SMOOTH: the 32 per-channel factors)
@@ -74,7 +74,7 @@ struct QuantParams {
   int64_t M;
   int nb;                 // blocks per row (d / 32)
   int n_row_tiles;        // ceil(M / 32)
-  int stages;             // shared-memory stages (<= kQMaxStages)
+  int coef_offset;        // bytes from the stage ring to the coefficient table (kQStages * kQStageBytes)
   const float* mats;      // KRON: fp32 [nb][32][32] (exact path)
   const float* factored;  // KRON: [nb][48]
   const float* inv_s;     // SMOOTH: [nb*32]
@@ -236,16 +236,18 @@ template <int MODE>
 __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* coef = reinterpret_cast<float*>(base + p.stages * kQStageBytes);  // [kQCols][kQCoef]
+  // [kQCols][kQCoef] after the stages; the offset comes from the host (kept out of
+  // the compile-time address arithmetic, which otherwise costs the loop a register)
+  float* coef = reinterpret_cast<float*>(base + p.coef_offset);
   uint64_t* full = reinterpret_cast<uint64_t*>(coef + kQCols * kQCoef);
-  uint64_t* empty = full + kQMaxStages;
+  uint64_t* empty = full + kQStages;
 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int col0 = int(blockIdx.x) * kQCols;
   const int my_tiles = (p.n_row_tiles - int(blockIdx.y) + int(gridDim.y) - 1) / int(gridDim.y);
 
   if (t == 0) {
-    for (int s = 0; s < p.stages; s++) {
+    for (int s = 0; s < kQStages; s++) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], uint32_t(kQConsWarps));
     }
@@ -258,15 +260,16 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_consta
       prefetch_tensormap(&tmap);
       int it = 0;
       for (; it < my_tiles; it++) {
-        const int s = it % p.stages;
-        if (it >= p.stages && !mbar_wait_bounded(&empty[s], uint32_t(it / p.stages - 1) & 1u, kWaitLimitNs)) break;
+        const int s = it % kQStages;
+        if (it >= kQStages && !mbar_wait_bounded(&empty[s], uint32_t(it / kQStages - 1) & 1u, kWaitLimitNs))
+          break;
         const int tile = int(blockIdx.y) + it * int(gridDim.y);
         mbar_arrive_expect_tx(&full[s], uint32_t(kQStageBytes));
         tma_load_3d(base + s * kQStageBytes, &tmap, &full[s], 0, tile * kQRows, col0);
       }
       if (it < my_tiles) {  // consumers stopped: let the loads still in flight land before exiting
-        for (int k = (it > p.stages ? it - p.stages : 0); k < it; k++)
-          mbar_wait_bounded(&full[k % p.stages], uint32_t(k / p.stages) & 1u, kWaitLimitNs / 4);
+        for (int k = (it > kQStages ? it - kQStages : 0); k < it; k++)
+          mbar_wait_bounded(&full[k % kQStages], uint32_t(k / kQStages) & 1u, kWaitLimitNs / 4);
       }
     }
     return;
@@ -307,8 +310,8 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_consta
   int64_t row = int64_t(blockIdx.y) * kQRows + rl;
 
   for (int it = 0; it < my_tiles; it++, row += row_step) {
-    const int s = it % p.stages;
-    if (!mbar_wait_bounded(&full[s], uint32_t(it / p.stages) & 1u, kWaitLimitNs)) break;
+    const int s = it % kQStages;  // compile-time ring size: no integer division per block
+    if (!mbar_wait_bounded(&full[s], uint32_t(it / kQStages) & 1u, kWaitLimitNs)) break;
     uint4 xr[4];
     const uint32_t blk = sbase + uint32_t(s) * kQStageBytes + xoff;
 #pragma unroll
