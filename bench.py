@@ -40,6 +40,7 @@ FLUX_DS = (3072, 12288)
 BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 32.0
 PROFILE_JSON = os.path.join(ROOT, "profiles", "kq_quant_flux_traffic.json")
 KERNEL_SOURCES = ["mxfp4_activations_b200/csrc/kq_quant.cuh", "mxfp4_activations_b200/csrc/kq_common.cuh",
+                  "mxfp4_activations_b200/csrc/kq_mx.cuh",
                   "mxfp4_activations_b200/csrc/kq_lib.cu"]
 
 
