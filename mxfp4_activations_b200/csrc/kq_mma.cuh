@@ -20,11 +20,13 @@
 //   warp 1      allocates the tensor memory; one lane issues the UMMAs (2 or 6 per
 //               block) and commits each tile to an mbarrier
 //   warps 2-9   epilogue: warp w handles block (w-2)/4 of the tile for tensor-memory
-//               lanes 32*(w%4)..+31: tcgen05.ld of 32 fp32 columns per row, the row's
-//               L1 bound and zero test from the staged tile, release of the
-//               accumulator buffer and the tile stage, then the certified MXFP4 step
-//               shared with the butterfly kernel (kq_mx.cuh); its rare exact
-//               recomputation re-reads x and K from global memory.
+//               lanes 32*(w%4)..+31.  As soon as the tile has landed it reads its
+//               row's inputs from the staged tile (L1 bound and zero test) while the
+//               UMMAs run; the stage is released by every epilogue warp plus a
+//               commit of the UMMAs that read it.  Then tcgen05.ld of 32 fp32
+//               columns per row, release of the accumulator buffer, and the
+//               certified MXFP4 step shared with the butterfly kernel (kq_mx.cuh);
+//               its rare exact recomputation re-reads x and K from global memory.
 // Three tile stages and two accumulator buffers per CTA keep load, MMA and
 // epilogue overlapped.  Every wait is bounded; on a timeout the CTA drains what it issued,
 // frees its tensor memory and exits with the device error flag set.
@@ -163,7 +165,7 @@ __global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(c
   uint8_t* b_smem = base + kMmaStages * kMmaAStageBytes;    // [Wb][nsplit][32][64 B]
   uint64_t* bars = reinterpret_cast<uint64_t*>(b_smem + kMmaWb * 3 * kMmaBBytes);
   uint64_t* full_a = bars;                                  // [stages]  TMA landed
-  uint64_t* empty_a = bars + kMmaStages;                    // [stages]  epilogue read the tile
+  uint64_t* empty_a = bars + kMmaStages;                    // [stages]  epilogue read x, UMMAs done
   uint64_t* mma_full = bars + 2 * kMmaStages;               // [bufs]    accumulators ready
   uint64_t* tmem_empty = bars + 2 * kMmaStages + kMmaAccBufs;  // [bufs] accumulators read
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kMmaStages + 2 * kMmaAccBufs);
@@ -176,7 +178,7 @@ __global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(c
   if (t == 0) {
     for (int s = 0; s < kMmaStages; s++) {
       mbar_init(&full_a[s], 1);
-      mbar_init(&empty_a[s], kMmaEpiWarps);
+      mbar_init(&empty_a[s], kMmaEpiWarps + 1);  // every epilogue warp + the MMA commit
     }
     for (int i = 0; i < kMmaAccBufs; i++) {
       mbar_init(&mma_full[i], 1);
@@ -294,11 +296,16 @@ __global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(c
           }
         }
         umma_commit(&mma_full[buf]);
+        umma_commit(&empty_a[s]);  // the stage is free for the producer once these UMMAs have read it
       }
       if (it > 0) {  // the last commit must have landed before tensor memory is freed
         const int k = it - 1;
         mbar_wait_bounded(&mma_full[k % kMmaAccBufs], uint32_t(k / kMmaAccBufs) & 1u, kWaitLimitNs / 4);
       }
+      // the stage-release commits of the last tiles arrive asynchronously too: let
+      // them land before the CTA's shared memory can be reused
+      for (int k = (it > kMmaStages ? it - kMmaStages : 0); k < it; k++)
+        mbar_wait_bounded(&empty_a[k % kMmaStages], uint32_t(k / kMmaStages) & 1u, kWaitLimitNs / 4);
     }
   } else {
     // ------------------------------------------------ epilogue
@@ -315,10 +322,9 @@ __global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(c
                          : static_cast<const void*>(static_cast<const float*>(p.mats) + int64_t(bc) * 1024);
     for (int it = 0; it < my_tiles; it++) {
       const int s = it % kMmaStages, buf = it % kMmaAccBufs;
-      if (!mbar_wait_bounded(&mma_full[buf], uint32_t(it / kMmaAccBufs) & 1u, kWaitLimitNs)) break;
-      tc_fence_after();
-      // this row's inputs from the staged tile first (their registers die before
-      // the accumulators arrive): L1 upper bound and exact zero test
+      // this row's inputs as soon as the tile has landed, overlapping the UMMAs:
+      // L1 upper bound and exact zero test
+      if (!mbar_wait_bounded(&full_a[s], uint32_t(it / kMmaStages) & 1u, kWaitLimitNs)) break;
       const uint4* xs = reinterpret_cast<const uint4*>(a_smem + s * kMmaAStageBytes + bw * kMmaATileBytes + rr * 64);
       float l1;
       bool zero_block;
@@ -332,15 +338,16 @@ __global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(c
         for (int k = 0; k < 4; k++) nz |= xv[k].x | xv[k].y | xv[k].z | xv[k].w;
         zero_block = (nz & 0x7FFF7FFFu) == 0u;
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_a[s]);
+      if (!mbar_wait_bounded(&mma_full[buf], uint32_t(it / kMmaAccBufs) & 1u, kWaitLimitNs)) break;
+      tc_fence_after();
       float y[32];
       tmem_ld32(tmem + (uint32_t(q * 32) << 16) + uint32_t(buf * kMmaAccCols + bw * 32), y);
-      // accumulators and tile are no longer needed: release them before the math
+      // the accumulators are no longer needed: release them before the math
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&tmem_empty[buf]);
-        mbar_arrive(&empty_a[s]);
-      }
+      if (lane == 0) mbar_arrive(&tmem_empty[buf]);
       const int64_t row = int64_t(int(blockIdx.y) + it * int(gridDim.y)) * kMmaRows + rr;
       const bool act = col_ok && row < p.M;
       const int64_t rowc = act ? row : 0;
