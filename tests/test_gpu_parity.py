@@ -213,6 +213,30 @@ def test_quantize_degenerate_blocks(kq, orc, variant, mdt):
 
 
 @pytest.mark.parametrize("variant,mdt", VARIANTS)
+def test_quantize_singular_and_exact_only_columns(kq, orc, variant, mdt):
+    """A factor with u = 0 puts inf and NaN into K, so even an all-zero block has
+    y = 0 * inf = NaN by definition (scale byte 0xFF); a factor with d = 0 keeps K
+    finite but has no butterfly form.  Both columns go through the exact path."""
+    rng = np.random.default_rng(31)
+    M, d = 40, 192
+    a = rng.standard_normal((M, d)).astype(np.float32)
+    a[0] = 0.0                    # an all-zero row crosses every column
+    a[1, 32:64] = 0.0             # zero block in the singular column
+    a[2, 64:96] = -0.0            # negative zeros in the d = 0 column
+    a[3, 0:32] = 0.0              # zero block in an ordinary column
+    x = inputs.f32_to_bf16_bits(a)
+    params = inputs.lu_params(d // 32, seed=32)
+    params[1, 2, 1] = 0.0         # u = 0: singular factor in block column 1
+    params[2, 1] = (-1.0, 1.0, 1.0)  # d = l v + 1/u = 0 in block column 2
+    q, s = gpu_quantize(kq, x, params, variant=variant, mdt=mdt)
+    assert kq.kq_get_device_error(clear=True) == 4  # the set-up kernels flag the singular factor
+    K = oracle_mats(orc, params, mdt)
+    qr, sr = orc.quantize(x, K)
+    check(q, s, qr, sr)
+    assert np.all(s[:, 1] == 0xFF) and np.all(qr[:, 16:32] == 0)  # every block of the singular column is NaN
+
+
+@pytest.mark.parametrize("variant,mdt", VARIANTS)
 def test_quantize_identity_all_bf16_patterns(kq, orc, variant, mdt):
     """K = I: every bf16 bit pattern (NaN/Inf included) goes through the scale and
     element steps as its own value; 2048 blocks of 32 consecutive patterns, plus a
