@@ -81,8 +81,13 @@ typedef enum { KQ_VAR_AUTO = 0, KQ_VAR_MMA = 1, KQ_VAR_BUTTERFLY = 2 } kq_varian
 /* ---------------------------------------------------------------- set-up (once per layer)
  *
  * kq_expand_blocks -- [KQ-sum, Approach]: K_b = F0 (x) F1 (x) F2 (x) F3 (x) F4
- * from the 15 LU parameters of each block; with inverse != 0,
- * K_b^-1 = F0^-1 (x) ... (x) F4^-1 (det F_k = 1, so F^-1 = [[d,-b],[-c,a]]).
+ * from the 15 LU parameters of each block.
+ *   inverse 0: K_b.
+ *           1: K_b^-1 = F0^-1 (x) ... (x) F4^-1 (det F_k = 1, so F^-1 = [[d,-b],[-c,a]]).
+ *           2: (K_b^-1)^T, the weight-side transform: quantizing each weight row w
+ *              with it ([KQ-abs] "its inverse to the weights") keeps products
+ *              invariant, (x K_b) . (w K_b^-T) = x . w ([LRQ] eq. 2).
+ *           any other value: KQ_ERR_INVALID_ARG.
  *   params  device fp32 [nb][5][3], 4-byte aligned.
  *   nb      number of blocks (>= 0; 0 is a no-op).
  *   mats    device [nb][32][32] row-major (row = input index i, column = output

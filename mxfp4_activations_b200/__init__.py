@@ -45,6 +45,17 @@ class BlockTransform:
     def quantize(self, x, variant: str = "auto", q=None, scales=None):
         return kq_quantize(x, self.mats, self.factored, variant=variant, q=q, scales=scales)
 
+    def quantize_weights(self, w, mat_dtype=None, q=None, scales=None):
+        """MXFP4 of the weight rows w [n_out, d] (bf16) times K_b^-T per block, the
+        weight side of the transform: dot products with quantize(x) rows then
+        approximate x . w.  Runs the tensor-core variant with the dense K^-T."""
+        import torch
+
+        key = mat_dtype or torch.float32
+        if getattr(self, "_inv_t", None) is None or self._inv_t.dtype != key:
+            self._inv_t = kq_expand_blocks(self.params, inverse=True, transpose=True, dtype=key)
+        return kq_quantize(w, self._inv_t, None, variant="mma", q=q, scales=scales)
+
     def dequantize(self, q, scales, undo_transform: bool = True, out_dtype=None):
         import torch
 

@@ -114,7 +114,8 @@ def _rows(x: torch.Tensor, name: str = "x"):
 # ---------------------------------------------------------------- set-up
 
 def kq_expand_blocks(params: torch.Tensor, inverse: bool = False, dtype: torch.dtype = torch.float32,
-                     out: torch.Tensor | None = None) -> torch.Tensor:
+                     out: torch.Tensor | None = None, transpose: bool = False) -> torch.Tensor:
+    """K_b, K_b^-1 (inverse=True) or the weight-side K_b^-T (inverse=True, transpose=True)."""
     _cuda(params, "params")
     params = params.contiguous()
     if params.dtype != torch.float32 or params.numel() % 15 != 0:
@@ -122,7 +123,10 @@ def kq_expand_blocks(params: torch.Tensor, inverse: bool = False, dtype: torch.d
     nb = params.numel() // 15
     if out is None:
         out = torch.empty((nb, 32, 32), dtype=dtype, device=params.device)
-    _check("kq_expand_blocks", load().kq_expand_blocks(_ptr(params), nb, int(bool(inverse)), _mat_dtype(out),
+    if transpose and not inverse:
+        raise ValueError("transpose is provided for the inverse (the weight-side transform) only")
+    mode = 2 if transpose else int(bool(inverse))
+    _check("kq_expand_blocks", load().kq_expand_blocks(_ptr(params), nb, mode, _mat_dtype(out),
                                                          _ptr(out), _stream(params.device)))
     return out
 

@@ -58,13 +58,18 @@ __device__ __forceinline__ uint16_t bf16_rne_from_f64(double a) {
 }
 
 // One thread per matrix entry: K[i][j] = F0[i4][j4] (F1[i3][j3] (F2 (F3 F4))),
-// the Kronecker product assembled from the innermost factor outward.
-__global__ void expand_kernel(const float* __restrict__ params, int64_t nb, int inverse, int out_bf16,
+// the Kronecker product assembled from the innermost factor outward.  mode 0:
+// K, 1: K^-1 (inverse factors), 2: (K^-1)^T (inverse factors, entry (i, j)
+// taken from (j, i): the transpose of a Kronecker product is the product of the
+// transposes).
+__global__ void expand_kernel(const float* __restrict__ params, int64_t nb, int mode, int out_bf16,
                               void* __restrict__ mats) {
   const int64_t gid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (gid >= nb * 1024) return;
   const int64_t b = gid >> 10;
-  const int i = int(gid >> 5) & 31, j = int(gid) & 31;
+  const int r = int(gid >> 5) & 31, c = int(gid) & 31;
+  const int i = mode == 2 ? c : r, j = mode == 2 ? r : c;
+  const bool inverse = mode != 0;
   double F[5][4];
   bool singular = false;
 #pragma unroll

@@ -255,12 +255,13 @@ const char* kq_status_string(kq_status s) {
 kq_status kq_expand_blocks(const float* params, int64_t nb, int inverse, kq_dtype out_dtype, void* mats,
                            kq_stream_t stream) {
   if (nb < 0 || (out_dtype != KQ_F32 && out_dtype != KQ_BF16)) return KQ_ERR_INVALID_ARG;
+  if (inverse < 0 || inverse > 2) return KQ_ERR_INVALID_ARG;
   if (nb == 0) return KQ_OK;
   if (params == nullptr || mats == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(params, 4) || !aligned(mats, 4)) return KQ_ERR_ALIGN;
   if (nb > (int64_t(1) << 30)) return KQ_ERR_SHAPE;
   const int64_t n = nb * 1024;
-  kq::expand_kernel<<<unsigned((n + 255) / 256), 256, 0, as_cuda(stream)>>>(params, nb, inverse ? 1 : 0,
+  kq::expand_kernel<<<unsigned((n + 255) / 256), 256, 0, as_cuda(stream)>>>(params, nb, inverse,
                                                                            out_dtype == KQ_BF16 ? 1 : 0, mats);
   return launch_status("expand_kernel launch");
 }

@@ -79,6 +79,8 @@ def test_other_entry_points_argument_errors(lib):
     assert lib.kq_expand_blocks(None, 4, 0, 0, P(64), None) == 1
     assert lib.kq_expand_blocks(P(64), -1, 0, 0, P(64), None) == 1
     assert lib.kq_expand_blocks(P(64), 4, 0, 5, P(64), None) == 1
+    assert lib.kq_expand_blocks(P(64), 4, 3, 0, P(64), None) == 1     # mode: 0 K, 1 K^-1, 2 K^-T
+    assert lib.kq_expand_blocks(P(64), 4, -1, 0, P(64), None) == 1
     assert lib.kq_expand_blocks(P(64), 0, 0, 0, P(64), None) == 0
     assert lib.kq_expand_factored(P(64), 4, P(68), None) == 3
     assert lib.kq_dequantize(P(16), P(16), 4, 48, None, 0, P(16), 0, None) == 2

@@ -89,13 +89,16 @@ def special_params():
     return p
 
 
-@pytest.mark.parametrize("inverse", [False, True])
+@pytest.mark.parametrize("mode", ["K", "K^-1", "K^-T"])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_expand_bit_exact(kq, orc, inverse, dtype):
+def test_expand_bit_exact(kq, orc, mode, dtype):
     params = special_params()
     tdt = torch.float32 if dtype == "f32" else torch.bfloat16
-    got = host(kq.kq_expand_blocks(dev_f32(params), inverse=inverse, dtype=tdt))
+    inverse, transpose = mode != "K", mode == "K^-T"
+    got = host(kq.kq_expand_blocks(dev_f32(params), inverse=inverse, dtype=tdt, transpose=transpose))
     want = orc.expand(params, dtype=orc.F32 if dtype == "f32" else orc.BF16, inverse=inverse)
+    if transpose:
+        want = np.ascontiguousarray(np.swapaxes(want, 1, 2))
     if dtype == "f32":
         assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
     else:
@@ -210,6 +213,22 @@ def test_quantize_degenerate_blocks(kq, orc, variant, mdt):
     K = oracle_mats(orc, params, mdt)
     qr, sr = orc.quantize(x, K)
     check(q, s, qr, sr)
+
+
+@pytest.mark.parametrize("mdt", ["f32", "bf16"])
+def test_weight_side_quantize(kq, orc, mdt):
+    """Weight rows quantized with the weight-side transform K_b^-T through the
+    public BlockTransform API, against the oracle on the same matrices."""
+    rng = np.random.default_rng(41)
+    n_out, d = 96, 320
+    w = inputs.f32_to_bf16_bits((rng.standard_normal((n_out, d)) * 0.02).astype(np.float32))
+    params = inputs.lu_params(d // 32, seed=42)
+    bt = kq.BlockTransform(dev_f32(params))
+    qd, sd = bt.quantize_weights(dev_bf16(w), mat_dtype=torch.float32 if mdt == "f32" else torch.bfloat16)
+    kit = np.ascontiguousarray(np.swapaxes(orc.expand(params, dtype=orc.F32 if mdt == "f32" else orc.BF16,
+                                                      inverse=True), 1, 2))
+    qr, sr = orc.quantize(w, kit)
+    check(host(qd), host(sd), qr, sr)
 
 
 @pytest.mark.parametrize("variant,mdt", VARIANTS)

@@ -262,6 +262,21 @@ def test_inverse_is_kron_of_factor_inverses(orc):
     assert np.abs(K @ Ki - eye).max() < 1e-12
 
 
+def test_weight_side_transform_keeps_products(orc):
+    """[LRQ] eq. 2: Y = X W^T = (X H)(W H)^T for orthogonal H; with an invertible
+    block transform the weight side takes K^-T instead: (x K)(w K^-T)^T = x w^T,
+    block by block, in exact arithmetic (checked in fp64 against numpy)."""
+    params = inputs.lu_params(8, seed=25)
+    K = orc.expand_f64(params)
+    KiT = np.swapaxes(orc.expand_f64(params, inverse=True), 1, 2)
+    rng = np.random.default_rng(26)
+    x = rng.standard_normal((16, 8, 32))
+    w = rng.standard_normal((12, 8, 32))
+    lhs = np.einsum("rbj,nbj->rn", np.einsum("rbi,bij->rbj", x, K), np.einsum("nbi,bij->nbj", w, KiT))
+    rhs = np.einsum("rbi,nbi->rn", x, w)
+    assert np.abs(lhs - rhs).max() < 1e-9 * np.abs(x).sum(axis=(1, 2)).max() * np.abs(w).max()
+
+
 def test_round_trip_fp32_below_1e_5(orc):
     params = inputs.lu_params(36, seed=23)
     K32 = orc.expand(params).astype(np.float32)
