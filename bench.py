@@ -193,13 +193,13 @@ class QuantStep:
         M, d = item["M"], item["d"]
         if kind == "kroquant":
             st = self.lib.kq_quantize(x.data_ptr(), M, d, d, item["mats"].data_ptr(), 0, item["fac"].data_ptr(),
-                                      q.data_ptr(), s.data_ptr(), 2, self.stream)
+                                      q.data_ptr(), s.data_ptr(), 2, 0, self.stream)
         elif kind == "kroquant_mma":
             st = self.lib.kq_quantize(x.data_ptr(), M, d, d, item["mats"].data_ptr(), 0, None,
-                                      q.data_ptr(), s.data_ptr(), 1, self.stream)
+                                      q.data_ptr(), s.data_ptr(), 1, 0, self.stream)
         elif kind == "kroquant_mma_bf16":
             st = self.lib.kq_quantize(x.data_ptr(), M, d, d, item["mats16"].data_ptr(), 1, None,
-                                      q.data_ptr(), s.data_ptr(), 1, self.stream)
+                                      q.data_ptr(), s.data_ptr(), 1, 0, self.stream)
         elif kind == "smooth":
             st = self.lib.kq_ref_smooth_quantize(x.data_ptr(), M, d, d, item["inv_s"].data_ptr(), q.data_ptr(),
                                                  s.data_ptr(), self.stream)
@@ -586,11 +586,11 @@ def run_sweep(args) -> None:
         mats16 = kq.kq_expand_blocks(pd, dtype=torch.bfloat16)
         calls = {
             "kroquant": lambda st: lib.kq_quantize(xd.data_ptr(), M, d, d, mats.data_ptr(), 0, fac.data_ptr(),
-                                                   q.data_ptr(), s.data_ptr(), 2, st),
+                                                   q.data_ptr(), s.data_ptr(), 2, 0, st),
             "kroquant_mma": lambda st: lib.kq_quantize(xd.data_ptr(), M, d, d, mats.data_ptr(), 0, None,
-                                                       q.data_ptr(), s.data_ptr(), 1, st),
+                                                       q.data_ptr(), s.data_ptr(), 1, 0, st),
             "kroquant_mma_bf16": lambda st: lib.kq_quantize(xd.data_ptr(), M, d, d, mats16.data_ptr(), 1, None,
-                                                            q.data_ptr(), s.data_ptr(), 1, st),
+                                                            q.data_ptr(), s.data_ptr(), 1, 0, st),
             "smooth": lambda st: lib.kq_ref_smooth_quantize(xd.data_ptr(), M, d, d, inv_s.data_ptr(), q.data_ptr(),
                                                             s.data_ptr(), st),
             "fwht": lambda st: lib.kq_ref_fwht_quantize(xd.data_ptr(), M, d, d, q.data_ptr(), s.data_ptr(), st),

@@ -73,6 +73,18 @@ typedef enum { KQ_F32 = 0, KQ_BF16 = 1 } kq_dtype;
  *   KQ_VAR_AUTO:      the faster provided variant for the shape and dtype. */
 typedef enum { KQ_VAR_AUTO = 0, KQ_VAR_MMA = 1, KQ_VAR_BUTTERFLY = 2 } kq_variant;
 
+/* Where kq_quantize writes the E8M0 scales.
+ *   KQ_SCALES_ROW_MAJOR: [M][d/32], scale of block b of row r at byte r*(d/32) + b.
+ *   KQ_SCALES_MMA_TILED: the layout that block-scaled tensor-core GEMMs read their
+ *     per-32-element scale factors in (tcgen05.mma kind::mxf4, cuBLASLt VEC32_UE8M0
+ *     scales).  The [M][d/32] scale matrix is padded to multiples of 128 rows and
+ *     4 columns and cut into 128x4 tiles of 512 bytes, stored tile row by tile row:
+ *     tile (R, C) starts at byte (R * ceil(d/128) + C) * 512, and inside it the scale
+ *     of row r and column c (r < 128, c < 4) sits at byte 16*(r % 32) + 4*(r / 32) + c.
+ *     The buffer holds ceil(M/128)*128 * ceil(d/128)*4 bytes; padding bytes are not
+ *     written. */
+typedef enum { KQ_SCALES_ROW_MAJOR = 0, KQ_SCALES_MMA_TILED = 1 } kq_scale_layout;
+
 #define KQ_BLOCK 32          /* elements per block / per E8M0 scale                */
 #define KQ_NFACTORS 5        /* 2x2 factors per block                              */
 #define KQ_PARAMS_PER_BLOCK 15
@@ -124,15 +136,19 @@ KQ_API kq_status kq_expand_factored(const float* params, int64_t nb, float* fact
  *   factored device [d/32][48] from kq_expand_factored for the same params, or
  *            NULL; required by KQ_VAR_BUTTERFLY.
  *   q        device [M][d/2] packed E2M1 codes, 16-byte aligned.
- *   scales   device [M][d/32] E8M0 bytes.
- * The butterfly variant computes y in fp32, bounds its rounding error from the
- * block's L1 norm and max|K_b|, and recomputes in fp64 (summing in increasing i)
- * exactly those scales and codes that the bound cannot certify, so its output
- * equals the fp64 definition.
+ *   scales   device E8M0 bytes in scale_layout (see kq_scale_layout for sizes).
+ *   variant  which kernel computes the transform (kq_variant).
+ *   scale_layout  KQ_SCALES_ROW_MAJOR or KQ_SCALES_MMA_TILED; anything else is
+ *            KQ_ERR_INVALID_ARG.
+ * Both variants compute y in fp32, bound its rounding error from the block's L1
+ * norm and max|K_b| (the butterfly by a proof, the tensor core by a calibrated
+ * allowance), and recompute in fp64 (summing in increasing i) exactly those
+ * scales and codes that the bound cannot certify, so the output equals the fp64
+ * definition.
  */
 KQ_API kq_status kq_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const void* mats,
                       kq_dtype mat_dtype, const float* factored, uint8_t* q, uint8_t* scales,
-                      kq_variant variant, kq_stream_t stream);
+                      kq_variant variant, kq_scale_layout scale_layout, kq_stream_t stream);
 
 /* kq_dequantize -- inverse of the MXFP4 step [KQ-abs]: yhat_j = E2M1(code_j) *
  * 2^(byte-127) (byte 0xFF gives NaN), and, when inv_mats != NULL, the block

@@ -10,6 +10,7 @@ thin ctypes binding plus seeded input generators (``inputs``).
 """
 from ._lib import (  # noqa: F401
     EXPORTED,
+    SCALE_LAYOUTS,
     KQError,
     kq_abi_version,
     kq_dequantize,
@@ -22,6 +23,7 @@ from ._lib import (  # noqa: F401
     kq_ref_smooth_quantize,
     kq_status_string,
     load,
+    scale_bytes,
 )
 
 
@@ -42,10 +44,11 @@ class BlockTransform:
             self._inv = kq_expand_blocks(self.params, inverse=True)
         return self._inv
 
-    def quantize(self, x, variant: str = "auto", q=None, scales=None):
-        return kq_quantize(x, self.mats, self.factored, variant=variant, q=q, scales=scales)
+    def quantize(self, x, variant: str = "auto", q=None, scales=None, scale_layout: str = "row"):
+        return kq_quantize(x, self.mats, self.factored, variant=variant, q=q, scales=scales,
+                           scale_layout=scale_layout)
 
-    def quantize_weights(self, w, mat_dtype=None, q=None, scales=None):
+    def quantize_weights(self, w, mat_dtype=None, q=None, scales=None, scale_layout: str = "row"):
         """MXFP4 of the weight rows w [n_out, d] (bf16) times K_b^-T per block, the
         weight side of the transform: dot products with quantize(x) rows then
         approximate x . w.  Runs the tensor-core variant with the dense K^-T."""
@@ -54,7 +57,7 @@ class BlockTransform:
         key = mat_dtype or torch.float32
         if getattr(self, "_inv_t", None) is None or self._inv_t.dtype != key:
             self._inv_t = kq_expand_blocks(self.params, inverse=True, transpose=True, dtype=key)
-        return kq_quantize(w, self._inv_t, None, variant="mma", q=q, scales=scales)
+        return kq_quantize(w, self._inv_t, None, variant="mma", q=q, scales=scales, scale_layout=scale_layout)
 
     def dequantize(self, q, scales, undo_transform: bool = True, out_dtype=None):
         import torch

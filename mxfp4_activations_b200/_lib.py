@@ -18,6 +18,14 @@ LIB_PATH = os.path.join(_PKG, "libkq.so")
 
 KQ_F32, KQ_BF16 = 0, 1
 VARIANTS = {"auto": 0, "mma": 1, "butterfly": 2}
+SCALE_LAYOUTS = {"row": 0, "mma": 1}  # row-major [M][d/32] / 128x4 tiles of block-scaled GEMMs
+
+
+def scale_bytes(M: int, d: int, layout: str = "row") -> int:
+    """Size of the scales buffer kq_quantize writes in the given layout."""
+    if layout == "row":
+        return M * (d // 32)
+    return ((M + 127) // 128) * 128 * ((d + 127) // 128) * 4
 STATUS = {
     0: "KQ_OK", 1: "KQ_ERR_INVALID_ARG", 2: "KQ_ERR_SHAPE", 3: "KQ_ERR_ALIGN", 4: "KQ_ERR_SINGULAR",
     5: "KQ_ERR_UNSUPPORTED", 6: "KQ_ERR_CUDA", 7: "KQ_ERR_DEVICE_TIMEOUT",
@@ -53,7 +61,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     sig = {
         "kq_expand_blocks": [P, I64, I, I, P, P],
         "kq_expand_factored": [P, I64, P, P],
-        "kq_quantize": [P, I64, I64, I64, P, I, P, P, P, I, P],
+        "kq_quantize": [P, I64, I64, I64, P, I, P, P, P, I, I, P],
         "kq_dequantize": [P, P, I64, I64, P, I, P, I, P],
         "kq_ref_smooth_quantize": [P, I64, I64, I64, P, P, P, P],
         "kq_ref_fwht_quantize": [P, I64, I64, I64, P, P, P],
@@ -145,26 +153,31 @@ def kq_expand_factored(params: torch.Tensor, out: torch.Tensor | None = None) ->
 
 # ---------------------------------------------------------------- hot path
 
-def _outputs(x: torch.Tensor, M: int, d: int, q, scales):
+def _outputs(x: torch.Tensor, M: int, d: int, q, scales, layout: str = "row"):
     if q is None:
         q = torch.empty((M, d // 2), dtype=torch.uint8, device=x.device)
     if scales is None:
-        scales = torch.empty((M, d // 32), dtype=torch.uint8, device=x.device)
+        if layout == "row":
+            scales = torch.empty((M, d // 32), dtype=torch.uint8, device=x.device)
+        else:  # padding bytes are not written: start from zeros
+            scales = torch.zeros(scale_bytes(M, d, layout), dtype=torch.uint8, device=x.device)
     if q.dtype != torch.uint8 or scales.dtype != torch.uint8 or not q.is_contiguous() or not scales.is_contiguous():
         raise ValueError("q and scales must be contiguous uint8")
-    if q.numel() < M * (d // 2) or scales.numel() < M * (d // 32):
+    if q.numel() < M * (d // 2) or scales.numel() < scale_bytes(M, d, layout):
         raise ValueError("q or scales too small")
     return q, scales
 
 
 def kq_quantize(x: torch.Tensor, mats: torch.Tensor, factored: torch.Tensor | None = None, variant: str = "auto",
-                q: torch.Tensor | None = None, scales: torch.Tensor | None = None):
-    """MXFP4 of x K_b per 32-element block -> (codes uint8 [M, d/2], E8M0 uint8 [M, d/32])."""
+                q: torch.Tensor | None = None, scales: torch.Tensor | None = None, scale_layout: str = "row"):
+    """MXFP4 of x K_b per 32-element block -> (codes uint8 [M, d/2], E8M0 scales: uint8
+    [M, d/32] for scale_layout="row", or the flat 128x4-tiled buffer for "mma")."""
     _cuda(x, "x")
     M, d, ldx = _rows(x)
-    q, scales = _outputs(x, M, d, q, scales)
+    q, scales = _outputs(x, M, d, q, scales, scale_layout)
     _check("kq_quantize", load().kq_quantize(_ptr(x), M, d, ldx, _ptr(mats), _mat_dtype(mats), _ptr(factored),
-                                             _ptr(q), _ptr(scales), VARIANTS[variant], _stream(x.device)))
+                                             _ptr(q), _ptr(scales), VARIANTS[variant], SCALE_LAYOUTS[scale_layout],
+                                             _stream(x.device)))
     return q, scales
 
 

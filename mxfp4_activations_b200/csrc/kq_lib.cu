@@ -96,7 +96,7 @@ int64_t row_stride(int64_t ncol, int64_t nrt, int sms, int per_sm) {
 
 template <int MODE>
 kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const float* mats, const float* factored,
-                       const float* inv_s, uint8_t* q, uint8_t* scales, cudaStream_t stream) {
+                       const float* inv_s, uint8_t* q, uint8_t* scales, int sf_tiled, cudaStream_t stream) {
   const DeviceInfo* dev = device_info();
   if (dev == nullptr) return cuda_fail("device query", cudaErrorInvalidDevice);
   EncodeTiledFn enc = encode_tiled();
@@ -148,6 +148,7 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   p.inv_s = inv_s;
   p.q = q;
   p.scales = scales;
+  p.sf_tiled = sf_tiled;
 
   const int64_t ncol = (nb + kq::kQCols - 1) / kq::kQCols;
   if (ncol > int64_t(INT32_MAX)) return KQ_ERR_SHAPE;
@@ -159,7 +160,7 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
 // Tensor-core variant: 128-row x 4-block tiles, one CTA per 4-block column group
 // and row-tile stride, two CTAs per SM (256 tensor-memory columns each).
 kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, const void* mats, bool mats_bf16,
-                           uint8_t* q, uint8_t* scales, cudaStream_t stream) {
+                           uint8_t* q, uint8_t* scales, int sf_tiled, cudaStream_t stream) {
   const DeviceInfo* dev = device_info();
   if (dev == nullptr) return cuda_fail("device query", cudaErrorInvalidDevice);
   EncodeTiledFn enc = encode_tiled();
@@ -197,6 +198,7 @@ kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, con
   p.mats = mats;
   p.q = q;
   p.scales = scales;
+  p.sf_tiled = sf_tiled;
   // Resident CTAs per SM.  The runtime's occupancy query reports one CTA per SM
   // for any kernel that touches tensor memory (it cannot know how many columns
   // the kernel allocates), so the count comes from the kernel's own budget:
@@ -236,7 +238,7 @@ int grid_for(int64_t work, int threads) {
 
 extern "C" {
 
-int kq_abi_version(void) { return 100; }
+int kq_abi_version(void) { return 200; }
 
 const char* kq_status_string(kq_status s) {
   switch (s) {
@@ -278,8 +280,10 @@ kq_status kq_expand_factored(const float* params, int64_t nb, float* factored, k
 
 kq_status kq_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const void* mats, kq_dtype mat_dtype,
                       const float* factored, uint8_t* q, uint8_t* scales, kq_variant variant,
-                      kq_stream_t stream) {
+                      kq_scale_layout scale_layout, kq_stream_t stream) {
   if (variant != KQ_VAR_AUTO && variant != KQ_VAR_MMA && variant != KQ_VAR_BUTTERFLY) return KQ_ERR_INVALID_ARG;
+  if (scale_layout != KQ_SCALES_ROW_MAJOR && scale_layout != KQ_SCALES_MMA_TILED) return KQ_ERR_INVALID_ARG;
+  const int sf_tiled = scale_layout == KQ_SCALES_MMA_TILED ? 1 : 0;
   if (mat_dtype != KQ_F32 && mat_dtype != KQ_BF16) return KQ_ERR_INVALID_ARG;
   kq_status st = check_x(x, M, d, ldx);
   if (st != KQ_OK) return st;
@@ -294,11 +298,11 @@ kq_status kq_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const vo
                        (variant == KQ_VAR_AUTO && factored == nullptr);
   if (variant == KQ_VAR_BUTTERFLY && mat_dtype == KQ_BF16) return KQ_ERR_UNSUPPORTED;
   if (use_mma)
-    return launch_quant_mma(x, M, d, ldx, mats, mat_dtype == KQ_BF16, q, scales, as_cuda(stream));
+    return launch_quant_mma(x, M, d, ldx, mats, mat_dtype == KQ_BF16, q, scales, sf_tiled, as_cuda(stream));
   if (factored == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(factored, 16)) return KQ_ERR_ALIGN;
   return launch_quant<kq::MODE_KRON>(x, M, d, ldx, static_cast<const float*>(mats), factored, nullptr, q, scales,
-                                     as_cuda(stream));
+                                     sf_tiled, as_cuda(stream));
 }
 
 kq_status kq_ref_smooth_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const float* inv_s,
@@ -310,7 +314,7 @@ kq_status kq_ref_smooth_quantize(const void* x, int64_t M, int64_t d, int64_t ld
   if (st != KQ_OK) return st;
   if (inv_s == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(inv_s, 16)) return KQ_ERR_ALIGN;
-  return launch_quant<kq::MODE_SMOOTH>(x, M, d, ldx, nullptr, nullptr, inv_s, q, scales, as_cuda(stream));
+  return launch_quant<kq::MODE_SMOOTH>(x, M, d, ldx, nullptr, nullptr, inv_s, q, scales, 0, as_cuda(stream));
 }
 
 kq_status kq_ref_fwht_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, uint8_t* q, uint8_t* scales,
@@ -320,7 +324,7 @@ kq_status kq_ref_fwht_quantize(const void* x, int64_t M, int64_t d, int64_t ldx,
   if (M == 0 || d == 0) return KQ_OK;
   st = check_out(q, scales);
   if (st != KQ_OK) return st;
-  return launch_quant<kq::MODE_FWHT>(x, M, d, ldx, nullptr, nullptr, nullptr, q, scales, as_cuda(stream));
+  return launch_quant<kq::MODE_FWHT>(x, M, d, ldx, nullptr, nullptr, nullptr, q, scales, 0, as_cuda(stream));
 }
 
 kq_status kq_dequantize(const uint8_t* q, const uint8_t* scales, int64_t M, int64_t d, const void* inv_mats,

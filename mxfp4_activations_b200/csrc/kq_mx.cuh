@@ -18,6 +18,16 @@ namespace kq {
 constexpr float kFwhtC = 0.17677669529663688f;    // fp32 nearest to 2^-2.5
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per bounded wait
 
+// Byte index of the scale of block column b of row `row` (nb block columns):
+// row-major, or the 128 x 4 tiled layout of block-scaled tensor-core GEMMs
+// (tile (row/128, b/4) of 512 bytes, stored tile row by tile row; inside it
+// 16*(row%32) + 4*((row/32)%4) + b%4).
+__device__ __forceinline__ int64_t scale_index(int64_t row, int b, int nb, int tiled) {
+  if (!tiled) return row * int64_t(nb) + b;
+  const int64_t tile = (row >> 7) * int64_t((nb + 3) >> 2) + (b >> 2);
+  return tile * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (b & 3);
+}
+
 // Where the exact path reads K[i][j] from.
 enum KSource { KSRC_F32 = 0, KSRC_BF16 = 1, KSRC_FWHT = 2 };
 

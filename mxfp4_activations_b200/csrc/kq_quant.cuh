@@ -79,7 +79,8 @@ struct QuantParams {
   const float* factored;  // KRON: [nb][48]
   const float* inv_s;     // SMOOTH: [nb*32]
   uint8_t* q;             // [M][nb*16]
-  uint8_t* scales;        // [M][nb]
+  uint8_t* scales;        // row-major [M][nb], or tiled (scale_index)
+  int sf_tiled;           // 1: scales in the 128 x 4 tiled layout
 };
 
 // Entry f of the coefficient record of block column b (fp32 bits as read by
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_consta
     const bool act = col_ok && row < p.M;
     const int64_t rowc = act ? row : 0;
     uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16;
-    uint8_t* sb = p.scales + rowc * int64_t(p.nb) + bc;
+    uint8_t* sb = p.scales + scale_index(rowc, bc, p.nb, p.sf_tiled);
     const uint16_t* xb = p.x + rowc * p.ldx + int64_t(bc) * kBlock;
     // every lane takes part (the exact path is warp-cooperative); only real blocks store
     quant_block<MODE>(cf, xr, act, qb, sb, xb, Kb);

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.kq_abi_version() == 100
+    assert lib.kq_abi_version() == 200
     for code in range(8):
         s = lib.kq_status_string(code).decode()
         assert s.startswith("KQ_")
@@ -52,9 +52,9 @@ P = ctypes.c_void_p
 
 
 def q(lib, x=16 * 1024, M=4, d=64, ldx=64, mats=16 * 2048, dtype=0, fac=16 * 4096, qq=16 * 8192,
-      sc=16 * 9000, var=2):
+      sc=16 * 9000, var=2, layout=0):
     return lib.kq_quantize(P(x) if x else None, M, d, ldx, P(mats) if mats else None, dtype,
-                           P(fac) if fac else None, P(qq) if qq else None, P(sc) if sc else None, var, None)
+                           P(fac) if fac else None, P(qq) if qq else None, P(sc) if sc else None, var, layout, None)
 
 
 def test_quantize_argument_errors_return_before_launch(lib):
@@ -68,6 +68,7 @@ def test_quantize_argument_errors_return_before_launch(lib):
     assert q(lib, qq=16 * 8192 + 4) == 3      # codes not 16-byte aligned
     assert q(lib, mats=0) == 1
     assert q(lib, var=9) == 1                 # bad variant enum
+    assert q(lib, layout=2) == 1              # bad scale layout enum
     assert q(lib, dtype=7) == 1               # bad dtype enum
     assert q(lib, fac=0) == 1                 # butterfly needs the factored form
     assert q(lib, dtype=1) == 5               # bf16 matrices need the tensor-core variant

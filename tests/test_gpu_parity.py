@@ -215,6 +215,73 @@ def test_quantize_degenerate_blocks(kq, orc, variant, mdt):
     check(q, s, qr, sr)
 
 
+def tiled_scales(s: np.ndarray) -> np.ndarray:
+    """Row-major [M][C] scales rearranged into 128 x 4 tiles (tile rows first; in a
+    tile, row r = 32 * r_hi + r_lo and column c go to 16 * r_lo + 4 * r_hi + c),
+    written as a reshape so that it shares no arithmetic with the kernels."""
+    M, C = s.shape
+    Mp, Cp = -(-M // 128) * 128, -(-C // 4) * 4
+    pad = np.zeros((Mp, Cp), np.uint8)
+    pad[:M, :C] = s
+    t = pad.reshape(Mp // 128, 4, 32, Cp // 4, 4)       # (R, r_hi, r_lo, C, c)
+    return np.ascontiguousarray(t.transpose(0, 3, 2, 1, 4)).reshape(-1)
+
+
+@pytest.mark.parametrize("variant,mdt", VARIANTS)
+@pytest.mark.parametrize("M,d", [(1, 32), (130, 96), (257, 1152), (64, 12288)])
+def test_quantize_tiled_scale_layout(kq, orc, M, d, variant, mdt):
+    x = inputs.activations(M, d, "t3", seed=[M, d, 5], outlier_frac=0.01, outlier_scale=(20.0, 100.0))
+    params = inputs.lu_params(d // 32, seed=[M, d, 6])
+    p = dev_f32(params)
+    mats = kq.kq_expand_blocks(p, dtype=torch.float32 if mdt == "f32" else torch.bfloat16)
+    fac = kq.kq_expand_factored(p) if variant == "butterfly" else None
+    qd, sd = kq.kq_quantize(dev_bf16(x), mats, fac, variant=variant, scale_layout="mma")
+    assert sd.numel() == kq.scale_bytes(M, d, "mma")
+    qr, sr = orc.quantize(x, oracle_mats(orc, params, mdt))
+    assert np.array_equal(host(qd), qr)
+    assert np.array_equal(host(sd), tiled_scales(sr))  # padding stays zero
+
+
+def test_w4a4_gemm_through_block_scaled_mma(kq, orc):
+    """End to end: activations quantized with K_b, weights with K_b^-T, both with
+    scales in the tiled layout, multiplied by cuBLAS's block-scaled FP4 GEMM
+    (through torch) -- the consumer the layout is for.  The product equals the
+    oracle's dequantized operands multiplied in fp64 up to fp32 accumulation and
+    the bf16 output rounding, and approximates x w^T (the transform cancels)."""
+    F = pytest.importorskip("torch.nn.functional")
+    if not hasattr(F, "scaled_mm") or not hasattr(torch, "float4_e2m1fn_x2"):
+        pytest.skip("this torch has no block-scaled FP4 matmul")
+    M, N, d = 256, 128, 512
+    x = inputs.activations(M, d, "t3", seed=51, outlier_frac=0.01, outlier_scale=(20.0, 100.0))
+    rng = np.random.default_rng(52)
+    w = inputs.f32_to_bf16_bits((rng.standard_normal((N, d)) * 0.05).astype(np.float32))
+    params = inputs.lu_params(d // 32, seed=53)
+    bt = kq.BlockTransform(dev_f32(params))
+    qa, sa = bt.quantize(dev_bf16(x), scale_layout="mma")
+    qb, sb = bt.quantize_weights(dev_bf16(w), scale_layout="mma")
+    try:
+        y = F.scaled_mm(qa.view(torch.float4_e2m1fn_x2), qb.view(torch.float4_e2m1fn_x2).t(),
+                        sa.view(torch.float8_e8m0fnu), F.ScalingType.BlockWise1x32,
+                        sb.view(torch.float8_e8m0fnu), F.ScalingType.BlockWise1x32,
+                        swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                        output_dtype=torch.bfloat16)
+    except (RuntimeError, NotImplementedError, TypeError, ValueError) as e:
+        pytest.skip(f"block-scaled FP4 matmul unavailable here: {str(e).splitlines()[0][:120]}")
+    y = y.float().cpu().numpy().astype(np.float64)
+    ka = orc.expand(params, dtype=orc.F32)
+    kbt = np.ascontiguousarray(np.swapaxes(orc.expand(params, dtype=orc.F32, inverse=True), 1, 2))
+    qar, sar = orc.quantize(x, ka)
+    qbr, sbr = orc.quantize(w, kbt)
+    a_hat = orc.dequantize(qar, sar).astype(np.float64)
+    b_hat = orc.dequantize(qbr, sbr).astype(np.float64)
+    yref = a_hat @ b_hat.T
+    mag = np.abs(a_hat) @ np.abs(b_hat).T
+    assert np.all(np.abs(y - yref) <= 2.0**-8 * np.abs(yref) + 2.0**-16 * mag), np.abs(y - yref).max()
+    xw = inputs.bf16_bits_to_f32(x).astype(np.float64) @ inputs.bf16_bits_to_f32(w).astype(np.float64).T
+    rel = np.linalg.norm(yref - xw) / np.linalg.norm(xw)
+    assert rel < 0.25, rel  # FP4 noise only: a wrong transform pair would not cancel
+
+
 @pytest.mark.parametrize("mdt", ["f32", "bf16"])
 def test_weight_side_quantize(kq, orc, mdt):
     """Weight rows quantized with the weight-side transform K_b^-T through the
