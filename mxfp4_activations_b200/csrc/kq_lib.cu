@@ -94,9 +94,9 @@ int64_t row_stride(int64_t ncol, int64_t nrt, int sms, int per_sm) {
   return gy;
 }
 
-template <int MODE>
+template <int MODE, int TILED>
 kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const float* mats, const float* factored,
-                       const float* inv_s, uint8_t* q, uint8_t* scales, int sf_tiled, cudaStream_t stream) {
+                       const float* inv_s, uint8_t* q, uint8_t* scales, cudaStream_t stream) {
   const DeviceInfo* dev = device_info();
   if (dev == nullptr) return cuda_fail("device query", cudaErrorInvalidDevice);
   EncodeTiledFn enc = encode_tiled();
@@ -116,7 +116,7 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cuda_fail("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
 
-  auto kern = kq::quant_kernel<MODE>;
+  auto kern = kq::quant_kernel<MODE, TILED>;
   static std::atomic<int> attr_set[kMaxDevices];
   int devid = 0;
   cudaGetDevice(&devid);
@@ -148,7 +148,6 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   p.inv_s = inv_s;
   p.q = q;
   p.scales = scales;
-  p.sf_tiled = sf_tiled;
 
   const int64_t ncol = (nb + kq::kQCols - 1) / kq::kQCols;
   if (ncol > int64_t(INT32_MAX)) return KQ_ERR_SHAPE;
@@ -177,14 +176,18 @@ kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, con
     return cuda_fail("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
   const int smem = 1024 + kq::kMmaStages * kq::kMmaAStageBytes + kq::kMmaWb * 3 * kq::kMmaBBytes + 256;
   if (smem > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
-  auto kern = mats_bf16 ? kq::quant_mma_kernel<kq::KSRC_BF16> : kq::quant_mma_kernel<kq::KSRC_F32>;
-  static std::atomic<int> attr_set[2][kMaxDevices];
+  const int which = (mats_bf16 ? 1 : 0) + (sf_tiled ? 2 : 0);
+  static void (*const kernels[4])(const CUtensorMap, const kq::MmaParams) = {
+      kq::quant_mma_kernel<kq::KSRC_F32, 0>, kq::quant_mma_kernel<kq::KSRC_BF16, 0>,
+      kq::quant_mma_kernel<kq::KSRC_F32, 1>, kq::quant_mma_kernel<kq::KSRC_BF16, 1>};
+  auto kern = kernels[which];
+  static std::atomic<int> attr_set[4][kMaxDevices];
   int devid = 0;
   cudaGetDevice(&devid);
-  if (!attr_set[mats_bf16][devid].load()) {
+  if (!attr_set[which][devid].load()) {
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
-    attr_set[mats_bf16][devid].store(1);
+    attr_set[which][devid].store(1);
   }
   kq::MmaParams p;
   p.x = static_cast<const uint16_t*>(x);
@@ -198,7 +201,6 @@ kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, con
   p.mats = mats;
   p.q = q;
   p.scales = scales;
-  p.sf_tiled = sf_tiled;
   // Resident CTAs per SM.  The runtime's occupancy query reports one CTA per SM
   // for any kernel that touches tensor memory (it cannot know how many columns
   // the kernel allocates), so the count comes from the kernel's own budget:
@@ -301,8 +303,9 @@ kq_status kq_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const vo
     return launch_quant_mma(x, M, d, ldx, mats, mat_dtype == KQ_BF16, q, scales, sf_tiled, as_cuda(stream));
   if (factored == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(factored, 16)) return KQ_ERR_ALIGN;
-  return launch_quant<kq::MODE_KRON>(x, M, d, ldx, static_cast<const float*>(mats), factored, nullptr, q, scales,
-                                     sf_tiled, as_cuda(stream));
+  const float* m32 = static_cast<const float*>(mats);
+  return sf_tiled ? launch_quant<kq::MODE_KRON, 1>(x, M, d, ldx, m32, factored, nullptr, q, scales, as_cuda(stream))
+                  : launch_quant<kq::MODE_KRON, 0>(x, M, d, ldx, m32, factored, nullptr, q, scales, as_cuda(stream));
 }
 
 kq_status kq_ref_smooth_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const float* inv_s,
@@ -314,7 +317,7 @@ kq_status kq_ref_smooth_quantize(const void* x, int64_t M, int64_t d, int64_t ld
   if (st != KQ_OK) return st;
   if (inv_s == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(inv_s, 16)) return KQ_ERR_ALIGN;
-  return launch_quant<kq::MODE_SMOOTH>(x, M, d, ldx, nullptr, nullptr, inv_s, q, scales, 0, as_cuda(stream));
+  return launch_quant<kq::MODE_SMOOTH, 0>(x, M, d, ldx, nullptr, nullptr, inv_s, q, scales, as_cuda(stream));
 }
 
 kq_status kq_ref_fwht_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, uint8_t* q, uint8_t* scales,
@@ -324,7 +327,7 @@ kq_status kq_ref_fwht_quantize(const void* x, int64_t M, int64_t d, int64_t ldx,
   if (M == 0 || d == 0) return KQ_OK;
   st = check_out(q, scales);
   if (st != KQ_OK) return st;
-  return launch_quant<kq::MODE_FWHT>(x, M, d, ldx, nullptr, nullptr, nullptr, q, scales, 0, as_cuda(stream));
+  return launch_quant<kq::MODE_FWHT, 0>(x, M, d, ldx, nullptr, nullptr, nullptr, q, scales, as_cuda(stream));
 }
 
 kq_status kq_dequantize(const uint8_t* q, const uint8_t* scales, int64_t M, int64_t d, const void* inv_mats,

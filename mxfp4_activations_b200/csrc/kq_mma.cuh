@@ -80,7 +80,6 @@ struct MmaParams {
   const void* mats;    // [nb][32][32] fp32 or bf16
   uint8_t* q;
   uint8_t* scales;     // row-major [M][nb], or tiled (scale_index)
-  int sf_tiled;
 };
 
 // Shared-memory matrix descriptor: start address, leading / stride byte
@@ -157,7 +156,7 @@ __device__ __forceinline__ float l1_upper_bf16(const uint4 (&v)[4]) {
   return __fmul_ru(s, 1.03125f);
 }
 
-template <int KSRC>
+template <int KSRC, int TILED>
 __global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                    const MmaParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -357,7 +356,7 @@ __global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(c
       for (int m2 = 0; m2 < 16; m2++) Y[m2] = pk2(y[2 * m2], y[2 * m2 + 1]);
       const float amax = block_amax(y);
       uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16;
-      uint8_t* sb = p.scales + scale_index(rowc, bc, p.nb, p.sf_tiled);
+      uint8_t* sb = p.scales + scale_index(rowc, bc, p.nb, TILED);
       const uint16_t* xb = p.x + rowc * p.ldx + int64_t(bc) * kBlock;
       certify_store(Y, amax, l1, zero_block, cfac, kMmaErrAbs, !(cfac <= FLT_MAX), act, qb, sb,
                     [&](bool need) { warp_exact_pass<KSRC>(need, xb, Kb, qb, sb); });

@@ -80,7 +80,6 @@ struct QuantParams {
   const float* inv_s;     // SMOOTH: [nb*32]
   uint8_t* q;             // [M][nb*16]
   uint8_t* scales;        // row-major [M][nb], or tiled (scale_index)
-  int sf_tiled;           // 1: scales in the 128 x 4 tiled layout
 };
 
 // Entry f of the coefficient record of block column b (fp32 bits as read by
@@ -233,7 +232,9 @@ __device__ __forceinline__ void quant_block(uint32_t cf, const uint4 (&xr)[4], b
 
 // ---------------------------------------------------------------- kernel
 
-template <int MODE>
+// TILED: scales in the 128 x 4 tiled layout of block-scaled GEMMs (a template
+// parameter, so the row-major store costs nothing extra).
+template <int MODE, int TILED>
 __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_consta
     const bool act = col_ok && row < p.M;
     const int64_t rowc = act ? row : 0;
     uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16;
-    uint8_t* sb = p.scales + scale_index(rowc, bc, p.nb, p.sf_tiled);
+    uint8_t* sb = p.scales + scale_index(rowc, bc, p.nb, TILED);
     const uint16_t* xb = p.x + rowc * p.ldx + int64_t(bc) * kBlock;
     // every lane takes part (the exact path is warp-cooperative); only real blocks store
     quant_block<MODE>(cf, xr, act, qb, sb, xb, Kb);
