@@ -49,7 +49,7 @@ constexpr int kMmaCtasPerSm = 3;
 static_assert(kMmaTmemCols * kMmaCtasPerSm <= 512, "co-resident CTAs must fit the tensor memory");
 static_assert((kMmaTmemCols & (kMmaTmemCols - 1)) == 0 && kMmaTmemCols >= 32, "tcgen05.alloc takes a power of 2 >= 32");
 constexpr int kMmaEpiWarps = 4 * kMmaWb;             // one warp per (block, lane quarter)
-constexpr int kMmaThreads = (2 + kMmaEpiWarps) * 32; // 576
+constexpr int kMmaThreads = (2 + kMmaEpiWarps) * 32; // 320
 constexpr int kMmaATileBytes = kMmaRows * 64;        // 8 KB per block of a tile
 constexpr int kMmaAStageBytes = kMmaWb * kMmaATileBytes;  // 16 KB per tile
 constexpr int kMmaBBytes = 32 * 64;                  // one 32x32 bf16 matrix
