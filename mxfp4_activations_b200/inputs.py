@@ -42,16 +42,17 @@ def bf16_bits_to_f32(h: np.ndarray) -> np.ndarray:
     return (np.ascontiguousarray(h, np.uint16).astype(np.uint32) << 16).view(np.float32)
 
 
-def lu_params(nb: int, seed, noise: float = 0.05) -> np.ndarray:
-    """Per-block params [nb, 5, 3] fp32: Hadamard initialisation + N(0, noise)."""
+def lu_params(nb: int, seed, noise: float = 0.05, factors: int = 5) -> np.ndarray:
+    """Per-block params [nb, factors, 3] fp32 (5 factors for 32-element blocks, 6
+    for 64): Hadamard initialisation + N(0, noise)."""
     rng = np.random.default_rng(seed)
     base = np.array(HADAMARD_INIT, np.float64)
-    p = base[None, None, :] + rng.normal(0.0, noise, size=(nb, 5, 3))
+    p = base[None, None, :] + rng.normal(0.0, noise, size=(nb, factors, 3))
     return p.astype(np.float32)
 
 
-def hadamard_params(nb: int) -> np.ndarray:
-    return np.tile(np.array(HADAMARD_INIT, np.float32), (nb, 5, 1))
+def hadamard_params(nb: int, factors: int = 5) -> np.ndarray:
+    return np.tile(np.array(HADAMARD_INIT, np.float32), (nb, factors, 1))
 
 
 def identity_params(nb: int) -> np.ndarray:

@@ -299,3 +299,72 @@ void kqo_dequantize(const uint8_t* q, const uint8_t* scales, int64_t M, int64_t 
       }
     }
 }
+
+/* ---- transform blocks of n = 2^log2n elements ------------------------------------ */
+
+/* [KQ-sum, Approach / Limitations]: the same construction with log2n factors,
+ * assembled from the innermost factor outward. */
+void kqo_expand_n_f64(const float* params, int64_t nt, int log2n, int inverse, double* K) {
+  const int n = 1 << log2n;
+  double* acc = (double*)malloc(sizeof(double) * (size_t)n * (size_t)n);
+  double* tmp = (double*)malloc(sizeof(double) * (size_t)n * (size_t)n);
+  for (int64_t c = 0; c < nt; c++) {
+    const float* p = params + c * 3 * log2n;
+    double F[4];
+    int m = 2;
+    if (inverse)
+      kqo_factor_inverse(p[3 * (log2n - 1)], p[3 * (log2n - 1) + 1], p[3 * (log2n - 1) + 2], F);
+    else
+      kqo_factor(p[3 * (log2n - 1)], p[3 * (log2n - 1) + 1], p[3 * (log2n - 1) + 2], F);
+    memcpy(acc, F, sizeof(F));
+    for (int k = log2n - 2; k >= 0; k--) {
+      if (inverse)
+        kqo_factor_inverse(p[3 * k], p[3 * k + 1], p[3 * k + 2], F);
+      else
+        kqo_factor(p[3 * k], p[3 * k + 1], p[3 * k + 2], F);
+      kqo_kron(F, 2, acc, m, tmp);
+      m *= 2;
+      memcpy(acc, tmp, sizeof(double) * (size_t)m * (size_t)m);
+    }
+    memcpy(K + c * (int64_t)n * n, acc, sizeof(double) * (size_t)n * (size_t)n);
+  }
+  free(acc);
+  free(tmp);
+}
+
+void kqo_expand_n(const float* params, int64_t nt, int log2n, int inverse, int dtype, void* out) {
+  const int64_t total = nt * ((int64_t)1 << (2 * log2n));
+  double* K = (double*)malloc(sizeof(double) * (size_t)(total > 0 ? total : 1));
+  kqo_expand_n_f64(params, nt, log2n, inverse, K);
+  if (dtype == KQO_F32) {
+    float* o = (float*)out;
+    for (int64_t i = 0; i < total; i++) o[i] = (float)K[i];
+  } else {
+    uint16_t* o = (uint16_t*)out;
+    for (int64_t i = 0; i < total; i++) o[i] = kqo_bf16_from_f64(K[i]);
+  }
+  free(K);
+}
+
+void kqo_transform_n(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const void* mats, int dtype,
+                     int n, float* y) {
+  const int64_t nt = d / n;
+  for (int64_t r = 0; r < M; r++)
+    for (int64_t c = 0; c < nt; c++)
+      for (int j = 0; j < n; j++) {
+        double acc = 0.0;
+        for (int i = 0; i < n; i++) {
+          const double xi = (double)f32_from_bf16(x[r * ldx + c * n + i]);
+          acc += xi * mat_entry(mats, dtype, c * (int64_t)n * n + (int64_t)i * n + j);
+        }
+        y[r * d + c * n + j] = (float)acc;
+      }
+}
+
+void kqo_quantize_n(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const void* mats, int dtype,
+                    int n, uint8_t* q, uint8_t* scales) {
+  float* y = (float*)malloc(sizeof(float) * (size_t)(M * d > 0 ? M * d : 1));
+  kqo_transform_n(x, M, d, ldx, mats, dtype, n, y);
+  kqo_mx_quantize(y, M, d, q, scales);
+  free(y);
+}

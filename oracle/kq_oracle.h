@@ -88,6 +88,24 @@ void kqo_fwht_quantize(const uint16_t* x, int64_t M, int64_t d, int64_t ldx,
 void kqo_dequantize(const uint8_t* q, const uint8_t* scales, int64_t M, int64_t d,
                     const void* inv_mats, int dtype, double* out);
 
+/* ---- transform blocks of n = 2^log2n elements (log2n in 4..7), MXFP4 still per 32
+ *
+ * [KQ-sum, Limitations]: the Kronecker parametrization has 3 log2(n) parameters
+ * per block of n elements.  K_c = F_0 (x) ... (x) F_{log2n-1} (F_0 on the most
+ * significant index bit) acts on elements [c n, c n + n) of a row; params are
+ * [nt][log2n][3].  The MX scale blocks stay 32 elements long. */
+/* K_c (or K_c^-1) in fp64, [nt][n][n]. */
+void kqo_expand_n_f64(const float* params, int64_t nt, int log2n, int inverse, double* K);
+/* Same, rounded once to fp32 (float out) or bf16 (uint16 out). */
+void kqo_expand_n(const float* params, int64_t nt, int log2n, int inverse, int dtype, void* out);
+/* y[r][c n + j] = fp32( sum_i x[r][c n + i] K_c[i][j] ), fp64 accumulation in
+ * index order from +0; d % n == 0. */
+void kqo_transform_n(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const void* mats, int dtype,
+                     int n, float* y);
+/* transform_n, then MXFP4 per 32 elements. */
+void kqo_quantize_n(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const void* mats, int dtype,
+                    int n, uint8_t* q, uint8_t* scales);
+
 #ifdef __cplusplus
 }
 #endif

@@ -47,6 +47,10 @@ def lib():
         L.kqo_kron.argtypes = [P, I, P, I, P]
         L.kqo_expand_f64.argtypes = [P, I64, I, P]
         L.kqo_expand.argtypes = [P, I64, I, I, P]
+        L.kqo_expand_n_f64.argtypes = [P, I64, I, I, P]
+        L.kqo_expand_n.argtypes = [P, I64, I, I, I, P]
+        L.kqo_transform_n.argtypes = [P, I64, I64, I64, P, I, I, P]
+        L.kqo_quantize_n.argtypes = [P, I64, I64, I64, P, I, I, P, P]
         L.kqo_bf16_from_f64.argtypes = [ctypes.c_double]
         L.kqo_bf16_from_f64.restype = ctypes.c_uint16
         L.kqo_hadamard.argtypes = [I, P]
@@ -220,3 +224,45 @@ def dequantize(q: np.ndarray, scales: np.ndarray, inv_mats: np.ndarray | None = 
         inv_mats = np.ascontiguousarray(inv_mats)
         lib().kqo_dequantize(_p(q), _p(scales), M, d, _p(inv_mats), _mats_dtype(inv_mats), _p(out))
     return out
+
+
+# ---- transform blocks of n = 2^log2n elements (MXFP4 still per 32) -------------------
+
+def expand_n_f64(params: np.ndarray, inverse: bool = False) -> np.ndarray:
+    """params [nt][log2n][3] -> K [nt][n][n] in fp64."""
+    params = np.ascontiguousarray(params, np.float32)
+    nt, log2n = params.shape[0], params.shape[1]
+    n = 1 << log2n
+    out = np.zeros((nt, n, n), np.float64)
+    lib().kqo_expand_n_f64(_p(params), nt, log2n, int(bool(inverse)), _p(out))
+    return out
+
+
+def expand_n(params: np.ndarray, dtype: int = F32, inverse: bool = False) -> np.ndarray:
+    params = np.ascontiguousarray(params, np.float32)
+    nt, log2n = params.shape[0], params.shape[1]
+    n = 1 << log2n
+    out = np.zeros((nt, n, n), np.float32 if dtype == F32 else np.uint16)
+    lib().kqo_expand_n(_p(params), nt, log2n, int(bool(inverse)), dtype, _p(out))
+    return out
+
+
+def transform_n(x: np.ndarray, mats: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, np.uint16)
+    mats = np.ascontiguousarray(mats)
+    M, d = x.shape
+    n = mats.shape[-1]
+    y = np.zeros((M, d), np.float32)
+    lib().kqo_transform_n(_p(x), M, d, d, _p(mats), _mats_dtype(mats), n, _p(y))
+    return y
+
+
+def quantize_n(x: np.ndarray, mats: np.ndarray):
+    x = np.ascontiguousarray(x, np.uint16)
+    mats = np.ascontiguousarray(mats)
+    M, d = x.shape
+    n = mats.shape[-1]
+    q = np.zeros((M, d // 2), np.uint8)
+    s = np.zeros((M, d // 32), np.uint8)
+    lib().kqo_quantize_n(_p(x), M, d, d, _p(mats), _mats_dtype(mats), n, _p(q), _p(s))
+    return q, s

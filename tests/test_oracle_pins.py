@@ -443,3 +443,69 @@ def test_fwht_equals_kroquant_with_sylvester_matrix(orc):
     H = np.broadcast_to(sylvester_closed_form(5).astype(np.float32), (3, 32, 32)).copy()
     q2, s2 = orc.quantize(x, H)
     assert np.array_equal(q, q2) and np.array_equal(s, s2)
+
+
+# ---------------------------------------------------------------- transform blocks of n = 2^k elements
+
+@pytest.mark.parametrize("log2n", [4, 6, 7])
+def test_expand_n_matches_numpy_kron(orc, log2n):
+    """[KQ-sum, Limitations]: 3 log2(n) parameters per n-element block; K is the
+    Kronecker product of the log2(n) LU factors, F_0 on the top index bit."""
+    params = inputs.lu_params(3, seed=60 + log2n, factors=log2n)
+    K = orc.expand_n_f64(params)
+    n = 1 << log2n
+    assert K.shape == (3, n, n) and params[0].size == 3 * log2n
+    for c in range(3):
+        ref = lu_numpy(*params[c, 0])
+        for k in range(1, log2n):
+            ref = np.kron(ref, lu_numpy(*params[c, k]))
+        assert np.allclose(K[c], ref, rtol=1e-13, atol=0)
+    sign, logdet = np.linalg.slogdet(K)
+    assert np.all(sign > 0) and np.abs(logdet).max() < 1e-9       # det = 1
+    Ki = orc.expand_n_f64(params, inverse=True)
+    assert np.allclose(Ki, np.linalg.inv(K), rtol=0, atol=1e-10)
+
+
+def test_expand_n_at_32_is_the_block_expansion(orc):
+    params = inputs.lu_params(4, seed=66)
+    assert np.array_equal(orc.expand_n(params).view(np.uint32), orc.expand(params).view(np.uint32))
+    assert np.array_equal(orc.expand_n(params, dtype=orc.BF16), orc.expand(params, dtype=orc.BF16))
+
+
+def test_hadamard_init_n64_reproduces_h64_up_to_signs(orc):
+    K = orc.expand_n_f64(inputs.hadamard_params(1, factors=6))[0]
+    D = np.diag([(-1.0) ** bin(i).count("1") for i in range(64)])
+    assert np.abs(K - D @ sylvester_closed_form(6)).max() < 1e-6
+    assert np.abs(K @ K.T - np.eye(64)).max() < 1e-6
+
+
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_transform_n64_exact_rational_brute_force(orc, dtype):
+    rng = np.random.default_rng(67 + dtype)
+    M, d = 2, 128
+    x = inputs.f32_to_bf16_bits((rng.standard_t(3, (M, d)) * rng.choice([1, 100], (M, d))).astype(np.float32))
+    params = inputs.lu_params(d // 64, seed=68, factors=6)
+    mats = orc.expand_n(params, dtype=dtype)
+    y = orc.transform_n(x, mats)
+    matf = mats if dtype == 0 else inputs.bf16_bits_to_f32(mats)
+    for r in range(M):
+        for c in range(d // 64):
+            xs = [bf16_bits_to_frac(int(h)) for h in x[r, 64 * c:64 * c + 64]]
+            for j in range(0, 64, 5):
+                exact = sum(xs[i] * Fraction(float(matf[c, i, j])) for i in range(64))
+                assert y[r, 64 * c + j] == f32_round_fraction(exact), (r, c, j)
+
+
+def test_quantize_n64_is_mx_of_the_transform(orc):
+    """MXFP4 per 32 elements of the n = 64 transform: scales by the bit-field
+    rule from each 32-block's amax, codes by the brute-force nearest value."""
+    rng = np.random.default_rng(69)
+    x = inputs.f32_to_bf16_bits(rng.standard_normal((3, 128)).astype(np.float32))
+    mats = orc.expand_n(inputs.lu_params(2, seed=70, factors=6))
+    y = orc.transform_n(x, mats)
+    q, s = orc.quantize_n(x, mats)
+    amax = np.abs(y.reshape(3, 4, 32)).max(axis=2)
+    assert np.array_equal(s, e8m0_from_bits(amax.astype(np.float32)).astype(np.uint8))
+    scale = np.exp2(s.astype(np.float64) - 127.0)
+    v = (y.reshape(3, 4, 32) / scale[:, :, None]).astype(np.float32).reshape(3, 128)
+    assert np.array_equal(unpack_nibbles(q).reshape(3, 128), brute_e2m1(v))
