@@ -112,6 +112,16 @@ typedef enum { KQ_SCALES_ROW_MAJOR = 0, KQ_SCALES_MMA_TILED = 1 } kq_scale_layou
 KQ_API kq_status kq_expand_blocks(const float* params, int64_t nb, int inverse, kq_dtype out_dtype,
                            void* mats, kq_stream_t stream);
 
+/* kq_expand_blocks_n -- the same for transform blocks of n = 2^log2n elements
+ * ([KQ-sum, Limitations]: 3 log2(n) parameters per block; log2n in 1..7):
+ * K_c = F0 (x) ... (x) F_{log2n-1}, F0 on the most significant index bit.
+ *   params  device fp32 [nt][log2n][3];  mats device [nt][n][n] in out_dtype.
+ *   inverse as for kq_expand_blocks (0: K, 1: K^-1, 2: K^-T).
+ * kq_expand_blocks(p, nb, ...) is kq_expand_blocks_n(p, nb, 5, ...).
+ */
+KQ_API kq_status kq_expand_blocks_n(const float* params, int64_t nt, int log2n, int inverse, kq_dtype out_dtype,
+                             void* mats, kq_stream_t stream);
+
 /* kq_expand_factored -- the same K_b in the form the butterfly kernel applies:
  * F_k = M_k diag(a_k, d_k) with M_k = [[1, b_k/d_k],[c_k/a_k, 1]], so that
  * K_b = (M_0 (x) ... (x) M_4) D_b with D_b = diag_j prod_k (a_k or d_k).
@@ -123,6 +133,17 @@ KQ_API kq_status kq_expand_blocks(const float* params, int64_t nb, int inverse, 
  *             [45..47] zero.  Coefficients are fp64 values rounded once.
  */
 KQ_API kq_status kq_expand_factored(const float* params, int64_t nb, float* factored, kq_stream_t stream);
+
+/* kq_expand_factored_n -- the butterfly form for transform blocks of 32 (log2n 5)
+ * or 64 (log2n 6) elements, one [48]-float record per 32-element block column
+ * (nt * n / 32 records): the five factors acting inside the 32-element block in
+ * [0..9] as above, this block's 32 entries of D in [10..41], max|K| bound, exact-only
+ * flag and absolute allowance in [42..44], and for 64-element blocks c/a, b/d of
+ * F0 (the factor that mixes the two halves) in [45], [46].  factored 16-byte aligned.
+ * kq_expand_factored(p, nb, ...) is kq_expand_factored_n(p, nb, 5, ...).
+ */
+KQ_API kq_status kq_expand_factored_n(const float* params, int64_t nt, int log2n, float* factored,
+                               kq_stream_t stream);
 
 /* ---------------------------------------------------------------- hot path
  *
@@ -149,6 +170,20 @@ KQ_API kq_status kq_expand_factored(const float* params, int64_t nb, float* fact
 KQ_API kq_status kq_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const void* mats,
                       kq_dtype mat_dtype, const float* factored, uint8_t* q, uint8_t* scales,
                       kq_variant variant, kq_scale_layout scale_layout, kq_stream_t stream);
+
+/* kq_quantize_n -- the same with transform blocks of n = 2^log2n elements, log2n 5
+ * or 6 ([KQ-sum, Limitations]); the MX scale blocks stay 32 elements long.
+ *   log2n 5: exactly kq_quantize.
+ *   log2n 6: d % 64 == 0 (else KQ_ERR_SHAPE); mats fp32 [d/64][64][64] from
+ *            kq_expand_blocks_n and factored from kq_expand_factored_n with the same
+ *            params are both required; only the butterfly serves it (KQ_VAR_MMA or
+ *            bf16 matrices: KQ_ERR_UNSUPPORTED).  y_j = fp32(sum over the 64 inputs
+ *            of the block), certified and recomputed exactly like kq_quantize.
+ *   log2n other: KQ_ERR_INVALID_ARG.
+ */
+KQ_API kq_status kq_quantize_n(const void* x, int64_t M, int64_t d, int64_t ldx, int log2n, const void* mats,
+                        kq_dtype mat_dtype, const float* factored, uint8_t* q, uint8_t* scales,
+                        kq_variant variant, kq_scale_layout scale_layout, kq_stream_t stream);
 
 /* kq_dequantize -- inverse of the MXFP4 step [KQ-abs]: yhat_j = E2M1(code_j) *
  * 2^(byte-127) (byte 0xFF gives NaN), and, when inv_mats != NULL, the block

@@ -29,8 +29,9 @@ from ._lib import (  # noqa: F401
 
 class BlockTransform:
     """The per-layer set-up of one KroQuant transform: the LU parameters
-    [d/32, 5, 3] expanded once into the dense block matrices (fp32 and bf16), their
-    inverses and the butterfly (factored) form, then reused for every call."""
+    [d/n, log2 n, 3] (n = 32: five factors per block; n = 64: six) expanded once into
+    the dense block matrices, their inverses and the butterfly (factored) form, then
+    reused for every call."""
 
     def __init__(self, params):
         self.params = params.contiguous()
@@ -54,6 +55,8 @@ class BlockTransform:
         approximate x . w.  Runs the tensor-core variant with the dense K^-T."""
         import torch
 
+        if self.mats.shape[-1] != 32:
+            raise NotImplementedError("the weight side is provided for 32-element transform blocks")
         key = mat_dtype or torch.float32
         if getattr(self, "_inv_t", None) is None or self._inv_t.dtype != key:
             self._inv_t = kq_expand_blocks(self.params, inverse=True, transpose=True, dtype=key)

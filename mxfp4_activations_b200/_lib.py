@@ -32,6 +32,7 @@ STATUS = {
 }
 EXPORTED = (
     "kq_expand_blocks", "kq_expand_factored", "kq_quantize", "kq_dequantize", "kq_ref_smooth_quantize",
+    "kq_expand_blocks_n", "kq_expand_factored_n", "kq_quantize_n",
     "kq_ref_fwht_quantize", "kq_e2m1_pack", "kq_get_device_error", "kq_status_string", "kq_abi_version",
     "kq_last_error",
 )
@@ -62,6 +63,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kq_expand_blocks": [P, I64, I, I, P, P],
         "kq_expand_factored": [P, I64, P, P],
         "kq_quantize": [P, I64, I64, I64, P, I, P, P, P, I, I, P],
+        "kq_expand_blocks_n": [P, I64, I, I, I, P, P],
+        "kq_expand_factored_n": [P, I64, I, P, P],
+        "kq_quantize_n": [P, I64, I64, I64, I, P, I, P, P, P, I, I, P],
         "kq_dequantize": [P, P, I64, I64, P, I, P, I, P],
         "kq_ref_smooth_quantize": [P, I64, I64, I64, P, P, P, P],
         "kq_ref_fwht_quantize": [P, I64, I64, I64, P, P, P],
@@ -121,33 +125,47 @@ def _rows(x: torch.Tensor, name: str = "x"):
 
 # ---------------------------------------------------------------- set-up
 
+def _params_shape(params: torch.Tensor, log2n: int | None):
+    """(transform blocks nt, log2n) of a params tensor [nt, log2n, 3] (a flat
+    tensor is read as 5 factors per block)."""
+    if log2n is None:
+        log2n = params.shape[-2] if params.dim() >= 2 else 5
+    per = 3 * log2n
+    if params.dtype != torch.float32 or params.numel() % per != 0:
+        raise ValueError(f"params must be float32 [nt, {log2n}, 3]")
+    return params.numel() // per, log2n
+
+
 def kq_expand_blocks(params: torch.Tensor, inverse: bool = False, dtype: torch.dtype = torch.float32,
-                     out: torch.Tensor | None = None, transpose: bool = False) -> torch.Tensor:
-    """K_b, K_b^-1 (inverse=True) or the weight-side K_b^-T (inverse=True, transpose=True)."""
+                     out: torch.Tensor | None = None, transpose: bool = False,
+                     log2n: int | None = None) -> torch.Tensor:
+    """K, K^-1 (inverse=True) or the weight-side K^-T (inverse=True, transpose=True)
+    per transform block of n = 2^log2n elements ([nt, n, n]; log2n from params [nt, log2n, 3])."""
     _cuda(params, "params")
     params = params.contiguous()
-    if params.dtype != torch.float32 or params.numel() % 15 != 0:
-        raise ValueError("params must be float32 [nb, 5, 3]")
-    nb = params.numel() // 15
+    nt, log2n = _params_shape(params, log2n)
+    n = 1 << log2n
     if out is None:
-        out = torch.empty((nb, 32, 32), dtype=dtype, device=params.device)
+        out = torch.empty((nt, n, n), dtype=dtype, device=params.device)
     if transpose and not inverse:
         raise ValueError("transpose is provided for the inverse (the weight-side transform) only")
     mode = 2 if transpose else int(bool(inverse))
-    _check("kq_expand_blocks", load().kq_expand_blocks(_ptr(params), nb, mode, _mat_dtype(out),
-                                                         _ptr(out), _stream(params.device)))
+    _check("kq_expand_blocks_n", load().kq_expand_blocks_n(_ptr(params), nt, log2n, mode, _mat_dtype(out),
+                                                             _ptr(out), _stream(params.device)))
     return out
 
 
-def kq_expand_factored(params: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+def kq_expand_factored(params: torch.Tensor, out: torch.Tensor | None = None,
+                       log2n: int | None = None) -> torch.Tensor:
+    """The butterfly form, one [48] record per 32-element block column."""
     _cuda(params, "params")
     params = params.contiguous()
-    if params.dtype != torch.float32 or params.numel() % 15 != 0:
-        raise ValueError("params must be float32 [nb, 5, 3]")
-    nb = params.numel() // 15
+    nt, log2n = _params_shape(params, log2n)
+    nb32 = nt << (log2n - 5) if log2n >= 5 else nt
     if out is None:
-        out = torch.empty((nb, 48), dtype=torch.float32, device=params.device)
-    _check("kq_expand_factored", load().kq_expand_factored(_ptr(params), nb, _ptr(out), _stream(params.device)))
+        out = torch.empty((nb32, 48), dtype=torch.float32, device=params.device)
+    _check("kq_expand_factored_n", load().kq_expand_factored_n(_ptr(params), nt, log2n, _ptr(out),
+                                                                 _stream(params.device)))
     return out
 
 
@@ -170,14 +188,19 @@ def _outputs(x: torch.Tensor, M: int, d: int, q, scales, layout: str = "row"):
 
 def kq_quantize(x: torch.Tensor, mats: torch.Tensor, factored: torch.Tensor | None = None, variant: str = "auto",
                 q: torch.Tensor | None = None, scales: torch.Tensor | None = None, scale_layout: str = "row"):
-    """MXFP4 of x K_b per 32-element block -> (codes uint8 [M, d/2], E8M0 scales: uint8
-    [M, d/32] for scale_layout="row", or the flat 128x4-tiled buffer for "mma")."""
+    """MXFP4 of x K per transform block -> (codes uint8 [M, d/2], E8M0 scales: uint8
+    [M, d/32] for scale_layout="row", or the flat 128x4-tiled buffer for "mma").
+    The transform block size comes from mats ([d/n, n, n], n = 32 or 64)."""
     _cuda(x, "x")
     M, d, ldx = _rows(x)
+    n = mats.shape[-1]
+    if n not in (32, 64):
+        raise ValueError("transform blocks of 32 or 64 elements")
     q, scales = _outputs(x, M, d, q, scales, scale_layout)
-    _check("kq_quantize", load().kq_quantize(_ptr(x), M, d, ldx, _ptr(mats), _mat_dtype(mats), _ptr(factored),
-                                             _ptr(q), _ptr(scales), VARIANTS[variant], SCALE_LAYOUTS[scale_layout],
-                                             _stream(x.device)))
+    _check("kq_quantize_n", load().kq_quantize_n(_ptr(x), M, d, ldx, n.bit_length() - 1, _ptr(mats),
+                                                 _mat_dtype(mats), _ptr(factored), _ptr(q), _ptr(scales),
+                                                 VARIANTS[variant], SCALE_LAYOUTS[scale_layout],
+                                                 _stream(x.device)))
     return q, scales
 
 
@@ -185,6 +208,8 @@ def kq_dequantize(q: torch.Tensor, scales: torch.Tensor, inv_mats: torch.Tensor 
                   out_dtype: torch.dtype = torch.float32, out: torch.Tensor | None = None) -> torch.Tensor:
     _cuda(q, "q")
     M, d = q.shape[0], q.shape[1] * 2
+    if inv_mats is not None and inv_mats.shape[-1] != 32:
+        raise ValueError("kq_dequantize undoes transforms of 32-element blocks only")
     if out is None:
         out = torch.empty((M, d), dtype=out_dtype, device=q.device)
     mdt = _mat_dtype(inv_mats) if inv_mats is not None else KQ_F32

@@ -12,6 +12,8 @@
 
 namespace kq {
 
+constexpr int kMaxFactors = 7;  // blocks of up to 128 elements
+
 // F = L U written as the 2x2 matrix product (row r, column c of F is
 // L[r][0] U[0][c] + L[r][1] U[1][c], zero terms included, so signed zeros
 // follow the same IEEE rules as the product written out).
@@ -57,34 +59,33 @@ __device__ __forceinline__ uint16_t bf16_rne_from_f64(double a) {
   return sign | uint16_t(__float_as_uint(r) >> 16);
 }
 
-// One thread per matrix entry: K[i][j] = F0[i4][j4] (F1[i3][j3] (F2 (F3 F4))),
-// the Kronecker product assembled from the innermost factor outward.  mode 0:
-// K, 1: K^-1 (inverse factors), 2: (K^-1)^T (inverse factors, entry (i, j)
-// taken from (j, i): the transpose of a Kronecker product is the product of the
-// transposes).
-__global__ void expand_kernel(const float* __restrict__ params, int64_t nb, int mode, int out_bf16,
+// One thread per matrix entry of an n x n block matrix, n = 2^log2n:
+// K[i][j] = F0[i_top][j_top] (F1 (... F_{log2n-1})), F0 on the most significant
+// index bit, assembled from the innermost factor outward.  mode 0: K, 1: K^-1
+// (inverse factors), 2: (K^-1)^T (inverse factors, entry (i, j) taken from (j, i):
+// the transpose of a Kronecker product is the product of the transposes).
+__global__ void expand_kernel(const float* __restrict__ params, int64_t nt, int log2n, int mode, int out_bf16,
                               void* __restrict__ mats) {
   const int64_t gid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (gid >= nb * 1024) return;
-  const int64_t b = gid >> 10;
-  const int r = int(gid >> 5) & 31, c = int(gid) & 31;
+  const int n = 1 << log2n;
+  if (gid >= (nt << (2 * log2n))) return;
+  const int64_t b = gid >> (2 * log2n);
+  const int r = int(gid >> log2n) & (n - 1), c = int(gid) & (n - 1);
   const int i = mode == 2 ? c : r, j = mode == 2 ? r : c;
   const bool inverse = mode != 0;
-  double F[5][4];
+  double F[kMaxFactors][4];
   bool singular = false;
-#pragma unroll
-  for (int k = 0; k < 5; k++) {
-    const float* prm = params + b * 15 + 3 * k;
+  for (int k = 0; k < log2n; k++) {
+    const float* prm = params + b * 3 * log2n + 3 * k;
     if (prm[1] == 0.0f) singular = true;
     if (inverse)
       lu_factor_inverse(prm, F[k]);
     else
       lu_factor(prm, F[k]);
   }
-  double acc = F[4][2 * (i & 1) + (j & 1)];
-#pragma unroll
-  for (int k = 3; k >= 0; k--) {
-    const int bi = (i >> (4 - k)) & 1, bj = (j >> (4 - k)) & 1;
+  double acc = F[log2n - 1][2 * (i & 1) + (j & 1)];
+  for (int k = log2n - 2; k >= 0; k--) {
+    const int bi = (i >> (log2n - 1 - k)) & 1, bj = (j >> (log2n - 1 - k)) & 1;
     acc = __dmul_rn(F[k][2 * bi + bj], acc);
   }
   if (singular && i == 0 && j == 0) record_error(kDevErrSingular);
@@ -94,19 +95,30 @@ __global__ void expand_kernel(const float* __restrict__ params, int64_t nb, int 
     static_cast<float*>(mats)[gid] = __double2float_rn(acc);
 }
 
-// One thread per block: the butterfly form F_k = M_k diag(a_k, d_k).
-__global__ void expand_factored_kernel(const float* __restrict__ params, int64_t nb, float* __restrict__ out) {
+// One thread per 32-element block column: the butterfly form F_k = M_k diag(a_k, d_k)
+// of its transform block of n = 2^log2n elements (log2n 5 or 6).  Record [48]:
+//   [0..4]  c_k/a_k and [5..9] b_k/d_k of the five factors acting inside the
+//           32-element block (factors log2n-5 .. log2n-1)
+//   [10..41] D_j for this block's 32 outputs
+//   [42]    upper bound of max|K|   [43] 1 if only the exact path may be used
+//   [44]    absolute allowance      [45], [46] c/a, b/d of factor 0 when log2n = 6
+//           (it mixes the two 32-element halves of the 64-element block)
+__global__ void expand_factored_kernel(const float* __restrict__ params, int64_t nb32, int log2n,
+                                       float* __restrict__ out) {
   const int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (b >= nb) return;
-  double a[5], d[5];
+  if (b >= nb32) return;
+  const int64_t c = b >> (log2n - 5);            // transform block
+  const int half = int(b & ((1 << (log2n - 5)) - 1));  // which 32 outputs of it
+  const int inner0 = log2n - 5;                   // first factor acting inside the 32-block
+  double a[kMaxFactors], d[kMaxFactors];
   double kmax = 1.0, gain = 1.0;
   bool exact_only = false;
   float* o = out + b * kFactored;
-#pragma unroll
-  for (int k = 0; k < 5; k++) {
-    const float* prm = params + b * 15 + 3 * k;
+  o[45] = o[46] = o[47] = 0.0f;
+  for (int k = 0; k < log2n; k++) {
+    const float* prm = params + c * 3 * log2n + 3 * k;
     if (prm[1] == 0.0f) {
-      record_error(kDevErrSingular);
+      if (half == 0) record_error(kDevErrSingular);
       exact_only = true;
     }
     double F[4];
@@ -118,32 +130,36 @@ __global__ void expand_factored_kernel(const float* __restrict__ params, int64_t
     const float lam32 = __double2float_rn(lam), bet32 = __double2float_rn(bet);
     // ratios must be finite and moderate for the fp32 butterfly to be usable
     if (!(fabsf(lam32) <= 1.8446744e19f) || !(fabsf(bet32) <= 1.8446744e19f)) exact_only = true;
-    o[k] = lam32;
-    o[5 + k] = bet32;
+    if (k >= inner0) {
+      o[k - inner0] = lam32;
+      o[5 + k - inner0] = bet32;
+    } else {
+      o[45] = lam32;
+      o[46] = bet32;
+    }
     const double mk = fmax(fmax(fabs(F[0]), fabs(F[1])), fmax(fabs(F[2]), fabs(F[3])));
     kmax = __dmul_rn(kmax, mk);
     gain = __dmul_rn(gain, 1.0 + fmax(fabs(double(lam32)), fabs(double(bet32))));
   }
   double dmax = 0.0;
   for (int j = 0; j < 32; j++) {
+    const int jj = half * 32 + j;  // output index inside the transform block
     double dj = 1.0;
-#pragma unroll
-    for (int k = 0; k < 5; k++) dj = __dmul_rn(dj, ((j >> (4 - k)) & 1) ? d[k] : a[k]);
+    for (int k = 0; k < log2n; k++) dj = __dmul_rn(dj, ((jj >> (log2n - 1 - k)) & 1) ? d[k] : a[k]);
     const float dj32 = __double2float_rn(dj);
     if (!(fabsf(dj32) <= 3.0e38f) || dj32 == 0.0f) exact_only = true;
     o[10 + j] = dj32;
     dmax = fmax(dmax, fabs(double(dj32)));
   }
-  // upper bound of max|K| (fp64 product error is far below the 2^-20 margin)
+  // upper bound of max|K| (fp64 product error is far below the allowance's margin)
   const float km = __fmul_ru(__double2float_ru(kmax), 1.00000095367431640625f);
   if (!(km <= 1.0e30f)) exact_only = true;
   o[42] = km;
   o[43] = exact_only ? 1.0f : 0.0f;
   // absolute error of results that fall in the fp32 subnormal range: each of the
-  // 6 roundings on an output's path adds at most 2^-150, amplified by at most
-  // max|D| * prod_k (1 + max(|c/a|, |b/d|)); 2^-145 leaves a margin.
+  // (log2n + 1 <= 7) roundings on an output's path adds at most 2^-150, amplified by
+  // at most max|D| * prod_k (1 + max(|c/a|, |b/d|)); 2^-145 leaves a margin.
   o[44] = __fmul_ru(__double2float_ru(__dmul_rn(dmax, gain)), 2.2420775429197073e-44f);
-  o[45] = o[46] = o[47] = 0.0f;
 }
 
 }  // namespace kq

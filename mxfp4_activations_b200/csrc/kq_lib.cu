@@ -94,7 +94,7 @@ int64_t row_stride(int64_t ncol, int64_t nrt, int sms, int per_sm) {
   return gy;
 }
 
-template <int MODE, int TILED>
+template <int MODE, int TILED, int NT = 32>
 kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const float* mats, const float* factored,
                        const float* inv_s, uint8_t* q, uint8_t* scales, cudaStream_t stream) {
   const DeviceInfo* dev = device_info();
@@ -116,7 +116,7 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cuda_fail("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
 
-  auto kern = kq::quant_kernel<MODE, TILED>;
+  auto kern = kq::quant_kernel<MODE, TILED, NT>;
   static std::atomic<int> attr_set[kMaxDevices];
   int devid = 0;
   cudaGetDevice(&devid);
@@ -256,44 +256,67 @@ const char* kq_status_string(kq_status s) {
   return "unknown kq_status";
 }
 
-kq_status kq_expand_blocks(const float* params, int64_t nb, int inverse, kq_dtype out_dtype, void* mats,
-                           kq_stream_t stream) {
-  if (nb < 0 || (out_dtype != KQ_F32 && out_dtype != KQ_BF16)) return KQ_ERR_INVALID_ARG;
-  if (inverse < 0 || inverse > 2) return KQ_ERR_INVALID_ARG;
-  if (nb == 0) return KQ_OK;
+kq_status kq_expand_blocks_n(const float* params, int64_t nt, int log2n, int inverse, kq_dtype out_dtype,
+                             void* mats, kq_stream_t stream) {
+  if (nt < 0 || (out_dtype != KQ_F32 && out_dtype != KQ_BF16)) return KQ_ERR_INVALID_ARG;
+  if (inverse < 0 || inverse > 2 || log2n < 1 || log2n > kq::kMaxFactors) return KQ_ERR_INVALID_ARG;
+  if (nt == 0) return KQ_OK;
   if (params == nullptr || mats == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(params, 4) || !aligned(mats, 4)) return KQ_ERR_ALIGN;
-  if (nb > (int64_t(1) << 30)) return KQ_ERR_SHAPE;
-  const int64_t n = nb * 1024;
-  kq::expand_kernel<<<unsigned((n + 255) / 256), 256, 0, as_cuda(stream)>>>(params, nb, inverse,
+  if (nt > (int64_t(INT32_MAX) * 256) >> (2 * log2n)) return KQ_ERR_SHAPE;  // grid of 256-thread blocks
+  const int64_t n = nt << (2 * log2n);
+  kq::expand_kernel<<<unsigned((n + 255) / 256), 256, 0, as_cuda(stream)>>>(params, nt, log2n, inverse,
                                                                            out_dtype == KQ_BF16 ? 1 : 0, mats);
   return launch_status("expand_kernel launch");
 }
 
-kq_status kq_expand_factored(const float* params, int64_t nb, float* factored, kq_stream_t stream) {
-  if (nb < 0) return KQ_ERR_INVALID_ARG;
-  if (nb == 0) return KQ_OK;
+kq_status kq_expand_blocks(const float* params, int64_t nb, int inverse, kq_dtype out_dtype, void* mats,
+                           kq_stream_t stream) {
+  return kq_expand_blocks_n(params, nb, 5, inverse, out_dtype, mats, stream);
+}
+
+kq_status kq_expand_factored_n(const float* params, int64_t nt, int log2n, float* factored, kq_stream_t stream) {
+  if (nt < 0 || (log2n != 5 && log2n != 6)) return KQ_ERR_INVALID_ARG;
+  if (nt == 0) return KQ_OK;
   if (params == nullptr || factored == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(params, 4) || !aligned(factored, 16)) return KQ_ERR_ALIGN;
-  if (nb > (int64_t(1) << 30)) return KQ_ERR_SHAPE;
-  kq::expand_factored_kernel<<<unsigned((nb + 127) / 128), 128, 0, as_cuda(stream)>>>(params, nb, factored);
+  if (nt > (int64_t(1) << 29)) return KQ_ERR_SHAPE;
+  const int64_t nb32 = nt << (log2n - 5);
+  kq::expand_factored_kernel<<<unsigned((nb32 + 127) / 128), 128, 0, as_cuda(stream)>>>(params, nb32, log2n,
+                                                                                        factored);
   return launch_status("expand_factored_kernel launch");
 }
 
-kq_status kq_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const void* mats, kq_dtype mat_dtype,
-                      const float* factored, uint8_t* q, uint8_t* scales, kq_variant variant,
-                      kq_scale_layout scale_layout, kq_stream_t stream) {
+kq_status kq_expand_factored(const float* params, int64_t nb, float* factored, kq_stream_t stream) {
+  return kq_expand_factored_n(params, nb, 5, factored, stream);
+}
+
+kq_status kq_quantize_n(const void* x, int64_t M, int64_t d, int64_t ldx, int log2n, const void* mats,
+                        kq_dtype mat_dtype, const float* factored, uint8_t* q, uint8_t* scales, kq_variant variant,
+                        kq_scale_layout scale_layout, kq_stream_t stream) {
   if (variant != KQ_VAR_AUTO && variant != KQ_VAR_MMA && variant != KQ_VAR_BUTTERFLY) return KQ_ERR_INVALID_ARG;
   if (scale_layout != KQ_SCALES_ROW_MAJOR && scale_layout != KQ_SCALES_MMA_TILED) return KQ_ERR_INVALID_ARG;
+  if (log2n != 5 && log2n != 6) return KQ_ERR_INVALID_ARG;
   const int sf_tiled = scale_layout == KQ_SCALES_MMA_TILED ? 1 : 0;
   if (mat_dtype != KQ_F32 && mat_dtype != KQ_BF16) return KQ_ERR_INVALID_ARG;
   kq_status st = check_x(x, M, d, ldx);
   if (st != KQ_OK) return st;
+  if (log2n == 6 && d % 64 != 0) return KQ_ERR_SHAPE;
   if (M == 0 || d == 0) return KQ_OK;
   st = check_out(q, scales);
   if (st != KQ_OK) return st;
   if (mats == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(mats, 16)) return KQ_ERR_ALIGN;
+  const float* m32 = static_cast<const float*>(mats);
+  if (log2n == 6) {
+    // 64-element blocks: the butterfly only (fp32 matrices and the factored form)
+    if (variant == KQ_VAR_MMA || mat_dtype == KQ_BF16) return KQ_ERR_UNSUPPORTED;
+    if (factored == nullptr) return KQ_ERR_INVALID_ARG;
+    if (!aligned(factored, 16)) return KQ_ERR_ALIGN;
+    return sf_tiled
+               ? launch_quant<kq::MODE_KRON, 1, 64>(x, M, d, ldx, m32, factored, nullptr, q, scales, as_cuda(stream))
+               : launch_quant<kq::MODE_KRON, 0, 64>(x, M, d, ldx, m32, factored, nullptr, q, scales, as_cuda(stream));
+  }
   // bf16 matrices are only served by the tensor-core variant; AUTO picks the
   // butterfly for fp32 matrices when the factored form is given
   const bool use_mma = variant == KQ_VAR_MMA || mat_dtype == KQ_BF16 ||
@@ -303,9 +326,14 @@ kq_status kq_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const vo
     return launch_quant_mma(x, M, d, ldx, mats, mat_dtype == KQ_BF16, q, scales, sf_tiled, as_cuda(stream));
   if (factored == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(factored, 16)) return KQ_ERR_ALIGN;
-  const float* m32 = static_cast<const float*>(mats);
-  return sf_tiled ? launch_quant<kq::MODE_KRON, 1>(x, M, d, ldx, m32, factored, nullptr, q, scales, as_cuda(stream))
-                  : launch_quant<kq::MODE_KRON, 0>(x, M, d, ldx, m32, factored, nullptr, q, scales, as_cuda(stream));
+  return sf_tiled ? launch_quant<kq::MODE_KRON, 1, 32>(x, M, d, ldx, m32, factored, nullptr, q, scales, as_cuda(stream))
+                  : launch_quant<kq::MODE_KRON, 0, 32>(x, M, d, ldx, m32, factored, nullptr, q, scales, as_cuda(stream));
+}
+
+kq_status kq_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const void* mats, kq_dtype mat_dtype,
+                      const float* factored, uint8_t* q, uint8_t* scales, kq_variant variant,
+                      kq_scale_layout scale_layout, kq_stream_t stream) {
+  return kq_quantize_n(x, M, d, ldx, 5, mats, mat_dtype, factored, q, scales, variant, scale_layout, stream);
 }
 
 kq_status kq_ref_smooth_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const float* inv_s,

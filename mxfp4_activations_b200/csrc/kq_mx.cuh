@@ -31,13 +31,6 @@ __device__ __forceinline__ int64_t scale_index(int64_t row, int b, int nb, int t
 // Where the exact path reads K[i][j] from.
 enum KSource { KSRC_F32 = 0, KSRC_BF16 = 1, KSRC_FWHT = 2 };
 
-template <int KSRC>
-__device__ __forceinline__ float k_entry(const void* __restrict__ Kb, int i, int j) {
-  if (KSRC == KSRC_FWHT) return (__popc(i & j) & 1) ? -kFwhtC : kFwhtC;
-  if (KSRC == KSRC_BF16) return bf16_to_f32(__ldg(static_cast<const unsigned short*>(Kb) + i * kBlock + j));
-  return __ldg(static_cast<const float*>(Kb) + i * kBlock + j);
-}
-
 // max_j |y_j| with NaN propagation: for each residue r = j mod 4, the eight
 // elements r, r+4, ..., r+28 through three-input maxima, then the four results.
 __device__ __forceinline__ float block_amax(const float (&y)[kBlock]) {
@@ -62,41 +55,52 @@ __device__ __forceinline__ uint32_t codes8(const uint64_t* Y) {
 
 // ---------------------------------------------------------------- exact fp64 path
 //
-// Only elements (or blocks) whose code (or scale) the fp32 bound cannot
-// certify come here.  Every load is issued before the arithmetic so that one
-// L2 round trip serves a whole recomputation.
+// Only blocks whose scale or some code the fp32 bound cannot certify come here.
+// Every load of a chunk is issued before its arithmetic, so that one L2 round
+// trip serves 32 rows of the recomputation.
 
-// Exact recomputation of one whole block by the whole warp: lane j computes
-// y32_j = fp32( sum_i x_i K[i][j] ) in fp64, summing in increasing i from +0
-// (each product of a bf16 and an fp32 or bf16 value is exact in fp64).  Row i of K is
-// one coalesced 128-byte load across the warp and all 32 rows are in flight
-// together; x is a broadcast load.  The block's scale then comes from the
-// exact maximum and every code from the exact value, and lane `owner` stores
-// them.  Must be called by all 32 lanes with the same arguments (taken from
-// the owner lane).
+// K[i][j] of a block matrix whose rows are `ld` entries apart.
 template <int KSRC>
+__device__ __forceinline__ float k_entry(const void* __restrict__ Kb, int i, int j, int ld) {
+  if (KSRC == KSRC_FWHT) return (__popc(i & j) & 1) ? -kFwhtC : kFwhtC;
+  if (KSRC == KSRC_BF16) return bf16_to_f32(__ldg(static_cast<const unsigned short*>(Kb) + i * ld + j));
+  return __ldg(static_cast<const float*>(Kb) + i * ld + j);
+}
+
+// Exact recomputation of one 32-element output block by the whole warp: lane j
+// computes y32_j = fp32( sum_{i < NT} x_i K[i][j] ) in fp64, summing in
+// increasing i from +0 (each product of a bf16 and an fp32 or bf16 value is
+// exact in fp64).  xb: the NT inputs of the transform block; Kb: column 0 of this
+// block's 32 outputs in the NT x NT matrix (rows NT entries apart).  Rows of K are
+// loaded 32 at a time, each row one coalesced 128-byte load across the warp; x is
+// a broadcast load.  The block's scale then comes from the exact maximum and
+// every code from the exact value, and lane `owner` stores them.  Must be called
+// by all 32 lanes with the same arguments (taken from the owner lane).
+template <int KSRC, int NT>
 __device__ __noinline__ void exact_block_warp(const uint16_t* __restrict__ xb, const void* __restrict__ Kb,
                                               uint8_t* __restrict__ qb, uint8_t* __restrict__ sb, int owner) {
   const int lane = threadIdx.x & 31;
-  float kc[kBlock];
-#pragma unroll
-  for (int i = 0; i < kBlock; i++)
-    kc[i] = k_entry<KSRC>(Kb, i, lane);
-  const uint4* px = reinterpret_cast<const uint4*>(xb);
-  uint32_t xw[16];
-#pragma unroll
-  for (int k = 0; k < 4; k++) {
-    const uint4 v = __ldg(px + k);
-    xw[4 * k] = v.x;
-    xw[4 * k + 1] = v.y;
-    xw[4 * k + 2] = v.z;
-    xw[4 * k + 3] = v.w;
-  }
   double acc = 0.0;
+#pragma unroll 1
+  for (int i0 = 0; i0 < NT; i0 += kBlock) {
+    float kc[kBlock];
 #pragma unroll
-  for (int i = 0; i < kBlock; i++) {
-    const float xi = (i & 1) ? bf16hi(xw[i >> 1]) : bf16lo(xw[i >> 1]);
-    acc = __dadd_rn(acc, __dmul_rn(double(xi), double(kc[i])));
+    for (int i = 0; i < kBlock; i++) kc[i] = k_entry<KSRC>(Kb, i0 + i, lane, NT);
+    const uint4* px = reinterpret_cast<const uint4*>(xb + i0);
+    uint32_t xw[16];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      const uint4 v = __ldg(px + k);
+      xw[4 * k] = v.x;
+      xw[4 * k + 1] = v.y;
+      xw[4 * k + 2] = v.z;
+      xw[4 * k + 3] = v.w;
+    }
+#pragma unroll
+    for (int i = 0; i < kBlock; i++) {
+      const float xi = (i & 1) ? bf16hi(xw[i >> 1]) : bf16lo(xw[i >> 1]);
+      acc = __dadd_rn(acc, __dmul_rn(double(xi), double(kc[i])));
+    }
   }
   const float y = __double2float_rn(acc);
   const bool finite = __all_sync(0xFFFFFFFFu, isfinite(y));
@@ -124,7 +128,7 @@ __device__ __noinline__ void exact_block_warp(const uint16_t* __restrict__ xb, c
 
 // Every lane whose block needs the exact path hands it to the whole warp, one
 // block at a time.  Called by all 32 lanes.
-template <int KSRC>
+template <int KSRC, int NT = kBlock>
 __device__ __forceinline__ void warp_exact_pass(bool need, const uint16_t* xb, const void* Kb, uint8_t* qb,
                                                 uint8_t* sb) {
   uint32_t pending = __ballot_sync(0xFFFFFFFFu, need);
@@ -137,7 +141,7 @@ __device__ __forceinline__ void warp_exact_pass(bool need, const uint16_t* xb, c
         __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(Kb), src));
     uint8_t* qs = reinterpret_cast<uint8_t*>(__shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(qb), src));
     uint8_t* ss = reinterpret_cast<uint8_t*>(__shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(sb), src));
-    exact_block_warp<KSRC>(xs, ks, qs, ss, src);
+    exact_block_warp<KSRC, NT>(xs, ks, qs, ss, src);
   }
 }
 

@@ -51,6 +51,7 @@ namespace kq {
 enum Mode { MODE_KRON = 0, MODE_FWHT = 1, MODE_SMOOTH = 2 };
 
 constexpr float kKronErrC = 9.5367431640625e-07f;   // 2^-20 = 16 u (14 u needed, see below)
+constexpr float kKronErrC64 = 1.9073486328125e-06f; // 2^-19 = 32 u for 64-element blocks (16 u needed)
 constexpr float kFwhtErrC = 4.76837158203125e-07f;  // 2^-21 = 8 u (7 u needed)
 constexpr float kErrAbs = 7.174648137343064e-43f;   // 2^-140: FWHT subnormal-range slack
 
@@ -66,6 +67,8 @@ constexpr int kQStages = 4;
 //   [16 .. 47]    D_0 .. D_31 (SMOOTH: the 32 per-channel factors)
 //   [48 .. 51]    lam and bet of factor 4 (index bit 0), C * max|K| (+inf: exact path
 //                 only), absolute allowance
+//   [52 .. 53]    lam and bet of the factor that mixes the two 32-element halves of a
+//                 64-element transform block (64-element blocks only)
 constexpr int kQCoef = 56;
 
 struct QuantParams {
@@ -84,7 +87,7 @@ struct QuantParams {
 
 // Entry f of the coefficient record of block column b (fp32 bits as read by
 // the consumer warps).
-template <int MODE>
+template <int MODE, int NT>
 __device__ __forceinline__ float coef_entry(const QuantParams& p, int b, int f) {
   if (MODE == MODE_KRON) {
     const float* fb = p.factored + int64_t(b) * kFactored;
@@ -95,8 +98,12 @@ __device__ __forceinline__ float coef_entry(const QuantParams& p, int b, int f) 
     if (f < 48) return __ldg(fb + 10 + (f - 16));  // D
     if (f == 48) return __ldg(fb + 4);
     if (f == 49) return __ldg(fb + 9);
-    if (f == 50) return __ldg(fb + 43) != 0.0f ? __int_as_float(0x7F800000) : __fmul_ru(kKronErrC, __ldg(fb + 42));
+    if (f == 50)
+      return __ldg(fb + 43) != 0.0f ? __int_as_float(0x7F800000)
+                                    : __fmul_ru(NT == 64 ? kKronErrC64 : kKronErrC, __ldg(fb + 42));
     if (f == 51) return __ldg(fb + 44);
+    if (NT == 64 && f == 52) return __ldg(fb + 45);
+    if (NT == 64 && f == 53) return __ldg(fb + 46);
     return 0.0f;
   }
   if (MODE == MODE_SMOOTH) return (f >= 16 && f < 48) ? __ldg(p.inv_s + int64_t(b) * kBlock + (f - 16)) : 0.0f;
@@ -105,10 +112,12 @@ __device__ __forceinline__ float coef_entry(const QuantParams& p, int b, int f) 
 
 // ---------------------------------------------------------------- one block of one row
 //
-// cf: shared-memory address of this block column's coefficient record.
-template <int MODE>
+// cf: shared-memory address of this block column's coefficient record.  NT = 64:
+// the block is one half of a 64-element transform block whose other half is held
+// by lane ^ 8 (same row, neighbouring column); `upper` marks the second half.
+template <int MODE, int NT>
 __device__ __forceinline__ void quant_block(uint32_t cf, const uint4 (&xr)[4], bool act, uint8_t* qb, uint8_t* sb,
-                                            const uint16_t* xb, const float* Kb) {
+                                            const uint16_t* xb, const float* Kb, bool upper) {
   float x[kBlock];
 #pragma unroll
   for (int k = 0; k < 4; k++) {
@@ -151,7 +160,9 @@ __device__ __forceinline__ void quant_block(uint32_t cf, const uint4 (&xr)[4], b
   float l1p[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
   for (int j = 0; j < kBlock; j++) l1p[j & 3] = __fadd_ru(l1p[j & 3], fabsf(x[j]));
-  const float l1 = __fadd_ru(__fadd_ru(l1p[0], l1p[1]), __fadd_ru(l1p[2], l1p[3]));
+  float l1 = __fadd_ru(__fadd_ru(l1p[0], l1p[1]), __fadd_ru(l1p[2], l1p[3]));
+  // every output of a 64-element block depends on all 64 inputs
+  if (NT == 64) l1 = __fadd_ru(l1, __shfl_xor_sync(0xFFFFFFFFu, l1, 8));
 
   float cfac, eabs;
   // stage on index bit 0 (factor 4), scalar: the pair partners share a register pair
@@ -204,6 +215,20 @@ __device__ __forceinline__ void quant_block(uint32_t cf, const uint4 (&xr)[4], b
       }
     }
   }
+  if (NT == 64) {
+    // factor 0 of a 64-element block: out_lo = y_lo + lam y_hi, out_hi = y_hi + bet y_lo,
+    // element by element between the two halves (held by lanes l and l ^ 8)
+    const uint4 cx = lds128(cf + 208);
+    const float cc = upper ? __uint_as_float(cx.y) : __uint_as_float(cx.x);
+    const uint64_t C2 = pk2(cc, cc);
+#pragma unroll
+    for (int m = 0; m < 16; m++) {
+      float lo, hi;
+      upk2(Y[m], lo, hi);
+      const float plo = __shfl_xor_sync(0xFFFFFFFFu, lo, 8), phi = __shfl_xor_sync(0xFFFFFFFFu, hi, 8);
+      Y[m] = fma2_rn(C2, pk2(plo, phi), Y[m]);
+    }
+  }
   // diagonal: D_j (FWHT: +-2^-2.5 with the sign of (-1)^popcount(j))
   if (MODE == MODE_FWHT) {
 #pragma unroll
@@ -227,14 +252,15 @@ __device__ __forceinline__ void quant_block(uint32_t cf, const uint4 (&xr)[4], b
   // l1 is an upward-rounded fp32 sum of |x| without flushing: 0 exactly when all inputs are +-0
   // cfac = +inf marks a column whose butterfly form is unusable: every block exact
   certify_store(Y, amax, l1, l1 == 0.0f, cfac, eabs, !(cfac <= FLT_MAX), act, qb, sb,
-                [&](bool need) { warp_exact_pass<KSRC>(need, xb, Kb, qb, sb); });
+                [&](bool need) { warp_exact_pass<KSRC, NT>(need, xb, Kb, qb, sb); });
 }
 
 // ---------------------------------------------------------------- kernel
 
 // TILED: scales in the 128 x 4 tiled layout of block-scaled GEMMs (a template
-// parameter, so the row-major store costs nothing extra).
-template <int MODE, int TILED>
+// parameter, so the row-major store costs nothing extra).  NT: transform block of
+// 32 or 64 elements (KRON only; 64 needs an even number of block columns).
+template <int MODE, int TILED, int NT>
 __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -287,7 +313,7 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_consta
     for (int i = 0; i < kPer; i++) {
       const int e = t + i * kQConsWarps * 32;
       const int c = e / kQCoef;
-      v[i] = (e < kN && col0 + c < p.nb) ? coef_entry<MODE>(p, col0 + c, e - c * kQCoef) : 0.0f;
+      v[i] = (e < kN && col0 + c < p.nb) ? coef_entry<MODE, NT>(p, col0 + c, e - c * kQCoef) : 0.0f;
     }
 #pragma unroll
     for (int i = 0; i < kPer; i++) {
@@ -306,7 +332,13 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_consta
   const uint32_t xoff = uint32_t(cl * kQRows + rl) * 64u;
   const int sw = (rl >> 1) & 3;
   const uint32_t sbase = smem_addr(base);
-  const float* Kb = (MODE == MODE_KRON) ? p.mats + int64_t(bc) * kBlock * kBlock : nullptr;
+  // exact path: this block's columns of its transform matrix ([nt][NT][NT]), and
+  // the transform block's first input
+  const float* Kb = (MODE == MODE_KRON)
+                        ? p.mats + int64_t(bc / (NT / kBlock)) * NT * NT + (bc % (NT / kBlock)) * kBlock
+                        : nullptr;
+  const int bx = bc - bc % (NT / kBlock);  // first block column of the transform block
+  const bool upper = (bc % (NT / kBlock)) != 0;
   // per-tile pointer steps: gridDim.y row tiles of kQRows rows
   const int64_t row_step = int64_t(gridDim.y) * kQRows;
   int64_t row = int64_t(blockIdx.y) * kQRows + rl;
@@ -324,9 +356,9 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_consta
     const int64_t rowc = act ? row : 0;
     uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16;
     uint8_t* sb = p.scales + scale_index(rowc, bc, p.nb, TILED);
-    const uint16_t* xb = p.x + rowc * p.ldx + int64_t(bc) * kBlock;
+    const uint16_t* xb = p.x + rowc * p.ldx + int64_t(bx) * kBlock;
     // every lane takes part (the exact path is warp-cooperative); only real blocks store
-    quant_block<MODE>(cf, xr, act, qb, sb, xb, Kb);
+    quant_block<MODE, NT>(cf, xr, act, qb, sb, xb, Kb, upper);
   }
 }
 

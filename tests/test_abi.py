@@ -69,6 +69,15 @@ def test_quantize_argument_errors_return_before_launch(lib):
     assert q(lib, mats=0) == 1
     assert q(lib, var=9) == 1                 # bad variant enum
     assert q(lib, layout=2) == 1              # bad scale layout enum
+    qn = lambda **kw: lib.kq_quantize_n(P(16 * 1024), kw.get("M", 4), kw.get("d", 128), kw.get("ldx", 128),
+                                        kw.get("log2n", 6), P(16 * 2048), kw.get("dtype", 0),
+                                        P(16 * 4096) if kw.get("fac", 1) else None, P(16 * 8192), P(16 * 9000),
+                                        kw.get("var", 2), 0, None)
+    assert qn(log2n=7) == 1                   # 32- or 64-element transform blocks
+    assert qn(d=96, ldx=96) == 2              # 64-element blocks need d % 64 == 0
+    assert qn(var=1) == 5                     # no tensor-core variant for 64-element blocks
+    assert qn(dtype=1) == 5                   # nor bf16 matrices
+    assert qn(fac=0) == 1                     # the butterfly needs the factored form
     assert q(lib, dtype=7) == 1               # bad dtype enum
     assert q(lib, fac=0) == 1                 # butterfly needs the factored form
     assert q(lib, dtype=1) == 5               # bf16 matrices need the tensor-core variant
@@ -81,6 +90,11 @@ def test_other_entry_points_argument_errors(lib):
     assert lib.kq_expand_blocks(P(64), -1, 0, 0, P(64), None) == 1
     assert lib.kq_expand_blocks(P(64), 4, 0, 5, P(64), None) == 1
     assert lib.kq_expand_blocks(P(64), 4, 3, 0, P(64), None) == 1     # mode: 0 K, 1 K^-1, 2 K^-T
+    assert lib.kq_expand_blocks_n(P(64), 4, 8, 0, 0, P(64), None) == 1  # at most 2^7-element blocks
+    assert lib.kq_expand_blocks_n(P(64), 4, 0, 0, 0, P(64), None) == 1
+    assert lib.kq_expand_blocks_n(P(64), 0, 6, 0, 0, P(64), None) == 0
+    assert lib.kq_expand_factored_n(P(64), 4, 7, P(64), None) == 1     # butterfly form for 32 or 64
+    assert lib.kq_expand_factored_n(P(64), 4, 6, P(72), None) == 3
     assert lib.kq_expand_blocks(P(64), 4, -1, 0, P(64), None) == 1
     assert lib.kq_expand_blocks(P(64), 0, 0, 0, P(64), None) == 0
     assert lib.kq_expand_factored(P(64), 4, P(68), None) == 3

@@ -467,3 +467,109 @@ def test_dequantize_inverse_within_fp32_bound(kq, orc):
 
 def test_no_device_error_after_suite(kq):
     assert kq.kq_get_device_error(clear=True) == 0
+
+
+# ---------------------------------------------------------------- 64-element transform blocks
+
+@pytest.mark.parametrize("log2n", [4, 6, 7])
+@pytest.mark.parametrize("mode", ["K", "K^-1", "K^-T"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_expand_n_bit_exact(kq, orc, log2n, mode, dtype):
+    params = inputs.lu_params(5, seed=80 + log2n, noise=0.3, factors=log2n)
+    params[1] = inputs.hadamard_params(1, factors=log2n)[0]
+    inverse, transpose = mode != "K", mode == "K^-T"
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    got = host(kq.kq_expand_blocks(dev_f32(params), inverse=inverse, dtype=tdt, transpose=transpose))
+    want = orc.expand_n(params, dtype=orc.F32 if dtype == "f32" else orc.BF16, inverse=inverse)
+    if transpose:
+        want = np.ascontiguousarray(np.swapaxes(want, 1, 2))
+    if dtype == "f32":
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    else:
+        assert np.array_equal(got, want)
+
+
+def test_expand_factored_n64_reproduces_matrix(kq, orc):
+    params = inputs.lu_params(6, seed=90, noise=0.3, factors=6)
+    params[5, 3] = (-1.0, 1.0, 1.0)  # d = 0 in one factor: no butterfly form
+    fac = host(kq.kq_expand_factored(dev_f32(params))).astype(np.float64)
+    assert fac.shape == (12, 48)
+    K = orc.expand_n_f64(params)
+    for c in range(6):
+        lo, hi = fac[2 * c], fac[2 * c + 1]
+        assert lo[43] == hi[43] and lo[42] == hi[42] and lo[42] >= np.abs(K[c]).max()
+        if lo[43]:
+            continue
+        assert np.array_equal(lo[:10], hi[:10]) and np.array_equal(lo[45:47], hi[45:47])
+        Mk = np.array([[1.0, lo[46]], [lo[45], 1.0]])
+        for k in range(5):
+            Mk = np.kron(Mk, np.array([[1.0, lo[5 + k]], [lo[k], 1.0]]))
+        Kf = Mk * np.concatenate([lo[10:42], hi[10:42]])[None, :]
+        assert np.all(np.abs(Kf - K[c]) <= 1e-6 * np.abs(K[c]) + 1e-30)
+    assert fac[10, 43] == 1.0 and fac[11, 43] == 1.0
+
+
+def gpu_quantize_n64(kq, x_bits, params, x_dev=None, scale_layout="row"):
+    p = dev_f32(params)
+    mats = kq.kq_expand_blocks(p)
+    fac = kq.kq_expand_factored(p)
+    x = dev_bf16(x_bits) if x_dev is None else x_dev
+    qd, sd = kq.kq_quantize(x, mats, fac, variant="butterfly", scale_layout=scale_layout)
+    return host(qd), host(sd)
+
+
+@pytest.mark.parametrize("M,d", [(1, 64), (3, 128), (65, 1152), (130, 2240), (33, 12288), (257, 3072), (300, 4608)])
+def test_quantize_n64_ragged_shapes(kq, orc, M, d):
+    x = inputs.activations(M, d, "t3", seed=[M, d, 64], outlier_frac=0.01, outlier_scale=(20.0, 100.0))
+    params = inputs.lu_params(d // 64, seed=[M, d, 65], factors=6)
+    q, s = gpu_quantize_n64(kq, x, params)
+    K = orc.expand_n(params)
+    qr, sr = orc.quantize_n(x, K)
+    check(q, s, qr, sr, orc.transform_n(x, K))
+
+
+def test_quantize_n64_flux_shape(kq, orc):
+    x, _ = inputs.config_case("flux", 3072)
+    params = inputs.lu_params(3072 // 64, seed=66, factors=6)
+    q, s = gpu_quantize_n64(kq, x, params)
+    qr, sr = orc.quantize_n(x, orc.expand_n(params))
+    check(q, s, qr, sr)
+
+
+def test_quantize_n64_degenerate_and_singular(kq, orc):
+    rng = np.random.default_rng(67)
+    M, d = 24, 384
+    a = rng.standard_normal((M, d)).astype(np.float32)
+    a[0] = 0.0                       # all-zero row
+    a[1, 64:128] = 0.0               # an all-zero 64-element block
+    a[2, 0:32] = 0.0                 # one zero half: its outputs still see the other half
+    a[3, 5] = np.inf
+    a[4, 100] = np.nan
+    a[6] *= 1e37
+    a[7] *= 1e-39
+    a[8, 33] = 3.4e38
+    a[9, 64:128] = 3.0               # constant block (exact cancellations)
+    x = inputs.f32_to_bf16_bits(a)
+    params = inputs.lu_params(d // 64, seed=68, factors=6)
+    params[2, 4, 1] = 0.0            # u = 0: singular factor in transform block 2
+    params[3, 0] = (-1.0, 1.0, 1.0)  # d = 0 in the half-mixing factor of block 3
+    q, s = gpu_quantize_n64(kq, x, params)
+    assert kq.kq_get_device_error(clear=True) == 4
+    qr, sr = orc.quantize_n(x, orc.expand_n(params))
+    check(q, s, qr, sr)
+
+
+def test_quantize_n64_strided_rows_and_tiled_scales(kq, orc):
+    M, d, ldx = 70, 1280, 1280 + 72
+    full = inputs.activations(M, ldx, "normal", seed=69, outlier_frac=0.01, outlier_scale=(50.0, 50.0))
+    params = inputs.lu_params(d // 64, seed=70, factors=6)
+    xd = dev_bf16(full)[:, :d]
+    qr, sr = orc.quantize_n(np.ascontiguousarray(full[:, :d]), orc.expand_n(params))
+    q, s = gpu_quantize_n64(kq, None, params, x_dev=xd)
+    check(q, s, qr, sr)
+    q, s = gpu_quantize_n64(kq, None, params, x_dev=xd, scale_layout="mma")
+    assert np.array_equal(q, qr) and np.array_equal(s, tiled_scales(sr))
+
+
+def test_no_device_error_after_n64(kq):
+    assert kq.kq_get_device_error(clear=True) == 0
