@@ -616,6 +616,9 @@ def run_sweep(args) -> None:
         q = torch.empty((M, d // 2), dtype=torch.uint8, device="cuda")
         s = torch.empty((M, d // 32), dtype=torch.uint8, device="cuda")
         mats16 = kq.kq_expand_blocks(pd, dtype=torch.bfloat16)
+        p64 = torch.from_numpy(inputs.lu_params(d // 64, seed=[M, d, 64], factors=6)).cuda() if d % 64 == 0 else None
+        mats64 = kq.kq_expand_blocks(p64) if p64 is not None else None
+        fac64 = kq.kq_expand_factored(p64) if p64 is not None else None
         calls = {
             "kroquant": lambda st: lib.kq_quantize(xd.data_ptr(), M, d, d, mats.data_ptr(), 0, fac.data_ptr(),
                                                    q.data_ptr(), s.data_ptr(), 2, 0, st),
@@ -627,6 +630,9 @@ def run_sweep(args) -> None:
                                                             s.data_ptr(), st),
             "fwht": lambda st: lib.kq_ref_fwht_quantize(xd.data_ptr(), M, d, d, q.data_ptr(), s.data_ptr(), st),
         }
+        if p64 is not None:  # 64-element transform blocks (six factors), butterfly
+            calls["kroquant64"] = lambda st: lib.kq_quantize_n(xd.data_ptr(), M, d, d, 6, mats64.data_ptr(), 0,
+                                                               fac64.data_ptr(), q.data_ptr(), s.data_ptr(), 2, 0, st)
         res = {}
         reps = 30 if M * d < 2**26 else 10
         for kind, fn in calls.items():
