@@ -344,7 +344,15 @@ def run_gpu(args) -> None:
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        total_ms, launch_ms = timed(torch, step, args.steps, "kroquant", per_launch=True)
+        # the K timed steps, back to back: events only around the whole loop (events
+        # between launches would serialise them and cost ~14 us per step)
+        total_ms, _ = timed(torch, step, args.steps, "kroquant", per_launch=False)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        # the same K steps again with events around every launch: per-kernel durations
+        # for the roofline
+        _, launch_ms = timed(torch, step, args.steps, "kroquant", per_launch=True)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()

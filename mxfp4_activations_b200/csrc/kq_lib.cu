@@ -78,6 +78,26 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
+// ---- launch with programmatic stream serialization: the kernel may start its
+// prologue while the previous kernel in the stream finishes; it waits for that
+// kernel's completion (griddepcontrol.wait) before reading global memory.
+template <typename Params>
+kq_status launch_pdl(void (*kern)(const CUtensorMap, const Params), dim3 grid, int threads, int smem,
+                     cudaStream_t stream, const char* what, const CUtensorMap& tmap, const Params& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(unsigned(threads));
+  cfg.dynamicSmemBytes = size_t(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmap, p);
+  return e == cudaSuccess ? launch_status(what) : cuda_fail(what, e);
+}
+
 // ---- launch of the quantizer kernels (tile: 8 block columns x 32 rows)
 
 // Row-tile stride for a grid of ncol column groups on sms SMs holding per_sm
@@ -152,8 +172,8 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   const int64_t ncol = (nb + kq::kQCols - 1) / kq::kQCols;
   if (ncol > int64_t(INT32_MAX)) return KQ_ERR_SHAPE;
   const int64_t gy = row_stride(ncol, nrt, dev->sms, per_sm);
-  kern<<<dim3(unsigned(ncol), unsigned(gy)), kq::kQThreads, smem, stream>>>(tmap, p);
-  return launch_status("quant_kernel launch");
+  return launch_pdl(kern, dim3(unsigned(ncol), unsigned(gy)), kq::kQThreads, smem, stream, "quant_kernel launch",
+                    tmap, p);
 }
 
 // Tensor-core variant: 128-row x 4-block tiles, one CTA per 4-block column group
@@ -209,8 +229,8 @@ kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, con
   const int per_sm = (smem + 1024) * kq::kMmaCtasPerSm <= dev->smem_per_sm ? kq::kMmaCtasPerSm : 1;
   const int64_t ngroups = (nb + kq::kMmaWb - 1) / kq::kMmaWb;
   const int64_t gy = row_stride(ngroups, nrt, dev->sms, per_sm);
-  kern<<<dim3(unsigned(ngroups), unsigned(gy)), kq::kMmaThreads, smem, stream>>>(tmap, p);
-  return launch_status("quant_mma_kernel launch");
+  return launch_pdl(kern, dim3(unsigned(ngroups), unsigned(gy)), kq::kMmaThreads, smem, stream,
+                    "quant_mma_kernel launch", tmap, p);
 }
 
 kq_status check_x(const void* x, int64_t M, int64_t d, int64_t ldx) {

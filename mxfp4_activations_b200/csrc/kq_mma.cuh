@@ -188,6 +188,7 @@ __global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(c
   }
   if (t < kMmaWb) kmax_bits[t] = 0u;
   __syncthreads();
+  grid_dependency_wait();  // inputs may come from the previous kernel in the stream
 
   if (warp >= 1) {
     // B operands, built by the MMA and epilogue warps while the producer streams
@@ -265,6 +266,7 @@ __global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(c
         mbar_arrive_expect_tx(&full_a[s], uint32_t(kMmaAStageBytes));
         tma_load_3d(a_smem + s * kMmaAStageBytes, &tmap, &full_a[s], 0, tile * kMmaRows, group * kMmaWb);
       }
+      grid_launch_dependents();  // every load issued: the next grid may start its prologue
       if (it < my_tiles) {
         for (int k = (it > kMmaStages ? it - kMmaStages : 0); k < it; k++)
           mbar_wait_bounded(&full_a[k % kMmaStages], uint32_t(k / kMmaStages) & 1u, kWaitLimitNs / 4);

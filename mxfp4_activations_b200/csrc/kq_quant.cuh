@@ -282,6 +282,7 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_consta
     fence_mbar_init();
   }
   __syncthreads();
+  grid_dependency_wait();  // inputs may come from the previous kernel in the stream
 
   if (warp == kQConsWarps) {  // producer warp: one thread issues every TMA load
     if (lane == 0) {
@@ -295,6 +296,7 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_consta
         mbar_arrive_expect_tx(&full[s], uint32_t(kQStageBytes));
         tma_load_3d(base + s * kQStageBytes, &tmap, &full[s], 0, tile * kQRows, col0);
       }
+      grid_launch_dependents();  // every load issued: the next grid may start its prologue
       if (it < my_tiles) {  // consumers stopped: let the loads still in flight land before exiting
         for (int k = (it > kQStages ? it - kQStages : 0); k < it; k++)
           mbar_wait_bounded(&full[k % kQStages], uint32_t(k / kQStages) & 1u, kWaitLimitNs / 4);
