@@ -110,6 +110,19 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// Hand a shared-memory stage back to the TMA producer once this warp's plain
+// (ld.shared) reads of it are done.  The producer's next TMA load into the stage
+// writes through the asynchronous proxy, so every lane first orders its reads
+// against such writes with a proxy fence; then one lane arrives.  Without the
+// fence, some reads were served after the next tile's TMA load had begun to
+// overwrite the stage: back-to-back launches of the butterfly quantizer at
+// 4608 x 12288 got one or a few blocks wrong in 6-16 % of launches.
+__device__ __forceinline__ void stage_release(uint64_t* bar, int lane) {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
+
 // One try_wait; the thread may sleep in hardware until the phase completes or
 // the suspend-time hint (ns) runs out, so a waiting warp does not spin on the
 // issue slots the computing warps need.

@@ -340,8 +340,7 @@ __global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(c
         for (int k = 0; k < 4; k++) nz |= xv[k].x | xv[k].y | xv[k].z | xv[k].w;
         zero_block = (nz & 0x7FFF7FFFu) == 0u;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_a[s]);
+      stage_release(&empty_a[s], lane);
       if (!mbar_wait_bounded(&mma_full[buf], uint32_t(it / kMmaAccBufs) & 1u, kWaitLimitNs)) break;
       tc_fence_after();
       float y[32];

@@ -162,7 +162,26 @@ __device__ __forceinline__ void quant_block(uint32_t cf, const uint4 (&xr)[4], b
   for (int j = 0; j < kBlock; j++) l1p[j & 3] = __fadd_ru(l1p[j & 3], fabsf(x[j]));
   float l1 = __fadd_ru(__fadd_ru(l1p[0], l1p[1]), __fadd_ru(l1p[2], l1p[3]));
   // every output of a 64-element block depends on all 64 inputs
-  if (NT == 64) l1 = __fadd_ru(l1, __shfl_xor_sync(0xFFFFFFFFu, l1, 8));
+  if (NT == 64) {
+    l1 = __fadd_ru(l1, __shfl_xor_sync(0xFFFFFFFFu, l1, 8));
+    // factor 0 of a 64-element block, applied first (the Kronecker factors act on
+    // different index bits and commute): x_lo + lam x_hi in the lower half, x_hi +
+    // bet x_lo in the upper one, element by element, with the partner half's inputs
+    // taken from lane ^ 8 as raw bf16 pairs (16 shuffles)
+    const uint4 cx = lds128(cf + 208);
+    const float cc = upper ? __uint_as_float(cx.y) : __uint_as_float(cx.x);
+    const uint64_t C2 = pk2(cc, cc);
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      const uint32_t w[4] = {xr[k].x, xr[k].y, xr[k].z, xr[k].w};
+#pragma unroll
+      for (int h = 0; h < 4; h++) {
+        const uint32_t pw = __shfl_xor_sync(0xFFFFFFFFu, w[h], 8);
+        const uint64_t X = fma2_rn(C2, pk2(bf16lo(pw), bf16hi(pw)), pk2(x[8 * k + 2 * h], x[8 * k + 2 * h + 1]));
+        upk2(X, x[8 * k + 2 * h], x[8 * k + 2 * h + 1]);
+      }
+    }
+  }
 
   float cfac, eabs;
   // stage on index bit 0 (factor 4), scalar: the pair partners share a register pair
@@ -213,20 +232,6 @@ __device__ __forceinline__ void quant_block(uint32_t cf, const uint4 (&xr)[4], b
         Y[m] = fma2_rn(L2, y1, y0);
         Y[m1] = fma2_rn(B2, y0, y1);
       }
-    }
-  }
-  if (NT == 64) {
-    // factor 0 of a 64-element block: out_lo = y_lo + lam y_hi, out_hi = y_hi + bet y_lo,
-    // element by element between the two halves (held by lanes l and l ^ 8)
-    const uint4 cx = lds128(cf + 208);
-    const float cc = upper ? __uint_as_float(cx.y) : __uint_as_float(cx.x);
-    const uint64_t C2 = pk2(cc, cc);
-#pragma unroll
-    for (int m = 0; m < 16; m++) {
-      float lo, hi;
-      upk2(Y[m], lo, hi);
-      const float plo = __shfl_xor_sync(0xFFFFFFFFu, lo, 8), phi = __shfl_xor_sync(0xFFFFFFFFu, hi, 8);
-      Y[m] = fma2_rn(C2, pk2(plo, phi), Y[m]);
     }
   }
   // diagonal: D_j (FWHT: +-2^-2.5 with the sign of (-1)^popcount(j))
@@ -352,8 +357,7 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_consta
     const uint32_t blk = sbase + uint32_t(s) * kQStageBytes + xoff;
 #pragma unroll
     for (int k = 0; k < 4; k++) xr[k] = lds128(blk + uint32_t((k ^ sw) << 4));
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+    stage_release(&empty[s], lane);
     const bool act = col_ok && row < p.M;
     const int64_t rowc = act ? row : 0;
     uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16;

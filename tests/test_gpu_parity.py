@@ -573,3 +573,43 @@ def test_quantize_n64_strided_rows_and_tiled_scales(kq, orc):
 
 def test_no_device_error_after_n64(kq):
     assert kq.kq_get_device_error(clear=True) == 0
+
+
+# ---------------------------------------------------------------- back-to-back launches
+
+@pytest.mark.parametrize("n,variant,mdt", [(32, "butterfly", "f32"), (64, "butterfly", "f32"),
+                                           (32, "mma", "f32"), (32, "mma", "bf16")])
+def test_back_to_back_launches_every_output_exact(kq, orc, n, variant, mdt):
+    """Launches queued back to back on one stream at the FLUX.1-schnell shape
+    4608 x 12288 (each may start while the previous one drains): every launch's
+    output must equal the oracle's, not only the last one.  Each launch of a round
+    writes its own buffer; the buffers are compared on the device between rounds,
+    and every other round starts after an L2-sized write."""
+    d = 12288
+    x, params = inputs.config_case("flux", d)
+    if n == 64:
+        params = inputs.lu_params(d // 64, seed=71, factors=6)
+        qr, sr = orc.quantize_n(x, orc.expand_n(params))
+    else:
+        qr, sr = orc.quantize(x, oracle_mats(orc, params, mdt))
+    p = dev_f32(params)
+    mats = kq.kq_expand_blocks(p, dtype=torch.float32 if mdt == "f32" else torch.bfloat16)
+    fac = kq.kq_expand_factored(p) if variant == "butterfly" else None
+    xd = dev_bf16(x)
+    qr_d, sr_d = torch.from_numpy(qr).cuda(), torch.from_numpy(sr).cuda()
+    nbuf = 8
+    qs = [torch.empty_like(qr_d) for _ in range(nbuf)]
+    ss = [torch.empty_like(sr_d) for _ in range(nbuf)]
+    flush = torch.empty(192 * 2**20, dtype=torch.uint8, device="cuda")
+    bad = []
+    for rnd in range(10):
+        if rnd % 2:
+            flush.fill_(rnd)
+        for i in range(nbuf):
+            kq.kq_quantize(xd, mats, fac, variant=variant, q=qs[i], scales=ss[i])
+        for i in range(nbuf):
+            nq, ns = int((qs[i] != qr_d).sum()), int((ss[i] != sr_d).sum())
+            if nq or ns:
+                bad.append((rnd * nbuf + i, nq, ns))
+    assert not bad, f"(launch, wrong code bytes, wrong scales): {bad}"
+    assert kq.kq_get_device_error(clear=True) == 0
