@@ -577,9 +577,9 @@ def test_no_device_error_after_n64(kq):
 
 # ---------------------------------------------------------------- back-to-back launches
 
-@pytest.mark.parametrize("n,variant,mdt", [(32, "butterfly", "f32"), (64, "butterfly", "f32"),
-                                           (32, "mma", "f32"), (32, "mma", "bf16")])
-def test_back_to_back_launches_every_output_exact(kq, orc, n, variant, mdt):
+@pytest.mark.parametrize("kind", ["butterfly", "butterfly64", "mma_f32", "mma_bf16", "butterfly_tiled", "smooth",
+                                  "fwht"])
+def test_back_to_back_launches_every_output_exact(kq, orc, kind):
     """Launches queued back to back on one stream at the FLUX.1-schnell shape
     4608 x 12288 (each may start while the previous one drains): every launch's
     output must equal the oracle's, not only the last one.  Each launch of a round
@@ -587,26 +587,41 @@ def test_back_to_back_launches_every_output_exact(kq, orc, n, variant, mdt):
     and every other round starts after an L2-sized write."""
     d = 12288
     x, params = inputs.config_case("flux", d)
-    if n == 64:
-        params = inputs.lu_params(d // 64, seed=71, factors=6)
-        qr, sr = orc.quantize_n(x, orc.expand_n(params))
-    else:
-        qr, sr = orc.quantize(x, oracle_mats(orc, params, mdt))
-    p = dev_f32(params)
-    mats = kq.kq_expand_blocks(p, dtype=torch.float32 if mdt == "f32" else torch.bfloat16)
-    fac = kq.kq_expand_factored(p) if variant == "butterfly" else None
     xd = dev_bf16(x)
+    layout = "mma" if kind == "butterfly_tiled" else "row"
+    if kind == "smooth":
+        inv_s = inputs.smooth_inv_scale(x)
+        inv_s_d = dev_f32(inv_s)
+        qr, sr = orc.smooth_quantize(x, inv_s)
+        launch = lambda q, s: kq.kq_ref_smooth_quantize(xd, inv_s_d, q=q, scales=s)
+    elif kind == "fwht":
+        qr, sr = orc.fwht_quantize(x)
+        launch = lambda q, s: kq.kq_ref_fwht_quantize(xd, q=q, scales=s)
+    else:
+        if kind == "butterfly64":
+            params = inputs.lu_params(d // 64, seed=71, factors=6)
+            qr, sr = orc.quantize_n(x, orc.expand_n(params))
+        else:
+            mdt = "bf16" if kind == "mma_bf16" else "f32"
+            qr, sr = orc.quantize(x, oracle_mats(orc, params, mdt))
+        p = dev_f32(params)
+        mats = kq.kq_expand_blocks(p, dtype=torch.bfloat16 if kind == "mma_bf16" else torch.float32)
+        variant = "mma" if kind.startswith("mma") else "butterfly"
+        fac = kq.kq_expand_factored(p) if variant == "butterfly" else None
+        launch = lambda q, s: kq.kq_quantize(xd, mats, fac, variant=variant, q=q, scales=s, scale_layout=layout)
+    if layout == "mma":
+        sr = tiled_scales(sr)
     qr_d, sr_d = torch.from_numpy(qr).cuda(), torch.from_numpy(sr).cuda()
     nbuf = 8
-    qs = [torch.empty_like(qr_d) for _ in range(nbuf)]
-    ss = [torch.empty_like(sr_d) for _ in range(nbuf)]
+    qs = [torch.zeros_like(qr_d) for _ in range(nbuf)]
+    ss = [torch.zeros_like(sr_d) for _ in range(nbuf)]
     flush = torch.empty(192 * 2**20, dtype=torch.uint8, device="cuda")
     bad = []
     for rnd in range(10):
         if rnd % 2:
             flush.fill_(rnd)
         for i in range(nbuf):
-            kq.kq_quantize(xd, mats, fac, variant=variant, q=qs[i], scales=ss[i])
+            launch(qs[i], ss[i])
         for i in range(nbuf):
             nq, ns = int((qs[i] != qr_d).sum()), int((ss[i] != sr_d).sum())
             if nq or ns:
