@@ -7,6 +7,7 @@ numpy arrays into the C oracle and back.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import subprocess
@@ -40,41 +41,67 @@ def lib():
     global _lib
     if _lib is None:
         build()
-        L = ctypes.CDLL(_LIB_PATH)
-        P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
-        L.kqo_factor.argtypes = [ctypes.c_float] * 3 + [P]
-        L.kqo_factor_inverse.argtypes = [ctypes.c_float] * 3 + [P]
-        L.kqo_kron.argtypes = [P, I, P, I, P]
-        L.kqo_expand_f64.argtypes = [P, I64, I, P]
-        L.kqo_expand.argtypes = [P, I64, I, I, P]
-        L.kqo_expand_n_f64.argtypes = [P, I64, I, I, P]
-        L.kqo_expand_n.argtypes = [P, I64, I, I, I, P]
-        L.kqo_transform_n.argtypes = [P, I64, I64, I64, P, I, I, P]
-        L.kqo_quantize_n.argtypes = [P, I64, I64, I64, P, I, I, P, P]
-        L.kqo_bf16_from_f64.argtypes = [ctypes.c_double]
-        L.kqo_bf16_from_f64.restype = ctypes.c_uint16
-        L.kqo_hadamard.argtypes = [I, P]
-        L.kqo_e8m0.argtypes = [ctypes.c_float]
-        L.kqo_e8m0.restype = I
-        L.kqo_e8m0_many.argtypes = [P, I64, P]
-        L.kqo_e8m0_many.restype = None
-        L.kqo_e2m1.argtypes = [ctypes.c_float]
-        L.kqo_e2m1.restype = I
-        L.kqo_e2m1_value.argtypes = [I]
-        L.kqo_e2m1_value.restype = ctypes.c_double
-        L.kqo_e2m1_pack.argtypes = [P, I64, P]
-        L.kqo_transform.argtypes = [P, I64, I64, I64, P, I, P]
-        L.kqo_mx_quantize.argtypes = [P, I64, I64, P, P]
-        L.kqo_quantize.argtypes = [P, I64, I64, I64, P, I, P, P]
-        L.kqo_smooth_quantize.argtypes = [P, I64, I64, I64, P, P, P]
-        L.kqo_fwht_quantize.argtypes = [P, I64, I64, I64, P, P]
-        L.kqo_dequantize.argtypes = [P, P, I64, I64, P, I, P]
-        for name in ("kqo_factor", "kqo_factor_inverse", "kqo_kron", "kqo_expand_f64", "kqo_expand",
-                     "kqo_hadamard", "kqo_e2m1_pack", "kqo_transform", "kqo_mx_quantize", "kqo_quantize",
-                     "kqo_smooth_quantize", "kqo_fwht_quantize", "kqo_dequantize"):
-            getattr(L, name).restype = None
-        _lib = L
+        _lib = _configure(ctypes.CDLL(_LIB_PATH))
     return _lib
+
+
+def compile_copy(src_text: str, out_path: str) -> str:
+    """Compile another text of kq_oracle.c, with the flags of ``build``, into
+    out_path (the tests plant mistakes in copies of the source)."""
+    c_path = os.path.splitext(out_path)[0] + ".c"
+    with open(c_path, "w") as f:
+        f.write(src_text)
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared", "-I", _HERE,
+                           "-o", out_path, c_path, "-lm"])
+    return out_path
+
+
+@contextlib.contextmanager
+def using_library(path: str):
+    """Route every call of this module through the oracle build at path."""
+    global _lib
+    saved = lib()
+    _lib = _configure(ctypes.CDLL(path))
+    try:
+        yield
+    finally:
+        _lib = saved
+
+
+def _configure(L):
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    L.kqo_factor.argtypes = [ctypes.c_float] * 3 + [P]
+    L.kqo_factor_inverse.argtypes = [ctypes.c_float] * 3 + [P]
+    L.kqo_kron.argtypes = [P, I, P, I, P]
+    L.kqo_expand_f64.argtypes = [P, I64, I, P]
+    L.kqo_expand.argtypes = [P, I64, I, I, P]
+    L.kqo_expand_n_f64.argtypes = [P, I64, I, I, P]
+    L.kqo_expand_n.argtypes = [P, I64, I, I, I, P]
+    L.kqo_transform_n.argtypes = [P, I64, I64, I64, P, I, I, P]
+    L.kqo_quantize_n.argtypes = [P, I64, I64, I64, P, I, I, P, P]
+    L.kqo_bf16_from_f64.argtypes = [ctypes.c_double]
+    L.kqo_bf16_from_f64.restype = ctypes.c_uint16
+    L.kqo_hadamard.argtypes = [I, P]
+    L.kqo_e8m0.argtypes = [ctypes.c_float]
+    L.kqo_e8m0.restype = I
+    L.kqo_e8m0_many.argtypes = [P, I64, P]
+    L.kqo_e8m0_many.restype = None
+    L.kqo_e2m1.argtypes = [ctypes.c_float]
+    L.kqo_e2m1.restype = I
+    L.kqo_e2m1_value.argtypes = [I]
+    L.kqo_e2m1_value.restype = ctypes.c_double
+    L.kqo_e2m1_pack.argtypes = [P, I64, P]
+    L.kqo_transform.argtypes = [P, I64, I64, I64, P, I, P]
+    L.kqo_mx_quantize.argtypes = [P, I64, I64, P, P]
+    L.kqo_quantize.argtypes = [P, I64, I64, I64, P, I, P, P]
+    L.kqo_smooth_quantize.argtypes = [P, I64, I64, I64, P, P, P]
+    L.kqo_fwht_quantize.argtypes = [P, I64, I64, I64, P, P]
+    L.kqo_dequantize.argtypes = [P, P, I64, I64, P, I, P]
+    for name in ("kqo_factor", "kqo_factor_inverse", "kqo_kron", "kqo_expand_f64", "kqo_expand",
+                 "kqo_hadamard", "kqo_e2m1_pack", "kqo_transform", "kqo_mx_quantize", "kqo_quantize",
+                 "kqo_smooth_quantize", "kqo_fwht_quantize", "kqo_dequantize"):
+        getattr(L, name).restype = None
+    return L
 
 
 def _p(a: np.ndarray):

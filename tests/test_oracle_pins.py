@@ -402,6 +402,25 @@ def test_nonfinite_block_rule(orc):
     assert s[0, 1] == orc.e8m0(1.0)
 
 
+def test_scale_and_nonfinite_rule_see_every_position(orc):
+    """Under K = I, a block whose largest magnitude sits at position j, for every
+    j: amax = 24 gives e = floor(log2 24) - 2 = 2 (byte 129); 24 / 4 = 6 is code 7
+    at j, and 0.5 / 4 = 0.125 (below the 0.25 midpoint) is code 0 elsewhere.  A
+    NaN at position j alone gives byte 0xFF and 32 zero codes."""
+    K = orc.expand(inputs.identity_params(1))
+    for j in range(32):
+        a = np.full((1, 32), 0.5, np.float32)
+        a[0, j] = 24.0
+        q, s = orc.quantize(inputs.f32_to_bf16_bits(a), K)
+        codes = np.stack([q[0] & 0xF, q[0] >> 4], axis=-1).reshape(-1)
+        expected = np.zeros(32, np.uint8)
+        expected[j] = 7
+        assert s[0, 0] == 129 and np.array_equal(codes, expected), j
+        a[0, j] = np.nan
+        q, s = orc.quantize(inputs.f32_to_bf16_bits(a), K)
+        assert s[0, 0] == 0xFF and not q.any(), j
+
+
 def test_dequantize_is_grid_value_times_scale(orc):
     rng = np.random.default_rng(61)
     y = (rng.standard_normal((8, 64)) * np.exp2(rng.integers(-10, 10, (8, 1)))).astype(np.float32)
