@@ -3,7 +3,8 @@
 The quantizer kernels take a scale or a code from their fp32 butterfly result
 y_f only when the whole interval y_f +- E maps to it, with
 
-    E = C * ||x||_1 * max|K|        (C = 16u for 32-element blocks, 32u for 64)
+    E = C * ||x||_1 * max|K|        (C = 16u for 32-element blocks, 32u for 64,
+                                     8u for the FWHT comparison kernel)
 
 ("KroQuant: Kronecker-Structured Block Transforms ...", Approach: K is the
 Kronecker product of 2x2 unit-determinant LU factors).  Exactness of the device
@@ -118,6 +119,30 @@ def test_bound_64_element_blocks_half_mixing_first(orc):
         for order in ([0, 5, 4, 3, 2, 1], [5, 4, 3, 2, 1, 0]):
             w = worst_error_in_u(orc, x, params, order=order, y32=y32)
             assert w <= 16.0, (order, w)   # the proven need; the kernel allows 32u
+
+
+def test_bound_fwht_comparison_kernel(orc):
+    """The FWHT comparison kernel runs the same butterfly with every ratio +-1
+    (exact add and subtract) and D_j = +-fp32(2^-2.5); its allowance is 8u
+    against a proven need of 7u."""
+    for x in cases(32):
+        d = x.shape[1]
+        R, nt = x.shape[0], d // 32
+        x32 = inputs.bf16_bits_to_f32(x).reshape(R, nt, 32)
+        lam = np.ones((nt, 5), np.float32)
+        bet = -np.ones((nt, 5), np.float32)
+        H = orc.hadamard(5)
+        c = np.float32(2.0 ** -2.5)
+        # the Sylvester H32 equals (M (x) ... (x) M) D with M = [[1, -1], [1, 1]] and D_j = c (-1)^popcount(j)
+        D = np.array([c if bin(j).count("1") % 2 == 0 else -c for j in range(32)], np.float32)
+        yf = butterfly(x32, lam, bet, np.tile(D, (nt, 1)), order=[4, 3, 2, 1, 0]).astype(np.float64)
+        H32 = H.astype(np.float32)
+        y32 = orc.transform(x, np.ascontiguousarray(np.tile(H32, (nt, 1, 1)))).reshape(R, nt, 32)
+        l1 = np.abs(x32.astype(np.float64)).sum(-1, keepdims=True)
+        kmax = float(np.abs(H32).max())
+        ok = l1 > 0
+        err = np.abs(yf - y32) / np.where(ok, l1 * kmax * U, 1.0)
+        assert err[np.broadcast_to(ok, err.shape)].max() <= 7.0
 
 
 @pytest.mark.parametrize("bad_constant", [0.25])
