@@ -28,8 +28,8 @@
  *           byte k of a row holds element 2k in its low nibble.
  *
  * Ownership: the caller owns every buffer (device memory unless stated).  No
- * entry point allocates, frees or synchronises; all device work is enqueued on
- * the given stream.  Argument errors are returned before anything is launched.
+ * entry point allocates or frees memory, and none but kq_get_device_error
+ * synchronises; all device work is enqueued on the given stream.  Argument errors are returned before anything is launched.
  * A launch failure returns KQ_ERR_CUDA.  Kernels that wait on asynchronous
  * copies bound every wait; a wait that runs out records a flag that
  * kq_get_device_error() reports.
