@@ -39,6 +39,9 @@ FLUX_M = 4608
 FLUX_DS = (3072, 12288)
 BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 32.0
 PROFILE_JSON = os.path.join(ROOT, "profiles", "kq_quant_flux_traffic.json")
+FLUX_WORKLOAD = ("FLUX.1-schnell-shaped activations, M=4608 tokens x d in {3072, 12288} bf16, "
+                 "Student-t(3) with 0.5% outlier channels x100, per-block LU params Hadamard+N(0,0.05)")
+
 KERNEL_SOURCES = ["mxfp4_activations_b200/csrc/kq_quant.cuh", "mxfp4_activations_b200/csrc/kq_common.cuh",
                   "mxfp4_activations_b200/csrc/kq_mx.cuh",
                   "mxfp4_activations_b200/csrc/kq_lib.cu"]
@@ -404,8 +407,7 @@ def run_gpu(args) -> None:
         "dtype": "f32",
         "data": "synthetic",
         "config": {
-            "workload": "FLUX.1-schnell-shaped activations, M=4608 tokens x d in {3072, 12288} bf16, "
-                        "Student-t(3) with 0.5% outlier channels x100, per-block LU params Hadamard+N(0,0.05)",
+            "workload": FLUX_WORKLOAD,
             "M": FLUX_M, "d": list(FLUX_DS), "variant": "butterfly",
             "l2": f"inputs rotated over 4 device copies ({resident_mb:.0f} MB > 126 MB L2)",
             "parallelism": f"dp{world} (rows sharded, no collective)",
@@ -566,8 +568,7 @@ def run_reference(args) -> None:
         "value": round(gbs, 6), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3 / max(1, args.steps), 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "FLUX.1-schnell-shaped activations, M=4608 tokens x d in {3072, 12288} bf16 "
-                               "(bounded row sample per step)", "M": FLUX_M, "d": list(FLUX_DS)},
+        "config": {"workload": FLUX_WORKLOAD, "M": FLUX_M, "d": list(FLUX_DS)},
         "tokens_per_s": round(rows * passes * pool.n * args.steps / dt, 3),
         "cpu_baseline": {"value": round(gbs, 6), "unit": "GB/s", "cores": pool.n, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(gbs, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
