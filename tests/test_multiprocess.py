@@ -69,3 +69,13 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["cpu_baseline"]["kind"] == "oracle"
+    # the contract's keys: the same metric, unit and workload as the device arm, an oracle
+    # cpu_baseline describing the run, and an e2e with no host-device traffic
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert rec["config"]["workload"] == bench.FLUX_WORKLOAD
+    assert rec["unit"] == "GB/s" and rec["higher_is_better"] is True and rec["value"] > 0
+    cb = rec["cpu_baseline"]
+    assert cb["value"] == rec["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert rec["e2e"] == {"value": rec["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
