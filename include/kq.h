@@ -70,7 +70,13 @@ typedef enum { KQ_F32 = 0, KQ_BF16 = 1 } kq_dtype;
  *   KQ_VAR_BUTTERFLY: 5-stage 2x2 butterfly over registers (needs KQ_F32
  *                     matrices and the factored form from kq_expand_factored).
  *   KQ_VAR_MMA:       tensor-core product with the dense block matrix.
- *   KQ_VAR_AUTO:      the faster provided variant for the shape and dtype. */
+ *   KQ_VAR_AUTO:      the faster provided variant for the shape and dtype: bf16
+ *                     matrices, or fp32 without the factored form, take the
+ *                     tensor core; fp32 with the factored form takes the winner
+ *                     measured at the nearest shape of the library's sweep table
+ *                     (log2 M, log2 d), unless the environment variable
+ *                     KQ_VARIANT=mma|butterfly (read once per process) names one.
+ *                     kq_select_variant reports the choice. */
 typedef enum { KQ_VAR_AUTO = 0, KQ_VAR_MMA = 1, KQ_VAR_BUTTERFLY = 2 } kq_variant;
 
 /* Where kq_quantize writes the E8M0 scales.
@@ -219,6 +225,16 @@ KQ_API kq_status kq_ref_fwht_quantize(const void* x, int64_t M, int64_t d, int64
  * code(v[2k+1]) << 4 for already scaled fp32 values (same rounding as
  * kq_quantize).  v device fp32 [n], out device [n/2]; n even. */
 KQ_API kq_status kq_e2m1_pack(const float* v, int64_t n, uint8_t* out, kq_stream_t stream);
+
+/* kq_select_variant -- the kernel kq_quantize_n(x, M, d, ..., log2n, ..., mat_dtype,
+ * factored, ..., KQ_VAR_AUTO, ...) runs for these sizes, without launching
+ * anything: *chosen = KQ_VAR_MMA or KQ_VAR_BUTTERFLY.  has_factored != 0 when the
+ * factored form will be passed.  KQ_ERR_INVALID_ARG for a NULL chosen, a negative
+ * size, a bad dtype or log2n other than 5 or 6; KQ_ERR_UNSUPPORTED when no
+ * variant serves the combination (64-element blocks need fp32 matrices and the
+ * factored form).  Host-only: needs no device. */
+KQ_API kq_status kq_select_variant(int64_t M, int64_t d, int log2n, kq_dtype mat_dtype, int has_factored,
+                                   kq_variant* chosen);
 
 /* ---------------------------------------------------------------- status
  *

@@ -21,6 +21,7 @@ from ._lib import (  # noqa: F401
     kq_quantize,
     kq_ref_fwht_quantize,
     kq_ref_smooth_quantize,
+    kq_select_variant,
     kq_status_string,
     load,
     scale_bytes,

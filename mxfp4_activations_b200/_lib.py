@@ -34,7 +34,7 @@ EXPORTED = (
     "kq_expand_blocks", "kq_expand_factored", "kq_quantize", "kq_dequantize", "kq_ref_smooth_quantize",
     "kq_expand_blocks_n", "kq_expand_factored_n", "kq_quantize_n",
     "kq_ref_fwht_quantize", "kq_e2m1_pack", "kq_get_device_error", "kq_status_string", "kq_abi_version",
-    "kq_last_error",
+    "kq_last_error", "kq_select_variant",
 )
 
 
@@ -74,6 +74,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kq_status_string": [I],
         "kq_abi_version": [],
         "kq_last_error": [],
+        "kq_select_variant": [I64, I64, I, I, I, P],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -101,26 +102,57 @@ def _stream(device: torch.device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-def _cuda(t: torch.Tensor, name: str):
+_BF16_LIKE = (torch.bfloat16, torch.int16, torch.uint16)
+_MAT_DTYPES = (torch.float32,) + _BF16_LIKE
+
+
+def _cuda(t, name: str, device: torch.device | None = None, dtypes=None, contiguous: bool = False,
+          min_numel: int | None = None) -> torch.Tensor:
+    """Checks that t is a CUDA tensor (on `device`, when given) of one of `dtypes`,
+    contiguous when required and holding at least `min_numel` elements, so that no
+    host pointer, foreign-device pointer or short buffer reaches a kernel."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the input on {device}")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name} must be one of {[str(d) for d in dtypes]}, not {t.dtype}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, {min_numel} are needed")
+    return t
 
 
 def _mat_dtype(t: torch.Tensor) -> int:
     if t.dtype == torch.float32:
         return KQ_F32
-    if t.dtype in (torch.bfloat16, torch.int16, torch.uint16):
+    if t.dtype in _BF16_LIKE:
         return KQ_BF16
     raise TypeError("matrices must be float32 or bfloat16")
 
 
-def _rows(x: torch.Tensor, name: str = "x"):
-    """(M, d, ldx) of a 2-D bf16 activation whose rows may be strided."""
-    if x.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
-        raise TypeError(f"{name} must be bfloat16 (or its 16-bit patterns)")
+def _rows(x, name: str = "x"):
+    """(M, d, ldx) of a 2-D bf16 CUDA activation whose rows may be strided."""
+    _cuda(x, name, dtypes=_BF16_LIKE)
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError(f"{name} must be 2-D with unit column stride")
     return x.shape[0], x.shape[1], x.stride(0)
+
+
+def _mats(mats, d: int, device: torch.device, name: str = "mats") -> int:
+    """Block size n of a contiguous [d/n, n, n] matrix tensor on `device`."""
+    _cuda(mats, name, device, _MAT_DTYPES, contiguous=True)
+    if mats.dim() != 3 or mats.shape[1] != mats.shape[2]:
+        raise ValueError(f"{name} must be [d/n, n, n]")
+    n = mats.shape[-1]
+    if n not in (32, 64):
+        raise ValueError("transform blocks of 32 or 64 elements")
+    if mats.shape[0] * n != d:
+        raise ValueError(f"{name} holds {mats.shape[0]} blocks of {n}, the input has d = {d}")
+    return n
 
 
 # ---------------------------------------------------------------- set-up
@@ -141,37 +173,43 @@ def kq_expand_blocks(params: torch.Tensor, inverse: bool = False, dtype: torch.d
                      log2n: int | None = None) -> torch.Tensor:
     """K, K^-1 (inverse=True) or the weight-side K^-T (inverse=True, transpose=True)
     per transform block of n = 2^log2n elements ([nt, n, n]; log2n from params [nt, log2n, 3])."""
-    _cuda(params, "params")
+    _cuda(params, "params", dtypes=(torch.float32,))
     params = params.contiguous()
     nt, log2n = _params_shape(params, log2n)
     n = 1 << log2n
     if out is None:
         out = torch.empty((nt, n, n), dtype=dtype, device=params.device)
+    _cuda(out, "out", params.device, _MAT_DTYPES, contiguous=True, min_numel=nt * n * n)
     if transpose and not inverse:
         raise ValueError("transpose is provided for the inverse (the weight-side transform) only")
     mode = 2 if transpose else int(bool(inverse))
-    _check("kq_expand_blocks_n", load().kq_expand_blocks_n(_ptr(params), nt, log2n, mode, _mat_dtype(out),
-                                                             _ptr(out), _stream(params.device)))
+    with torch.cuda.device(params.device):
+        _check("kq_expand_blocks_n", load().kq_expand_blocks_n(_ptr(params), nt, log2n, mode, _mat_dtype(out),
+                                                                 _ptr(out), _stream(params.device)))
     return out
 
 
 def kq_expand_factored(params: torch.Tensor, out: torch.Tensor | None = None,
                        log2n: int | None = None) -> torch.Tensor:
     """The butterfly form, one [48] record per 32-element block column."""
-    _cuda(params, "params")
+    _cuda(params, "params", dtypes=(torch.float32,))
     params = params.contiguous()
     nt, log2n = _params_shape(params, log2n)
     nb32 = nt << (log2n - 5) if log2n >= 5 else nt
     if out is None:
         out = torch.empty((nb32, 48), dtype=torch.float32, device=params.device)
-    _check("kq_expand_factored_n", load().kq_expand_factored_n(_ptr(params), nt, log2n, _ptr(out),
-                                                                 _stream(params.device)))
+    _cuda(out, "out", params.device, (torch.float32,), contiguous=True, min_numel=nb32 * 48)
+    with torch.cuda.device(params.device):
+        _check("kq_expand_factored_n", load().kq_expand_factored_n(_ptr(params), nt, log2n, _ptr(out),
+                                                                     _stream(params.device)))
     return out
 
 
 # ---------------------------------------------------------------- hot path
 
 def _outputs(x: torch.Tensor, M: int, d: int, q, scales, layout: str = "row"):
+    if layout not in SCALE_LAYOUTS:
+        raise ValueError(f"scale_layout must be one of {list(SCALE_LAYOUTS)}")
     if q is None:
         q = torch.empty((M, d // 2), dtype=torch.uint8, device=x.device)
     if scales is None:
@@ -179,10 +217,8 @@ def _outputs(x: torch.Tensor, M: int, d: int, q, scales, layout: str = "row"):
             scales = torch.empty((M, d // 32), dtype=torch.uint8, device=x.device)
         else:  # padding bytes are not written: start from zeros
             scales = torch.zeros(scale_bytes(M, d, layout), dtype=torch.uint8, device=x.device)
-    if q.dtype != torch.uint8 or scales.dtype != torch.uint8 or not q.is_contiguous() or not scales.is_contiguous():
-        raise ValueError("q and scales must be contiguous uint8")
-    if q.numel() < M * (d // 2) or scales.numel() < scale_bytes(M, d, layout):
-        raise ValueError("q or scales too small")
+    _cuda(q, "q", x.device, (torch.uint8,), contiguous=True, min_numel=M * (d // 2))
+    _cuda(scales, "scales", x.device, (torch.uint8,), contiguous=True, min_numel=scale_bytes(M, d, layout))
     return q, scales
 
 
@@ -191,60 +227,84 @@ def kq_quantize(x: torch.Tensor, mats: torch.Tensor, factored: torch.Tensor | No
     """MXFP4 of x K per transform block -> (codes uint8 [M, d/2], E8M0 scales: uint8
     [M, d/32] for scale_layout="row", or the flat 128x4-tiled buffer for "mma").
     The transform block size comes from mats ([d/n, n, n], n = 32 or 64)."""
-    _cuda(x, "x")
     M, d, ldx = _rows(x)
-    n = mats.shape[-1]
-    if n not in (32, 64):
-        raise ValueError("transform blocks of 32 or 64 elements")
+    n = _mats(mats, d, x.device)
+    if factored is not None:
+        _cuda(factored, "factored", x.device, (torch.float32,), contiguous=True, min_numel=(d // 32) * 48)
+    if variant not in VARIANTS:
+        raise ValueError(f"variant must be one of {list(VARIANTS)}")
     q, scales = _outputs(x, M, d, q, scales, scale_layout)
-    _check("kq_quantize_n", load().kq_quantize_n(_ptr(x), M, d, ldx, n.bit_length() - 1, _ptr(mats),
-                                                 _mat_dtype(mats), _ptr(factored), _ptr(q), _ptr(scales),
-                                                 VARIANTS[variant], SCALE_LAYOUTS[scale_layout],
-                                                 _stream(x.device)))
+    with torch.cuda.device(x.device):
+        _check("kq_quantize_n", load().kq_quantize_n(_ptr(x), M, d, ldx, n.bit_length() - 1, _ptr(mats),
+                                                     _mat_dtype(mats), _ptr(factored), _ptr(q), _ptr(scales),
+                                                     VARIANTS[variant], SCALE_LAYOUTS[scale_layout],
+                                                     _stream(x.device)))
     return q, scales
 
 
 def kq_dequantize(q: torch.Tensor, scales: torch.Tensor, inv_mats: torch.Tensor | None = None,
                   out_dtype: torch.dtype = torch.float32, out: torch.Tensor | None = None) -> torch.Tensor:
-    _cuda(q, "q")
+    """E2M1 value x 2^(scale - 127) per element, then (with inv_mats [d/32, 32, 32])
+    the inverse block transform.  Takes row-major scales [M, d/32] only."""
+    _cuda(q, "q", dtypes=(torch.uint8,), contiguous=True)
+    if q.dim() != 2:
+        raise ValueError("q must be [M, d/2]")
     M, d = q.shape[0], q.shape[1] * 2
-    if inv_mats is not None and inv_mats.shape[-1] != 32:
-        raise ValueError("kq_dequantize undoes transforms of 32-element blocks only")
+    _cuda(scales, "scales", q.device, (torch.uint8,), contiguous=True)
+    if scales.dim() != 2 or tuple(scales.shape) != (M, d // 32):
+        raise ValueError(f"scales must be row-major [M, d/32] = [{M}, {d // 32}] (the 128x4-tiled layout is "
+                         "for block-scaled GEMMs and is not read here)")
+    if inv_mats is not None:
+        n = _mats(inv_mats, d, q.device, "inv_mats")
+        if n != 32:
+            raise ValueError("kq_dequantize undoes transforms of 32-element blocks only")
     if out is None:
         out = torch.empty((M, d), dtype=out_dtype, device=q.device)
+    _cuda(out, "out", q.device, (torch.float32,) + _BF16_LIKE, contiguous=True, min_numel=M * d)
     mdt = _mat_dtype(inv_mats) if inv_mats is not None else KQ_F32
-    _check("kq_dequantize", load().kq_dequantize(_ptr(q), _ptr(scales), M, d, _ptr(inv_mats), mdt, _ptr(out),
-                                                 _mat_dtype(out), _stream(q.device)))
+    with torch.cuda.device(q.device):
+        _check("kq_dequantize", load().kq_dequantize(_ptr(q), _ptr(scales), M, d, _ptr(inv_mats), mdt, _ptr(out),
+                                                     _mat_dtype(out), _stream(q.device)))
     return out
 
 
 def kq_ref_smooth_quantize(x: torch.Tensor, inv_s: torch.Tensor, q=None, scales=None):
-    _cuda(x, "x")
     M, d, ldx = _rows(x)
+    _cuda(inv_s, "inv_s", x.device, (torch.float32,), contiguous=True, min_numel=d)
     q, scales = _outputs(x, M, d, q, scales)
-    _check("kq_ref_smooth_quantize", load().kq_ref_smooth_quantize(_ptr(x), M, d, ldx, _ptr(inv_s), _ptr(q),
-                                                                   _ptr(scales), _stream(x.device)))
+    with torch.cuda.device(x.device):
+        _check("kq_ref_smooth_quantize", load().kq_ref_smooth_quantize(_ptr(x), M, d, ldx, _ptr(inv_s), _ptr(q),
+                                                                       _ptr(scales), _stream(x.device)))
     return q, scales
 
 
 def kq_ref_fwht_quantize(x: torch.Tensor, q=None, scales=None):
-    _cuda(x, "x")
     M, d, ldx = _rows(x)
     q, scales = _outputs(x, M, d, q, scales)
-    _check("kq_ref_fwht_quantize", load().kq_ref_fwht_quantize(_ptr(x), M, d, ldx, _ptr(q), _ptr(scales),
-                                                               _stream(x.device)))
+    with torch.cuda.device(x.device):
+        _check("kq_ref_fwht_quantize", load().kq_ref_fwht_quantize(_ptr(x), M, d, ldx, _ptr(q), _ptr(scales),
+                                                                   _stream(x.device)))
     return q, scales
 
 
 def kq_e2m1_pack(v: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
-    _cuda(v, "v")
+    _cuda(v, "v", dtypes=(torch.float32,))
     v = v.contiguous()
-    if v.dtype != torch.float32:
-        raise TypeError("v must be float32")
     if out is None:
         out = torch.empty(v.numel() // 2, dtype=torch.uint8, device=v.device)
-    _check("kq_e2m1_pack", load().kq_e2m1_pack(_ptr(v), v.numel(), _ptr(out), _stream(v.device)))
+    _cuda(out, "out", v.device, (torch.uint8,), contiguous=True, min_numel=v.numel() // 2)
+    with torch.cuda.device(v.device):
+        _check("kq_e2m1_pack", load().kq_e2m1_pack(_ptr(v), v.numel(), _ptr(out), _stream(v.device)))
     return out
+
+
+def kq_select_variant(M: int, d: int, mat_dtype=None, has_factored: bool = True, log2n: int = 5) -> str:
+    """The variant ("mma" or "butterfly") that variant="auto" runs for these sizes."""
+    mdt = KQ_BF16 if mat_dtype in _BF16_LIKE else KQ_F32
+    out = ctypes.c_int(-1)
+    _check("kq_select_variant", load().kq_select_variant(M, d, log2n, mdt, int(bool(has_factored)),
+                                                         ctypes.byref(out)))
+    return {v: k for k, v in VARIANTS.items()}[out.value]
 
 
 def kq_get_device_error(clear: bool = True) -> int:

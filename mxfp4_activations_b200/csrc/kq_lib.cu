@@ -5,10 +5,14 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
+#include <cstdlib>
 #include <cstdio>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "kq.h"
 #include "kq_common.cuh"
@@ -81,9 +85,9 @@ EncodeTiledFn encode_tiled() {
 // ---- launch with programmatic stream serialization: the kernel may start its
 // prologue while the previous kernel in the stream finishes; it waits for that
 // kernel's completion (griddepcontrol.wait) before reading global memory.
-template <typename Params>
-kq_status launch_pdl(void (*kern)(const CUtensorMap, const Params), dim3 grid, int threads, int smem,
-                     cudaStream_t stream, const char* what, const CUtensorMap& tmap, const Params& p) {
+template <typename... Args>
+kq_status launch_pdl(void (*kern)(Args...), dim3 grid, int threads, int smem, cudaStream_t stream, const char* what,
+                     const Args&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(unsigned(threads));
@@ -94,11 +98,90 @@ kq_status launch_pdl(void (*kern)(const CUtensorMap, const Params), dim3 grid, i
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmap, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
   return e == cudaSuccess ? launch_status(what) : cuda_fail(what, e);
 }
 
-// ---- launch of the quantizer kernels (tile: 8 block columns x 32 rows)
+// ---- launch of the butterfly / comparison quantizer kernels
+
+// Resident CTAs per SM of a kernel launched with `threads` threads and `smem`
+// bytes of dynamic shared memory (the occupancy query, cached per kernel and device).
+kq_status resident_ctas(const void* kern, int threads, int smem, int devid, int* out) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find({kern, devid});
+  if (it != cache.end()) {
+    *out = it->second;
+    return KQ_OK;
+  }
+  int per_sm = 0;
+  const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+  if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveBlocksPerMultiprocessor", e);
+  if (per_sm < 1) return cuda_fail("occupancy: no resident CTA", cudaErrorInvalidConfiguration);
+  cache[{kern, devid}] = per_sm;
+  *out = per_sm;
+  return KQ_OK;
+}
+
+// Lane layout of the streaming quantizer: every lane owns one block column and
+// walks rows r0, r0 + k, ...; one wave of resident threads takes the lanes.
+// k is the largest row count that fits the wave, then lowered to the smallest
+// value with the same number of row steps (same makespan, fewer threads).  When
+// the block columns alone exceed the wave, k = 1 and threads walk several lanes.
+void lane_layout(int64_t M, int64_t nb, int64_t slots, kq::QuantParams& p) {
+  if (nb <= slots) {
+    int64_t k = slots / nb;
+    if (k > M) k = M;
+    const int64_t n_iter = (M + k - 1) / k;
+    k = (M + n_iter - 1) / n_iter;
+    p.k = k;
+    p.n_iter = n_iter;
+    p.lanes = k * nb;
+    p.threads = p.lanes;
+    p.passes = 1;
+  } else {
+    p.k = 1;
+    p.n_iter = M;
+    p.lanes = nb;
+    p.threads = slots;
+    p.passes = int((nb + slots - 1) / slots);
+  }
+}
+
+template <int MODE, int TILED, int NT = 32>
+kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const float* mats, const float* factored,
+                       const float* inv_s, uint8_t* q, uint8_t* scales, cudaStream_t stream) {
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return cuda_fail("device query", cudaErrorInvalidDevice);
+  int devid = 0;
+  cudaGetDevice(&devid);
+  const int64_t nb = d / 32;
+  void (*kern)(const kq::QuantParams) = kq::quant_kernel<MODE, TILED, NT>;
+  static std::atomic<int> attr_set[kMaxDevices];
+  if (!attr_set[devid].load()) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kq::kSSmemBytes);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
+    attr_set[devid].store(1);
+  }
+  int per_sm = 0;
+  kq_status st = resident_ctas(reinterpret_cast<const void*>(kern), kq::kSThreads, kq::kSSmemBytes, devid, &per_sm);
+  if (st != KQ_OK) return st;
+
+  kq::QuantParams p;
+  p.x = static_cast<const uint16_t*>(x);
+  p.ldx = ldx;
+  p.M = M;
+  p.nb = int(nb);
+  p.mats = mats;
+  p.factored = factored;
+  p.inv_s = inv_s;
+  p.q = q;
+  p.scales = scales;
+  lane_layout(M, nb, int64_t(dev->sms) * per_sm * kq::kSThreads, p);
+  const int64_t grid = (p.threads + kq::kSThreads - 1) / kq::kSThreads;
+  return launch_pdl(kern, dim3(unsigned(grid)), kq::kSThreads, kq::kSSmemBytes, stream, "quant_kernel launch", p);
+}
 
 // Row-tile stride for a grid of ncol column groups on sms SMs holding per_sm
 // CTAs each: fill the resident slots once, then balance the row tiles.
@@ -112,68 +195,6 @@ int64_t row_stride(int64_t ncol, int64_t nrt, int sms, int per_sm) {
   gy = (nrt + per - 1) / per;
   if (gy > 65535) gy = 65535;
   return gy;
-}
-
-template <int MODE, int TILED, int NT = 32>
-kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const float* mats, const float* factored,
-                       const float* inv_s, uint8_t* q, uint8_t* scales, cudaStream_t stream) {
-  const DeviceInfo* dev = device_info();
-  if (dev == nullptr) return cuda_fail("device query", cudaErrorInvalidDevice);
-  EncodeTiledFn enc = encode_tiled();
-  if (enc == nullptr) return cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
-  const int nb = int(d / 32);
-  const int smem = 1024 /*alignment slack*/ + kq::kQStages * kq::kQStageBytes + kq::kQCols * kq::kQCoef * 4 +
-                   2 * kq::kQStages * 8;
-  if (smem > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
-
-  CUtensorMap tmap;
-  const cuuint64_t gdim[3] = {32, cuuint64_t(M), cuuint64_t(nb)};
-  const cuuint64_t gstride[2] = {cuuint64_t(ldx) * 2, 64};
-  const cuuint32_t box[3] = {32, cuuint32_t(kq::kQRows), cuuint32_t(kq::kQCols)};
-  const cuuint32_t estride[3] = {1, 1, 1};
-  if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), gdim, gstride, box, estride,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cuda_fail("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
-
-  auto kern = kq::quant_kernel<MODE, TILED, NT>;
-  static std::atomic<int> attr_set[kMaxDevices];
-  int devid = 0;
-  cudaGetDevice(&devid);
-  if (!attr_set[devid].load()) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
-    attr_set[devid].store(1);
-  }
-  static std::atomic<int> occ[kMaxDevices];
-  int per_sm = occ[devid].load();
-  if (per_sm == 0) {
-    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kq::kQThreads, smem);
-    if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveBlocksPerMultiprocessor", e);
-    if (per_sm < 1) return cuda_fail("occupancy: no resident CTA", cudaErrorInvalidConfiguration);
-    occ[devid].store(per_sm);
-  }
-
-  kq::QuantParams p;
-  p.x = static_cast<const uint16_t*>(x);
-  p.ldx = ldx;
-  p.M = M;
-  p.nb = nb;
-  const int64_t nrt = (M + kq::kQRows - 1) / kq::kQRows;
-  if (nrt > int64_t(INT32_MAX) / kq::kQRows) return KQ_ERR_SHAPE;  // TMA row coordinates are int32
-  p.n_row_tiles = int(nrt);
-  p.coef_offset = kq::kQStages * kq::kQStageBytes;
-  p.mats = mats;
-  p.factored = factored;
-  p.inv_s = inv_s;
-  p.q = q;
-  p.scales = scales;
-
-  const int64_t ncol = (nb + kq::kQCols - 1) / kq::kQCols;
-  if (ncol > int64_t(INT32_MAX)) return KQ_ERR_SHAPE;
-  const int64_t gy = row_stride(ncol, nrt, dev->sms, per_sm);
-  return launch_pdl(kern, dim3(unsigned(ncol), unsigned(gy)), kq::kQThreads, smem, stream, "quant_kernel launch",
-                    tmap, p);
 }
 
 // Tensor-core variant: 128-row x 4-block tiles, one CTA per 4-block column group
@@ -256,11 +277,70 @@ int grid_for(int64_t work, int threads) {
   return g < 1 ? 1 : int(g);
 }
 
+// ---- variant selection for KQ_VAR_AUTO
+//
+// The faster variant for fp32 matrices with the factored form given, as measured
+// at the shapes of the quantizer sweep (rows M x channels d, 32-element blocks;
+// the sweep table of every kernel kind at every shape is the source).  A shape
+// takes the entry of the nearest swept shape, distance measured in log2 M and
+// log2 d.  bf16 matrices, and fp32 matrices without the factored form, have only
+// the tensor-core variant.
+struct AutoRule {
+  int64_t M, d;
+  kq_variant v;
+};
+constexpr AutoRule kAutoTable[] = {
+    {1, 1152, KQ_VAR_BUTTERFLY},     {1, 3072, KQ_VAR_BUTTERFLY},     {1, 12288, KQ_VAR_BUTTERFLY},
+    {16, 1152, KQ_VAR_BUTTERFLY},    {16, 3072, KQ_VAR_MMA},          {16, 12288, KQ_VAR_BUTTERFLY},
+    {256, 1152, KQ_VAR_BUTTERFLY},   {256, 3072, KQ_VAR_BUTTERFLY},   {256, 12288, KQ_VAR_BUTTERFLY},
+    {4096, 1152, KQ_VAR_BUTTERFLY},  {4096, 3072, KQ_VAR_BUTTERFLY},  {4096, 12288, KQ_VAR_BUTTERFLY},
+    {16384, 1152, KQ_VAR_BUTTERFLY}, {16384, 3072, KQ_VAR_BUTTERFLY}, {16384, 12288, KQ_VAR_BUTTERFLY},
+    {65536, 1152, KQ_VAR_BUTTERFLY}, {65536, 3072, KQ_VAR_BUTTERFLY}, {65536, 12288, KQ_VAR_BUTTERFLY},
+};
+
+kq_variant table_variant(int64_t M, int64_t d) {
+  const double lm = std::log2(double(M > 0 ? M : 1)), ld = std::log2(double(d > 0 ? d : 1));
+  double best = 1e300;
+  kq_variant v = KQ_VAR_BUTTERFLY;
+  for (const AutoRule& r : kAutoTable) {
+    const double dm = std::log2(double(r.M)) - lm, dd = std::log2(double(r.d)) - ld;
+    const double dist = dm * dm + dd * dd;
+    if (dist < best) {
+      best = dist;
+      v = r.v;
+    }
+  }
+  return v;
+}
+
+// KQ_VARIANT=mma|butterfly in the environment replaces the table's choice for
+// KQ_VAR_AUTO where that variant can serve the call (read once per process).
+kq_variant env_variant() {
+  static const kq_variant v = []() {
+    const char* e = std::getenv("KQ_VARIANT");
+    if (e == nullptr) return KQ_VAR_AUTO;
+    if (std::strcmp(e, "mma") == 0) return KQ_VAR_MMA;
+    if (std::strcmp(e, "butterfly") == 0) return KQ_VAR_BUTTERFLY;
+    return KQ_VAR_AUTO;
+  }();
+  return v;
+}
+
+// The variant kq_quantize runs: an explicit request as given; KQ_VAR_AUTO through
+// the override, then the table, within what the matrices allow.
+kq_variant resolve_variant(int64_t M, int64_t d, kq_dtype mat_dtype, bool has_factored, kq_variant requested) {
+  if (requested != KQ_VAR_AUTO) return requested;
+  if (mat_dtype == KQ_BF16 || !has_factored) return KQ_VAR_MMA;
+  const kq_variant e = env_variant();
+  if (e != KQ_VAR_AUTO) return e;
+  return table_variant(M, d);
+}
+
 }  // namespace
 
 extern "C" {
 
-int kq_abi_version(void) { return 200; }
+int kq_abi_version(void) { return 201; }
 
 const char* kq_status_string(kq_status s) {
   switch (s) {
@@ -337,11 +417,9 @@ kq_status kq_quantize_n(const void* x, int64_t M, int64_t d, int64_t ldx, int lo
                ? launch_quant<kq::MODE_KRON, 1, 64>(x, M, d, ldx, m32, factored, nullptr, q, scales, as_cuda(stream))
                : launch_quant<kq::MODE_KRON, 0, 64>(x, M, d, ldx, m32, factored, nullptr, q, scales, as_cuda(stream));
   }
-  // bf16 matrices are only served by the tensor-core variant; AUTO picks the
-  // butterfly for fp32 matrices when the factored form is given
-  const bool use_mma = variant == KQ_VAR_MMA || mat_dtype == KQ_BF16 ||
-                       (variant == KQ_VAR_AUTO && factored == nullptr);
+  // bf16 matrices are only served by the tensor-core variant; AUTO resolves per shape
   if (variant == KQ_VAR_BUTTERFLY && mat_dtype == KQ_BF16) return KQ_ERR_UNSUPPORTED;
+  const bool use_mma = resolve_variant(M, d, mat_dtype, factored != nullptr, variant) == KQ_VAR_MMA;
   if (use_mma)
     return launch_quant_mma(x, M, d, ldx, mats, mat_dtype == KQ_BF16, q, scales, sf_tiled, as_cuda(stream));
   if (factored == nullptr) return KQ_ERR_INVALID_ARG;
@@ -402,6 +480,19 @@ kq_status kq_e2m1_pack(const float* v, int64_t n, uint8_t* out, kq_stream_t stre
   if (!aligned(v, 16) || !aligned(out, 4)) return KQ_ERR_ALIGN;
   kq::e2m1_pack_kernel<<<grid_for(n / 8 + 1, 256), 256, 0, as_cuda(stream)>>>(v, n, out);
   return launch_status("e2m1_pack_kernel launch");
+}
+
+kq_status kq_select_variant(int64_t M, int64_t d, int log2n, kq_dtype mat_dtype, int has_factored,
+                            kq_variant* chosen) {
+  if (chosen == nullptr || M < 0 || d < 0 || (mat_dtype != KQ_F32 && mat_dtype != KQ_BF16)) return KQ_ERR_INVALID_ARG;
+  if (log2n != 5 && log2n != 6) return KQ_ERR_INVALID_ARG;
+  if (log2n == 6) {  // 64-element blocks: the butterfly only
+    if (mat_dtype == KQ_BF16 || !has_factored) return KQ_ERR_UNSUPPORTED;
+    *chosen = KQ_VAR_BUTTERFLY;
+    return KQ_OK;
+  }
+  *chosen = resolve_variant(M, d, mat_dtype, has_factored != 0, KQ_VAR_AUTO);
+  return KQ_OK;
 }
 
 const char* kq_last_error(void) { return g_last_error; }

@@ -359,8 +359,8 @@ __global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(c
       uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16;
       uint8_t* sb = p.scales + scale_index(rowc, bc, p.nb, TILED);
       const uint16_t* xb = p.x + rowc * p.ldx + int64_t(bc) * kBlock;
-      certify_store(Y, amax, l1, zero_block, cfac, kMmaErrAbs, !(cfac <= FLT_MAX), act, qb, sb,
-                    [&](bool need) { warp_exact_pass<KSRC>(need, xb, Kb, qb, sb); });
+      const bool need = certify_store(Y, amax, l1, zero_block, cfac, kMmaErrAbs, !(cfac <= FLT_MAX), act, qb, sb);
+      if (__any_sync(0xFFFFFFFFu, need)) warp_exact_pass<KSRC>(need, xb, Kb, qb, sb);
     }
   }
   tc_fence_before();

@@ -96,10 +96,12 @@ __device__ __noinline__ void exact_block_warp(const uint16_t* __restrict__ xb, c
       xw[4 * k + 2] = v.z;
       xw[4 * k + 3] = v.w;
     }
+    // every product is exact in fp64, so the fused multiply-add rounds exactly as
+    // the addition of the product would
 #pragma unroll
     for (int i = 0; i < kBlock; i++) {
       const float xi = (i & 1) ? bf16hi(xw[i >> 1]) : bf16lo(xw[i >> 1]);
-      acc = __dadd_rn(acc, __dmul_rn(double(xi), double(kc[i])));
+      acc = __fma_rn(double(xi), double(kc[i]), acc);
     }
   }
   const float y = __double2float_rn(acc);
@@ -149,17 +151,17 @@ __device__ __forceinline__ void warp_exact_pass(bool need, const uint16_t* xb, c
 // amax = max|y| (NaN-propagating), and E = cfac * l1 + eabs bounds |y - y32|
 // for every element, y32 being the definition's value; zero_block is the exact
 // test that every input of the block is +-0 (then y = +0 when every matrix entry
-// is finite).  exact_only sends every block, zero or not, to the exact path.  The scale is taken from
-// amax only when amax - E and amax + E (directed rounding) give the same E8M0
-// byte; each code only when (y - E) 2^-e rounded down and (y + E) 2^-e rounded
-// up give the same E2M1 code.  Any block that fails either test is recomputed
-// exactly by the warp.  Must be called by all 32 lanes; act marks real blocks.
-// exact_pass(need) must recompute, warp-cooperatively, the block of every lane
-// with need == true and store its codes and scale.
-template <class ExactPass>
-__device__ __forceinline__ void certify_store(const uint64_t (&Y)[16], float amax, float l1, bool zero_block,
+// is finite).  exact_only sends every block, zero or not, to the exact path.  The
+// scale is taken from amax only when amax - E and amax + E (directed rounding)
+// give the same E8M0 byte; each code only when (y - E) 2^-e rounded down and
+// (y + E) 2^-e rounded up give the same E2M1 code.  For a real block (act) the
+// fast codes and scale are stored either way; the return value says whether the
+// block is uncertain, in which case the caller must recompute it exactly and
+// store over them (warp_exact_pass).  Keeping the recomputation out of this step
+// leaves nothing of it on the per-block path but one vote.
+__device__ __forceinline__ bool certify_store(const uint64_t (&Y)[16], float amax, float l1, bool zero_block,
                                               float cfac, float eabs, bool exact_only, bool act, uint8_t* qb,
-                                              uint8_t* sb, const ExactPass& exact_pass) {
+                                              uint8_t* sb) {
   // zero_block: all inputs +-0, so every y is +0 by definition (byte 0, codes 0)
   const float E = __fmaf_ru(cfac, l1, eabs);
   bool exact = exact_only || !(amax <= FLT_MAX) || !(E <= FLT_MAX);
@@ -182,18 +184,14 @@ __device__ __forceinline__ void certify_store(const uint64_t (&Y)[16], float ama
     cp[k] = codes8(V);
   }
   const uint32_t diff = (cm[0] ^ cp[0]) | (cm[1] ^ cp[1]) | (cm[2] ^ cp[2]) | (cm[3] ^ cp[3]);
+  if (act) {
+    const uint32_t keep = zero_block ? 0u : 0xFFFFFFFFu;
+    *reinterpret_cast<uint4*>(qb) = make_uint4(cm[0] & keep, cm[1] & keep, cm[2] & keep, cm[3] & keep);
+    *sb = uint8_t(zero_block ? 0 : byte);
+  }
   // a block with an uncertain scale or an uncertain code is recomputed exactly;
   // with exact_only (matrix entries possibly non-finite) so is an all-zero block
-  const bool need = act && (exact_only || (!zero_block && (exact || diff != 0u)));
-  exact_pass(need);
-  if (!act || need) return;
-  if (zero_block) {
-    *reinterpret_cast<uint4*>(qb) = make_uint4(0u, 0u, 0u, 0u);
-    *sb = 0;
-    return;
-  }
-  *reinterpret_cast<uint4*>(qb) = make_uint4(cm[0], cm[1], cm[2], cm[3]);
-  *sb = uint8_t(byte);
+  return act && (exact_only || (!zero_block && (exact || diff != 0u)));
 }
 
 }  // namespace kq

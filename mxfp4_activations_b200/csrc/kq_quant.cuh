@@ -10,22 +10,26 @@
 //               form (c/a = 1, b/d = -1, D_j = +-2^-2.5): the FWHT comparison point.
 //   MODE_SMOOTH per-channel scaling y_j = x_j s_j: the SmoothQuant comparison point.
 //
-// Data movement: a tile is 8 block columns x 32 rows (16 KB of bf16), fetched by
-// one 3-D TMA load (box {32 elements, 32 rows, 8 blocks}, 64-byte swizzle, no
-// multicast) into a ring of shared-memory stages; in shared memory the tile is
-// [block column][row][64 B].  A CTA owns one group of 8 block columns and walks
-// a stride of row tiles.  Its last warp only issues the loads; a stage is
-// refilled when every consumer warp has arrived on its "empty" barrier, so
-// consumer warps never wait for each other.  Consumer warp w holds block
-// columns 4(w&1)..4(w&1)+3 and rows 8(w>>1)..8(w>>1)+7 of each tile: lane l
-// takes column 4(w&1) + l/8 and row 8(w>>1) + l%8.  Eight lanes share a column,
-// so the per-column coefficients are read from a shared table by broadcast loads
-// (four distinct addresses per warp, in distinct banks) instead of living in
-// registers, and the four 16-byte shared loads of a block stay conflict-free
-// under the swizzle (chunk k of 64-byte row t sits at chunk k ^ ((t >> 1) & 3)).
-// Each row's four blocks give 64 contiguous bytes of codes per warp store.
-// The butterfly stages on index bits 1..4 run as packed f32x2 FMAs on element
-// pairs (2m, 2m+1).
+// Work mapping.  The [M][nb] grid of 32-element blocks is cut into "lanes": lane
+// v owns block column c = v % nb and the rows r0 = v / nb, r0 + k, r0 + 2k, ...
+// (k rows in flight, k * nb lanes).  Thread t takes lane t, so a thread keeps one
+// block column for its whole life: its butterfly coefficients (or per-channel
+// factors) are loaded once into registers and no per-block coefficient traffic
+// remains.  Consecutive threads hold consecutive block columns of one row, so a
+// warp reads 2 KB of contiguous input and writes 512 contiguous bytes of codes and
+// 32 contiguous scale bytes per row step.  When nb exceeds the threads of one
+// wave, threads walk several lanes.
+//
+// Data movement.  Each thread streams its own blocks through a private ring of
+// kSStages 64-byte slots in shared memory with asynchronous copies (cp.async, four
+// 16-byte pieces per block): kSStages - 1 blocks are in flight while one is
+// computed, without holding registers.  Piece k of thread t's slot sits at 16-byte
+// position k ^ ((t >> 1) & 3), so the four 16-byte reads of a block are free of
+// bank conflicts across each group of eight threads.
+//
+// A row step stores every block's fast result; the rare blocks that the fp32 bound
+// cannot certify (below) are then recomputed exactly by the whole warp, which
+// overwrites their fast results.
 //
 // Exactness (KRON, FWHT): the fp32 result y_f differs from the definition
 // y32 = fp32(sum_i x_i K32[i][j]) by at most E = C * ||x||_1 * max|K|.  KRON:
@@ -50,102 +54,143 @@ namespace kq {
 
 enum Mode { MODE_KRON = 0, MODE_FWHT = 1, MODE_SMOOTH = 2 };
 
-constexpr float kKronErrC = 9.5367431640625e-07f;   // 2^-20 = 16 u (14 u needed, see below)
+constexpr float kKronErrC = 9.5367431640625e-07f;   // 2^-20 = 16 u (14 u needed, see above)
 constexpr float kKronErrC64 = 1.9073486328125e-06f; // 2^-19 = 32 u for 64-element blocks (16 u needed)
 constexpr float kFwhtErrC = 4.76837158203125e-07f;  // 2^-21 = 8 u (7 u needed)
 constexpr float kErrAbs = 7.174648137343064e-43f;   // 2^-140: FWHT subnormal-range slack
 
-// Tile geometry (see "Data movement" above).
-constexpr int kQCols = 8;                        // block columns per tile
-constexpr int kQRows = 32;                       // rows per tile
-constexpr int kQConsWarps = 8;                   // consumer warps (4 columns x 8 rows each)
-constexpr int kQThreads = (kQConsWarps + 1) * 32;  // + the TMA producer warp
-constexpr int kQStageBytes = kQCols * kQRows * 64;  // 16 KB
-constexpr int kQStages = 4;
-// Shared coefficient table, one record of kQCoef floats per block column:
-//   [4s .. 4s+3]  (lam, lam, bet, bet) of the stage on index bit s+1 (factor 3-s), s = 0..3
-//   [16 .. 47]    D_0 .. D_31 (SMOOTH: the 32 per-channel factors)
-//   [48 .. 51]    lam and bet of factor 4 (index bit 0), C * max|K| (+inf: exact path
-//                 only), absolute allowance
-//   [52 .. 53]    lam and bet of the factor that mixes the two 32-element halves of a
-//                 64-element transform block (64-element blocks only)
-constexpr int kQCoef = 56;
+constexpr int kSThreads = 256;    // threads per CTA
+constexpr int kSCtasPerSm = 2;    // resident CTAs per SM the register budget is written for
+constexpr int kSStages = 4;       // 64-byte slots per thread (blocks in flight + 1)
+constexpr int kSSmemBytes = kSStages * kSThreads * 64;
 
 struct QuantParams {
-  const uint16_t* x;      // bf16 bits [M][ldx] (exact path re-reads rows from here)
+  const uint16_t* x;      // bf16 bits [M][ldx]
   int64_t ldx;
   int64_t M;
+  int64_t k;              // rows in flight per lane pass (row step of a lane)
+  int64_t lanes;          // k * nb (every lane: one block column, rows r0 + i k)
+  int64_t threads;        // threads that take lanes (lane v is taken by thread v % threads)
+  int64_t n_iter;         // row steps per lane: ceil(M / k)
+  int passes;             // lanes per thread: ceil(lanes / threads)
   int nb;                 // blocks per row (d / 32)
-  int n_row_tiles;        // ceil(M / 32)
-  int coef_offset;        // bytes from the stage ring to the coefficient table (kQStages * kQStageBytes)
-  const float* mats;      // KRON: fp32 [nb][32][32] (exact path)
+  const float* mats;      // KRON: fp32 [nb/(NT/32)][NT][NT] (exact path)
   const float* factored;  // KRON: [nb][48]
   const float* inv_s;     // SMOOTH: [nb*32]
   uint8_t* q;             // [M][nb*16]
   uint8_t* scales;        // row-major [M][nb], or tiled (scale_index)
 };
 
-// Entry f of the coefficient record of block column b (fp32 bits as read by
-// the consumer warps).
+// Coefficients of one block column, held in registers by the thread that owns it.
+struct ColCoef {
+  float l4, b4;         // stage on index bit 0 (factor 4): lam, bet
+  uint64_t L[4], B[4];  // stages on index bits 1..4 (factors 3..0): (lam, lam), (bet, bet)
+  uint64_t D[16];       // (D_2m, D_2m+1); SMOOTH: the per-channel factors
+  float cfac;           // C * max|K| (+inf: the column takes the exact path only)
+  float eabs;           // absolute allowance (results in the fp32 subnormal range)
+  float mix;            // 64-element blocks: lam (lower half) or bet (upper half) of F0
+};
+
 template <int MODE, int NT>
-__device__ __forceinline__ float coef_entry(const QuantParams& p, int b, int f) {
+__device__ __forceinline__ void load_coef(const QuantParams& p, int c, ColCoef& cf) {
+  cf.l4 = 1.0f;
+  cf.b4 = -1.0f;
+  cf.cfac = kFwhtErrC * kFwhtC;
+  cf.eabs = kErrAbs;
+  cf.mix = 0.0f;
+#pragma unroll
+  for (int s = 0; s < 4; s++) cf.L[s] = cf.B[s] = 0;
   if (MODE == MODE_KRON) {
-    const float* fb = p.factored + int64_t(b) * kFactored;
-    if (f < 16) {
-      const int k = 3 - (f >> 2);                  // factor of this stage
-      return __ldg(fb + ((f & 2) ? 5 + k : k));    // bet_k = b/d, lam_k = c/a
+    const float4* fb = reinterpret_cast<const float4*>(p.factored + int64_t(c) * kFactored);
+    float r[kFactored];
+#pragma unroll
+    for (int i = 0; i < kFactored / 4; i++) {
+      const float4 v = __ldg(fb + i);
+      r[4 * i] = v.x;
+      r[4 * i + 1] = v.y;
+      r[4 * i + 2] = v.z;
+      r[4 * i + 3] = v.w;
     }
-    if (f < 48) return __ldg(fb + 10 + (f - 16));  // D
-    if (f == 48) return __ldg(fb + 4);
-    if (f == 49) return __ldg(fb + 9);
-    if (f == 50)
-      return __ldg(fb + 43) != 0.0f ? __int_as_float(0x7F800000)
-                                    : __fmul_ru(NT == 64 ? kKronErrC64 : kKronErrC, __ldg(fb + 42));
-    if (f == 51) return __ldg(fb + 44);
-    if (NT == 64 && f == 52) return __ldg(fb + 45);
-    if (NT == 64 && f == 53) return __ldg(fb + 46);
-    return 0.0f;
+    cf.l4 = r[4];
+    cf.b4 = r[9];
+#pragma unroll
+    for (int s = 0; s < 4; s++) {  // stage on bit s+1 uses factor 3-s
+      cf.L[s] = pk2(r[3 - s], r[3 - s]);
+      cf.B[s] = pk2(r[8 - s], r[8 - s]);
+    }
+#pragma unroll
+    for (int m = 0; m < 16; m++) cf.D[m] = pk2(r[10 + 2 * m], r[11 + 2 * m]);
+    cf.cfac = r[43] != 0.0f ? __int_as_float(0x7F800000) : __fmul_ru(NT == 64 ? kKronErrC64 : kKronErrC, r[42]);
+    cf.eabs = r[44];
+    cf.mix = (c & 1) ? r[46] : r[45];
+  } else if (MODE == MODE_SMOOTH) {
+    const float4* sp = reinterpret_cast<const float4*>(p.inv_s + int64_t(c) * kBlock);
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const float4 v = __ldg(sp + i);
+      cf.D[2 * i] = pk2(v.x, v.y);
+      cf.D[2 * i + 1] = pk2(v.z, v.w);
+    }
   }
-  if (MODE == MODE_SMOOTH) return (f >= 16 && f < 48) ? __ldg(p.inv_s + int64_t(b) * kBlock + (f - 16)) : 0.0f;
-  return 0.0f;
+}
+
+// Asynchronous copy of one block (64 bytes at p, 16-byte aligned) into the slot
+// whose 16-byte pieces are at slot + ((k ^ sw) << 4); completes with the thread's
+// next commit group.
+__device__ __forceinline__ void copy_block_async(uint32_t slot, int sw, const uint16_t* p) {
+#pragma unroll
+  for (int k = 0; k < 4; k++)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(slot + uint32_t((k ^ sw) << 4)), "l"(p + 8 * k)
+                 : "memory");
+}
+__device__ __forceinline__ void copy_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's commit groups are still in flight.
+template <int N>
+__device__ __forceinline__ void copy_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// The 64 bytes of a landed slot as 16 words: word h holds elements 2h (low half)
+// and 2h+1 (high half) of the block.
+__device__ __forceinline__ void read_slot(uint32_t slot, int sw, uint32_t (&w)[16]) {
+#pragma unroll
+  for (int k = 0; k < 4; k++) {
+    const uint4 v = lds128(slot + uint32_t((k ^ sw) << 4));
+    w[4 * k] = v.x;
+    w[4 * k + 1] = v.y;
+    w[4 * k + 2] = v.z;
+    w[4 * k + 3] = v.w;
+  }
 }
 
 // ---------------------------------------------------------------- one block of one row
 //
-// cf: shared-memory address of this block column's coefficient record.  NT = 64:
-// the block is one half of a 64-element transform block whose other half is held
-// by lane ^ 8 (same row, neighbouring column); `upper` marks the second half.
+// NT = 64: the block is one half of a 64-element transform block whose other half
+// is held by lane ^ 1 (same row, neighbouring column); (c & 1) marks the upper half.
+// act marks the lanes whose block is real.  Stores the fast result of a real
+// block and returns whether it must be recomputed exactly (never for SMOOTH, whose
+// fp32 product is the definition itself).
 template <int MODE, int NT>
-__device__ __forceinline__ void quant_block(uint32_t cf, const uint4 (&xr)[4], bool act, uint8_t* qb, uint8_t* sb,
-                                            const uint16_t* xb, const float* Kb, bool upper) {
+__device__ __forceinline__ bool quant_block(const ColCoef& cf, const uint32_t (&w)[16], bool act, uint8_t* qb,
+                                            uint8_t* sb) {
   float x[kBlock];
 #pragma unroll
-  for (int k = 0; k < 4; k++) {
-    const uint32_t w[4] = {xr[k].x, xr[k].y, xr[k].z, xr[k].w};
-#pragma unroll
-    for (int h = 0; h < 4; h++) {
-      x[8 * k + 2 * h] = bf16lo(w[h]);
-      x[8 * k + 2 * h + 1] = bf16hi(w[h]);
-    }
+  for (int h = 0; h < 16; h++) {
+    x[2 * h] = bf16lo(w[h]);
+    x[2 * h + 1] = bf16hi(w[h]);
   }
   uint64_t Y[16];
   float y[kBlock];
 
   if (MODE == MODE_SMOOTH) {
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-      const uint4 dv = lds128(cf + 64 + 16 * i);
-      Y[2 * i] = mul2_rn(pk2(x[4 * i], x[4 * i + 1]), pk2(__uint_as_float(dv.x), __uint_as_float(dv.y)));
-      Y[2 * i + 1] = mul2_rn(pk2(x[4 * i + 2], x[4 * i + 3]), pk2(__uint_as_float(dv.z), __uint_as_float(dv.w)));
-    }
+    for (int m = 0; m < 16; m++) Y[m] = mul2_rn(pk2(x[2 * m], x[2 * m + 1]), cf.D[m]);
 #pragma unroll
     for (int m = 0; m < 16; m++) upk2(Y[m], y[2 * m], y[2 * m + 1]);
     const float amax = block_amax(y);
-    if (!act) return;
+    if (!act) return false;
     if (!(amax <= FLT_MAX)) {
       *reinterpret_cast<uint4*>(qb) = make_uint4(0u, 0u, 0u, 0u);
       *sb = 0xFF;
-      return;
+      return false;
     }
     const int byte = e8m0_byte(amax);
     const uint64_t S2 = pk2(inv_scale_of_byte(byte), inv_scale_of_byte(byte));
@@ -153,7 +198,7 @@ __device__ __forceinline__ void quant_block(uint32_t cf, const uint4 (&xr)[4], b
     for (int m = 0; m < 16; m++) Y[m] = mul2_rn(Y[m], S2);
     *reinterpret_cast<uint4*>(qb) = make_uint4(codes8(Y), codes8(Y + 4), codes8(Y + 8), codes8(Y + 12));
     *sb = uint8_t(byte);
-    return;
+    return false;
   }
 
   // ||x||_1 rounded upward (four partial sums for ILP)
@@ -161,52 +206,32 @@ __device__ __forceinline__ void quant_block(uint32_t cf, const uint4 (&xr)[4], b
 #pragma unroll
   for (int j = 0; j < kBlock; j++) l1p[j & 3] = __fadd_ru(l1p[j & 3], fabsf(x[j]));
   float l1 = __fadd_ru(__fadd_ru(l1p[0], l1p[1]), __fadd_ru(l1p[2], l1p[3]));
-  // every output of a 64-element block depends on all 64 inputs
   if (NT == 64) {
-    l1 = __fadd_ru(l1, __shfl_xor_sync(0xFFFFFFFFu, l1, 8));
+    // every output of a 64-element block depends on all 64 inputs
+    l1 = __fadd_ru(l1, __shfl_xor_sync(0xFFFFFFFFu, l1, 1));
     // factor 0 of a 64-element block, applied first (the Kronecker factors act on
     // different index bits and commute): x_lo + lam x_hi in the lower half, x_hi +
     // bet x_lo in the upper one, element by element, with the partner half's inputs
-    // taken from lane ^ 8 as raw bf16 pairs (16 shuffles)
-    const uint4 cx = lds128(cf + 208);
-    const float cc = upper ? __uint_as_float(cx.y) : __uint_as_float(cx.x);
-    const uint64_t C2 = pk2(cc, cc);
+    // taken from lane ^ 1 as raw bf16 pairs (16 shuffles)
+    const uint64_t C2 = pk2(cf.mix, cf.mix);
 #pragma unroll
-    for (int k = 0; k < 4; k++) {
-      const uint32_t w[4] = {xr[k].x, xr[k].y, xr[k].z, xr[k].w};
-#pragma unroll
-      for (int h = 0; h < 4; h++) {
-        const uint32_t pw = __shfl_xor_sync(0xFFFFFFFFu, w[h], 8);
-        const uint64_t X = fma2_rn(C2, pk2(bf16lo(pw), bf16hi(pw)), pk2(x[8 * k + 2 * h], x[8 * k + 2 * h + 1]));
-        upk2(X, x[8 * k + 2 * h], x[8 * k + 2 * h + 1]);
-      }
+    for (int h = 0; h < 16; h++) {
+      const uint32_t pw = __shfl_xor_sync(0xFFFFFFFFu, w[h], 1);
+      const uint64_t X = fma2_rn(C2, pk2(bf16lo(pw), bf16hi(pw)), pk2(x[2 * h], x[2 * h + 1]));
+      upk2(X, x[2 * h], x[2 * h + 1]);
     }
   }
 
-  float cfac, eabs;
   // stage on index bit 0 (factor 4), scalar: the pair partners share a register pair
-  {
-    float l4 = 1.0f, b4 = -1.0f;
-    if (MODE == MODE_KRON) {
-      const uint4 s0 = lds128(cf + 192);
-      l4 = __uint_as_float(s0.x);
-      b4 = __uint_as_float(s0.y);
-      cfac = __uint_as_float(s0.z);
-      eabs = __uint_as_float(s0.w);
-    } else {
-      cfac = kFwhtErrC * kFwhtC;
-      eabs = kErrAbs;
-    }
 #pragma unroll
-    for (int m = 0; m < 16; m++) {
-      const float x0 = x[2 * m], x1 = x[2 * m + 1];
-      if (MODE == MODE_FWHT) {
-        x[2 * m] = __fadd_rn(x0, x1);
-        x[2 * m + 1] = __fsub_rn(x1, x0);
-      } else {
-        x[2 * m] = __fmaf_rn(l4, x1, x0);
-        x[2 * m + 1] = __fmaf_rn(b4, x0, x1);
-      }
+  for (int m = 0; m < 16; m++) {
+    const float x0 = x[2 * m], x1 = x[2 * m + 1];
+    if (MODE == MODE_FWHT) {
+      x[2 * m] = __fadd_rn(x0, x1);
+      x[2 * m + 1] = __fsub_rn(x1, x0);
+    } else {
+      x[2 * m] = __fmaf_rn(cf.l4, x1, x0);
+      x[2 * m + 1] = __fmaf_rn(cf.b4, x0, x1);
     }
   }
 #pragma unroll
@@ -214,12 +239,6 @@ __device__ __forceinline__ void quant_block(uint32_t cf, const uint4 (&xr)[4], b
   // stages on index bits 1..4 (factors 3..0) on packed pairs
 #pragma unroll
   for (int pb = 1; pb < 5; pb++) {
-    uint64_t L2 = 0, B2 = 0;
-    if (MODE == MODE_KRON) {
-      const uint4 c = lds128(cf + 16 * (pb - 1));
-      L2 = pk2(__uint_as_float(c.x), __uint_as_float(c.y));
-      B2 = pk2(__uint_as_float(c.z), __uint_as_float(c.w));
-    }
 #pragma unroll
     for (int m = 0; m < 16; m++) {
       if (m & (1 << (pb - 1))) continue;
@@ -229,142 +248,113 @@ __device__ __forceinline__ void quant_block(uint32_t cf, const uint4 (&xr)[4], b
         Y[m] = add2_rn(y0, y1);
         Y[m1] = sub2_rn(y1, y0);
       } else {
-        Y[m] = fma2_rn(L2, y1, y0);
-        Y[m1] = fma2_rn(B2, y0, y1);
+        Y[m] = fma2_rn(cf.L[pb - 1], y1, y0);
+        Y[m1] = fma2_rn(cf.B[pb - 1], y0, y1);
       }
     }
   }
   // diagonal: D_j (FWHT: +-2^-2.5 with the sign of (-1)^popcount(j))
-  if (MODE == MODE_FWHT) {
 #pragma unroll
-    for (int m = 0; m < 16; m++) {
+  for (int m = 0; m < 16; m++) {
+    if (MODE == MODE_FWHT) {
       const float sg = (__popc(m) & 1) ? -kFwhtC : kFwhtC;
       Y[m] = mul2_rn(pk2(sg, -sg), Y[m]);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-      const uint4 dv = lds128(cf + 64 + 16 * i);
-      Y[2 * i] = mul2_rn(pk2(__uint_as_float(dv.x), __uint_as_float(dv.y)), Y[2 * i]);
-      Y[2 * i + 1] = mul2_rn(pk2(__uint_as_float(dv.z), __uint_as_float(dv.w)), Y[2 * i + 1]);
+    } else {
+      Y[m] = mul2_rn(cf.D[m], Y[m]);
     }
   }
 #pragma unroll
   for (int m = 0; m < 16; m++) upk2(Y[m], y[2 * m], y[2 * m + 1]);
   const float amax = block_amax(y);
 
-  constexpr int KSRC = (MODE == MODE_FWHT) ? KSRC_FWHT : KSRC_F32;
   // l1 is an upward-rounded fp32 sum of |x| without flushing: 0 exactly when all inputs are +-0
   // cfac = +inf marks a column whose butterfly form is unusable: every block exact
-  certify_store(Y, amax, l1, l1 == 0.0f, cfac, eabs, !(cfac <= FLT_MAX), act, qb, sb,
-                [&](bool need) { warp_exact_pass<KSRC, NT>(need, xb, Kb, qb, sb); });
+  return certify_store(Y, amax, l1, l1 == 0.0f, cf.cfac, cf.eabs, !(cf.cfac <= FLT_MAX), act, qb, sb);
 }
 
 // ---------------------------------------------------------------- kernel
+
+// One row step of a lane: wait for the block of ring slot `slot` (offset of the
+// stage from the thread's slot base), refill the slot read one step earlier with
+// the block kSStages - 1 rows ahead, quantize, and recompute exactly every block
+// of the warp that the fp32 bound could not certify.
+template <int MODE, int TILED, int NT>
+__device__ __forceinline__ void row_step(const QuantParams& p, const ColCoef& cf, uint32_t cbase, int sw,
+                                         uint32_t slot, uint32_t refill, bool lane_ok, int c, int64_t r, int64_t f,
+                                         int64_t f_end, int64_t f_ahead, const uint16_t* xr, const uint16_t* xi) {
+  copy_wait<kSStages - 2>();  // this step's block has landed
+  uint32_t cur[16];
+  read_slot(cbase + slot, sw, cur);
+  if (lane_ok && f + f_ahead < f_end) copy_block_async(cbase + refill, sw, xi);
+  copy_commit();
+  const bool act = lane_ok && f < f_end;
+  const int64_t fc = act ? f : c;
+  uint8_t* qb = p.q + fc * 16;
+  uint8_t* sb = p.scales + (TILED ? scale_index(act ? r : 0, c, p.nb, 1) : fc);
+  const bool need = quant_block<MODE, NT>(cf, cur, act, qb, sb);
+  if (MODE != MODE_SMOOTH && __any_sync(0xFFFFFFFFu, need)) {
+    // rare: the transform block's first input and this block's columns of its matrix
+    const int cx = c - c % (NT / kBlock);
+    const uint16_t* xb = xr - (c - cx) * kBlock;
+    const float* Kb = (MODE == MODE_KRON)
+                          ? p.mats + int64_t(c / (NT / kBlock)) * NT * NT + (c % (NT / kBlock)) * kBlock
+                          : nullptr;
+    constexpr int KSRC = (MODE == MODE_FWHT) ? KSRC_FWHT : KSRC_F32;
+    warp_exact_pass<KSRC, NT>(need, xb, Kb, qb, sb);
+  }
+}
 
 // TILED: scales in the 128 x 4 tiled layout of block-scaled GEMMs (a template
 // parameter, so the row-major store costs nothing extra).  NT: transform block of
 // 32 or 64 elements (KRON only; 64 needs an even number of block columns).
 template <int MODE, int TILED, int NT>
-__global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // [kQCols][kQCoef] after the stages; the offset comes from the host (kept out of
-  // the compile-time address arithmetic, which otherwise costs the loop a register)
-  float* coef = reinterpret_cast<float*>(base + p.coef_offset);
-  uint64_t* full = reinterpret_cast<uint64_t*>(coef + kQCols * kQCoef);
-  uint64_t* empty = full + kQStages;
-
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int col0 = int(blockIdx.x) * kQCols;
-  const int my_tiles = (p.n_row_tiles - int(blockIdx.y) + int(gridDim.y) - 1) / int(gridDim.y);
-
-  if (t == 0) {
-    for (int s = 0; s < kQStages; s++) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], uint32_t(kQConsWarps));
-    }
-    fence_mbar_init();
-  }
-  __syncthreads();
+__global__ void __launch_bounds__(kSThreads, kSCtasPerSm) quant_kernel(const __grid_constant__ QuantParams p) {
+  static_assert(kSStages == 4, "the row loop below is written for a ring of four slots");
+  extern __shared__ __align__(128) uint8_t ring[];
+  const int64_t t = int64_t(blockIdx.x) * kSThreads + threadIdx.x;
+  const int sw = (threadIdx.x >> 1) & 3;
+  const uint32_t cbase = smem_addr(ring) + threadIdx.x * 64u;
+  constexpr uint32_t kStage = kSThreads * 64u;  // bytes between the stages of one thread's ring
   grid_dependency_wait();  // inputs may come from the previous kernel in the stream
-
-  if (warp == kQConsWarps) {  // producer warp: one thread issues every TMA load
-    if (lane == 0) {
-      prefetch_tensormap(&tmap);
-      int it = 0;
-      for (; it < my_tiles; it++) {
-        const int s = it % kQStages;
-        if (it >= kQStages && !mbar_wait_bounded(&empty[s], uint32_t(it / kQStages - 1) & 1u, kWaitLimitNs))
-          break;
-        const int tile = int(blockIdx.y) + it * int(gridDim.y);
-        mbar_arrive_expect_tx(&full[s], uint32_t(kQStageBytes));
-        tma_load_3d(base + s * kQStageBytes, &tmap, &full[s], 0, tile * kQRows, col0);
-      }
-      grid_launch_dependents();  // every load issued: the next grid may start its prologue
-      if (it < my_tiles) {  // consumers stopped: let the loads still in flight land before exiting
-        for (int k = (it > kQStages ? it - kQStages : 0); k < it; k++)
-          mbar_wait_bounded(&full[k % kQStages], uint32_t(k / kQStages) & 1u, kWaitLimitNs / 4);
-      }
-    }
-    return;
-  }
-
-  // coefficient table of this CTA's columns (consumer warps only; the producer
-  // is already streaming the first tiles)
-  if (MODE != MODE_FWHT) {
-    constexpr int kN = kQCols * kQCoef;
-    constexpr int kPer = (kN + kQConsWarps * 32 - 1) / (kQConsWarps * 32);
-    float v[kPer];
+  for (int pass = 0; pass < p.passes; pass++) {
+    const int64_t v = t + int64_t(pass) * p.threads;
+    const bool lane_ok = t < p.threads && v < p.lanes;
+    const int64_t vc = lane_ok ? v : 0;
+    const int c = int(vc % p.nb);
+    const int64_t r0 = vc / p.nb;
+    const int64_t xstep = p.k * p.ldx;
+    const int64_t fstep = p.k * int64_t(p.nb);
+    const int64_t f_end = p.M * int64_t(p.nb);  // row r is real iff its flat index r nb + c < f_end
+    const uint16_t* xr = p.x + r0 * p.ldx + int64_t(c) * kBlock;  // this lane's block in row r
+    int64_t r = r0;                                                   // row of the step
+    int64_t f = r0 * int64_t(p.nb) + c;                               // flat block index of row r
+    // the first kSStages - 1 blocks of the lane go in flight before anything else
 #pragma unroll
-    for (int i = 0; i < kPer; i++) {
-      const int e = t + i * kQConsWarps * 32;
-      const int c = e / kQCoef;
-      v[i] = (e < kN && col0 + c < p.nb) ? coef_entry<MODE, NT>(p, col0 + c, e - c * kQCoef) : 0.0f;
+    for (int s = 0; s < kSStages - 1; s++) {
+      if (lane_ok && f + s * fstep < f_end) copy_block_async(cbase + s * kStage, sw, xr + s * xstep);
+      copy_commit();
     }
-#pragma unroll
-    for (int i = 0; i < kPer; i++) {
-      const int e = t + i * kQConsWarps * 32;
-      if (e < kN) coef[e] = v[i];
+    if (pass == 0) grid_launch_dependents();
+    ColCoef cf;
+    load_coef<MODE, NT>(p, c, cf);
+    const int64_t f_ahead = (kSStages - 1) * fstep;
+    const uint16_t* xi = xr + (kSStages - 1) * xstep;  // next block to put in flight
+    // two row steps per trip: step i uses stage i & 3, so the pair (i, i + 1) uses
+    // stages (h, h + 1) with h = 0 or 2 and refills (h + 3, h) & 3
+    uint32_t h = 0;
+    for (int64_t i = 0; i < p.n_iter; i += 2) {
+      row_step<MODE, TILED, NT>(p, cf, cbase, sw, h, (h + 3 * kStage) & (4 * kStage - 1), lane_ok, c, r, f, f_end,
+                                f_ahead, xr, xi);
+      if (i + 1 < p.n_iter)
+        row_step<MODE, TILED, NT>(p, cf, cbase, sw, h + kStage, h, lane_ok, c, r + p.k, f + fstep, f_end, f_ahead,
+                                  xr + xstep, xi + xstep);
+      h ^= 2 * kStage;
+      r += 2 * p.k;
+      f += 2 * fstep;
+      xr += 2 * xstep;
+      xi += 2 * xstep;
     }
-    asm volatile("bar.sync 1, %0;" ::"r"(kQConsWarps * 32) : "memory");
-  }
-
-  const int cl = (warp & 1) * 4 + (lane >> 3);  // block column inside the tile
-  const int rl = (warp >> 1) * 8 + (lane & 7);  // row inside the tile
-  const int b = col0 + cl;
-  const bool col_ok = b < p.nb;
-  const int bc = col_ok ? b : 0;
-  const uint32_t cf = smem_addr(coef + cl * kQCoef);
-  const uint32_t xoff = uint32_t(cl * kQRows + rl) * 64u;
-  const int sw = (rl >> 1) & 3;
-  const uint32_t sbase = smem_addr(base);
-  // exact path: this block's columns of its transform matrix ([nt][NT][NT]), and
-  // the transform block's first input
-  const float* Kb = (MODE == MODE_KRON)
-                        ? p.mats + int64_t(bc / (NT / kBlock)) * NT * NT + (bc % (NT / kBlock)) * kBlock
-                        : nullptr;
-  const int bx = bc - bc % (NT / kBlock);  // first block column of the transform block
-  const bool upper = (bc % (NT / kBlock)) != 0;
-  // per-tile pointer steps: gridDim.y row tiles of kQRows rows
-  const int64_t row_step = int64_t(gridDim.y) * kQRows;
-  int64_t row = int64_t(blockIdx.y) * kQRows + rl;
-
-  for (int it = 0; it < my_tiles; it++, row += row_step) {
-    const int s = it % kQStages;  // compile-time ring size: no integer division per block
-    if (!mbar_wait_bounded(&full[s], uint32_t(it / kQStages) & 1u, kWaitLimitNs)) break;
-    uint4 xr[4];
-    const uint32_t blk = sbase + uint32_t(s) * kQStageBytes + xoff;
-#pragma unroll
-    for (int k = 0; k < 4; k++) xr[k] = lds128(blk + uint32_t((k ^ sw) << 4));
-    stage_release(&empty[s], lane);
-    const bool act = col_ok && row < p.M;
-    const int64_t rowc = act ? row : 0;
-    uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16;
-    uint8_t* sb = p.scales + scale_index(rowc, bc, p.nb, TILED);
-    const uint16_t* xb = p.x + rowc * p.ldx + int64_t(bx) * kBlock;
-    // every lane takes part (the exact path is warp-cooperative); only real blocks store
-    quant_block<MODE, NT>(cf, xr, act, qb, sb, xb, Kb, upper);
+    copy_wait<0>();  // no copy of this pass still writes the ring
   }
 }
 

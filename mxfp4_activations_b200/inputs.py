@@ -30,8 +30,9 @@ SWEEP_D = (1152, 3072, 12288)
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """Round fp32 to bf16 (nearest, ties to even) and return the 16-bit patterns."""
     a = np.ascontiguousarray(a, np.float32)
-    w = a.view(np.uint32).astype(np.uint64)
-    rounded = ((w + 0x7FFF + ((w >> 16) & 1)) >> 16).astype(np.uint16)
+    w = a.view(np.uint32)
+    # only NaN patterns can wrap around in 32 bits; they are replaced below
+    rounded = ((w + np.uint32(0x7FFF) + ((w >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)
     nan = np.isnan(a)
     if nan.any():
         rounded[nan] = 0x7FC0

@@ -14,7 +14,7 @@ torch = pytest.importorskip("torch")
 
 from mxfp4_activations_b200 import inputs  # noqa: E402
 
-from .parity import compare, unpack  # noqa: E402
+from .parity import compare, guarded, guards_intact, oracle_rows, unpack  # noqa: E402
 
 pytestmark = [
     pytest.mark.gpu,
@@ -54,13 +54,34 @@ def host(t: "torch.Tensor") -> np.ndarray:
 VARIANTS = [("butterfly", "f32"), ("mma", "f32"), ("mma", "bf16")]
 
 
+def guarded_outputs(M: int, d: int, layout: str = "row"):
+    """q [M, d/2] and scales inside canary bytes (see tests/parity.py), plus the
+    backing buffers to check afterwards."""
+    from mxfp4_activations_b200 import scale_bytes
+
+    qv, qbuf = guarded(torch, M * (d // 2))
+    sv, sbuf = guarded(torch, scale_bytes(M, d, layout))
+    if layout == "mma":
+        sv.zero_()  # padding bytes of the tiled layout are not written
+    return qv.view(M, d // 2), (sv.view(M, d // 32) if layout == "row" else sv), (qbuf, sbuf)
+
+
+def assert_guards(bufs):
+    for b in bufs:
+        assert guards_intact(torch, b), "a kernel wrote outside its output buffer"
+
+
 def gpu_quantize(kq, x_bits, params, x_dev=None, variant="butterfly", mdt="f32"):
     p = dev_f32(params)
     mats = kq.kq_expand_blocks(p, dtype=torch.float32 if mdt == "f32" else torch.bfloat16)
     fac = kq.kq_expand_factored(p) if variant == "butterfly" else None
     x = dev_bf16(x_bits) if x_dev is None else x_dev
-    qd, sd = kq.kq_quantize(x, mats, fac, variant=variant)
-    return host(qd), host(sd)
+    M, d = x.shape
+    q, s, bufs = guarded_outputs(M, d)
+    kq.kq_quantize(x, mats, fac, variant=variant, q=q, scales=s)
+    torch.cuda.synchronize()
+    assert_guards(bufs)
+    return host(q), host(s)
 
 
 def oracle_mats(orc, params, mdt):
@@ -368,38 +389,40 @@ def test_quantize_hadamard_init_onehot(kq, orc, variant, mdt):
     assert np.all(s == 127) and np.all((unpack(q) & 7) == 7)
 
 
-def sampled_rows(M: int, n: int, seed: int) -> np.ndarray:
-    rng = np.random.default_rng(seed)
-    rows = set([0, M - 1, M // 2]) | set(rng.choice(M, size=min(n, M), replace=False).tolist())
-    return np.array(sorted(rows))
+_CASE_CACHE = {}
+
+
+def case_full(orc, key, make, mdt):
+    """(x, params, oracle codes, oracle scales) of one input, every row; the oracle
+    runs over the host cores.  Cached per input and matrix precision, so the
+    variants that share a matrix share one oracle run (the variants are the
+    fastest-varying parameter of the tests below)."""
+    if key not in _CASE_CACHE:
+        _CASE_CACHE.clear()
+        _CASE_CACHE[key] = {"input": make()}
+    entry = _CASE_CACHE[key]
+    x, params = entry["input"]
+    if mdt not in entry:
+        entry[mdt] = oracle_rows("quantize", x, oracle_mats(orc, params, mdt))
+    return (x, params) + entry[mdt]
 
 
 @pytest.mark.parametrize("variant,mdt", VARIANTS)
 @pytest.mark.parametrize("name,d", [("pixart", 1152), ("pixart", 4608), ("sana", 2240), ("sana", 5600),
                                     ("flux", 3072), ("flux", 12288)])
-def test_quantize_full_config_sampled(kq, orc, name, d, variant, mdt):
-    x, params = inputs.config_case(name, d)
+def test_quantize_full_config_every_row(kq, orc, name, d, variant, mdt):
+    x, params, qr, sr = case_full(orc, (name, d), lambda: inputs.config_case(name, d), mdt)
     q, s = gpu_quantize(kq, x, params, variant=variant, mdt=mdt)
-    rows = sampled_rows(x.shape[0], 40, seed=d)
-    K = oracle_mats(orc, params, mdt)
-    xs = np.ascontiguousarray(x[rows])
-    qr, sr = orc.quantize(xs, K)
-    check(q[rows], s[rows], qr, sr, orc.transform(xs, K))
+    check(q, s, qr, sr)
 
 
 @pytest.mark.parametrize("variant,mdt", VARIANTS)
+@pytest.mark.parametrize("d", inputs.SWEEP_D)
 @pytest.mark.parametrize("M", inputs.SWEEP_M)
-def test_quantize_sweep_shapes_sampled(kq, orc, M, variant, mdt):
-    for d in inputs.SWEEP_D:
-        if M * d > 2**28 and d != inputs.SWEEP_D[0]:
-            # largest shapes: only the first d runs here; the bench sweep covers the rest
-            continue
-        x, params = inputs.sweep_case(M, d)
-        q, s = gpu_quantize(kq, x, params, variant=variant, mdt=mdt)
-        rows = sampled_rows(M, 12, seed=M + d)
-        K = oracle_mats(orc, params, mdt)
-        qr, sr = orc.quantize(np.ascontiguousarray(x[rows]), K)
-        check(q[rows], s[rows], qr, sr)
+def test_quantize_sweep_shapes_every_row(kq, orc, M, d, variant, mdt):
+    x, params, qr, sr = case_full(orc, ("sweep", M, d), lambda: inputs.sweep_case(M, d), mdt)
+    q, s = gpu_quantize(kq, x, params, variant=variant, mdt=mdt)
+    check(q, s, qr, sr)
 
 
 # ---------------------------------------------------------------- comparison kernels
@@ -408,17 +431,21 @@ def test_quantize_sweep_shapes_sampled(kq, orc, M, variant, mdt):
 def test_smooth_parity(kq, orc, M, d):
     x = inputs.activations(M, d, "t4", seed=[M, d, 2], outlier_frac=0.01, outlier_scale=(20.0, 100.0))
     inv_s = inputs.smooth_inv_scale(x)
-    qd, sd = kq.kq_ref_smooth_quantize(dev_bf16(x), dev_f32(inv_s))
+    qd, sd, bufs = guarded_outputs(M, d)
+    kq.kq_ref_smooth_quantize(dev_bf16(x), dev_f32(inv_s), q=qd, scales=sd)
     qr, sr = orc.smooth_quantize(x, inv_s)
     check(host(qd), host(sd), qr, sr)
+    assert_guards(bufs)
 
 
 @pytest.mark.parametrize("M,d", [(64, 1152), (7, 5600), (1, 32), (300, 3072)])
 def test_fwht_parity(kq, orc, M, d):
     x = inputs.activations(M, d, "t3", seed=[M, d, 3], outlier_frac=0.01, outlier_scale=(20.0, 100.0))
-    qd, sd = kq.kq_ref_fwht_quantize(dev_bf16(x))
+    qd, sd, bufs = guarded_outputs(M, d)
+    kq.kq_ref_fwht_quantize(dev_bf16(x), q=qd, scales=sd)
     qr, sr = orc.fwht_quantize(x)
     check(host(qd), host(sd), qr, sr)
+    assert_guards(bufs)
 
 
 def test_fwht_degenerate_blocks(kq, orc):
