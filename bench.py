@@ -43,8 +43,7 @@ FLUX_WORKLOAD = ("FLUX.1-schnell-shaped activations, M=4608 tokens x d in {3072,
                  "Student-t(3) with 0.5% outlier channels x100, per-block LU params Hadamard+N(0,0.05)")
 
 KERNEL_SOURCES = ["mxfp4_activations_b200/csrc/kq_quant.cuh", "mxfp4_activations_b200/csrc/kq_common.cuh",
-                  "mxfp4_activations_b200/csrc/kq_mx.cuh",
-                  "mxfp4_activations_b200/csrc/kq_lib.cu"]
+                  "mxfp4_activations_b200/csrc/kq_mx.cuh"]
 
 
 def algo_bytes(M: int, d: int) -> float:
@@ -68,16 +67,20 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "source": "fallback"}
 
 
-def recorded_traffic():
-    """dram bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
+def recorded_traffic(d: int):
+    """DRAM bytes (read + write) of one launch of the dominant kernel at width d,
+    from the committed ncu summary, if it was taken on the current kernel sources;
+    else None."""
     if not os.path.exists(PROFILE_JSON):
         return None
     with open(PROFILE_JSON) as f:
-        d = json.load(f)
-    if d.get("source_hash") != kernel_source_hash():
+        rec = json.load(f)
+    if rec.get("source_hash") != kernel_source_hash():
         return None
-    return d.get("dram_bytes_per_step")
+    for launch in rec.get("launches", []):
+        if launch.get("d") == d:
+            return launch["dram_read_bytes"] + launch["dram_write_bytes"]
+    return None
 
 
 # ---------------------------------------------------------------- clocks
@@ -238,6 +241,23 @@ def timed(torch, step: QuantStep, K: int, kind: str, per_launch: bool):
     return total_ms, launch_ms
 
 
+def timed_b2b(torch, step: QuantStep, j: int, kind: str, K: int) -> float:
+    """Average duration (microseconds) of one launch of `kind` on item j (one d),
+    from K launches queued back to back on the launching stream with CUDA events
+    around the whole loop (inputs rotate over the resident copies, so every launch
+    reads from HBM)."""
+    item = step.items[j]
+    for it in range(3):
+        step.launch(it, item, kind)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for it in range(K):
+        step.launch(it, item, kind)
+    b.record()
+    b.synchronize()
+    return a.elapsed_time(b) * 1e3 / K
+
+
 def e2e_run(torch, kq, step: QuantStep, xs_host, K: int):
     """Same metric through the public API with host buffers: every step copies
     that step's activations from pinned host memory, quantizes them, and reads the
@@ -353,8 +373,15 @@ def run_gpu(args) -> None:
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        # the same K steps again with events around every launch: per-kernel durations
-        # for the roofline
+        # the dominant kernel (the d = 12288 launch) alone, back to back: its average
+        # launch duration for the roofline
+        dom = max(range(len(step.items)), key=lambda j: step.items[j]["d"])
+        dom_us = timed_b2b(torch, step, dom, "kroquant", args.steps)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        # the K steps once more with events around every launch (these serialise the
+        # launches and add each launch's start-up; reported beside the roofline)
         _, launch_ms = timed(torch, step, args.steps, "kroquant", per_launch=True)
         torch.cuda.synchronize()
         if world > 1:
@@ -366,14 +393,13 @@ def run_gpu(args) -> None:
     if err != 0:
         raise RuntimeError(f"device error in timed region: {kq.kq_status_string(err)}")
 
-    # comparison kernels on the same inputs (after the timed region)
+    # comparison kernels on the same inputs (after the timed region): every kind,
+    # each shape back to back on its own
     comp = {}
+    n_cmp = max(50, args.steps)
     for kind in ("smooth", "fwht", "kroquant", "kroquant_mma", "kroquant_mma_bf16"):
-        timed(torch, step, 20, kind, per_launch=False)
-        ms, lm = timed(torch, step, max(50, args.steps), kind, per_launch=True)
-        n = max(50, args.steps)
-        comp[kind] = {"gbs": bytes_step * n / (sum(lm) * 1e-3) / 1e9,
-                      "us_per_launch": {str(it["d"]): lm[j] * 1e3 / n for j, it in enumerate(step.items)}}
+        us = {str(it["d"]): timed_b2b(torch, step, j, kind, n_cmp) for j, it in enumerate(step.items)}
+        comp[kind] = {"gbs": bytes_step / (sum(us.values()) * 1e-6) / 1e9, "us_per_launch": us}
 
     e2e_steps = max(3, min(args.steps, 20))
     e2e_ms, h2d, d2h = e2e_run(torch, kq, step, xs, e2e_steps)
@@ -389,9 +415,10 @@ def run_gpu(args) -> None:
 
     peaks = measured_peaks()
     value = world * bytes_step * args.steps / (total_ms * 1e-3) / 1e9
-    launch_total_ms = sum(launch_ms)
-    achieved = bytes_step * args.steps / (launch_total_ms * 1e-3) / 1e9
-    traffic = recorded_traffic()
+    dom_item = step.items[dom]
+    dom_bytes = algo_bytes(dom_item["M"], dom_item["d"])
+    achieved = dom_bytes / (dom_us * 1e-6) / 1e9
+    traffic = recorded_traffic(dom_item["d"])
     clocks = clk.summary()
     out = {
         "metric": "quantizer GB/s (bf16 in + FP4/E8M0 out) and % of B200 HBM peak; tokens/s",
@@ -419,9 +446,13 @@ def run_gpu(args) -> None:
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
             "traffic": traffic,
-            "algorithmic_bytes_per_step": bytes_step,
-            "us_per_launch": {str(it["d"]): round(launch_ms[j] * 1e3 / args.steps, 3)
-                              for j, it in enumerate(step.items)},
+            "kernel": "quant_kernel<MODE_KRON, row-major scales, 32-element blocks>",
+            "launch": f"M={dom_item['M']}, d={dom_item['d']}",
+            "algorithmic_bytes_per_launch": dom_bytes,
+            "us_per_launch": round(dom_us, 3),
+            "timing": f"{args.steps} launches of this kernel back to back, CUDA events around the loop",
+            "us_per_launch_serialised": {str(it["d"]): round(launch_ms[j] * 1e3 / args.steps, 3)
+                                         for j, it in enumerate(step.items)},
         },
         "comparison": {k: {"gbs": round(v["gbs"], 1),
                            "us_per_launch": {dk: round(dv, 3) for dk, dv in v["us_per_launch"].items()}}
@@ -603,72 +634,84 @@ def graph_time(torch, fn, n: int) -> float:
 
 
 def run_sweep(args) -> None:
+    """Every quantizer kind on every named config and sweep shape: average launch
+    duration over launches queued back to back (CUDA events around the loop).
+    Inputs rotate over enough device copies that a loop touches more than 256 MB
+    (so each launch reads from HBM) unless a copy is under 1 MB (launch-bound
+    shapes, where the inputs stay in L2 as they would in use)."""
     import torch
 
     import mxfp4_activations_b200 as kq
     from mxfp4_activations_b200 import build
 
     build.build()
-    kq.load()
     lib = kq.load()
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     cases = [(name, M, d) for name, c in inputs.CONFIGS.items() for d in c["ds"] for M in [c["M"]]]
     cases += [("sweep", M, d) for M in inputs.SWEEP_M for d in inputs.SWEEP_D]
-    # clean-L2 flush: reading a buffer larger than L2 leaves no dirty lines behind
-    flush = torch.ones(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
     for name, M, d in cases:
         x, p = inputs.sweep_case(M, d) if name == "sweep" else inputs.config_case(name, d)
-        xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+        nbytes = x.nbytes
+        ncopy = 1 if nbytes < 2**20 else max(1, min(8, -(-(256 * 2**20) // nbytes)))
+        x0 = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+        xs = [x0] + [x0.clone() for _ in range(ncopy - 1)]
         pd = torch.from_numpy(p).cuda()
         mats, fac = kq.kq_expand_blocks(pd), kq.kq_expand_factored(pd)
         inv_s = torch.from_numpy(inputs.smooth_inv_scale(x)).cuda()
         q = torch.empty((M, d // 2), dtype=torch.uint8, device="cuda")
         s = torch.empty((M, d // 32), dtype=torch.uint8, device="cuda")
         mats16 = kq.kq_expand_blocks(pd, dtype=torch.bfloat16)
-        p64 = torch.from_numpy(inputs.lu_params(d // 64, seed=[M, d, 64], factors=6)).cuda() if d % 64 == 0 else None
-        mats64 = kq.kq_expand_blocks(p64) if p64 is not None else None
-        fac64 = kq.kq_expand_factored(p64) if p64 is not None else None
-        calls = {
-            "kroquant": lambda st: lib.kq_quantize(xd.data_ptr(), M, d, d, mats.data_ptr(), 0, fac.data_ptr(),
-                                                   q.data_ptr(), s.data_ptr(), 2, 0, st),
-            "kroquant_mma": lambda st: lib.kq_quantize(xd.data_ptr(), M, d, d, mats.data_ptr(), 0, None,
-                                                       q.data_ptr(), s.data_ptr(), 1, 0, st),
-            "kroquant_mma_bf16": lambda st: lib.kq_quantize(xd.data_ptr(), M, d, d, mats16.data_ptr(), 1, None,
-                                                            q.data_ptr(), s.data_ptr(), 1, 0, st),
-            "smooth": lambda st: lib.kq_ref_smooth_quantize(xd.data_ptr(), M, d, d, inv_s.data_ptr(), q.data_ptr(),
-                                                            s.data_ptr(), st),
-            "fwht": lambda st: lib.kq_ref_fwht_quantize(xd.data_ptr(), M, d, d, q.data_ptr(), s.data_ptr(), st),
-        }
-        if p64 is not None:  # 64-element transform blocks (six factors), butterfly
-            calls["kroquant64"] = lambda st: lib.kq_quantize_n(xd.data_ptr(), M, d, d, 6, mats64.data_ptr(), 0,
-                                                               fac64.data_ptr(), q.data_ptr(), s.data_ptr(), 2, 0, st)
+        extra = {}
+        for log2n in (4, 6, 7):
+            if d % max(32, 1 << log2n) == 0:
+                pn = torch.from_numpy(inputs.lu_params(d >> log2n, seed=[M, d, 1 << log2n], factors=log2n)).cuda()
+                extra[log2n] = (kq.kq_expand_blocks(pn), kq.kq_expand_factored(pn))
+
+        def calls(xd):
+            c = {
+                "kroquant": lambda st: lib.kq_quantize(xd.data_ptr(), M, d, d, mats.data_ptr(), 0, fac.data_ptr(),
+                                                       q.data_ptr(), s.data_ptr(), 2, 0, st),
+                "kroquant_mma": lambda st: lib.kq_quantize(xd.data_ptr(), M, d, d, mats.data_ptr(), 0, None,
+                                                           q.data_ptr(), s.data_ptr(), 1, 0, st),
+                "kroquant_mma_bf16": lambda st: lib.kq_quantize(xd.data_ptr(), M, d, d, mats16.data_ptr(), 1, None,
+                                                                q.data_ptr(), s.data_ptr(), 1, 0, st),
+                "smooth": lambda st: lib.kq_ref_smooth_quantize(xd.data_ptr(), M, d, d, inv_s.data_ptr(),
+                                                                q.data_ptr(), s.data_ptr(), st),
+                "fwht": lambda st: lib.kq_ref_fwht_quantize(xd.data_ptr(), M, d, d, q.data_ptr(), s.data_ptr(), st),
+            }
+            for log2n, (mn, fn) in extra.items():
+                c[f"kroquant{1 << log2n}"] = (lambda mn, fn, log2n: lambda st: lib.kq_quantize_n(
+                    xd.data_ptr(), M, d, d, log2n, mn.data_ptr(), 0, fn.data_ptr(), q.data_ptr(), s.data_ptr(),
+                    2, 0, st))(mn, fn, log2n)
+            return c
+
+        per_copy = [calls(xd) for xd in xs]
+        reps = 60 if M * d < 2**24 else (30 if M * d < 2**28 else 10)
         res = {}
-        reps = 30 if M * d < 2**26 else 10
-        for kind, fn in calls.items():
-            for _ in range(3):
-                assert fn(stream) == 0
-            times = []
-            for _ in range(reps):
-                flush.sum()  # evict L2 between launches
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record()
-                assert fn(stream) == 0
-                b.record()
-                b.synchronize()
-                times.append(a.elapsed_time(b) * 1e3)
-            med = statistics.median(times)
-            res[kind] = {"us_median": round(med, 3), "us_best": round(min(times), 3),
-                         "gbs_median": round(algo_bytes(M, d) / (med * 1e-6) / 1e9, 1)}
+        for kind in per_copy[0]:
+            fns = [pc[kind] for pc in per_copy]
+            for i in range(3):
+                assert fns[i % ncopy](stream) == 0
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for i in range(reps):
+                assert fns[i % ncopy](stream) == 0
+            b.record()
+            b.synchronize()
+            us = a.elapsed_time(b) * 1e3 / reps
+            res[kind] = {"us": round(us, 3), "gbs": round(algo_bytes(M, d) / (us * 1e-6) / 1e9, 1)}
             if M <= 256:
                 # launch-latency-bound shapes: back-to-back launches replayed from a CUDA graph
-                # (inputs stay in L2 here; the point is the per-launch floor)
-                res[kind]["graph_us_per_launch"] = round(graph_time(torch, fn, 50), 3)
-        best_f32 = min(("kroquant", "kroquant_mma"), key=lambda k: res[k]["us_median"])
-        line = {"sweep": name, "M": M, "d": d, "bytes": algo_bytes(M, d), **res, "best_f32_variant": best_f32,
-                "kroquant_vs_smooth_speed": round(res["smooth"]["us_median"] / res[best_f32]["us_median"], 3),
-                "kroquant_vs_fwht_speed": round(res["fwht"]["us_median"] / res[best_f32]["us_median"], 3)}
+                res[kind]["graph_us_per_launch"] = round(graph_time(torch, fns[0], 50), 3)
+        best_f32 = min(("kroquant", "kroquant_mma"), key=lambda k: res[k]["us"])
+        line = {"sweep": name, "M": M, "d": d, "bytes": algo_bytes(M, d), "input_copies": ncopy, "launches": reps,
+                **res, "best_f32_variant": best_f32,
+                "kroquant_vs_smooth_speed": round(res["smooth"]["us"] / res["kroquant"]["us"], 3),
+                "kroquant_vs_fwht_speed": round(res["fwht"]["us"] / res["kroquant"]["us"], 3)}
         print(json.dumps(line), flush=True)
-        del xd, q, s
+        del xs, x0, q, s
+        torch.cuda.empty_cache()
     assert kq.kq_get_device_error(clear=True) == 0
 
 

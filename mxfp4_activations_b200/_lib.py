@@ -148,8 +148,8 @@ def _mats(mats, d: int, device: torch.device, name: str = "mats") -> int:
     if mats.dim() != 3 or mats.shape[1] != mats.shape[2]:
         raise ValueError(f"{name} must be [d/n, n, n]")
     n = mats.shape[-1]
-    if n not in (32, 64):
-        raise ValueError("transform blocks of 32 or 64 elements")
+    if n not in (16, 32, 64, 128):
+        raise ValueError("transform blocks of 16, 32, 64 or 128 elements")
     if mats.shape[0] * n != d:
         raise ValueError(f"{name} holds {mats.shape[0]} blocks of {n}, the input has d = {d}")
     return n
@@ -189,16 +189,25 @@ def kq_expand_blocks(params: torch.Tensor, inverse: bool = False, dtype: torch.d
     return out
 
 
+def factored_floats(log2n: int) -> int:
+    """Floats per butterfly record of one 32-element block column."""
+    return 64 if log2n == 4 else 48
+
+
 def kq_expand_factored(params: torch.Tensor, out: torch.Tensor | None = None,
                        log2n: int | None = None) -> torch.Tensor:
-    """The butterfly form, one [48] record per 32-element block column."""
+    """The butterfly form, one record per 32-element block column ([48] floats;
+    [64] for 16-element transform blocks, two per column)."""
     _cuda(params, "params", dtypes=(torch.float32,))
     params = params.contiguous()
     nt, log2n = _params_shape(params, log2n)
-    nb32 = nt << (log2n - 5) if log2n >= 5 else nt
+    if log2n < 4 or log2n > 7:
+        raise ValueError("the butterfly form covers transform blocks of 16 to 128 elements")
+    nb32 = nt << (log2n - 5) if log2n >= 5 else nt // 2
+    rec = factored_floats(log2n)
     if out is None:
-        out = torch.empty((nb32, 48), dtype=torch.float32, device=params.device)
-    _cuda(out, "out", params.device, (torch.float32,), contiguous=True, min_numel=nb32 * 48)
+        out = torch.empty((nb32, rec), dtype=torch.float32, device=params.device)
+    _cuda(out, "out", params.device, (torch.float32,), contiguous=True, min_numel=nb32 * rec)
     with torch.cuda.device(params.device):
         _check("kq_expand_factored_n", load().kq_expand_factored_n(_ptr(params), nt, log2n, _ptr(out),
                                                                      _stream(params.device)))
@@ -230,7 +239,8 @@ def kq_quantize(x: torch.Tensor, mats: torch.Tensor, factored: torch.Tensor | No
     M, d, ldx = _rows(x)
     n = _mats(mats, d, x.device)
     if factored is not None:
-        _cuda(factored, "factored", x.device, (torch.float32,), contiguous=True, min_numel=(d // 32) * 48)
+        _cuda(factored, "factored", x.device, (torch.float32,), contiguous=True,
+              min_numel=(d // 32) * factored_floats(n.bit_length() - 1))
     if variant not in VARIANTS:
         raise ValueError(f"variant must be one of {list(VARIANTS)}")
     q, scales = _outputs(x, M, d, q, scales, scale_layout)

@@ -95,71 +95,120 @@ __global__ void expand_kernel(const float* __restrict__ params, int64_t nt, int 
     static_cast<float*>(mats)[gid] = __double2float_rn(acc);
 }
 
+// Floats per butterfly record of one 32-element block column.
+__host__ __device__ constexpr int factored_floats(int log2n) { return log2n == 4 ? 64 : kFactored; }
+
 // One thread per 32-element block column: the butterfly form F_k = M_k diag(a_k, d_k)
-// of its transform block of n = 2^log2n elements (log2n 5 or 6).  Record [48]:
-//   [0..4]  c_k/a_k and [5..9] b_k/d_k of the five factors acting inside the
-//           32-element block (factors log2n-5 .. log2n-1)
-//   [10..41] D_j for this block's 32 outputs
-//   [42]    upper bound of max|K|   [43] 1 if only the exact path may be used
-//   [44]    absolute allowance      [45], [46] c/a, b/d of factor 0 when log2n = 6
-//           (it mixes the two 32-element halves of the 64-element block)
+// of its transform block(s) of n = 2^log2n elements (log2n 4..7), as the records
+// documented with kq_expand_factored_n:
+//   log2n 5..7, [48] floats:
+//     [0..4]  c_k/a_k and [5..9] b_k/d_k of the five factors acting inside the
+//             32-element block (factors log2n-5 .. log2n-1)
+//     [10..41] D_j for this block's 32 outputs
+//     [42]    upper bound of max|K|   [43] 1 if only the exact path may be used
+//     [44]    absolute allowance
+//     log2n 6: [45], [46] c/a, b/d of factor 0 (it mixes the two 32-element halves)
+//     log2n 7: [45] the coefficient of factor 1 (index bit 5) that this column uses:
+//              c/a when the column is the lower one of its pair, else b/d;
+//              [46] the same for factor 0 (index bit 6) and the column's 64-element half
+//   log2n 4, [64] floats (two 16-element transform blocks h = 0, 1 per column):
+//     [0..3] c/a and [4..7] b/d of factors 0..3 of block h = 0, [8..15] those of h = 1
+//     [16..47] D_j for the 32 outputs   [48] upper bound of max|K| over both blocks
+//     [49] 1 if only the exact path may be used   [50] absolute allowance   [51..63] zero
+__device__ void butterfly_factors(const float* __restrict__ prm, int nf, double* a, double* dd, float* lam,
+                                  float* bet, bool& exact_only, bool report, double& kmax, double& gain) {
+  for (int k = 0; k < nf; k++) {
+    if (prm[3 * k + 1] == 0.0f) {
+      if (report) record_error(kDevErrSingular);
+      exact_only = true;
+    }
+    double F[4];
+    lu_factor(prm + 3 * k, F);
+    a[k] = F[0];
+    dd[k] = F[3];
+    lam[k] = __double2float_rn(__ddiv_rn(F[2], F[0]));
+    bet[k] = __double2float_rn(__ddiv_rn(F[1], F[3]));
+    // ratios must be finite and moderate for the fp32 butterfly to be usable
+    if (!(fabsf(lam[k]) <= 1.8446744e19f) || !(fabsf(bet[k]) <= 1.8446744e19f)) exact_only = true;
+    const double mk = fmax(fmax(fabs(F[0]), fabs(F[1])), fmax(fabs(F[2]), fabs(F[3])));
+    kmax = __dmul_rn(kmax, mk);
+    gain = __dmul_rn(gain, 1.0 + fmax(fabs(double(lam[k])), fabs(double(bet[k]))));
+  }
+}
+
 __global__ void expand_factored_kernel(const float* __restrict__ params, int64_t nb32, int log2n,
                                        float* __restrict__ out) {
   const int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (b >= nb32) return;
-  const int64_t c = b >> (log2n - 5);            // transform block
-  const int half = int(b & ((1 << (log2n - 5)) - 1));  // which 32 outputs of it
-  const int inner0 = log2n - 5;                   // first factor acting inside the 32-block
-  double a[kMaxFactors], d[kMaxFactors];
-  double kmax = 1.0, gain = 1.0;
+  const int rec = factored_floats(log2n);
+  float* o = out + b * rec;
+  double a[2][kMaxFactors], dd[2][kMaxFactors];
+  float lam[2][kMaxFactors], bet[2][kMaxFactors];
+  double kmax[2] = {1.0, 1.0}, gain[2] = {1.0, 1.0};
   bool exact_only = false;
-  float* o = out + b * kFactored;
-  o[45] = o[46] = o[47] = 0.0f;
-  for (int k = 0; k < log2n; k++) {
-    const float* prm = params + c * 3 * log2n + 3 * k;
-    if (prm[1] == 0.0f) {
-      if (half == 0) record_error(kDevErrSingular);
-      exact_only = true;
-    }
-    double F[4];
-    lu_factor(prm, F);
-    a[k] = F[0];
-    d[k] = F[3];
-    const double lam = __ddiv_rn(F[2], F[0]);
-    const double bet = __ddiv_rn(F[1], F[3]);
-    const float lam32 = __double2float_rn(lam), bet32 = __double2float_rn(bet);
-    // ratios must be finite and moderate for the fp32 butterfly to be usable
-    if (!(fabsf(lam32) <= 1.8446744e19f) || !(fabsf(bet32) <= 1.8446744e19f)) exact_only = true;
-    if (k >= inner0) {
-      o[k - inner0] = lam32;
-      o[5 + k - inner0] = bet32;
-    } else {
-      o[45] = lam32;
-      o[46] = bet32;
-    }
-    const double mk = fmax(fmax(fabs(F[0]), fabs(F[1])), fmax(fabs(F[2]), fabs(F[3])));
-    kmax = __dmul_rn(kmax, mk);
-    gain = __dmul_rn(gain, 1.0 + fmax(fabs(double(lam32)), fabs(double(bet32))));
-  }
   double dmax = 0.0;
+  if (log2n == 4) {  // two 16-element transform blocks: 2b and 2b + 1
+    for (int h = 0; h < 2; h++)
+      butterfly_factors(params + (2 * b + h) * 12, 4, a[h], dd[h], lam[h], bet[h], exact_only, true, kmax[h],
+                        gain[h]);
+    for (int h = 0; h < 2; h++)
+      for (int k = 0; k < 4; k++) {
+        o[8 * h + k] = lam[h][k];
+        o[8 * h + 4 + k] = bet[h][k];
+      }
+    for (int j = 0; j < 32; j++) {
+      const int h = j >> 4, jj = j & 15;
+      double dj = 1.0;
+      for (int k = 0; k < 4; k++) dj = __dmul_rn(dj, ((jj >> (3 - k)) & 1) ? dd[h][k] : a[h][k]);
+      const float dj32 = __double2float_rn(dj);
+      if (!(fabsf(dj32) <= 3.0e38f) || dj32 == 0.0f) exact_only = true;
+      o[16 + j] = dj32;
+      dmax = fmax(dmax, fabs(double(dj32)));
+    }
+    const double km = fmax(kmax[0], kmax[1]);
+    const float kmf = __fmul_ru(__double2float_ru(km), 1.00000095367431640625f);
+    if (!(kmf <= 1.0e30f)) exact_only = true;
+    o[48] = kmf;
+    o[49] = exact_only ? 1.0f : 0.0f;
+    o[50] = __fmul_ru(__double2float_ru(__dmul_rn(dmax, fmax(gain[0], gain[1]))), 2.2420775429197073e-44f);
+    for (int i = 51; i < 64; i++) o[i] = 0.0f;
+    return;
+  }
+  const int64_t c = b >> (log2n - 5);                    // transform block
+  const int part = int(b & ((1 << (log2n - 5)) - 1));    // which 32 outputs of it
+  const int inner0 = log2n - 5;                          // first factor acting inside the 32-block
+  butterfly_factors(params + c * 3 * log2n, log2n, a[0], dd[0], lam[0], bet[0], exact_only, part == 0, kmax[0],
+                    gain[0]);
+  for (int k = inner0; k < log2n; k++) {
+    o[k - inner0] = lam[0][k];
+    o[5 + k - inner0] = bet[0][k];
+  }
+  o[45] = o[46] = o[47] = 0.0f;
+  if (log2n == 6) {
+    o[45] = lam[0][0];
+    o[46] = bet[0][0];
+  } else if (log2n == 7) {
+    o[45] = (part & 1) ? bet[0][1] : lam[0][1];
+    o[46] = (part & 2) ? bet[0][0] : lam[0][0];
+  }
   for (int j = 0; j < 32; j++) {
-    const int jj = half * 32 + j;  // output index inside the transform block
+    const int jj = part * 32 + j;  // output index inside the transform block
     double dj = 1.0;
-    for (int k = 0; k < log2n; k++) dj = __dmul_rn(dj, ((jj >> (log2n - 1 - k)) & 1) ? d[k] : a[k]);
+    for (int k = 0; k < log2n; k++) dj = __dmul_rn(dj, ((jj >> (log2n - 1 - k)) & 1) ? dd[0][k] : a[0][k]);
     const float dj32 = __double2float_rn(dj);
     if (!(fabsf(dj32) <= 3.0e38f) || dj32 == 0.0f) exact_only = true;
     o[10 + j] = dj32;
     dmax = fmax(dmax, fabs(double(dj32)));
   }
   // upper bound of max|K| (fp64 product error is far below the allowance's margin)
-  const float km = __fmul_ru(__double2float_ru(kmax), 1.00000095367431640625f);
+  const float km = __fmul_ru(__double2float_ru(kmax[0]), 1.00000095367431640625f);
   if (!(km <= 1.0e30f)) exact_only = true;
   o[42] = km;
   o[43] = exact_only ? 1.0f : 0.0f;
   // absolute error of results that fall in the fp32 subnormal range: each of the
-  // (log2n + 1 <= 7) roundings on an output's path adds at most 2^-150, amplified by
+  // (log2n + 1 <= 8) roundings on an output's path adds at most 2^-150, amplified by
   // at most max|D| * prod_k (1 + max(|c/a|, |b/d|)); 2^-145 leaves a margin.
-  o[44] = __fmul_ru(__double2float_ru(__dmul_rn(dmax, gain)), 2.2420775429197073e-44f);
+  o[44] = __fmul_ru(__double2float_ru(__dmul_rn(dmax, gain[0])), 2.2420775429197073e-44f);
 }
 
 }  // namespace kq

@@ -290,12 +290,12 @@ struct AutoRule {
   kq_variant v;
 };
 constexpr AutoRule kAutoTable[] = {
-    {1, 1152, KQ_VAR_BUTTERFLY},     {1, 3072, KQ_VAR_BUTTERFLY},     {1, 12288, KQ_VAR_BUTTERFLY},
-    {16, 1152, KQ_VAR_BUTTERFLY},    {16, 3072, KQ_VAR_MMA},          {16, 12288, KQ_VAR_BUTTERFLY},
-    {256, 1152, KQ_VAR_BUTTERFLY},   {256, 3072, KQ_VAR_BUTTERFLY},   {256, 12288, KQ_VAR_BUTTERFLY},
-    {4096, 1152, KQ_VAR_BUTTERFLY},  {4096, 3072, KQ_VAR_BUTTERFLY},  {4096, 12288, KQ_VAR_BUTTERFLY},
-    {16384, 1152, KQ_VAR_BUTTERFLY}, {16384, 3072, KQ_VAR_BUTTERFLY}, {16384, 12288, KQ_VAR_BUTTERFLY},
-    {65536, 1152, KQ_VAR_BUTTERFLY}, {65536, 3072, KQ_VAR_BUTTERFLY}, {65536, 12288, KQ_VAR_BUTTERFLY},
+    {1, 1152, KQ_VAR_MMA},            {1, 3072, KQ_VAR_MMA},            {1, 12288, KQ_VAR_BUTTERFLY},
+    {16, 1152, KQ_VAR_BUTTERFLY},     {16, 3072, KQ_VAR_BUTTERFLY},     {16, 12288, KQ_VAR_BUTTERFLY},
+    {256, 1152, KQ_VAR_BUTTERFLY},    {256, 3072, KQ_VAR_MMA},          {256, 12288, KQ_VAR_BUTTERFLY},
+    {4096, 1152, KQ_VAR_BUTTERFLY},   {4096, 3072, KQ_VAR_BUTTERFLY},   {4096, 12288, KQ_VAR_BUTTERFLY},
+    {16384, 1152, KQ_VAR_BUTTERFLY},  {16384, 3072, KQ_VAR_BUTTERFLY},  {16384, 12288, KQ_VAR_BUTTERFLY},
+    {65536, 1152, KQ_VAR_BUTTERFLY},  {65536, 3072, KQ_VAR_BUTTERFLY},  {65536, 12288, KQ_VAR_BUTTERFLY},
 };
 
 kq_variant table_variant(int64_t M, int64_t d) {
@@ -376,12 +376,13 @@ kq_status kq_expand_blocks(const float* params, int64_t nb, int inverse, kq_dtyp
 }
 
 kq_status kq_expand_factored_n(const float* params, int64_t nt, int log2n, float* factored, kq_stream_t stream) {
-  if (nt < 0 || (log2n != 5 && log2n != 6)) return KQ_ERR_INVALID_ARG;
+  if (nt < 0 || log2n < 4 || log2n > 7) return KQ_ERR_INVALID_ARG;
+  if (log2n == 4 && nt % 2 != 0) return KQ_ERR_SHAPE;  // two 16-element blocks per record
   if (nt == 0) return KQ_OK;
   if (params == nullptr || factored == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(params, 4) || !aligned(factored, 16)) return KQ_ERR_ALIGN;
   if (nt > (int64_t(1) << 29)) return KQ_ERR_SHAPE;
-  const int64_t nb32 = nt << (log2n - 5);
+  const int64_t nb32 = log2n == 4 ? nt / 2 : nt << (log2n - 5);
   kq::expand_factored_kernel<<<unsigned((nb32 + 127) / 128), 128, 0, as_cuda(stream)>>>(params, nb32, log2n,
                                                                                         factored);
   return launch_status("expand_factored_kernel launch");
@@ -396,26 +397,32 @@ kq_status kq_quantize_n(const void* x, int64_t M, int64_t d, int64_t ldx, int lo
                         kq_scale_layout scale_layout, kq_stream_t stream) {
   if (variant != KQ_VAR_AUTO && variant != KQ_VAR_MMA && variant != KQ_VAR_BUTTERFLY) return KQ_ERR_INVALID_ARG;
   if (scale_layout != KQ_SCALES_ROW_MAJOR && scale_layout != KQ_SCALES_MMA_TILED) return KQ_ERR_INVALID_ARG;
-  if (log2n != 5 && log2n != 6) return KQ_ERR_INVALID_ARG;
+  if (log2n < 4 || log2n > 7) return KQ_ERR_INVALID_ARG;
   const int sf_tiled = scale_layout == KQ_SCALES_MMA_TILED ? 1 : 0;
   if (mat_dtype != KQ_F32 && mat_dtype != KQ_BF16) return KQ_ERR_INVALID_ARG;
   kq_status st = check_x(x, M, d, ldx);
   if (st != KQ_OK) return st;
-  if (log2n == 6 && d % 64 != 0) return KQ_ERR_SHAPE;
+  if (log2n > 5 && d % (int64_t(1) << log2n) != 0) return KQ_ERR_SHAPE;
   if (M == 0 || d == 0) return KQ_OK;
   st = check_out(q, scales);
   if (st != KQ_OK) return st;
   if (mats == nullptr) return KQ_ERR_INVALID_ARG;
   if (!aligned(mats, 16)) return KQ_ERR_ALIGN;
   const float* m32 = static_cast<const float*>(mats);
-  if (log2n == 6) {
-    // 64-element blocks: the butterfly only (fp32 matrices and the factored form)
+  if (log2n != 5) {
+    // 16-, 64- and 128-element blocks: the butterfly only (fp32 matrices and the factored form)
     if (variant == KQ_VAR_MMA || mat_dtype == KQ_BF16) return KQ_ERR_UNSUPPORTED;
     if (factored == nullptr) return KQ_ERR_INVALID_ARG;
     if (!aligned(factored, 16)) return KQ_ERR_ALIGN;
-    return sf_tiled
-               ? launch_quant<kq::MODE_KRON, 1, 64>(x, M, d, ldx, m32, factored, nullptr, q, scales, as_cuda(stream))
-               : launch_quant<kq::MODE_KRON, 0, 64>(x, M, d, ldx, m32, factored, nullptr, q, scales, as_cuda(stream));
+    const cudaStream_t cs = as_cuda(stream);
+    switch (log2n * 2 + sf_tiled) {
+      case 8: return launch_quant<kq::MODE_KRON, 0, 16>(x, M, d, ldx, m32, factored, nullptr, q, scales, cs);
+      case 9: return launch_quant<kq::MODE_KRON, 1, 16>(x, M, d, ldx, m32, factored, nullptr, q, scales, cs);
+      case 12: return launch_quant<kq::MODE_KRON, 0, 64>(x, M, d, ldx, m32, factored, nullptr, q, scales, cs);
+      case 13: return launch_quant<kq::MODE_KRON, 1, 64>(x, M, d, ldx, m32, factored, nullptr, q, scales, cs);
+      case 14: return launch_quant<kq::MODE_KRON, 0, 128>(x, M, d, ldx, m32, factored, nullptr, q, scales, cs);
+      default: return launch_quant<kq::MODE_KRON, 1, 128>(x, M, d, ldx, m32, factored, nullptr, q, scales, cs);
+    }
   }
   // bf16 matrices are only served by the tensor-core variant; AUTO resolves per shape
   if (variant == KQ_VAR_BUTTERFLY && mat_dtype == KQ_BF16) return KQ_ERR_UNSUPPORTED;
@@ -467,7 +474,16 @@ kq_status kq_dequantize(const uint8_t* q, const uint8_t* scales, int64_t M, int6
   if (!aligned(q, 16) || !aligned(out, 16) || (inv_mats != nullptr && !aligned(inv_mats, 4))) return KQ_ERR_ALIGN;
   const int64_t nb = d / 32;
   if (nb > int64_t(INT32_MAX)) return KQ_ERR_SHAPE;
-  kq::dequant_kernel<<<grid_for(M * nb, 256), 256, 0, as_cuda(stream)>>>(
+  // block columns across x; groups of 8 warps x 8 rows across y, about four waves
+  // of resident CTAs
+  const DeviceInfo* dev = device_info();
+  const int64_t want = (dev ? int64_t(dev->sms) : 148) * 8 * 4;
+  int64_t gy = (want + nb - 1) / nb;
+  const int64_t row_groups = (M + kq::kDqWarps * kq::kDqRows - 1) / (kq::kDqWarps * kq::kDqRows);
+  if (gy > row_groups) gy = row_groups;
+  if (gy > 65535) gy = 65535;
+  auto kern = inv_mats != nullptr ? kq::dequant_kernel<1> : kq::dequant_kernel<0>;
+  kern<<<dim3(unsigned(nb), unsigned(gy)), kq::kDqWarps * 32, 0, as_cuda(stream)>>>(
       q, scales, M, int(nb), inv_mats, mat_dtype == KQ_BF16 ? 1 : 0, out, out_dtype == KQ_BF16 ? 1 : 0);
   return launch_status("dequant_kernel launch");
 }
@@ -485,8 +501,8 @@ kq_status kq_e2m1_pack(const float* v, int64_t n, uint8_t* out, kq_stream_t stre
 kq_status kq_select_variant(int64_t M, int64_t d, int log2n, kq_dtype mat_dtype, int has_factored,
                             kq_variant* chosen) {
   if (chosen == nullptr || M < 0 || d < 0 || (mat_dtype != KQ_F32 && mat_dtype != KQ_BF16)) return KQ_ERR_INVALID_ARG;
-  if (log2n != 5 && log2n != 6) return KQ_ERR_INVALID_ARG;
-  if (log2n == 6) {  // 64-element blocks: the butterfly only
+  if (log2n < 4 || log2n > 7) return KQ_ERR_INVALID_ARG;
+  if (log2n != 5) {  // 16-, 64- and 128-element blocks: the butterfly only
     if (mat_dtype == KQ_BF16 || !has_factored) return KQ_ERR_UNSUPPORTED;
     *chosen = KQ_VAR_BUTTERFLY;
     return KQ_OK;

@@ -22,55 +22,72 @@ __device__ __forceinline__ float scale_of_byte(uint32_t byte) {
   return __uint_as_float(byte << 23);
 }
 
-// One thread per (row, block): yhat = value(code) * 2^(byte-127); with inv
-// (fp32 or bf16 [nb][32][32]) xhat_i = sum_j yhat_j inv[j][i], fp32 FMAs in j order.
-__global__ void dequant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ scales, int64_t M,
-                               int nb, const void* __restrict__ inv, int inv_bf16, void* __restrict__ out,
-                               int out_bf16) {
-  const int64_t total = M * nb;
-  for (int64_t g = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; g < total;
-       g += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t row = g / nb;
-    const int b = int(g - row * nb);
-    const uint4 cw = *reinterpret_cast<const uint4*>(q + g * 16);
-    const float sc = scale_of_byte(scales[g]);
-    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-    float yh[32];
+constexpr int kDqWarps = 8;  // warps per CTA of dequant_kernel
+constexpr int kDqRows = 8;   // rows a warp has in flight
+
+// CTA (b, g) handles block column b; its warp w takes the rows (g*8 + w)*8 + i,
+// i < 8, then steps by gridDim.y*64 rows; lane l computes element l of each row:
+// yhat_l = value(code_l) * 2^(byte-127).  The codes and scales of a warp's eight
+// rows are loaded before any of them is used.  With inv (fp32 or bf16
+// [nb][32][32]), lane i keeps column i of block b's inverse in registers (loaded
+// once, one coalesced row of the matrix per step) and forms xhat_i = sum_j yhat_j
+// inv[j][i] with fp32 FMAs in j order from +0, the row's yhat broadcast through
+// shared memory.  Each row's 32 outputs are one contiguous store of the warp.
+// INV: an inverse is applied (a template parameter, so the plain decode keeps few
+// registers and many warps in flight).
+template <int INV>
+__global__ void __launch_bounds__(kDqWarps * 32, INV ? 2 : 3) dequant_kernel(
+    const uint8_t* __restrict__ q, const uint8_t* __restrict__ scales, int64_t M, int nb,
+    const void* __restrict__ inv, int inv_bf16, void* __restrict__ out, int out_bf16) {
+  __shared__ __align__(16) float ys[kDqWarps][kBlock];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int b = blockIdx.x;
+  float kcol[kBlock];
+  if (INV) {
 #pragma unroll
-    for (int k = 0; k < 4; k++)
-#pragma unroll
-      for (int n = 0; n < 8; n++) yh[8 * k + n] = __fmul_rn(e2m1_value((words[k] >> (4 * n)) & 0xFu), sc);
-    float xo[32];
-    if (inv == nullptr) {
-#pragma unroll
-      for (int i = 0; i < 32; i++) xo[i] = yh[i];
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; i++) xo[i] = 0.0f;
-      for (int j = 0; j < 32; j++) {
-        const int64_t off = (int64_t(b) * 32 + j) * 32;
-#pragma unroll
-        for (int i = 0; i < 32; i++) {
-          const float kji = inv_bf16 ? bf16_to_f32(static_cast<const uint16_t*>(inv)[off + i])
-                                     : static_cast<const float*>(inv)[off + i];
-          xo[i] = __fmaf_rn(yh[j], kji, xo[i]);
-        }
-      }
+    for (int j = 0; j < kBlock; j++) {
+      const int64_t off = (int64_t(b) * kBlock + j) * kBlock + lane;
+      kcol[j] = inv_bf16 ? bf16_to_f32(static_cast<const uint16_t*>(inv)[off]) : static_cast<const float*>(inv)[off];
     }
-    if (out_bf16) {
-      uint32_t pk[16];
+  }
+  const int64_t d = int64_t(nb) * kBlock;
+  const int64_t step = int64_t(gridDim.y) * kDqWarps * kDqRows;
+  for (int64_t r0 = (int64_t(blockIdx.y) * kDqWarps + warp) * kDqRows; r0 < M; r0 += step) {
+    uint32_t w[kDqRows];
+    uint32_t sc[kDqRows];
 #pragma unroll
-      for (int h = 0; h < 16; h++) {
-        const __nv_bfloat162 v = __floats2bfloat162_rn(xo[2 * h], xo[2 * h + 1]);
-        pk[h] = *reinterpret_cast<const uint32_t*>(&v);
+    for (int i = 0; i < kDqRows; i++) {
+      const int64_t r = r0 + i < M ? r0 + i : r0;
+      const int64_t g = r * nb + b;
+      w[i] = reinterpret_cast<const uint32_t*>(q + g * 16)[lane >> 3];
+      sc[i] = scales[g];
+    }
+#pragma unroll
+    for (int i = 0; i < kDqRows; i++) {
+      if (r0 + i >= M) break;
+      const float yh = __fmul_rn(e2m1_value((w[i] >> (4 * (lane & 7))) & 0xFu), scale_of_byte(sc[i]));
+      float xo = yh;
+      if (INV) {
+        ys[warp][lane] = yh;
+        __syncwarp();
+        const float4* yv = reinterpret_cast<const float4*>(ys[warp]);
+        float acc = 0.0f;
+#pragma unroll
+        for (int k = 0; k < kBlock / 4; k++) {
+          const float4 v = yv[k];
+          acc = __fmaf_rn(v.x, kcol[4 * k], acc);
+          acc = __fmaf_rn(v.y, kcol[4 * k + 1], acc);
+          acc = __fmaf_rn(v.z, kcol[4 * k + 2], acc);
+          acc = __fmaf_rn(v.w, kcol[4 * k + 3], acc);
+        }
+        __syncwarp();  // the row's yhat is read by every lane before the next row overwrites it
+        xo = acc;
       }
-      uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + g * 32);
-#pragma unroll
-      for (int h = 0; h < 4; h++) o[h] = make_uint4(pk[4 * h], pk[4 * h + 1], pk[4 * h + 2], pk[4 * h + 3]);
-    } else {
-      float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + g * 32);
-#pragma unroll
-      for (int h = 0; h < 8; h++) o[h] = make_float4(xo[4 * h], xo[4 * h + 1], xo[4 * h + 2], xo[4 * h + 3]);
+      const int64_t o = (r0 + i) * d + int64_t(b) * kBlock + lane;
+      if (out_bf16)
+        static_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(xo);
+      else
+        static_cast<float*>(out)[o] = xo;
     }
   }
 }

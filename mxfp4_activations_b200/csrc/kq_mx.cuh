@@ -71,18 +71,43 @@ __device__ __forceinline__ float k_entry(const void* __restrict__ Kb, int i, int
 // computes y32_j = fp32( sum_{i < NT} x_i K[i][j] ) in fp64, summing in
 // increasing i from +0 (each product of a bf16 and an fp32 or bf16 value is
 // exact in fp64).  xb: the NT inputs of the transform block; Kb: column 0 of this
-// block's 32 outputs in the NT x NT matrix (rows NT entries apart).  Rows of K are
+// block's 32 outputs in the NT x NT matrix (rows NT entries apart).  NT = 16: xb is
+// the 32-element block, which holds two transform blocks, and Kb their two 16 x 16
+// matrices; lane j sums over the 16 inputs of its own half.  Rows of K are
 // loaded 32 at a time, each row one coalesced 128-byte load across the warp; x is
 // a broadcast load.  The block's scale then comes from the exact maximum and
 // every code from the exact value, and lane `owner` stores them.  Must be called
 // by all 32 lanes with the same arguments (taken from the owner lane).
 template <int KSRC, int NT>
-__device__ __noinline__ void exact_block_warp(const uint16_t* __restrict__ xb, const void* __restrict__ Kb,
+__device__ __forceinline__ void exact_block_warp(const uint16_t* __restrict__ xb, const void* __restrict__ Kb,
                                               uint8_t* __restrict__ qb, uint8_t* __restrict__ sb, int owner) {
   const int lane = threadIdx.x & 31;
   double acc = 0.0;
+  if (NT == 16) {
+    // two 16-element transform blocks: lane j sums over its half's 16 inputs,
+    // with the half's 16 x 16 matrix (Kb: the first of the column's two)
+    const int h = lane >> 4;
+    float kc[16];
+#pragma unroll
+    for (int i = 0; i < 16; i++) kc[i] = k_entry<KSRC>(Kb, h * 16 + i, lane & 15, 16);
+    const uint4* px = reinterpret_cast<const uint4*>(xb + 16 * h);
+    uint32_t xw[8];
+#pragma unroll
+    for (int k = 0; k < 2; k++) {
+      const uint4 v = __ldg(px + k);
+      xw[4 * k] = v.x;
+      xw[4 * k + 1] = v.y;
+      xw[4 * k + 2] = v.z;
+      xw[4 * k + 3] = v.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+      const float xi = (i & 1) ? bf16hi(xw[i >> 1]) : bf16lo(xw[i >> 1]);
+      acc = __fma_rn(double(xi), double(kc[i]), acc);
+    }
+  }
 #pragma unroll 1
-  for (int i0 = 0; i0 < NT; i0 += kBlock) {
+  for (int i0 = 0; i0 < (NT == 16 ? 0 : NT); i0 += kBlock) {
     float kc[kBlock];
 #pragma unroll
     for (int i = 0; i < kBlock; i++) kc[i] = k_entry<KSRC>(Kb, i0 + i, lane, NT);

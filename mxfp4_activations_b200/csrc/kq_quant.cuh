@@ -54,8 +54,8 @@ namespace kq {
 
 enum Mode { MODE_KRON = 0, MODE_FWHT = 1, MODE_SMOOTH = 2 };
 
-constexpr float kKronErrC = 9.5367431640625e-07f;   // 2^-20 = 16 u (14 u needed, see above)
-constexpr float kKronErrC64 = 1.9073486328125e-06f; // 2^-19 = 32 u for 64-element blocks (16 u needed)
+constexpr float kKronErrC = 9.5367431640625e-07f;   // 2^-20 = 16 u (14 u needed, see above; 12 u for 16-element blocks)
+constexpr float kKronErrC64 = 1.9073486328125e-06f; // 2^-19 = 32 u for 64- and 128-element blocks (16 u, 18 u needed)
 constexpr float kFwhtErrC = 4.76837158203125e-07f;  // 2^-21 = 8 u (7 u needed)
 constexpr float kErrAbs = 7.174648137343064e-43f;   // 2^-140: FWHT subnormal-range slack
 
@@ -88,8 +88,27 @@ struct ColCoef {
   uint64_t D[16];       // (D_2m, D_2m+1); SMOOTH: the per-channel factors
   float cfac;           // C * max|K| (+inf: the column takes the exact path only)
   float eabs;           // absolute allowance (results in the fp32 subnormal range)
-  float mix;            // 64-element blocks: lam (lower half) or bet (upper half) of F0
+  float mix;            // 64-element blocks: lam (lower half) or bet (upper half) of F0;
+                        // 128-element blocks: this column's coefficient of the factor on index bit 5
+  float mix2;           // 128-element blocks: this column's coefficient of the factor on index bit 6
+  float l16[2], b16[2];        // 16-element blocks: stage on index bit 0 of each half
+  uint64_t L16[3][2], B16[3][2];  // 16-element blocks: stages on index bits 1..3 of each half
 };
+
+// Offset of column c's first output column in its transform matrix array, and the
+// first block column of its transform block (n = 16: the column's two 16 x 16
+// matrices; n >= 32: one n x n matrix per n / 32 columns).
+template <int NT>
+__device__ __forceinline__ int64_t kmat_offset(int c) {
+  constexpr int g = NT >= kBlock ? NT / kBlock : 1;  // block columns per transform block
+  if (NT == 16) return int64_t(c) * 512;
+  return int64_t(c / g) * NT * NT + (c % g) * kBlock;
+}
+template <int NT>
+__device__ __forceinline__ int first_column(int c) {
+  constexpr int g = NT >= kBlock ? NT / kBlock : 1;
+  return c - c % g;
+}
 
 template <int MODE, int NT>
 __device__ __forceinline__ void load_coef(const QuantParams& p, int c, ColCoef& cf) {
@@ -97,10 +116,35 @@ __device__ __forceinline__ void load_coef(const QuantParams& p, int c, ColCoef& 
   cf.b4 = -1.0f;
   cf.cfac = kFwhtErrC * kFwhtC;
   cf.eabs = kErrAbs;
-  cf.mix = 0.0f;
+  cf.mix = cf.mix2 = 0.0f;
 #pragma unroll
   for (int s = 0; s < 4; s++) cf.L[s] = cf.B[s] = 0;
-  if (MODE == MODE_KRON) {
+  if (MODE == MODE_KRON && NT == 16) {
+    const float4* fb = reinterpret_cast<const float4*>(p.factored + int64_t(c) * 64);
+    float r[64];
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+      const float4 v = __ldg(fb + i);
+      r[4 * i] = v.x;
+      r[4 * i + 1] = v.y;
+      r[4 * i + 2] = v.z;
+      r[4 * i + 3] = v.w;
+    }
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+      cf.l16[h] = r[8 * h + 3];  // factor 3 acts on index bit 0
+      cf.b16[h] = r[8 * h + 7];
+#pragma unroll
+      for (int s = 0; s < 3; s++) {  // stage on bit s+1 uses factor 2-s
+        cf.L16[s][h] = pk2(r[8 * h + 2 - s], r[8 * h + 2 - s]);
+        cf.B16[s][h] = pk2(r[8 * h + 6 - s], r[8 * h + 6 - s]);
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < 16; m++) cf.D[m] = pk2(r[16 + 2 * m], r[17 + 2 * m]);
+    cf.cfac = r[49] != 0.0f ? __int_as_float(0x7F800000) : __fmul_ru(kKronErrC, r[48]);
+    cf.eabs = r[50];
+  } else if (MODE == MODE_KRON) {
     const float4* fb = reinterpret_cast<const float4*>(p.factored + int64_t(c) * kFactored);
     float r[kFactored];
 #pragma unroll
@@ -120,9 +164,13 @@ __device__ __forceinline__ void load_coef(const QuantParams& p, int c, ColCoef& 
     }
 #pragma unroll
     for (int m = 0; m < 16; m++) cf.D[m] = pk2(r[10 + 2 * m], r[11 + 2 * m]);
-    cf.cfac = r[43] != 0.0f ? __int_as_float(0x7F800000) : __fmul_ru(NT == 64 ? kKronErrC64 : kKronErrC, r[42]);
+    cf.cfac = r[43] != 0.0f ? __int_as_float(0x7F800000) : __fmul_ru(NT >= 64 ? kKronErrC64 : kKronErrC, r[42]);
     cf.eabs = r[44];
-    cf.mix = (c & 1) ? r[46] : r[45];
+    if (NT == 64) cf.mix = (c & 1) ? r[46] : r[45];
+    if (NT == 128) {
+      cf.mix = r[45];
+      cf.mix2 = r[46];
+    }
   } else if (MODE == MODE_SMOOTH) {
     const float4* sp = reinterpret_cast<const float4*>(p.inv_s + int64_t(c) * kBlock);
 #pragma unroll
@@ -163,8 +211,11 @@ __device__ __forceinline__ void read_slot(uint32_t slot, int sw, uint32_t (&w)[1
 
 // ---------------------------------------------------------------- one block of one row
 //
-// NT = 64: the block is one half of a 64-element transform block whose other half
-// is held by lane ^ 1 (same row, neighbouring column); (c & 1) marks the upper half.
+// NT = 16: the block holds two 16-element transform blocks (its halves).  NT = 64:
+// the block is one half of a 64-element transform block whose other half is held
+// by lane ^ 1 (same row, neighbouring column).  NT = 128: a quarter of a 128-element
+// transform block, the others held by lanes ^ 1, ^ 2 and ^ 3 (bits 5 and 6 of the
+// index inside the transform block are bits 0 and 1 of the lane).
 // act marks the lanes whose block is real.  Stores the fast result of a real
 // block and returns whether it must be recomputed exactly (never for SMOOTH, whose
 // fp32 product is the definition itself).
@@ -206,13 +257,15 @@ __device__ __forceinline__ bool quant_block(const ColCoef& cf, const uint32_t (&
 #pragma unroll
   for (int j = 0; j < kBlock; j++) l1p[j & 3] = __fadd_ru(l1p[j & 3], fabsf(x[j]));
   float l1 = __fadd_ru(__fadd_ru(l1p[0], l1p[1]), __fadd_ru(l1p[2], l1p[3]));
-  if (NT == 64) {
-    // every output of a 64-element block depends on all 64 inputs
+  if (NT >= 64) {
+    // every output of the transform block depends on all of its inputs
     l1 = __fadd_ru(l1, __shfl_xor_sync(0xFFFFFFFFu, l1, 1));
-    // factor 0 of a 64-element block, applied first (the Kronecker factors act on
-    // different index bits and commute): x_lo + lam x_hi in the lower half, x_hi +
-    // bet x_lo in the upper one, element by element, with the partner half's inputs
-    // taken from lane ^ 1 as raw bf16 pairs (16 shuffles)
+    if (NT == 128) l1 = __fadd_ru(l1, __shfl_xor_sync(0xFFFFFFFFu, l1, 2));
+    // the factor on index bit 5 (64-element blocks: factor 0; 128: factor 1), applied
+    // first (the Kronecker factors act on different index bits and commute): x_lo +
+    // lam x_hi in the lower column, x_hi + bet x_lo in the upper one, element by
+    // element, with the partner column's inputs taken from lane ^ 1 as raw bf16
+    // pairs (16 shuffles)
     const uint64_t C2 = pk2(cf.mix, cf.mix);
 #pragma unroll
     for (int h = 0; h < 16; h++) {
@@ -220,15 +273,31 @@ __device__ __forceinline__ bool quant_block(const ColCoef& cf, const uint32_t (&
       const uint64_t X = fma2_rn(C2, pk2(bf16lo(pw), bf16hi(pw)), pk2(x[2 * h], x[2 * h + 1]));
       upk2(X, x[2 * h], x[2 * h + 1]);
     }
+    if (NT == 128) {
+      // factor 0 (index bit 6) with the 64-element half held by lanes ^ 2, on the
+      // fp32 results of the step above (32 shuffles)
+      const uint64_t C4 = pk2(cf.mix2, cf.mix2);
+#pragma unroll
+      for (int h = 0; h < 16; h++) {
+        const float p0 = __shfl_xor_sync(0xFFFFFFFFu, x[2 * h], 2);
+        const float p1 = __shfl_xor_sync(0xFFFFFFFFu, x[2 * h + 1], 2);
+        const uint64_t X = fma2_rn(C4, pk2(p0, p1), pk2(x[2 * h], x[2 * h + 1]));
+        upk2(X, x[2 * h], x[2 * h + 1]);
+      }
+    }
   }
 
-  // stage on index bit 0 (factor 4), scalar: the pair partners share a register pair
+  // stage on index bit 0 (factor 4; 16-element blocks: factor 3 of each half),
+  // scalar: the pair partners share a register pair
 #pragma unroll
   for (int m = 0; m < 16; m++) {
     const float x0 = x[2 * m], x1 = x[2 * m + 1];
     if (MODE == MODE_FWHT) {
       x[2 * m] = __fadd_rn(x0, x1);
       x[2 * m + 1] = __fsub_rn(x1, x0);
+    } else if (NT == 16) {
+      x[2 * m] = __fmaf_rn(cf.l16[m >> 3], x1, x0);
+      x[2 * m + 1] = __fmaf_rn(cf.b16[m >> 3], x0, x1);
     } else {
       x[2 * m] = __fmaf_rn(cf.l4, x1, x0);
       x[2 * m + 1] = __fmaf_rn(cf.b4, x0, x1);
@@ -236,9 +305,10 @@ __device__ __forceinline__ bool quant_block(const ColCoef& cf, const uint32_t (&
   }
 #pragma unroll
   for (int m = 0; m < 16; m++) Y[m] = pk2(x[2 * m], x[2 * m + 1]);
-  // stages on index bits 1..4 (factors 3..0) on packed pairs
+  // stages on index bits 1..4 (factors 3..0; 16-element blocks: bits 1..3, factors
+  // 2..0 of each half) on packed pairs
 #pragma unroll
-  for (int pb = 1; pb < 5; pb++) {
+  for (int pb = 1; pb < (NT == 16 ? 4 : 5); pb++) {
 #pragma unroll
     for (int m = 0; m < 16; m++) {
       if (m & (1 << (pb - 1))) continue;
@@ -247,6 +317,9 @@ __device__ __forceinline__ bool quant_block(const ColCoef& cf, const uint32_t (&
       if (MODE == MODE_FWHT) {
         Y[m] = add2_rn(y0, y1);
         Y[m1] = sub2_rn(y1, y0);
+      } else if (NT == 16) {
+        Y[m] = fma2_rn(cf.L16[pb - 1][m >> 3], y1, y0);
+        Y[m1] = fma2_rn(cf.B16[pb - 1][m >> 3], y0, y1);
       } else {
         Y[m] = fma2_rn(cf.L[pb - 1], y1, y0);
         Y[m1] = fma2_rn(cf.B[pb - 1], y0, y1);
@@ -294,11 +367,8 @@ __device__ __forceinline__ void row_step(const QuantParams& p, const ColCoef& cf
   const bool need = quant_block<MODE, NT>(cf, cur, act, qb, sb);
   if (MODE != MODE_SMOOTH && __any_sync(0xFFFFFFFFu, need)) {
     // rare: the transform block's first input and this block's columns of its matrix
-    const int cx = c - c % (NT / kBlock);
-    const uint16_t* xb = xr - (c - cx) * kBlock;
-    const float* Kb = (MODE == MODE_KRON)
-                          ? p.mats + int64_t(c / (NT / kBlock)) * NT * NT + (c % (NT / kBlock)) * kBlock
-                          : nullptr;
+    const uint16_t* xb = xr - (c - first_column<NT>(c)) * kBlock;
+    const float* Kb = (MODE == MODE_KRON) ? p.mats + kmat_offset<NT>(c) : nullptr;
     constexpr int KSRC = (MODE == MODE_FWHT) ? KSRC_FWHT : KSRC_F32;
     warp_exact_pass<KSRC, NT>(need, xb, Kb, qb, sb);
   }
@@ -306,7 +376,7 @@ __device__ __forceinline__ void row_step(const QuantParams& p, const ColCoef& cf
 
 // TILED: scales in the 128 x 4 tiled layout of block-scaled GEMMs (a template
 // parameter, so the row-major store costs nothing extra).  NT: transform block of
-// 32 or 64 elements (KRON only; 64 needs an even number of block columns).
+// 16, 32, 64 or 128 elements (KRON only; n > 32 needs d % n == 0).
 template <int MODE, int TILED, int NT>
 __global__ void __launch_bounds__(kSThreads, kSCtasPerSm) quant_kernel(const __grid_constant__ QuantParams p) {
   static_assert(kSStages == 4, "the row loop below is written for a ring of four slots");

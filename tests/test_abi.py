@@ -73,7 +73,9 @@ def test_quantize_argument_errors_return_before_launch(lib):
                                         kw.get("log2n", 6), P(16 * 2048), kw.get("dtype", 0),
                                         P(16 * 4096) if kw.get("fac", 1) else None, P(16 * 8192), P(16 * 9000),
                                         kw.get("var", 2), 0, None)
-    assert qn(log2n=7) == 1                   # 32- or 64-element transform blocks
+    assert qn(log2n=8) == 1                   # transform blocks of 16 to 128 elements
+    assert qn(log2n=3) == 1
+    assert qn(log2n=7, d=96, ldx=96) == 2     # 128-element blocks need d % 128 == 0
     assert qn(d=96, ldx=96) == 2              # 64-element blocks need d % 64 == 0
     assert qn(var=1) == 5                     # no tensor-core variant for 64-element blocks
     assert qn(dtype=1) == 5                   # nor bf16 matrices
@@ -93,7 +95,8 @@ def test_other_entry_points_argument_errors(lib):
     assert lib.kq_expand_blocks_n(P(64), 4, 8, 0, 0, P(64), None) == 1  # at most 2^7-element blocks
     assert lib.kq_expand_blocks_n(P(64), 4, 0, 0, 0, P(64), None) == 1
     assert lib.kq_expand_blocks_n(P(64), 0, 6, 0, 0, P(64), None) == 0
-    assert lib.kq_expand_factored_n(P(64), 4, 7, P(64), None) == 1     # butterfly form for 32 or 64
+    assert lib.kq_expand_factored_n(P(64), 4, 8, P(64), None) == 1     # butterfly form for 16 to 128
+    assert lib.kq_expand_factored_n(P(64), 3, 4, P(64), None) == 2     # 16-element blocks come in pairs
     assert lib.kq_expand_factored_n(P(64), 4, 6, P(72), None) == 3
     assert lib.kq_expand_blocks(P(64), 4, -1, 0, P(64), None) == 1
     assert lib.kq_expand_blocks(P(64), 0, 0, 0, P(64), None) == 0

@@ -536,69 +536,129 @@ def test_expand_factored_n64_reproduces_matrix(kq, orc):
     assert fac[10, 43] == 1.0 and fac[11, 43] == 1.0
 
 
-def gpu_quantize_n64(kq, x_bits, params, x_dev=None, scale_layout="row"):
+def test_expand_factored_n16_reproduces_matrices(kq, orc):
+    """16-element transform blocks: one [64] record per 32-element column holds the
+    butterfly of both of its 16-element blocks."""
+    params = inputs.lu_params(12, seed=91, noise=0.3, factors=4)
+    params[9, 1] = (-1.0, 1.0, 1.0)  # d = 0 in one factor: no butterfly form for column 4
+    fac = host(kq.kq_expand_factored(dev_f32(params))).astype(np.float64)
+    assert fac.shape == (6, 64) and np.all(fac[:, 51:] == 0.0)
+    K = orc.expand_n_f64(params)
+    for c in range(6):
+        r = fac[c]
+        assert r[48] >= max(np.abs(K[2 * c]).max(), np.abs(K[2 * c + 1]).max())
+        if r[49]:
+            continue
+        for h in range(2):
+            Mk = np.ones((1, 1))
+            for k in range(4):
+                Mk = np.kron(Mk, np.array([[1.0, r[8 * h + 4 + k]], [r[8 * h + k], 1.0]]))
+            Kf = Mk * r[16 + 16 * h:32 + 16 * h][None, :]
+            assert np.all(np.abs(Kf - K[2 * c + h]) <= 1e-6 * np.abs(K[2 * c + h]) + 1e-30)
+    assert fac[4, 49] == 1.0
+
+
+def test_expand_factored_n128_reproduces_matrix(kq, orc):
+    """128-element transform blocks: each of the four columns of a block carries the
+    five inner factors, its 32 entries of D, and the coefficients of the two
+    cross-column factors that its position uses."""
+    params = inputs.lu_params(3, seed=92, noise=0.3, factors=7)
+    fac = host(kq.kq_expand_factored(dev_f32(params))).astype(np.float64)
+    assert fac.shape == (12, 48)
+    K = orc.expand_n_f64(params)
+    for t in range(3):
+        rec = fac[4 * t:4 * t + 4]
+        assert np.all(rec[:, 43] == 0.0) and np.all(rec[:, 42] >= np.abs(K[t]).max())
+        assert all(np.array_equal(rec[0, :10], rec[q, :10]) for q in range(4))
+        lam1, bet1 = rec[0, 45], rec[1, 45]   # factor 1 (index bit 5): lower / upper column
+        lam0, bet0 = rec[0, 46], rec[2, 46]   # factor 0 (index bit 6): lower / upper 64-element half
+        assert rec[2, 45] == lam1 and rec[3, 45] == bet1 and rec[1, 46] == lam0 and rec[3, 46] == bet0
+        Mk = np.kron(np.array([[1.0, bet0], [lam0, 1.0]]), np.array([[1.0, bet1], [lam1, 1.0]]))
+        for k in range(5):
+            Mk = np.kron(Mk, np.array([[1.0, rec[0, 5 + k]], [rec[0, k], 1.0]]))
+        Kf = Mk * np.concatenate([rec[q, 10:42] for q in range(4)])[None, :]
+        assert np.all(np.abs(Kf - K[t]) <= 1e-6 * np.abs(K[t]) + 1e-30)
+
+
+def gpu_quantize_n(kq, x_bits, params, x_dev=None, scale_layout="row"):
     p = dev_f32(params)
     mats = kq.kq_expand_blocks(p)
     fac = kq.kq_expand_factored(p)
     x = dev_bf16(x_bits) if x_dev is None else x_dev
-    qd, sd = kq.kq_quantize(x, mats, fac, variant="butterfly", scale_layout=scale_layout)
-    return host(qd), host(sd)
+    M, d = x.shape
+    q, s, bufs = guarded_outputs(M, d, scale_layout)
+    kq.kq_quantize(x, mats, fac, variant="butterfly", q=q, scales=s, scale_layout=scale_layout)
+    torch.cuda.synchronize()
+    assert_guards(bufs)
+    return host(q), host(s)
 
 
-@pytest.mark.parametrize("M,d", [(1, 64), (3, 128), (65, 1152), (130, 2240), (33, 12288), (257, 3072), (300, 4608)])
-def test_quantize_n64_ragged_shapes(kq, orc, M, d):
-    x = inputs.activations(M, d, "t3", seed=[M, d, 64], outlier_frac=0.01, outlier_scale=(20.0, 100.0))
-    params = inputs.lu_params(d // 64, seed=[M, d, 65], factors=6)
-    q, s = gpu_quantize_n64(kq, x, params)
+# (log2 n, shapes): d a multiple of max(32, n)
+N_SHAPES = {
+    4: [(1, 32), (3, 96), (65, 1152), (130, 2240), (33, 12288), (257, 3072)],
+    6: [(1, 64), (3, 128), (65, 1152), (130, 2240), (33, 12288), (257, 3072), (300, 4608)],
+    7: [(1, 128), (3, 256), (65, 1152), (33, 12288), (257, 3072), (300, 4608)],
+}
+
+
+@pytest.mark.parametrize("log2n,M,d", [(k, M, d) for k, v in N_SHAPES.items() for M, d in v])
+def test_quantize_n_ragged_shapes(kq, orc, log2n, M, d):
+    x = inputs.activations(M, d, "t3", seed=[M, d, 64 + log2n], outlier_frac=0.01, outlier_scale=(20.0, 100.0))
+    params = inputs.lu_params(d >> log2n, seed=[M, d, 65 + log2n], factors=log2n)
+    q, s = gpu_quantize_n(kq, x, params)
     K = orc.expand_n(params)
     qr, sr = orc.quantize_n(x, K)
     check(q, s, qr, sr, orc.transform_n(x, K))
 
 
-def test_quantize_n64_flux_shape(kq, orc):
+@pytest.mark.parametrize("log2n", [4, 6, 7])
+def test_quantize_n_flux_shape(kq, orc, log2n):
     x, _ = inputs.config_case("flux", 3072)
-    params = inputs.lu_params(3072 // 64, seed=66, factors=6)
-    q, s = gpu_quantize_n64(kq, x, params)
-    qr, sr = orc.quantize_n(x, orc.expand_n(params))
+    params = inputs.lu_params(3072 >> log2n, seed=66 + log2n, factors=log2n)
+    q, s = gpu_quantize_n(kq, x, params)
+    qr, sr = oracle_rows("quantize_n", x, orc.expand_n(params))
     check(q, s, qr, sr)
 
 
-def test_quantize_n64_degenerate_and_singular(kq, orc):
-    rng = np.random.default_rng(67)
+@pytest.mark.parametrize("log2n", [4, 6, 7])
+def test_quantize_n_degenerate_and_singular(kq, orc, log2n):
+    n = 1 << log2n
+    rng = np.random.default_rng(67 + log2n)
     M, d = 24, 384
     a = rng.standard_normal((M, d)).astype(np.float32)
     a[0] = 0.0                       # all-zero row
-    a[1, 64:128] = 0.0               # an all-zero 64-element block
-    a[2, 0:32] = 0.0                 # one zero half: its outputs still see the other half
+    a[1, 128:256] = 0.0              # all-zero transform blocks
+    a[2, 0:16] = 0.0                 # a zero part: its outputs still see the rest of the block
     a[3, 5] = np.inf
     a[4, 100] = np.nan
     a[6] *= 1e37
     a[7] *= 1e-39
     a[8, 33] = 3.4e38
-    a[9, 64:128] = 3.0               # constant block (exact cancellations)
+    a[9, 128:256] = 3.0              # constant blocks (exact cancellations)
     x = inputs.f32_to_bf16_bits(a)
-    params = inputs.lu_params(d // 64, seed=68, factors=6)
-    params[2, 4, 1] = 0.0            # u = 0: singular factor in transform block 2
-    params[3, 0] = (-1.0, 1.0, 1.0)  # d = 0 in the half-mixing factor of block 3
-    q, s = gpu_quantize_n64(kq, x, params)
+    params = inputs.lu_params(d // n, seed=68 + log2n, factors=log2n)
+    params[1, log2n - 2, 1] = 0.0    # u = 0: singular factor in transform block 1
+    params[2, 0] = (-1.0, 1.0, 1.0)  # d = 0 in the outermost factor of block 2
+    q, s = gpu_quantize_n(kq, x, params)
     assert kq.kq_get_device_error(clear=True) == 4
     qr, sr = orc.quantize_n(x, orc.expand_n(params))
     check(q, s, qr, sr)
 
 
-def test_quantize_n64_strided_rows_and_tiled_scales(kq, orc):
+@pytest.mark.parametrize("log2n", [4, 6, 7])
+def test_quantize_n_strided_rows_and_tiled_scales(kq, orc, log2n):
     M, d, ldx = 70, 1280, 1280 + 72
-    full = inputs.activations(M, ldx, "normal", seed=69, outlier_frac=0.01, outlier_scale=(50.0, 50.0))
-    params = inputs.lu_params(d // 64, seed=70, factors=6)
+    full = inputs.activations(M, ldx, "normal", seed=69 + log2n, outlier_frac=0.01, outlier_scale=(50.0, 50.0))
+    params = inputs.lu_params(d >> log2n, seed=70 + log2n, factors=log2n)
     xd = dev_bf16(full)[:, :d]
     qr, sr = orc.quantize_n(np.ascontiguousarray(full[:, :d]), orc.expand_n(params))
-    q, s = gpu_quantize_n64(kq, None, params, x_dev=xd)
+    q, s = gpu_quantize_n(kq, None, params, x_dev=xd)
     check(q, s, qr, sr)
-    q, s = gpu_quantize_n64(kq, None, params, x_dev=xd, scale_layout="mma")
+    q, s = gpu_quantize_n(kq, None, params, x_dev=xd, scale_layout="mma")
     assert np.array_equal(q, qr) and np.array_equal(s, tiled_scales(sr))
 
 
-def test_no_device_error_after_n64(kq):
+def test_no_device_error_after_n_blocks(kq):
     assert kq.kq_get_device_error(clear=True) == 0
 
 

@@ -498,33 +498,40 @@ def test_hadamard_init_n64_reproduces_h64_up_to_signs(orc):
     assert np.abs(K @ K.T - np.eye(64)).max() < 1e-6
 
 
+@pytest.mark.parametrize("log2n", [4, 6, 7])
 @pytest.mark.parametrize("dtype", [0, 1])
-def test_transform_n64_exact_rational_brute_force(orc, dtype):
-    rng = np.random.default_rng(67 + dtype)
-    M, d = 2, 128
+def test_transform_n_exact_rational_brute_force(orc, dtype, log2n):
+    n = 1 << log2n
+    rng = np.random.default_rng(67 + dtype + 10 * log2n)
+    M, d = 2, 2 * n if n >= 32 else 64
     x = inputs.f32_to_bf16_bits((rng.standard_t(3, (M, d)) * rng.choice([1, 100], (M, d))).astype(np.float32))
-    params = inputs.lu_params(d // 64, seed=68, factors=6)
+    params = inputs.lu_params(d // n, seed=68 + log2n, factors=log2n)
     mats = orc.expand_n(params, dtype=dtype)
     y = orc.transform_n(x, mats)
     matf = mats if dtype == 0 else inputs.bf16_bits_to_f32(mats)
     for r in range(M):
-        for c in range(d // 64):
-            xs = [bf16_bits_to_frac(int(h)) for h in x[r, 64 * c:64 * c + 64]]
-            for j in range(0, 64, 5):
-                exact = sum(xs[i] * Fraction(float(matf[c, i, j])) for i in range(64))
-                assert y[r, 64 * c + j] == f32_round_fraction(exact), (r, c, j)
+        for c in range(d // n):
+            xs = [bf16_bits_to_frac(int(h)) for h in x[r, n * c:n * c + n]]
+            for j in range(0, n, 5 if n <= 64 else 11):
+                exact = sum(xs[i] * Fraction(float(matf[c, i, j])) for i in range(n))
+                assert y[r, n * c + j] == f32_round_fraction(exact), (r, c, j)
 
 
-def test_quantize_n64_is_mx_of_the_transform(orc):
-    """MXFP4 per 32 elements of the n = 64 transform: scales by the bit-field
-    rule from each 32-block's amax, codes by the brute-force nearest value."""
-    rng = np.random.default_rng(69)
-    x = inputs.f32_to_bf16_bits(rng.standard_normal((3, 128)).astype(np.float32))
-    mats = orc.expand_n(inputs.lu_params(2, seed=70, factors=6))
+@pytest.mark.parametrize("log2n", [4, 6, 7])
+def test_quantize_n_is_mx_of_the_transform(orc, log2n):
+    """MXFP4 per 32 elements of the n-element block transform: scales by the
+    bit-field rule from each 32-block's amax, codes by the brute-force nearest
+    value."""
+    n = 1 << log2n
+    rng = np.random.default_rng(69 + log2n)
+    d = max(128, 2 * n)
+    x = inputs.f32_to_bf16_bits(rng.standard_normal((3, d)).astype(np.float32))
+    mats = orc.expand_n(inputs.lu_params(d // n, seed=70 + log2n, factors=log2n))
     y = orc.transform_n(x, mats)
     q, s = orc.quantize_n(x, mats)
-    amax = np.abs(y.reshape(3, 4, 32)).max(axis=2)
+    nb = d // 32
+    amax = np.abs(y.reshape(3, nb, 32)).max(axis=2)
     assert np.array_equal(s, e8m0_from_bits(amax.astype(np.float32)).astype(np.uint8))
     scale = np.exp2(s.astype(np.float64) - 127.0)
-    v = (y.reshape(3, 4, 32) / scale[:, :, None]).astype(np.float32).reshape(3, 128)
-    assert np.array_equal(unpack_nibbles(q).reshape(3, 128), brute_e2m1(v))
+    v = (y.reshape(3, nb, 32) / scale[:, :, None]).astype(np.float32).reshape(3, d)
+    assert np.array_equal(unpack_nibbles(q).reshape(3, d), brute_e2m1(v))

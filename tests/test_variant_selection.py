@@ -64,7 +64,8 @@ def test_auto_fixed_choices(kq):
 
     out = ctypes.c_int(-1)
     assert lib.kq_select_variant(4, 64, 6, 1, 1, ctypes.byref(out)) == 5   # 64-element blocks: fp32 only
-    assert lib.kq_select_variant(4, 64, 7, 0, 1, ctypes.byref(out)) == 1
+    assert lib.kq_select_variant(4, 64, 8, 0, 1, ctypes.byref(out)) == 1
+    assert lib.kq_select_variant(4, 64, 4, 0, 1, ctypes.byref(out)) == 0 and out.value == 2
     assert lib.kq_select_variant(-1, 64, 5, 0, 1, ctypes.byref(out)) == 1
     assert lib.kq_select_variant(4, 64, 5, 0, 1, None) == 1
 
