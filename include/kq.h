@@ -140,12 +140,22 @@ KQ_API kq_status kq_expand_blocks_n(const float* params, int64_t nt, int log2n, 
  */
 KQ_API kq_status kq_expand_factored(const float* params, int64_t nb, float* factored, kq_stream_t stream);
 
-/* kq_expand_factored_n -- the butterfly form for transform blocks of 32 (log2n 5)
- * or 64 (log2n 6) elements, one [48]-float record per 32-element block column
- * (nt * n / 32 records): the five factors acting inside the 32-element block in
- * [0..9] as above, this block's 32 entries of D in [10..41], max|K| bound, exact-only
- * flag and absolute allowance in [42..44], and for 64-element blocks c/a, b/d of
- * F0 (the factor that mixes the two halves) in [45], [46].  factored 16-byte aligned.
+/* kq_expand_factored_n -- the butterfly form for transform blocks of n = 2^log2n
+ * elements, log2n 4..7 ([KQ-sum, Limitations]), one record per 32-element block
+ * column, factored 16-byte aligned:
+ *   log2n 5..7: nt * n / 32 records of [48] floats: the five factors acting inside
+ *     the 32-element block in [0..9] as above (factors log2n-5 .. log2n-1), this
+ *     block's 32 entries of D in [10..41], max|K| bound, exact-only flag and absolute
+ *     allowance in [42..44];
+ *     log2n 6: c/a, b/d of F0 (it mixes the two 32-element halves) in [45], [46];
+ *     log2n 7: [45] the coefficient of F1 (index bit 5) that this column applies
+ *       (c/a if it is the lower column of its pair, else b/d), [46] the same for F0
+ *       (index bit 6) and the column's 64-element half.
+ *   log2n 4: nt / 2 records of [64] floats (nt even; a 32-element column holds two
+ *     16-element blocks h = 0, 1): [8h .. 8h+3] c/a and [8h+4 .. 8h+7] b/d of factors
+ *     0..3 of block h, [16..47] D for the 32 outputs, [48] max|K| bound over both
+ *     blocks, [49] exact-only flag, [50] absolute allowance, [51..63] zero.
+ * log2n outside 4..7: KQ_ERR_INVALID_ARG; odd nt with log2n 4: KQ_ERR_SHAPE.
  * kq_expand_factored(p, nb, ...) is kq_expand_factored_n(p, nb, 5, ...).
  */
 KQ_API kq_status kq_expand_factored_n(const float* params, int64_t nt, int log2n, float* factored,
@@ -177,14 +187,16 @@ KQ_API kq_status kq_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, c
                       kq_dtype mat_dtype, const float* factored, uint8_t* q, uint8_t* scales,
                       kq_variant variant, kq_scale_layout scale_layout, kq_stream_t stream);
 
-/* kq_quantize_n -- the same with transform blocks of n = 2^log2n elements, log2n 5
- * or 6 ([KQ-sum, Limitations]); the MX scale blocks stay 32 elements long.
+/* kq_quantize_n -- the same with transform blocks of n = 2^log2n elements, log2n 4..7
+ * ([KQ-sum, Limitations]: 3 log2(n) parameters per block); the MX scale blocks stay
+ * 32 elements long.
  *   log2n 5: exactly kq_quantize.
- *   log2n 6: d % 64 == 0 (else KQ_ERR_SHAPE); mats fp32 [d/64][64][64] from
- *            kq_expand_blocks_n and factored from kq_expand_factored_n with the same
- *            params are both required; only the butterfly serves it (KQ_VAR_MMA or
- *            bf16 matrices: KQ_ERR_UNSUPPORTED).  y_j = fp32(sum over the 64 inputs
- *            of the block), certified and recomputed exactly like kq_quantize.
+ *   log2n 4, 6, 7: d % max(32, n) == 0 (else KQ_ERR_SHAPE); mats fp32 [d/n][n][n]
+ *            from kq_expand_blocks_n and factored from kq_expand_factored_n with the
+ *            same params are both required; only the butterfly serves them
+ *            (KQ_VAR_MMA or bf16 matrices: KQ_ERR_UNSUPPORTED).  y_j = fp32(sum over
+ *            the n inputs of the block), certified and recomputed exactly like
+ *            kq_quantize.
  *   log2n other: KQ_ERR_INVALID_ARG.
  */
 KQ_API kq_status kq_quantize_n(const void* x, int64_t M, int64_t d, int64_t ldx, int log2n, const void* mats,
@@ -230,9 +242,9 @@ KQ_API kq_status kq_e2m1_pack(const float* v, int64_t n, uint8_t* out, kq_stream
  * factored, ..., KQ_VAR_AUTO, ...) runs for these sizes, without launching
  * anything: *chosen = KQ_VAR_MMA or KQ_VAR_BUTTERFLY.  has_factored != 0 when the
  * factored form will be passed.  KQ_ERR_INVALID_ARG for a NULL chosen, a negative
- * size, a bad dtype or log2n other than 5 or 6; KQ_ERR_UNSUPPORTED when no
- * variant serves the combination (64-element blocks need fp32 matrices and the
- * factored form).  Host-only: needs no device. */
+ * size, a bad dtype or log2n outside 4..7; KQ_ERR_UNSUPPORTED when no variant
+ * serves the combination (16-, 64- and 128-element blocks need fp32 matrices and
+ * the factored form).  Host-only: needs no device. */
 KQ_API kq_status kq_select_variant(int64_t M, int64_t d, int log2n, kq_dtype mat_dtype, int has_factored,
                                    kq_variant* chosen);
 
