@@ -216,6 +216,30 @@ KQ_API kq_status kq_dequantize(const uint8_t* q, const uint8_t* scales, int64_t 
                         const void* inv_mats, kq_dtype mat_dtype, void* out, kq_dtype out_dtype,
                         kq_stream_t stream);
 
+/* ---------------------------------------------------------------- consumer
+ *
+ * kq_gemm_mxf4 -- the W4A4 product the quantizer feeds [KQ-sum, Approach; KQ-abs,
+ * "W4A4 (MXFP4e2)"]: activations quantized with K_b and weights with K_b^-T, so
+ *   C[m][n] = sum_k A(m,k) B(n,k),  A(m,k) = E2M1(a_q code) * 2^(a_scale byte - 127),
+ *                                   B(n,k) = E2M1(b_q code) * 2^(b_scale byte - 127),
+ * computed on the tensor cores (tcgen05.mma kind::mxf4, block scales of 32
+ * elements) with fp32 accumulation, then rounded to c_dtype.
+ *   a_q       device [M][K/2] codes as written by kq_quantize (x rows), 16-byte aligned.
+ *   a_scales  device, KQ_SCALES_MMA_TILED layout for M rows and K/32 blocks, 16-byte
+ *             aligned; its padding bytes are never used.
+ *   b_q       device [N][K/2] codes of the weight rows (BlockTransform.quantize_weights).
+ *   b_scales  device, KQ_SCALES_MMA_TILED layout for N rows, 16-byte aligned.
+ *   c         device [M][ldc] fp32 (KQ_F32) or bf16 bits (KQ_BF16), element aligned;
+ *             ldc >= N.  Only columns < N are written.
+ * K must be a positive multiple of 32 (KQ_ERR_SHAPE otherwise); M or N = 0 is a
+ * no-op.  A block whose scale byte is 0xFF (non-finite input) yields NaN in the rows
+ * or columns it touches.  The sum of each 64-element step is formed by the tensor
+ * core and added to an fp32 accumulator; the result is within the fp32 rounding of
+ * K/64 such additions of the exact product.  Bounded waits (kq_get_device_error). */
+KQ_API kq_status kq_gemm_mxf4(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, const uint8_t* b_q,
+                              const uint8_t* b_scales, int64_t N, int64_t K, void* c, int64_t ldc, kq_dtype c_dtype,
+                              kq_stream_t stream);
+
 /* ---------------------------------------------------------------- comparison points
  *
  * kq_ref_smooth_quantize -- per-channel scaling (SmoothQuant) then MXFP4, the

@@ -34,7 +34,7 @@ EXPORTED = (
     "kq_expand_blocks", "kq_expand_factored", "kq_quantize", "kq_dequantize", "kq_ref_smooth_quantize",
     "kq_expand_blocks_n", "kq_expand_factored_n", "kq_quantize_n",
     "kq_ref_fwht_quantize", "kq_e2m1_pack", "kq_get_device_error", "kq_status_string", "kq_abi_version",
-    "kq_last_error", "kq_select_variant",
+    "kq_last_error", "kq_select_variant", "kq_gemm_mxf4",
 )
 
 
@@ -75,6 +75,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kq_abi_version": [],
         "kq_last_error": [],
         "kq_select_variant": [I64, I64, I, I, I, P],
+        "kq_gemm_mxf4": [P, P, I64, P, P, I64, I64, P, I64, I, P],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -275,6 +276,26 @@ def kq_dequantize(q: torch.Tensor, scales: torch.Tensor, inv_mats: torch.Tensor 
     with torch.cuda.device(q.device):
         _check("kq_dequantize", load().kq_dequantize(_ptr(q), _ptr(scales), M, d, _ptr(inv_mats), mdt, _ptr(out),
                                                      _mat_dtype(out), _stream(q.device)))
+    return out
+
+
+def kq_gemm_mxf4(a_q: torch.Tensor, a_scales: torch.Tensor, b_q: torch.Tensor, b_scales: torch.Tensor,
+                 out_dtype: torch.dtype = torch.float32, out: torch.Tensor | None = None) -> torch.Tensor:
+    """C [M, N] = A . B^T on the tensor cores from two MXFP4 operands as kq_quantize
+    writes them with scale_layout="mma": codes [M, K/2] and [N, K/2], tiled scales."""
+    _cuda(a_q, "a_q", dtypes=(torch.uint8,), contiguous=True)
+    _cuda(b_q, "b_q", a_q.device, (torch.uint8,), contiguous=True)
+    if a_q.dim() != 2 or b_q.dim() != 2 or a_q.shape[1] != b_q.shape[1]:
+        raise ValueError("a_q and b_q must be [M, K/2] and [N, K/2] with the same K")
+    M, N, K = a_q.shape[0], b_q.shape[0], a_q.shape[1] * 2
+    _cuda(a_scales, "a_scales", a_q.device, (torch.uint8,), contiguous=True, min_numel=scale_bytes(M, K, "mma"))
+    _cuda(b_scales, "b_scales", a_q.device, (torch.uint8,), contiguous=True, min_numel=scale_bytes(N, K, "mma"))
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=a_q.device)
+    _cuda(out, "out", a_q.device, (torch.float32,) + _BF16_LIKE, contiguous=True, min_numel=M * N)
+    with torch.cuda.device(a_q.device):
+        _check("kq_gemm_mxf4", load().kq_gemm_mxf4(_ptr(a_q), _ptr(a_scales), M, _ptr(b_q), _ptr(b_scales), N, K,
+                                                   _ptr(out), N, _mat_dtype(out), _stream(a_q.device)))
     return out
 
 

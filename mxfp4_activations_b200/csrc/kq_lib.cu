@@ -17,6 +17,7 @@
 #include "kq.h"
 #include "kq_common.cuh"
 #include "kq_expand.cuh"
+#include "kq_gemm.cuh"
 #include "kq_misc.cuh"
 #include "kq_mma.cuh"
 #include "kq_quant.cuh"
@@ -254,6 +255,55 @@ kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, con
                     "quant_mma_kernel launch", tmap, p);
 }
 
+// W4A4 GEMM: one 128 x 128 tile of C per CTA, N tiles across x, M tiles across y.
+kq_status launch_gemm(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, const uint8_t* b_q,
+                      const uint8_t* b_scales, int64_t N, int64_t K, void* c, int64_t ldc, bool c_bf16,
+                      cudaStream_t stream) {
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return cuda_fail("device query", cudaErrorInvalidDevice);
+  EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
+  if (kq::kGmSmemBytes > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
+  // codes as a 2-D byte tensor [rows][K/2], 128-row x 64-byte boxes, 64-byte swizzle
+  CUtensorMap maps[2];
+  const uint8_t* codes[2] = {a_q, b_q};
+  const int64_t rows[2] = {M, N};
+  for (int i = 0; i < 2; i++) {
+    const cuuint64_t gdim[2] = {cuuint64_t(K / 2), cuuint64_t(rows[i])};
+    const cuuint64_t gstride[1] = {cuuint64_t(K / 2)};
+    const cuuint32_t box[2] = {64, cuuint32_t(kq::kGmTile)};
+    const cuuint32_t estride[2] = {1, 1};
+    if (enc(&maps[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes[i]), gdim, gstride, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cuda_fail("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
+  }
+  static std::atomic<int> attr_set[kMaxDevices];
+  int devid = 0;
+  cudaGetDevice(&devid);
+  if (!attr_set[devid].load()) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kq::mxf4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kq::kGmSmemBytes);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
+    attr_set[devid].store(1);
+  }
+  kq::GemmParams p;
+  p.sa = a_scales;
+  p.sb = b_scales;
+  p.c = c;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.ldc = ldc;
+  p.c_bf16 = c_bf16 ? 1 : 0;
+  p.n_ktiles = int((K + kq::kGmKStage - 1) / kq::kGmKStage);
+  p.k_tail_blocks = int((K / 32 - 1) % 4) + 1;
+  p.c_vec = (aligned(c, 16) && (ldc * (c_bf16 ? 2 : 4)) % 16 == 0) ? 1 : 0;
+  const int64_t gx = (N + kq::kGmTile - 1) / kq::kGmTile, gy = (M + kq::kGmTile - 1) / kq::kGmTile;
+  return launch_pdl(kq::mxf4_gemm_kernel, dim3(unsigned(gx), unsigned(gy)), kq::kGmThreads, kq::kGmSmemBytes, stream,
+                    "mxf4_gemm_kernel launch", maps[0], maps[1], p);
+}
+
 kq_status check_x(const void* x, int64_t M, int64_t d, int64_t ldx) {
   if (M < 0 || d < 0) return KQ_ERR_INVALID_ARG;
   if (d % 32 != 0 || ldx < d) return KQ_ERR_SHAPE;
@@ -340,7 +390,7 @@ kq_variant resolve_variant(int64_t M, int64_t d, kq_dtype mat_dtype, bool has_fa
 
 extern "C" {
 
-int kq_abi_version(void) { return 201; }
+int kq_abi_version(void) { return 202; }
 
 const char* kq_status_string(kq_status s) {
   switch (s) {
@@ -486,6 +536,24 @@ kq_status kq_dequantize(const uint8_t* q, const uint8_t* scales, int64_t M, int6
   kern<<<dim3(unsigned(nb), unsigned(gy)), kq::kDqWarps * 32, 0, as_cuda(stream)>>>(
       q, scales, M, int(nb), inv_mats, mat_dtype == KQ_BF16 ? 1 : 0, out, out_dtype == KQ_BF16 ? 1 : 0);
   return launch_status("dequant_kernel launch");
+}
+
+kq_status kq_gemm_mxf4(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, const uint8_t* b_q,
+                       const uint8_t* b_scales, int64_t N, int64_t K, void* c, int64_t ldc, kq_dtype c_dtype,
+                       kq_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0) return KQ_ERR_INVALID_ARG;
+  if (c_dtype != KQ_F32 && c_dtype != KQ_BF16) return KQ_ERR_INVALID_ARG;
+  if (K % 32 != 0 || ldc < N) return KQ_ERR_SHAPE;
+  if (M == 0 || N == 0) return KQ_OK;
+  if (K == 0) return KQ_ERR_SHAPE;
+  if (a_q == nullptr || a_scales == nullptr || b_q == nullptr || b_scales == nullptr || c == nullptr)
+    return KQ_ERR_INVALID_ARG;
+  if (!aligned(a_q, 16) || !aligned(b_q, 16) || !aligned(a_scales, 16) || !aligned(b_scales, 16) ||
+      !aligned(c, c_dtype == KQ_BF16 ? 2 : 4))
+    return KQ_ERR_ALIGN;
+  if (K / 2 > int64_t(INT32_MAX) - 128 || M > int64_t(65535) * kq::kGmTile || N > int64_t(INT32_MAX) - kq::kGmTile)
+    return KQ_ERR_SHAPE;
+  return launch_gemm(a_q, a_scales, M, b_q, b_scales, N, K, c, ldc, c_dtype == KQ_BF16, as_cuda(stream));
 }
 
 kq_status kq_e2m1_pack(const float* v, int64_t n, uint8_t* out, kq_stream_t stream) {

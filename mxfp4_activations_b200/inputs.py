@@ -24,6 +24,13 @@ CONFIGS = {
     "flux": dict(M=4608, ds=(3072, 12288), law="t3", outlier_frac=0.005, outlier_scale=(100.0, 100.0), token_lognormal=None, seed=3),
 }
 SWEEP_M = (1, 16, 256, 4096, 16384, 65536)
+# W4A4 products of the FLUX.1-schnell-shaped workload (4608 tokens of width 3072):
+# name: (M tokens, N outputs, K inputs) of the linear layer the quantized rows feed.
+GEMM_SHAPES = {
+    "flux_proj": (4608, 3072, 3072),
+    "flux_fc1": (4608, 12288, 3072),
+    "flux_fc2": (4608, 3072, 12288),
+}
 SWEEP_D = (1152, 3072, 12288)
 
 
@@ -116,3 +123,13 @@ def smooth_inv_scale(x_bits: np.ndarray) -> np.ndarray:
     a = np.abs(bf16_bits_to_f32(x_bits)).max(axis=0).astype(np.float64)
     a = np.maximum(a, 1e-6)
     return (1.0 / np.sqrt(a)).astype(np.float32)
+
+
+def mx_operand(rows: int, K: int, seed, scale_range=(118, 136)):
+    """A random MXFP4 operand: codes [rows, K/2] (uniform bytes: every E2M1 code and
+    sign in both nibbles) and row-major E8M0 scale bytes [rows, K/32] drawn uniformly
+    from scale_range (inclusive)."""
+    rng = np.random.default_rng(seed)
+    q = rng.integers(0, 256, (rows, K // 2), dtype=np.uint8)
+    s = rng.integers(scale_range[0], scale_range[1] + 1, (rows, K // 32), dtype=np.uint8)
+    return q, s

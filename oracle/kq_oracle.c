@@ -368,3 +368,27 @@ void kqo_quantize_n(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const 
   kqo_mx_quantize(y, M, d, q, scales);
   free(y);
 }
+
+/* ---- the consumer: W4A4 product of two MXFP4 operands --------------------------- */
+
+/* Value of element k of an MXFP4 row: its E2M1 code times its block's power of two. */
+static double mx_value(const uint8_t* q, const uint8_t* scales, int64_t row, int64_t k, int64_t K) {
+  const int byte = scales[row * (K / KQO_N) + k / KQO_N];
+  const uint8_t pair = q[row * (K / 2) + k / 2];
+  const int code = (k & 1) ? (pair >> 4) : (pair & 0xF);
+  if (byte == 0xFF) return NAN;
+  return ldexp(kqo_e2m1_value(code), byte - 127);
+}
+
+/* [KQ-sum, Approach]; [KQ-abs] W4A4: the plain dot product of every activation row
+ * with every weight row, both as MXFP4 values, summed in fp64 in index order. */
+void kqo_mx_gemm(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, const uint8_t* b_q,
+                 const uint8_t* b_scales, int64_t N, int64_t K, double* c) {
+  for (int64_t m = 0; m < M; m++)
+    for (int64_t n = 0; n < N; n++) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; k++)
+        acc += mx_value(a_q, a_scales, m, k, K) * mx_value(b_q, b_scales, n, k, K);
+      c[m * N + n] = acc;
+    }
+}

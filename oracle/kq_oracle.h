@@ -106,6 +106,17 @@ void kqo_transform_n(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const
 void kqo_quantize_n(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const void* mats, int dtype,
                     int n, uint8_t* q, uint8_t* scales);
 
+/* ---- the consumer: W4A4 product of two MXFP4 operands
+ *
+ * [KQ-sum, Approach] and [KQ-abs] ("W4A4 (MXFP4e2)"): activations quantized with
+ * K_b, weights with K_b^-T, so the layer's product is taken between the two MXFP4
+ * tensors.  c[m][n] = sum_k A(m,k) B(n,k) in fp64 with
+ * A(m,k) = value(code of a_q[m], element k) * 2^(a_scales[m][k/32] - 127) and B alike;
+ * a scale byte 0xFF makes its values NaN.  Codes [rows][K/2] (element 2j in the low
+ * nibble of byte j), scales row-major [rows][K/32], c fp64 [M][N]. */
+void kqo_mx_gemm(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, const uint8_t* b_q,
+                 const uint8_t* b_scales, int64_t N, int64_t K, double* c);
+
 #ifdef __cplusplus
 }
 #endif

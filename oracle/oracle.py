@@ -97,9 +97,10 @@ def _configure(L):
     L.kqo_smooth_quantize.argtypes = [P, I64, I64, I64, P, P, P]
     L.kqo_fwht_quantize.argtypes = [P, I64, I64, I64, P, P]
     L.kqo_dequantize.argtypes = [P, P, I64, I64, P, I, P]
+    L.kqo_mx_gemm.argtypes = [P, P, I64, P, P, I64, I64, P]
     for name in ("kqo_factor", "kqo_factor_inverse", "kqo_kron", "kqo_expand_f64", "kqo_expand",
                  "kqo_hadamard", "kqo_e2m1_pack", "kqo_transform", "kqo_mx_quantize", "kqo_quantize",
-                 "kqo_smooth_quantize", "kqo_fwht_quantize", "kqo_dequantize"):
+                 "kqo_smooth_quantize", "kqo_fwht_quantize", "kqo_dequantize", "kqo_mx_gemm"):
         getattr(L, name).restype = None
     return L
 
@@ -293,3 +294,16 @@ def quantize_n(x: np.ndarray, mats: np.ndarray):
     s = np.zeros((M, d // 32), np.uint8)
     lib().kqo_quantize_n(_p(x), M, d, d, _p(mats), _mats_dtype(mats), n, _p(q), _p(s))
     return q, s
+
+
+# ---- the consumer: W4A4 product ------------------------------------------------------
+
+def mx_gemm(a_q: np.ndarray, a_scales: np.ndarray, b_q: np.ndarray, b_scales: np.ndarray) -> np.ndarray:
+    """c [M, N] fp64 = sum_k A(m, k) B(n, k) over MXFP4 operands with row-major scales."""
+    a_q, b_q = np.ascontiguousarray(a_q, np.uint8), np.ascontiguousarray(b_q, np.uint8)
+    a_scales, b_scales = np.ascontiguousarray(a_scales, np.uint8), np.ascontiguousarray(b_scales, np.uint8)
+    M, N, K = a_q.shape[0], b_q.shape[0], a_q.shape[1] * 2
+    assert b_q.shape[1] * 2 == K and a_scales.shape == (M, K // 32) and b_scales.shape == (N, K // 32)
+    c = np.zeros((M, N), np.float64)
+    lib().kqo_mx_gemm(_p(a_q), _p(a_scales), M, _p(b_q), _p(b_scales), N, K, _p(c))
+    return c

@@ -179,3 +179,23 @@ def oracle_rows(fn: str, x: np.ndarray, K: np.ndarray | None = None, extra=None,
         for h in blocks:
             h.close()
             h.unlink()
+
+
+def tiled_scales(s: np.ndarray, pad: int = 0) -> np.ndarray:
+    """Row-major [M][C] scales rearranged into 128 x 4 tiles (tile rows first; in a
+    tile, row r = 32 * r_hi + r_lo and column c go to 16 * r_lo + 4 * r_hi + c),
+    written as a reshape so that it shares no arithmetic with the kernels.  Padding
+    bytes get the value `pad`."""
+    M, C = s.shape
+    Mp, Cp = -(-M // 128) * 128, -(-C // 4) * 4
+    full = np.full((Mp, Cp), pad, np.uint8)
+    full[:M, :C] = s
+    t = full.reshape(Mp // 128, 4, 32, Cp // 4, 4)       # (R, r_hi, r_lo, C, c)
+    return np.ascontiguousarray(t.transpose(0, 3, 2, 1, 4)).reshape(-1)
+
+
+def untiled_scales(t: np.ndarray, M: int, C: int) -> np.ndarray:
+    """Inverse of tiled_scales: the row-major [M][C] scales of a tiled buffer."""
+    Mp, Cp = -(-M // 128) * 128, -(-C // 4) * 4
+    full = np.asarray(t, np.uint8).reshape(-1)[: Mp * Cp].reshape(Mp // 128, Cp // 4, 32, 4, 4)  # (R, C, r_lo, r_hi, c)
+    return np.ascontiguousarray(full.transpose(0, 3, 2, 1, 4)).reshape(Mp, Cp)[:M, :C]

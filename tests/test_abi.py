@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.kq_abi_version() == 201
+    assert lib.kq_abi_version() == 202
     for code in range(8):
         s = lib.kq_status_string(code).decode()
         assert s.startswith("KQ_")
@@ -110,6 +110,17 @@ def test_other_entry_points_argument_errors(lib):
     assert lib.kq_e2m1_pack(P(16), 7, P(16), None) == 2
     assert lib.kq_e2m1_pack(P(16), 0, P(16), None) == 0
     assert lib.kq_e2m1_pack(P(20), 8, P(16), None) == 3
+    # kq_gemm_mxf4(a_q, a_scales, M, b_q, b_scales, N, K, c, ldc, c_dtype, stream)
+    g = lib.kq_gemm_mxf4
+    assert g(P(16), P(16), 4, P(16), P(16), 4, 48, P(16), 4, 0, None) == 2    # K not a multiple of 32
+    assert g(P(16), P(16), 4, P(16), P(16), 4, 64, P(16), 3, 0, None) == 2    # ldc < N
+    assert g(P(16), P(16), 4, P(16), P(16), 4, 0, P(16), 4, 0, None) == 2     # K = 0 with work to do
+    assert g(P(16), P(16), 0, P(16), P(16), 4, 64, P(16), 4, 0, None) == 0    # M = 0: no-op
+    assert g(P(16), P(16), 4, P(16), P(16), -1, 64, P(16), 4, 0, None) == 1
+    assert g(P(16), P(16), 4, P(16), P(16), 4, 64, P(16), 4, 2, None) == 1    # bad output dtype
+    assert g(None, P(16), 4, P(16), P(16), 4, 64, P(16), 4, 0, None) == 1
+    assert g(P(16), P(16), 4, P(24), P(16), 4, 64, P(16), 4, 0, None) == 3    # codes 16-byte aligned
+    assert g(P(16), P(16), 4, P(16), P(16), 4, 64, P(18), 4, 0, None) == 3    # fp32 C 4-byte aligned
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

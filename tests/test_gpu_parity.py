@@ -14,7 +14,7 @@ torch = pytest.importorskip("torch")
 
 from mxfp4_activations_b200 import inputs  # noqa: E402
 
-from .parity import compare, guarded, guards_intact, oracle_rows, unpack  # noqa: E402
+from .parity import compare, guarded, guards_intact, oracle_rows, tiled_scales, unpack  # noqa: E402
 
 pytestmark = [
     pytest.mark.gpu,
@@ -234,18 +234,6 @@ def test_quantize_degenerate_blocks(kq, orc, variant, mdt):
     K = oracle_mats(orc, params, mdt)
     qr, sr = orc.quantize(x, K)
     check(q, s, qr, sr)
-
-
-def tiled_scales(s: np.ndarray) -> np.ndarray:
-    """Row-major [M][C] scales rearranged into 128 x 4 tiles (tile rows first; in a
-    tile, row r = 32 * r_hi + r_lo and column c go to 16 * r_lo + 4 * r_hi + c),
-    written as a reshape so that it shares no arithmetic with the kernels."""
-    M, C = s.shape
-    Mp, Cp = -(-M // 128) * 128, -(-C // 4) * 4
-    pad = np.zeros((Mp, Cp), np.uint8)
-    pad[:M, :C] = s
-    t = pad.reshape(Mp // 128, 4, 32, Cp // 4, 4)       # (R, r_hi, r_lo, C, c)
-    return np.ascontiguousarray(t.transpose(0, 3, 2, 1, 4)).reshape(-1)
 
 
 @pytest.mark.parametrize("variant,mdt", VARIANTS)

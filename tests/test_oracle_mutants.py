@@ -11,6 +11,7 @@ grid and the random-pattern pins cover the E2M1 cases).
 from __future__ import annotations
 
 import inspect
+import itertools
 import os
 
 import pytest
@@ -55,6 +56,15 @@ MUTANTS = {
                               "(float)((double)f32_from_bf16(x[r * ldx + c]))"),
     "dequantize_scale_inverted": ("ldexp(1.0, byte - 127)", "ldexp(1.0, 127 - byte)"),
     "dequantize_inverse_transposed": ("(int64_t)j * KQO_N + i);", "(int64_t)i * KQO_N + j);"),
+    # the W4A4 product
+    # (a nibble swap on both operands leaves every dot product unchanged: not a mistake here)
+    "mx_gemm_high_nibble_twice": ("const int code = (k & 1) ? (pair >> 4) : (pair & 0xF);\n  if (byte == 0xFF)",
+                                  "const int code = (k & 1) ? (pair >> 4) : (pair >> 4);\n  if (byte == 0xFF)"),
+    "mx_gemm_scale_of_next_block": ("scales[row * (K / KQO_N) + k / KQO_N];",
+                                    "scales[row * (K / KQO_N) + (k / KQO_N + 1) % (K / KQO_N)];"),
+    "mx_gemm_scale_sign": ("ldexp(kqo_e2m1_value(code), byte - 127)", "ldexp(kqo_e2m1_value(code), 127 - byte)"),
+    "mx_gemm_last_element_dropped": ("for (int64_t k = 0; k < K; k++)\n        acc +=",
+                                     "for (int64_t k = 0; k < K - 1; k++)\n        acc +="),
 }
 
 SKIP = {"test_e2m1_exhaustive_core_binades"}
@@ -71,9 +81,10 @@ def pin_calls():
         if not marks:
             calls.append((name, (lambda f: lambda orc: f(orc) if "orc" in inspect.signature(f).parameters else f())(fn)))
             continue
-        argname, values = marks[0].args[0], marks[0].args[1]
-        for v in values:
-            calls.append((f"{name}[{v}]", (lambda f, a, v: lambda orc: f(orc, **{a: v}))(fn, argname, v)))
+        names = [m.args[0] for m in marks]
+        for combo in itertools.product(*(m.args[1] for m in marks)):
+            kw = dict(zip(names, combo))
+            calls.append((f"{name}{list(combo)}", (lambda f, kw: lambda orc: f(orc, **kw))(fn, kw)))
         assert params[0] == "orc"
     return calls
 

@@ -535,3 +535,74 @@ def test_quantize_n_is_mx_of_the_transform(orc, log2n):
     scale = np.exp2(s.astype(np.float64) - 127.0)
     v = (y.reshape(3, nb, 32) / scale[:, :, None]).astype(np.float32).reshape(3, d)
     assert np.array_equal(unpack_nibbles(q).reshape(3, d), brute_e2m1(v))
+
+
+# ---------------------------------------------------------------- the W4A4 product (consumer of the codes)
+
+def _golden_e2m1_values() -> dict:
+    vals = {}
+    with open(os.path.join(GOLDEN, "e2m1_grid.txt")) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) == 2 and parts[0].isdigit():
+                vals[int(parts[0])] = Fraction(parts[1])
+    assert len(vals) == 16
+    return vals
+
+
+def test_mx_gemm_exact_rational_brute_force(orc):
+    """Every entry of the oracle's W4A4 product against an exact rational sum written
+    from the E2M1 table of the OCP definition (tests/golden/e2m1_grid.txt) and the
+    header's nibble order, with ragged K (three 32-blocks) and scales of both signs
+    of exponent.  A swapped nibble, a scale read from the wrong block or row, or a
+    transposed operand changes some entry."""
+    vals = _golden_e2m1_values()
+    rng = np.random.default_rng(71)
+    M, N, K = 3, 4, 96
+    aq = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    bq = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    sa = rng.integers(100, 150, (M, K // 32), dtype=np.uint8)
+    sb = rng.integers(100, 150, (N, K // 32), dtype=np.uint8)
+    c = orc.mx_gemm(aq, sa, bq, sb)
+
+    def elem(q, s, r, k):
+        byte = int(q[r, k // 2])
+        code = byte >> 4 if k % 2 else byte & 0xF
+        return vals[code] * Fraction(2) ** (int(s[r, k // 32]) - 127)
+
+    for m in range(M):
+        for n in range(N):
+            exact = sum(elem(aq, sa, m, k) * elem(bq, sb, n, k) for k in range(K))
+            assert c[m, n] == float(exact), (m, n)  # fp64 holds every partial sum exactly here
+
+
+def test_mx_gemm_one_hot_closed_form(orc):
+    """A single nonzero element on each side: c = value_a value_b 2^(sa + sb - 254)
+    at exactly one (m, n), zero elsewhere."""
+    M, N, K = 2, 3, 64
+    aq = np.zeros((M, K // 2), np.uint8)
+    bq = np.zeros((N, K // 2), np.uint8)
+    aq[1, 37 // 2] = 0x7 << 4          # element 37 (odd: high nibble) = +6
+    bq[2, 37 // 2] = 0xB << 4          # element 37 of weight row 2 = -1.5
+    sa = np.full((M, K // 32), 127, np.uint8)
+    sb = np.full((N, K // 32), 127, np.uint8)
+    sa[1, 1], sb[2, 1] = 130, 120     # block 1 holds element 37
+    c = orc.mx_gemm(aq, sa, bq, sb)
+    want = np.zeros((M, N))
+    want[1, 2] = 6.0 * -1.5 * 2.0 ** (3 - 7)
+    assert np.array_equal(c, want)
+
+
+def test_mx_gemm_nan_scale_poisons_its_row_and_column(orc):
+    """Scale byte 0xFF is NaN (OCP MX): every product that reads such a block is NaN."""
+    rng = np.random.default_rng(72)
+    M, N, K = 3, 3, 64
+    aq = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    bq = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    sa = np.full((M, 2), 127, np.uint8)
+    sb = np.full((N, 2), 127, np.uint8)
+    sa[0, 1] = 0xFF
+    sb[2, 0] = 0xFF
+    c = orc.mx_gemm(aq, sa, bq, sb)
+    assert np.isnan(c[0]).all() and np.isnan(c[:, 2]).all()
+    assert np.isfinite(c[1:, :2]).all()
