@@ -63,8 +63,76 @@ def measured_peaks() -> dict:
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "source": "fallback"}
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+FP4_OVER_BF16 = 4.0  # nominal dense ratio on B200: 9 PFLOP/s FP4 / 2.25 PFLOP/s bf16
+
+
+def gemm_leg(torch, kq, n: int, device) -> dict:
+    """The quantizer's consumer, kq_gemm_mxf4 (bf16 C), on the FLUX linear-layer
+    shapes: random MXFP4 operands, four copies of each rotated so that the operands
+    of consecutive launches are not all in L2, back-to-back launches between CUDA
+    events.  cuBLAS's block-scaled FP4 GEMM (through torch) on the same operands
+    is timed beside it as a cross-check."""
+    F = torch.nn.functional
+    peaks = measured_peaks()
+    peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    out = {"peak_tflops": round(peak, 1),
+           "peak_source": f"{peaks['source']} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/bf16 ratio)",
+           "output": "bf16", "timing": f"{n} launches back to back over 4 rotated operand copies", "shapes": {}}
+    for name, (M, N, K) in inputs.GEMM_SHAPES.items():
+        sets = []
+        for c in range(4):
+            aq, _ = inputs.mx_operand(M, K, seed=[M, N, K, c, 1])
+            bq, _ = inputs.mx_operand(N, K, seed=[M, N, K, c, 2])
+            rng = np.random.default_rng([M, N, K, c, 3])
+            sa = rng.integers(118, 137, kq.scale_bytes(M, K, "mma"), dtype=np.uint8)
+            sb = rng.integers(118, 137, kq.scale_bytes(N, K, "mma"), dtype=np.uint8)
+            sets.append([torch.from_numpy(a).to(device) for a in (aq, sa, bq, sb)])
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+
+        def ours(i):
+            a, sa_, b, sb_ = sets[i % 4]
+            kq.kq_gemm_mxf4(a, sa_, b, sb_, out=C)
+
+        def cublas(i):
+            a, sa_, b, sb_ = sets[i % 4]
+            F.scaled_mm(a.view(torch.float4_e2m1fn_x2), b.view(torch.float4_e2m1fn_x2).t(),
+                        sa_.view(torch.float8_e8m0fnu), F.ScalingType.BlockWise1x32,
+                        sb_.view(torch.float8_e8m0fnu), F.ScalingType.BlockWise1x32,
+                        swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                        output_dtype=torch.bfloat16)
+
+        def loop(fn) -> float:
+            for i in range(8):
+                fn(i)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(n):
+                fn(i)
+            e1.record()
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) * 1e3 / n
+
+        flops = 2.0 * M * N * K
+        us = loop(ours)
+        rec = {"M": M, "N": N, "K": K, "us": round(us, 2), "tflops": round(flops / us / 1e6, 1),
+               "frac": round(flops / us / 1e6 / peak, 4)}
+        try:
+            cus = loop(cublas)
+            rec["cublas_us"] = round(cus, 2)
+            rec["cublas_tflops"] = round(flops / cus / 1e6, 1)
+        except (RuntimeError, AttributeError, TypeError, ValueError) as e:
+            rec["cublas_us"] = f"unavailable: {str(e).splitlines()[0][:80]}"
+        out["shapes"][name] = rec
+        del sets, C
+    err = kq.kq_get_device_error(clear=True)
+    if err != 0:
+        raise RuntimeError(f"device error in the GEMM leg: {kq.kq_status_string(err)}")
+    return out
 
 
 def recorded_traffic(d: int):
@@ -401,6 +469,8 @@ def run_gpu(args) -> None:
         us = {str(it["d"]): timed_b2b(torch, step, j, kind, n_cmp) for j, it in enumerate(step.items)}
         comp[kind] = {"gbs": bytes_step / (sum(us.values()) * 1e-6) / 1e9, "us_per_launch": us}
 
+    gemm = gemm_leg(torch, kq, max(20, min(args.steps, 50)), device)
+
     e2e_steps = max(3, min(args.steps, 20))
     e2e_ms, h2d, d2h = e2e_run(torch, kq, step, xs, e2e_steps)
     if world > 1:
@@ -463,6 +533,7 @@ def run_gpu(args) -> None:
                 "streams": "upload / quantize / download overlapped across steps, double-buffered"},
         "gpu_launches": len(FLUX_DS) * args.steps,
         "clocks": clocks,
+        "gemm_w4a4": gemm,
     }
     if not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
@@ -728,13 +799,30 @@ def run_profile(args) -> None:
     xs, ps = zip(*(inputs.config_case("flux", d) for d in FLUX_DS))
     step = QuantStep(torch, kq, list(xs), list(ps), n_copies=1, device=torch.device("cuda", 0))
     kinds = args.profile_kinds.split(",")
+    launches = 0
     for kind in kinds:
+        if kind.startswith("gemm"):
+            # gemm or gemm:<shape name>: the W4A4 product on random operands
+            names = [kind.split(":", 1)[1]] if ":" in kind else list(inputs.GEMM_SHAPES)
+            for name in names:
+                M, N, K = inputs.GEMM_SHAPES[name]
+                aq, _ = inputs.mx_operand(M, K, seed=1)
+                bq, _ = inputs.mx_operand(N, K, seed=2)
+                sa = torch.full((kq.scale_bytes(M, K, "mma"),), 127, dtype=torch.uint8, device="cuda")
+                sb = torch.full((kq.scale_bytes(N, K, "mma"),), 127, dtype=torch.uint8, device="cuda")
+                a, b = torch.from_numpy(aq).cuda(), torch.from_numpy(bq).cuda()
+                c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+                for it in range(args.steps):
+                    kq.kq_gemm_mxf4(a, sa, b, sb, out=c)
+                    launches += 1
+            continue
         for it in range(args.steps):
             for item in step.items:
                 step.launch(it, item, kind)
+                launches += 1
     torch.cuda.synchronize()
     assert kq.kq_get_device_error(clear=True) == 0
-    print(json.dumps({"profile": kinds, "launches": len(kinds) * args.steps * len(FLUX_DS)}))
+    print(json.dumps({"profile": kinds, "launches": launches}))
 
 
 def main():

@@ -240,6 +240,15 @@ KQ_API kq_status kq_gemm_mxf4(const uint8_t* a_q, const uint8_t* a_scales, int64
                               const uint8_t* b_scales, int64_t N, int64_t K, void* c, int64_t ldc, kq_dtype c_dtype,
                               kq_stream_t stream);
 
+/* kq_select_gemm_kernel -- which kernel kq_gemm_mxf4 runs for M x N x K on the current
+ * device, without launching: *two_sm = 1 for the persistent two-SM kernel (tcgen05
+ * cta_group::2, 256 x 256 tiles; needs K % 128 == 0 and at least one tile per SM
+ * pair), 0 for the one-SM kernel (128 x 128 tiles).  The environment variable
+ * KQ_GEMM=1sm|2sm (read once per process) overrides the choice where both apply.
+ * KQ_ERR_INVALID_ARG for a NULL two_sm or a negative size, KQ_ERR_SHAPE for
+ * K % 32 != 0, KQ_ERR_CUDA without a device. */
+KQ_API kq_status kq_select_gemm_kernel(int64_t M, int64_t N, int64_t K, int* two_sm);
+
 /* ---------------------------------------------------------------- comparison points
  *
  * kq_ref_smooth_quantize -- per-channel scaling (SmoothQuant) then MXFP4, the

@@ -17,6 +17,7 @@ from ._lib import (  # noqa: F401
     kq_e2m1_pack,
     kq_expand_blocks,
     kq_expand_factored,
+    kq_gemm_kernel,
     kq_gemm_mxf4,
     kq_get_device_error,
     kq_quantize,

@@ -34,7 +34,7 @@ EXPORTED = (
     "kq_expand_blocks", "kq_expand_factored", "kq_quantize", "kq_dequantize", "kq_ref_smooth_quantize",
     "kq_expand_blocks_n", "kq_expand_factored_n", "kq_quantize_n",
     "kq_ref_fwht_quantize", "kq_e2m1_pack", "kq_get_device_error", "kq_status_string", "kq_abi_version",
-    "kq_last_error", "kq_select_variant", "kq_gemm_mxf4",
+    "kq_last_error", "kq_select_variant", "kq_gemm_mxf4", "kq_select_gemm_kernel",
 )
 
 
@@ -76,6 +76,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kq_last_error": [],
         "kq_select_variant": [I64, I64, I, I, I, P],
         "kq_gemm_mxf4": [P, P, I64, P, P, I64, I64, P, I64, I, P],
+        "kq_select_gemm_kernel": [I64, I64, I64, P],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -297,6 +298,13 @@ def kq_gemm_mxf4(a_q: torch.Tensor, a_scales: torch.Tensor, b_q: torch.Tensor, b
         _check("kq_gemm_mxf4", load().kq_gemm_mxf4(_ptr(a_q), _ptr(a_scales), M, _ptr(b_q), _ptr(b_scales), N, K,
                                                    _ptr(out), N, _mat_dtype(out), _stream(a_q.device)))
     return out
+
+
+def kq_gemm_kernel(M: int, N: int, K: int) -> str:
+    """"2sm" or "1sm": the kernel kq_gemm_mxf4 runs for this shape on the current device."""
+    v = ctypes.c_int(0)
+    _check("kq_select_gemm_kernel", load().kq_select_gemm_kernel(M, N, K, ctypes.byref(v)))
+    return "2sm" if v.value else "1sm"
 
 
 def kq_ref_smooth_quantize(x: torch.Tensor, inv_s: torch.Tensor, q=None, scales=None):

@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdlib>
@@ -255,6 +256,140 @@ kq_status launch_quant_mma(const void* x, int64_t M, int64_t d, int64_t ldx, con
                     "quant_mma_kernel launch", tmap, p);
 }
 
+// Which GEMM kernel serves a shape: the two-SM persistent kernel needs K % 128 == 0
+// and pays off once its 256 x 256 tiles give every SM pair work; smaller products
+// take the one-SM kernel's 128 x 128 tiles.  KQ_GEMM=1sm|2sm (read once) overrides
+// the choice where both apply.
+int gemm_env() {
+  static const int v = []() {
+    const char* e = std::getenv("KQ_GEMM");
+    if (e == nullptr) return 0;
+    if (std::strcmp(e, "1sm") == 0) return 1;
+    if (std::strcmp(e, "2sm") == 0) return 2;
+    if (std::strcmp(e, "2sm128") == 0) return 3;
+    return 0;
+  }();
+  return v;
+}
+
+bool gemm_uses_pair(int64_t M, int64_t N, int64_t K, int sms) {
+  if (K % 128 != 0) return false;
+  const int e = gemm_env();
+  if (e != 0) return e >= 2;
+  const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  return tiles >= sms / 2;
+}
+
+// Codes as a byte matrix [rows][K/2]: boxes of 128 rows x row_bytes (64 or 128) with
+// the swizzle of the same width.
+kq_status encode_codes_map(EncodeTiledFn enc, CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K,
+                           int row_bytes) {
+  const cuuint64_t gdim[2] = {cuuint64_t(K / 2), cuuint64_t(rows)};
+  const cuuint64_t gstride[1] = {cuuint64_t(K / 2)};
+  const cuuint32_t box[2] = {cuuint32_t(row_bytes), cuuint32_t(kq::kGmTile)};
+  const cuuint32_t estride[2] = {1, 1};
+  if (enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), gdim, gstride, box, estride,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cuda_fail("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
+  return KQ_OK;
+}
+
+// Tiled scales as a byte matrix of 256-byte half tiles: a box of 2 * n_tiles rows is
+// n_tiles consecutive 512-byte 128 x 4 tiles; tiles past the buffer read as zeros.
+kq_status encode_scales_map(EncodeTiledFn enc, CUtensorMap* map, const uint8_t* scales, int64_t rows, int64_t K,
+                            int n_tiles) {
+  const int64_t tiles = ((rows + 127) / 128) * (K / 128);
+  const cuuint64_t gdim[2] = {256, cuuint64_t(2 * tiles)};
+  const cuuint64_t gstride[1] = {256};
+  const cuuint32_t box[2] = {256, cuuint32_t(2 * n_tiles)};
+  const cuuint32_t estride[2] = {1, 1};
+  if (enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(scales), gdim, gstride, box, estride,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cuda_fail("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
+  return KQ_OK;
+}
+
+// C as a [M][ldc] matrix of bf16 or fp32 for TMA tensor stores of 32 x 32 boxes with
+// the swizzle of the box's row width (64 or 128 bytes).  False when C's base or row
+// stride is not 16-byte aligned or the encoder refuses; the kernels then store
+// directly.
+bool encode_c_map(EncodeTiledFn enc, CUtensorMap* map, void* c, int64_t M, int64_t N, int64_t ldc, bool bf16) {
+  const int64_t esz = bf16 ? 2 : 4;
+  if (!aligned(c, 16) || (ldc * esz) % 16 != 0) return false;
+  const cuuint64_t gdim[2] = {cuuint64_t(N), cuuint64_t(M)};
+  const cuuint64_t gstride[1] = {cuuint64_t(ldc * esz)};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estride[2] = {1, 1};
+  return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, c, gdim, gstride, box,
+             estride, CU_TENSOR_MAP_INTERLEAVE_NONE, bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Two-SM persistent W4A4 GEMM: one cluster of two CTAs per SM pair, 256 x 256 tiles,
+// KS K-elements per stage.
+template <int KS>
+kq_status launch_gemm_pair(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, const uint8_t* b_q,
+                           const uint8_t* b_scales, int64_t N, int64_t K, void* c, int64_t ldc, bool c_bf16,
+                           cudaStream_t stream) {
+  using C = kq::G2Cfg<KS>;
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return cuda_fail("device query", cudaErrorInvalidDevice);
+  EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
+  if (C::kSmemBytes > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
+  CUtensorMap ma, mb, msa, msb;
+  kq_status st;
+  if ((st = encode_codes_map(enc, &ma, a_q, M, K, C::kRowBytes)) != KQ_OK ||
+      (st = encode_codes_map(enc, &mb, b_q, N, K, C::kRowBytes)) != KQ_OK ||
+      (st = encode_scales_map(enc, &msa, a_scales, M, K, C::kTiles)) != KQ_OK ||
+      (st = encode_scales_map(enc, &msb, b_scales, N, K, C::kTiles)) != KQ_OK)
+    return st;
+  static std::atomic<int> attr_set[kMaxDevices];
+  int devid = 0;
+  cudaGetDevice(&devid);
+  if (!attr_set[devid].load()) {
+    const cudaError_t e = cudaFuncSetAttribute(kq::mxf4_gemm2_kernel<KS>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
+    attr_set[devid].store(1);
+  }
+  CUtensorMap mc;
+  std::memset(&mc, 0, sizeof(mc));
+  kq::Gemm2Params p;
+  p.c = c;
+  p.M = M;
+  p.N = N;
+  p.ldc = ldc;
+  p.c_bf16 = c_bf16 ? 1 : 0;
+  p.c_tma = encode_c_map(enc, &mc, c, M, N, ldc, c_bf16) ? 1 : 0;
+  p.n_ktiles = int(K / KS);
+  p.n_ctiles = int(K / 128);
+  p.tiles_m = int((M + 255) / 256);
+  p.tiles_n = int((N + 255) / 256);
+  const int64_t tiles = int64_t(p.tiles_m) * p.tiles_n;
+  const int64_t clusters = std::min<int64_t>(tiles, dev->sms / 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(2 * clusters));
+  cfg.blockDim = dim3(unsigned(kq::kG2Threads));
+  cfg.dynamicSmemBytes = size_t(C::kSmemBytes);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kq::mxf4_gemm2_kernel<KS>, ma, mb, msa, msb, mc, p);
+  if (e != cudaSuccess) return cuda_fail("mxf4_gemm2_kernel launch", e);
+  return KQ_OK;
+}
+
 // W4A4 GEMM: one 128 x 128 tile of C per CTA, N tiles across x, M tiles across y.
 kq_status launch_gemm(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, const uint8_t* b_q,
                       const uint8_t* b_scales, int64_t N, int64_t K, void* c, int64_t ldc, bool c_bf16,
@@ -287,6 +422,8 @@ kq_status launch_gemm(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, co
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
     attr_set[devid].store(1);
   }
+  CUtensorMap mc;
+  std::memset(&mc, 0, sizeof(mc));
   kq::GemmParams p;
   p.sa = a_scales;
   p.sb = b_scales;
@@ -296,12 +433,12 @@ kq_status launch_gemm(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, co
   p.K = K;
   p.ldc = ldc;
   p.c_bf16 = c_bf16 ? 1 : 0;
+  p.c_tma = encode_c_map(enc, &mc, c, M, N, ldc, c_bf16) ? 1 : 0;
   p.n_ktiles = int((K + kq::kGmKStage - 1) / kq::kGmKStage);
   p.k_tail_blocks = int((K / 32 - 1) % 4) + 1;
-  p.c_vec = (aligned(c, 16) && (ldc * (c_bf16 ? 2 : 4)) % 16 == 0) ? 1 : 0;
   const int64_t gx = (N + kq::kGmTile - 1) / kq::kGmTile, gy = (M + kq::kGmTile - 1) / kq::kGmTile;
   return launch_pdl(kq::mxf4_gemm_kernel, dim3(unsigned(gx), unsigned(gy)), kq::kGmThreads, kq::kGmSmemBytes, stream,
-                    "mxf4_gemm_kernel launch", maps[0], maps[1], p);
+                    "mxf4_gemm_kernel launch", maps[0], maps[1], mc, p);
 }
 
 kq_status check_x(const void* x, int64_t M, int64_t d, int64_t ldx) {
@@ -553,7 +690,24 @@ kq_status kq_gemm_mxf4(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, c
     return KQ_ERR_ALIGN;
   if (K / 2 > int64_t(INT32_MAX) - 128 || M > int64_t(65535) * kq::kGmTile || N > int64_t(INT32_MAX) - kq::kGmTile)
     return KQ_ERR_SHAPE;
+  const DeviceInfo* dev = device_info();
+  if (dev != nullptr && gemm_uses_pair(M, N, K, dev->sms)) {
+    if (K % 256 == 0 && gemm_env() != 3)
+      return launch_gemm_pair<256>(a_q, a_scales, M, b_q, b_scales, N, K, c, ldc, c_dtype == KQ_BF16,
+                                   as_cuda(stream));
+    return launch_gemm_pair<128>(a_q, a_scales, M, b_q, b_scales, N, K, c, ldc, c_dtype == KQ_BF16,
+                                 as_cuda(stream));
+  }
   return launch_gemm(a_q, a_scales, M, b_q, b_scales, N, K, c, ldc, c_dtype == KQ_BF16, as_cuda(stream));
+}
+
+kq_status kq_select_gemm_kernel(int64_t M, int64_t N, int64_t K, int* two_sm) {
+  if (two_sm == nullptr || M < 0 || N < 0 || K < 0) return KQ_ERR_INVALID_ARG;
+  if (K % 32 != 0) return KQ_ERR_SHAPE;
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return cuda_fail("device query", cudaErrorInvalidDevice);
+  *two_sm = gemm_uses_pair(M, N, K, dev->sms) ? 1 : 0;
+  return KQ_OK;
 }
 
 kq_status kq_e2m1_pack(const float* v, int64_t n, uint8_t* out, kq_stream_t stream) {

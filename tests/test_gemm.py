@@ -79,6 +79,7 @@ SMALL = [(1, 1, 32), (1, 8, 64), (127, 129, 96), (130, 260, 160), (256, 128, 128
 
 @pytest.mark.parametrize("M,N,K", SMALL)
 def test_gemm_random_operands_every_entry(kq, orc, M, N, K):
+    assert kq.kq_gemm_kernel(M, N, K) == "1sm"
     """Every entry, shapes spanning several 128 x 128 tiles, ragged M and N, K ending
     inside a 128-element stage (tiled-scale padding filled with 0xFF), K longer than
     the stage ring."""
@@ -119,23 +120,50 @@ def sample_rows(M: int) -> np.ndarray:
     return np.unique(np.concatenate([fixed, rng.choice(M, 14, replace=False)]))
 
 
-@pytest.mark.parametrize("name", sorted(inputs.GEMM_SHAPES))
-def test_gemm_flux_layer_shapes_sampled_rows(kq, orc, name):
-    """The FLUX-shaped products at full size, in the launch configuration the bench
-    times; the oracle checks 24 sampled rows (tile edges included) against every
-    column, from its dequantized operands multiplied in fp64."""
-    M, N, K = inputs.GEMM_SHAPES[name]
-    aq, sa = inputs.mx_operand(M, K, seed=[M, N, K, 7])
-    bq, sb = inputs.mx_operand(N, K, seed=[M, N, K, 8])
-    c = run_gemm(kq, aq, sa, bq, sb)
-    rows = sample_rows(M)
+def check_sampled(orc, c, aq, sa, bq, sb, bf16: bool):
+    K = aq.shape[1] * 2
+    rows = sample_rows(aq.shape[0])
     a_hat = orc.dequantize(aq[rows], sa[rows])
     b_hat = orc.dequantize(bq, sb)
     ref = a_hat @ b_hat.T
     mag = np.abs(a_hat) @ np.abs(b_hat).T
     err = np.abs(c[rows] - ref)
-    assert np.all(err <= bound(K, mag, ref, False)), err.max()
+    assert np.all(err <= bound(K, mag, ref, bf16)), err.max()
     assert np.isfinite(c).all()
+
+
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+@pytest.mark.parametrize("name", sorted(inputs.GEMM_SHAPES))
+def test_gemm_flux_layer_shapes_sampled_rows(kq, orc, name, out):
+    """The FLUX-shaped products at full size, in the launch configuration the bench
+    times (the two-SM kernel); the oracle checks 24 sampled rows (tile edges
+    included) against every column, from its dequantized operands multiplied in
+    fp64."""
+    M, N, K = inputs.GEMM_SHAPES[name]
+    aq, sa = inputs.mx_operand(M, K, seed=[M, N, K, 7])
+    bq, sb = inputs.mx_operand(N, K, seed=[M, N, K, 8])
+    c = run_gemm(kq, aq, sa, bq, sb, out_dtype=torch.float32 if out == "f32" else torch.bfloat16)
+    check_sampled(orc, c, aq, sa, bq, sb, out == "bf16")
+
+
+# two-SM kernel (K % 128 == 0 and at least one 256 x 256 tile per SM pair): ragged M
+# and N (a pair whose second CTA lies wholly past M), several tiles per cluster, and
+# K % 256 == 128 (stages of 128 K-elements instead of 256)
+PAIR = [(3900, 2000, 1024), (2304, 4352, 512), (4608, 9216, 3072), (2304, 4352, 640)]
+
+
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+@pytest.mark.parametrize("M,N,K", PAIR)
+def test_gemm_pair_kernel_ragged_and_persistent(kq, orc, M, N, K, out):
+    assert kq.kq_gemm_kernel(M, N, K) == "2sm"
+    aq, sa = inputs.mx_operand(M, K, seed=[M, N, K, 9])
+    bq, sb = inputs.mx_operand(N, K, seed=[M, N, K, 10])
+    c = run_gemm(kq, aq, sa, bq, sb, out_dtype=torch.float32 if out == "f32" else torch.bfloat16)
+    check_sampled(orc, c, aq, sa, bq, sb, out == "bf16")
+    cols = np.random.default_rng(M).choice(N, 16, replace=False)
+    ref = orc.mx_gemm(aq, sa, bq[cols], sb[cols])  # every row against 16 columns
+    mag = orc.mx_gemm(magnitudes(aq), sa, magnitudes(bq[cols]), sb[cols])
+    assert np.all(np.abs(c[:, cols] - ref) <= bound(K, mag, ref, out == "bf16"))
 
 
 def test_gemm_end_to_end_with_the_quantizer(kq, orc):
