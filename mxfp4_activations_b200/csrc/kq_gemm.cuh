@@ -112,6 +112,19 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Non-blocking test of an mbarrier phase (acquire semantics when it reports completion).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // TMA tensor store from shared memory, tracked by this thread's bulk async-group.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int c0, int c1) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
@@ -452,6 +465,27 @@ __device__ __forceinline__ void pair_commit(uint64_t* bar) {
       : "memory");
 }
 
+// One stage's scale tiles from both CTAs' shared memory into their tensor memory:
+// A tile c to sfa + 4c, B tiles of tile column c (rows 0..127, 128..255) to sfb + 8c
+// and sfb + 8c + 4.  Scale tiles are 32 rows of 16 bytes, no swizzle (core matrices of
+// 8 rows x 16 bytes stacked every 128 bytes); each row lands in one lane of every
+// lane quarter.
+template <class C>
+__device__ __forceinline__ void pair_scale_copies(uint32_t st, uint32_t sfa_col, uint32_t sfb_col) {
+#pragma unroll
+  for (int c = 0; c < C::kTiles; c++) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(sfa_col + 4 * c),
+                 "l"(gemm_sdesc(st + C::kSfaOff + 512 * c, 128, 128, 0))
+                 : "memory");
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(sfb_col + 8 * c),
+                 "l"(gemm_sdesc(st + C::kSfbOff + 512 * c, 128, 128, 0))
+                 : "memory");
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(sfb_col + 8 * c + 4),
+                 "l"(gemm_sdesc(st + C::kSfbOff + 512 * (C::kTiles + c), 128, 128, 0))
+                 : "memory");
+  }
+}
+
 template <int KS>
 __global__ void __launch_bounds__(kG2Threads, 1)
     mxf4_gemm2_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
@@ -512,7 +546,7 @@ __global__ void __launch_bounds__(kG2Threads, 1)
         const int sfa_tile = tm * 2 + int(rank), sfb_tile = tn * 2;
         for (int kt = 0; kt < p.n_ktiles; kt++, it++) {
           const int s = it % C::kStages;
-          if (it >= C::kStages &&
+          if (it >= C::kStages && !mbar_test(&empty[s], uint32_t(it / C::kStages - 1) & 1u) &&
               (*abort_flag || !mbar_wait_bounded(&empty[s], uint32_t(it / C::kStages - 1) & 1u, kWaitLimitNs))) {
             *abort_flag = 1;
             ok = false;
@@ -547,30 +581,24 @@ __global__ void __launch_bounds__(kG2Threads, 1)
           break;
         }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        // The issuing thread is held by the tensor pipe while it issues a stage, so
+        // the next stage's barrier is tested (without blocking) before that, and the
+        // full wait with its time-outs runs only when the test found it incomplete.
+        bool ready = mbar_test(&full[it % C::kStages], uint32_t(it / C::kStages) & 1u);
         for (int kt = 0; kt < p.n_ktiles; kt++, it++) {
           const int s = it % C::kStages;
-          if (*abort_flag || !mbar_wait_bounded(&full[s], uint32_t(it / C::kStages) & 1u, kWaitLimitNs)) {
+          if (!ready &&
+              (*abort_flag || !mbar_wait_bounded(&full[s], uint32_t(it / C::kStages) & 1u, kWaitLimitNs))) {
             *abort_flag = 1;
             ok = false;
             break;
           }
           asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          ready = kt + 1 < p.n_ktiles &&
+                  mbar_test(&full[(it + 1) % C::kStages], uint32_t((it + 1) / C::kStages) & 1u);
           const uint32_t st = smem_addr(base + s * C::kStageBytes);
-          // tensor-memory scale columns of the stage: A tile c at sfa + 4c; B scales of
-          // tile column c at sfb + 8c (rows 0..127, then 128..255)
           const uint32_t sfa_col = tmem + 256 + uint32_t(C::kSfCols * s), sfb_col = sfa_col + 4 * C::kTiles;
-#pragma unroll
-          for (int c = 0; c < C::kTiles; c++) {
-            asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(sfa_col + 4 * c),
-                         "l"(gemm_sdesc(st + C::kSfaOff + 512 * c, 128, 128, 0))
-                         : "memory");
-            asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(sfb_col + 8 * c),
-                         "l"(gemm_sdesc(st + C::kSfbOff + 512 * c, 128, 128, 0))
-                         : "memory");
-            asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(sfb_col + 8 * c + 4),
-                         "l"(gemm_sdesc(st + C::kSfbOff + 512 * (C::kTiles + c), 128, 128, 0))
-                         : "memory");
-          }
+          pair_scale_copies<C>(st, sfa_col, sfb_col);
 #pragma unroll
           for (int j = 0; j < C::kMmas; j++) {
             const uint64_t ad = gemm_sdesc(st + j * 32, 16, C::kSbo, C::kLayout);
