@@ -135,6 +135,20 @@ def gemm_leg(torch, kq, n: int, device) -> dict:
     return out
 
 
+def recorded_exact_path_share():
+    """Share of blocks the certified kernels send to their exact path at the bench's
+    FLUX inputs: the host estimate committed by tests/exact_path_rate.py."""
+    path = os.path.join(ROOT, "profiles", "kq_exact_path_rate.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    return {"kind": "host estimate (tests/exact_path_rate.py)",
+            "butterfly": {d: round(r["butterfly"], 5) for d, r in rec["rates"].items()},
+            "tensor_core_bf16_K": {d: round(r["tensor_core_bf16_K"], 5) for d, r in rec["rates"].items()},
+            "tensor_core_fp32_K": {d: round(r["tensor_core_fp32_K"], 5) for d, r in rec["rates"].items()}}
+
+
 def recorded_traffic(d: int):
     """DRAM bytes (read + write) of one launch of the dominant kernel at width d,
     from the committed ncu summary, if it was taken on the current kernel sources;
@@ -534,6 +548,7 @@ def run_gpu(args) -> None:
         "gpu_launches": len(FLUX_DS) * args.steps,
         "clocks": clocks,
         "gemm_w4a4": gemm,
+        "exact_path_share": recorded_exact_path_share(),
     }
     if not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)

@@ -53,17 +53,29 @@ constexpr int kMmaThreads = (2 + kMmaEpiWarps) * 32; // 320
 constexpr int kMmaATileBytes = kMmaRows * 64;        // 8 KB per block of a tile
 constexpr int kMmaAStageBytes = kMmaWb * kMmaATileBytes;  // 16 KB per tile
 constexpr int kMmaBBytes = 32 * 64;                  // one 32x32 bf16 matrix
-// Error allowance of the tensor-core sum, relative to sum_i |x_i| * max|K|.
-// Model: each kind::f16 UMMA adds its 16 exact bf16 x bf16 products to the fp32
-// accumulator with an error of at most about 2u of the magnitudes involved
-// (u = 2^-24; measured on B200 at most 11u in total for the six UMMAs of the
-// fp32 three-part mode and 5.3u for the two of the bf16 mode, over 8 M
-// elements including blocks spanning 2^40 in magnitude).  With the final fp32
-// rounding of the definition this gives 13u and 5u; the allowances below keep a
-// margin of 2.5x or more.
-constexpr float kMmaErrC_F32 = 1.9073486328125e-06f;  // 2^-19 = 32u
-constexpr float kMmaErrC_BF16 = 9.5367431640625e-07f; // 2^-20 = 16u
-constexpr float kMmaErrAbs = 7.703719777548943e-34f;  // 2^-110: flushed subnormal partial sums
+// Error allowance of the tensor-core sum, derived (not measured):
+//   E = (C max|K| + kMmaErrL1) ||x||_1 + kMmaErrAbsK max|K| + kMmaErrAbs  >=  |y_fast - fp32(x K)|.
+// Model: one kind::f16 UMMA (K = 16) forms d + sum of 16 products; every bf16 x bf16
+// product is exact in fp32, and the 16 additions may run in any order, each rounded
+// or truncated to at least 24 significant bits (relative error below 2u, u = 2^-24).
+// Then |error| <= g (|d| + sum |p|) with g = 16 (2u) / (1 - 32u).  A block chains J
+// UMMAs from d = 0 (J = 2 for bf16 K; J = 6 for fp32 K split exactly into three bf16
+// parts, whose magnitudes add up to at most (1 + 2^-6) |K|), so the chain's error is
+// at most J g (1 + g)^J sum_i |x_i| |K_ij|, and the definition's own rounding of y
+// adds u |y|.  With sum_i |x_i||K_ij| <= ||x||_1 max|K|:
+//   bf16 K: 2 g (1 + g)^2 + u < 65.1u  -> C = 66u
+//   fp32 K: 6 g (1 + g)^6 (1 + 2^-6) + u < 196.1u -> C = 198u.
+// Absolute terms for a tensor core that flushes fp32 subnormals: flushed K parts lose
+// at most 3 x 2^-126 per unit of ||x||_1 (kMmaErrL1 = 2^-124); flushed subnormal
+// inputs at most 32 x 2^-126 x (1 + 2^-6) max|K| (kMmaErrAbsK = 2^-120); flushed
+// subnormal products and partial sums at most 2 x 96 x 2^-126 (kMmaErrAbs = 2^-118).
+// A fast result that overflowed is non-finite and always takes the exact path.
+// (Measured on B200 the worst error was 11u and 5.3u: the bound holds with room.)
+constexpr float kMmaErrC_F32 = 1.1801719665527344e-05f;  // 198u
+constexpr float kMmaErrC_BF16 = 3.933906555175781e-06f;  // 66u
+constexpr float kMmaErrL1 = 4.701977403289208e-38f;      // 2^-124
+constexpr float kMmaErrAbsK = 7.52316384526264e-37f;     // 2^-120
+constexpr float kMmaErrAbs = 3.009265538105056e-36f;     // 2^-118
 
 // UMMA instruction descriptor, kind::f16: D fp32, A and B bf16, A K-major,
 // B N-major, N = 32, M = 128.
@@ -134,7 +146,7 @@ __device__ __forceinline__ uint32_t sw64_offset(int row, int col) {
 // rounding to nearest: relative error at most 2^-8 per level, four levels plus
 // one upward fp32 addition), then scaled up by 1 + 2^-5 > 1 / (1 - 2^-8)^4.
 // Sums that land in the subnormal range may lose up to 2^-126 per addition;
-// the absolute allowance kMmaErrAbs covers that.
+// the absolute allowance kMmaErrAbsK max|K| covers that (C max|K| 2^-122 is far smaller).
 __device__ __forceinline__ float l1_upper_bf16(const uint4 (&v)[4]) {
   uint32_t w[16];
 #pragma unroll
@@ -318,7 +330,9 @@ __global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(c
     const int b = group * kMmaWb + bw;
     const bool col_ok = b < p.nb;
     const int bc = col_ok ? b : 0;
-    const float cfac = __fmul_ru(KSRC == KSRC_BF16 ? kMmaErrC_BF16 : kMmaErrC_F32, __uint_as_float(kmax_bits[bw]));
+    const float kmax = __uint_as_float(kmax_bits[bw]);
+    const float cfac = __fmaf_ru(KSRC == KSRC_BF16 ? kMmaErrC_BF16 : kMmaErrC_F32, kmax, kMmaErrL1);
+    const float eabs = __fmaf_ru(kMmaErrAbsK, kmax, kMmaErrAbs);
     const void* Kb = (KSRC == KSRC_BF16)
                          ? static_cast<const void*>(static_cast<const uint16_t*>(p.mats) + int64_t(bc) * 1024)
                          : static_cast<const void*>(static_cast<const float*>(p.mats) + int64_t(bc) * 1024);
@@ -359,7 +373,7 @@ __global__ void __launch_bounds__(kMmaThreads, kMmaCtasPerSm) quant_mma_kernel(c
       uint8_t* qb = p.q + rowc * int64_t(p.nb) * 16 + int64_t(bc) * 16;
       uint8_t* sb = p.scales + scale_index(rowc, bc, p.nb, TILED);
       const uint16_t* xb = p.x + rowc * p.ldx + int64_t(bc) * kBlock;
-      const bool need = certify_store(Y, amax, l1, zero_block, cfac, kMmaErrAbs, !(cfac <= FLT_MAX), act, qb, sb);
+      const bool need = certify_store(Y, amax, l1, zero_block, cfac, eabs, !(cfac <= FLT_MAX), act, qb, sb);
       if (__any_sync(0xFFFFFFFFu, need)) warp_exact_pass<KSRC>(need, xb, Kb, qb, sb);
     }
   }

@@ -154,3 +154,21 @@ def test_bound_check_detects_a_wrong_bound(orc, bad_constant):
     params = inputs.lu_params(d // 32, seed=[d, 7])
     y32 = orc.transform(x, orc.expand(params))
     assert worst_error_in_u(orc, x, params, order=[4, 3, 2, 1, 0], y32=y32) > bad_constant
+
+
+def test_exact_path_rate_estimate_orders_the_allowances(orc):
+    """The host estimate of the exact-path share (tests/exact_path_rate.py) on 256 rows
+    of the FLUX d=3072 input: wider allowances send more blocks to the exact path, the
+    derived tensor-core allowances stay below a few per cent, and the butterfly's
+    stays near the 0.15 % measured on the device."""
+    from . import exact_path_rate as epr
+
+    x, params = inputs.config_case("flux", 3072)
+    x = x[:256]
+    k32 = orc.expand(params, dtype=orc.F32)
+    k16 = orc.expand(params, dtype=orc.BF16)
+    r = {name: epr.rate(orc, x, k16 if dt == "bf16" else k32, c, e1, ek, e0)
+         for name, (dt, c, e1, ek, e0) in epr.ALLOWANCES.items()}
+    assert r["tensor_core_bf16_K_calibrated_16u"] <= r["tensor_core_bf16_K"] < 0.02
+    assert r["tensor_core_fp32_K_calibrated_32u"] <= r["tensor_core_fp32_K"] < 0.05
+    assert 0.0005 < r["butterfly"] < 0.005
