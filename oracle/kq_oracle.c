@@ -392,3 +392,58 @@ void kqo_mx_gemm(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, const u
       c[m * N + n] = acc;
     }
 }
+
+/* ---- the producer: AdaLN normalisation fused in front of the quantizer ------------ */
+
+/* Pairwise sum in fp64: a[0..n) padded with +0 to a power of two, then neighbours
+ * added level by level.  tmp holds at least that power of two. */
+static double pairwise_sum(const double* a, int64_t n, double* tmp) {
+  int64_t p = 1;
+  while (p < n) p *= 2;
+  for (int64_t i = 0; i < p; i++) tmp[i] = (i < n) ? a[i] : 0.0;
+  for (int64_t w = p; w > 1; w /= 2)
+    for (int64_t j = 0; j < w / 2; j++) tmp[j] = tmp[2 * j] + tmp[2 * j + 1];
+  return tmp[0];
+}
+
+/* [KQ §Problem], [KQ abstract]: the modulated LayerNorm whose output the quantizer
+ * receives, in the step order stated in the header. */
+void kqo_adaln(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const uint16_t* shift,
+               const uint16_t* scale, int64_t rows_per_group, double eps, uint16_t* h, double* stats) {
+  int64_t p = 1;
+  while (p < d) p *= 2;
+  double* v = (double*)malloc(sizeof(double) * (size_t)(d > 0 ? d : 1));
+  double* tmp = (double*)malloc(sizeof(double) * (size_t)p);
+  for (int64_t r = 0; r < M; r++) {
+    for (int64_t i = 0; i < d; i++) v[i] = (double)f32_from_bf16(x[r * ldx + i]);
+    const double mu = pairwise_sum(v, d, tmp) / (double)d;
+    for (int64_t i = 0; i < d; i++) {
+      const double t = v[i] - mu;
+      v[i] = t * t;
+    }
+    const double var = pairwise_sum(v, d, tmp) / (double)d;
+    const double rstd = 1.0 / sqrt(var + eps);
+    const int64_t g = r / rows_per_group;
+    for (int64_t i = 0; i < d; i++) {
+      const double t = (double)f32_from_bf16(x[r * ldx + i]) - mu;
+      const double a = 1.0 + (double)f32_from_bf16(scale[g * d + i]);
+      const double b = (double)f32_from_bf16(shift[g * d + i]);
+      h[r * d + i] = kqo_bf16_from_f64((t * rstd) * a + b);
+    }
+    if (stats != NULL) {
+      stats[2 * r] = mu;
+      stats[2 * r + 1] = rstd;
+    }
+  }
+  free(v);
+  free(tmp);
+}
+
+void kqo_adaln_quantize(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const uint16_t* shift,
+                        const uint16_t* scale, int64_t rows_per_group, double eps, const void* mats,
+                        int dtype, uint8_t* q, uint8_t* scales, double* stats) {
+  uint16_t* h = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(M * d > 0 ? M * d : 1));
+  kqo_adaln(x, M, d, ldx, shift, scale, rows_per_group, eps, h, stats);
+  kqo_quantize(h, M, d, d, mats, dtype, q, scales);
+  free(h);
+}

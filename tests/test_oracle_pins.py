@@ -606,3 +606,93 @@ def test_mx_gemm_nan_scale_poisons_its_row_and_column(orc):
     c = orc.mx_gemm(aq, sa, bq, sb)
     assert np.isnan(c[0]).all() and np.isnan(c[:, 2]).all()
     assert np.isfinite(c[1:, :2]).all()
+
+
+# ---------------------------------------------------------------- AdaLN normalisation (the quantizer's producer)
+
+def _nearest_bf16_ok(h_bits: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    """True where the bf16 value h is a nearest bf16 value to the fp64 reference (both
+    neighbours accepted within 1e-9 of a midpoint, where fp64 evaluations that differ in
+    the last bits may round either way)."""
+    h = inputs.bf16_bits_to_f32(h_bits).astype(np.float64)
+    err = np.abs(h - ref)
+    # spacing of bf16 values at |ref|: 2^(floor(log2|ref|) - 7), at least 2^-133
+    mag = np.maximum(np.abs(ref), 2.0**-126)
+    ulp = np.exp2(np.floor(np.log2(mag)) - 7)
+    return (err <= 0.5 * ulp * (1 + 1e-9)) | ~np.isfinite(ref)
+
+
+def test_adaln_matches_torch_fp64_layer_norm(orc):
+    """The oracle's modulated LayerNorm against torch's fp64 layer_norm (a library
+    routine with its own reduction order): the statistics agree to fp64 rounding, and
+    every bf16 output is a nearest bf16 value to torch's fp64 result.  Rows with
+    outliers of 2^12, two samples' modulation vectors, ragged d."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(81)
+    for d, rpg in ((96, 3), (1152, 5), (3104, 4)):
+        M = 8
+        a = rng.standard_normal((M, d)).astype(np.float32)
+        a[:, rng.choice(d, 3, replace=False)] *= 4096.0
+        a[2] += 1000.0                                  # a large mean
+        x = inputs.f32_to_bf16_bits(a)
+        G = -(-M // rpg)
+        shift = inputs.f32_to_bf16_bits(rng.standard_normal((G, d)).astype(np.float32))
+        scale = inputs.f32_to_bf16_bits((0.3 * rng.standard_normal((G, d))).astype(np.float32))
+        eps = 1e-6
+        h, stats = orc.adaln(x, shift, scale, rpg, eps)
+        xt = torch.from_numpy(inputs.bf16_bits_to_f32(x).astype(np.float64))
+        ln = torch.nn.functional.layer_norm(xt, (d,), eps=eps)
+        g = np.arange(M) // rpg
+        sc = torch.from_numpy(inputs.bf16_bits_to_f32(scale).astype(np.float64))[g]
+        sh = torch.from_numpy(inputs.bf16_bits_to_f32(shift).astype(np.float64))[g]
+        ref = (ln * (1 + sc) + sh).numpy()
+        assert _nearest_bf16_ok(h, ref).all(), d
+        mu = xt.mean(dim=1).numpy()
+        var = xt.var(dim=1, unbiased=False).numpy()
+        assert np.allclose(stats[:, 0], mu, rtol=1e-13, atol=1e-13 * np.abs(xt.numpy()).max())
+        assert np.allclose(stats[:, 1], 1 / np.sqrt(var + eps), rtol=1e-12)
+
+
+def test_adaln_constant_row_is_the_shift(orc):
+    """A constant row has mean equal to the constant and variance 0, so its normalised
+    values are 0 and the output is the shift vector exactly (any d, any eps > 0)."""
+    d = 160
+    x = np.full((3, d), 0x4049, np.uint16)               # 3.140625
+    x[1] = 0xC2C8                                          # -100
+    rng = np.random.default_rng(82)
+    shift = inputs.f32_to_bf16_bits(rng.standard_normal((1, d)).astype(np.float32))
+    scale = inputs.f32_to_bf16_bits(rng.standard_normal((1, d)).astype(np.float32))
+    h, stats = orc.adaln(x, shift, scale, 3, 1e-5)
+    assert np.array_equal(inputs.bf16_bits_to_f32(h), np.repeat(inputs.bf16_bits_to_f32(shift), 3, axis=0))
+    assert stats[0, 0] == 3.140625 and stats[1, 0] == -100.0
+    assert stats[0, 1] == 1 / np.sqrt(1e-5)
+
+
+def test_adaln_group_of_each_row(orc):
+    """Rows take the modulation vectors of group row // rows_per_group: constant rows
+    with group g's shift equal to g give h = g."""
+    d, M, rpg = 64, 11, 4
+    x = np.full((M, d), 0x3F80, np.uint16)                # 1.0
+    shift = inputs.f32_to_bf16_bits(np.repeat(np.arange(3, dtype=np.float32)[:, None] + 10, d, axis=1))
+    scale = np.zeros((3, d), np.uint16)
+    h, _ = orc.adaln(x, shift, scale, rpg, 1e-6)
+    assert np.array_equal(inputs.bf16_bits_to_f32(h)[:, 0], 10.0 + np.arange(M) // rpg)
+
+
+def test_adaln_symmetric_row_closed_form(orc):
+    """x = (+a, -a, +a, ...): mean 0 and variance a^2 exactly, so h_i = +-a (1 + s_i) /
+    sqrt(a^2 + eps) + b_i, checked against exact rational arithmetic (the nearest bf16
+    value of the real result, away from midpoints)."""
+    d, a = 256, 3.5
+    x = np.where(np.arange(d) % 2 == 0, 0x4060, 0xC060).astype(np.uint16)[None, :]  # +-3.5
+    rng = np.random.default_rng(83)
+    shift = inputs.f32_to_bf16_bits(rng.standard_normal((1, d)).astype(np.float32))
+    scale = inputs.f32_to_bf16_bits((0.5 * rng.standard_normal((1, d))).astype(np.float32))
+    eps = 2.0**-20
+    h, stats = orc.adaln(x, shift, scale, 1, eps)
+    assert stats[0, 0] == 0.0
+    rstd = 1.0 / math.sqrt(a * a + eps)
+    sgn = np.where(np.arange(d) % 2 == 0, 1.0, -1.0)
+    ref = sgn * a * rstd * (1 + inputs.bf16_bits_to_f32(scale)[0].astype(np.float64)) + \
+        inputs.bf16_bits_to_f32(shift)[0].astype(np.float64)
+    assert _nearest_bf16_ok(h[0], ref).all()
