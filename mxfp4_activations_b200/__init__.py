@@ -10,6 +10,7 @@ thin ctypes binding plus seeded input generators (``inputs``).
 """
 from ._lib import (  # noqa: F401
     EXPORTED,
+    kq_adaln_quantize,
     SCALE_LAYOUTS,
     KQError,
     kq_abi_version,
@@ -64,6 +65,15 @@ class BlockTransform:
         if getattr(self, "_inv_t", None) is None or self._inv_t.dtype != key:
             self._inv_t = kq_expand_blocks(self.params, inverse=True, transpose=True, dtype=key)
         return kq_quantize(w, self._inv_t, None, variant="mma", q=q, scales=scales, scale_layout=scale_layout)
+
+    def adaln_quantize(self, x, shift, scale, rows_per_group: int, eps: float = 1e-6, q=None, scales=None,
+                       scale_layout: str = "row", stats=None):
+        """The DiT block's modulated LayerNorm fused in front of the quantizer: MXFP4 of
+        bf16(LN(x) (1 + scale[g]) + shift[g]) K_b, g = row // rows_per_group."""
+        if self.mats.shape[-1] != 32:
+            raise NotImplementedError("the fused AdaLN quantizer is provided for 32-element transform blocks")
+        return kq_adaln_quantize(x, shift, scale, rows_per_group, self.mats, self.factored, eps=eps, q=q,
+                                 scales=scales, scale_layout=scale_layout, stats=stats)
 
     def dequantize(self, q, scales, undo_transform: bool = True, out_dtype=None):
         import torch

@@ -34,7 +34,7 @@ EXPORTED = (
     "kq_expand_blocks", "kq_expand_factored", "kq_quantize", "kq_dequantize", "kq_ref_smooth_quantize",
     "kq_expand_blocks_n", "kq_expand_factored_n", "kq_quantize_n",
     "kq_ref_fwht_quantize", "kq_e2m1_pack", "kq_get_device_error", "kq_status_string", "kq_abi_version",
-    "kq_last_error", "kq_select_variant", "kq_gemm_mxf4", "kq_select_gemm_kernel",
+    "kq_last_error", "kq_select_variant", "kq_gemm_mxf4", "kq_select_gemm_kernel", "kq_adaln_quantize",
 )
 
 
@@ -77,6 +77,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kq_select_variant": [I64, I64, I, I, I, P],
         "kq_gemm_mxf4": [P, P, I64, P, P, I64, I64, P, I64, I, P],
         "kq_select_gemm_kernel": [I64, I64, I64, P],
+        "kq_adaln_quantize": [P, I64, I64, I64, P, P, I64, ctypes.c_double, P, P, P, P, I, P, P],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -252,6 +253,35 @@ def kq_quantize(x: torch.Tensor, mats: torch.Tensor, factored: torch.Tensor | No
                                                      VARIANTS[variant], SCALE_LAYOUTS[scale_layout],
                                                      _stream(x.device)))
     return q, scales
+
+
+def kq_adaln_quantize(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor, rows_per_group: int,
+                      mats: torch.Tensor, factored: torch.Tensor, eps: float = 1e-6, q: torch.Tensor | None = None,
+                      scales: torch.Tensor | None = None, scale_layout: str = "row", stats: torch.Tensor | None = None):
+    """The quantizer fused with the AdaLN-modulated LayerNorm in front of it:
+    h = bf16(LN(x) (1 + scale[g]) + shift[g]) with g = row // rows_per_group, then MXFP4
+    of h K per 32-element block (butterfly variant) -> (codes, scales, stats), stats the
+    fp64 (mean, 1/sqrt(var + eps)) of each row when a [M, 2] float64 tensor is given."""
+    M, d, ldx = _rows(x)
+    G = -(-M // max(1, int(rows_per_group)))
+    for name, t in (("shift", shift), ("scale", scale)):
+        _cuda(t, name, x.device, _BF16_LIKE, contiguous=True)
+        if t.dim() != 2 or t.shape[1] != d or t.shape[0] < G:
+            raise ValueError(f"{name} must be [ceil(M / rows_per_group), d] = [{G}, {d}]")
+    n = _mats(mats, d, x.device)
+    if n != 32 or mats.dtype != torch.float32:
+        raise ValueError("the fused AdaLN quantizer takes fp32 matrices of 32-element blocks")
+    _cuda(factored, "factored", x.device, (torch.float32,), contiguous=True, min_numel=(d // 32) * factored_floats(5))
+    q, scales = _outputs(x, M, d, q, scales, scale_layout)
+    if stats is not None:
+        _cuda(stats, "stats", x.device, (torch.float64,), contiguous=True, min_numel=2 * M)
+    with torch.cuda.device(x.device):
+        _check("kq_adaln_quantize", load().kq_adaln_quantize(_ptr(x), M, d, ldx, _ptr(shift), _ptr(scale),
+                                                             int(rows_per_group), float(eps), _ptr(mats),
+                                                             _ptr(factored), _ptr(q), _ptr(scales),
+                                                             SCALE_LAYOUTS[scale_layout], _ptr(stats),
+                                                             _stream(x.device)))
+    return q, scales, stats
 
 
 def kq_dequantize(q: torch.Tensor, scales: torch.Tensor, inv_mats: torch.Tensor | None = None,

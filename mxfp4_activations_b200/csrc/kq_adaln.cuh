@@ -1,0 +1,230 @@
+// kq_adaln.cuh -- the KroQuant quantizer fused with the AdaLN-modulated LayerNorm that
+// produces its input in a DiT block ("KroQuant: Kronecker-Structured Block Transforms
+// ...", Problem: AdaLN blocks keep the transform from being absorbed offline; the
+// KroQuant abstract: normalisation layers between blocks force it to run online).
+//
+// Per row of x (bf16, d = 32 nb):
+//   S1 = pairwise sum of the d inputs in fp64 (padded with +0 to a power of two,
+//        neighbours added level by level), mu = S1 / d
+//   S2 = pairwise sum of (x_i - mu)^2, var = S2 / d, rstd = 1 / sqrt(var + eps)
+//   h_i = bf16( ((x_i - mu) * rstd) * (1 + scale[g][i]) + shift[g][i] ),  g = row / rows_per_group
+// every step one IEEE fp64 operation rounded to nearest even (no contraction), so the
+// statistics and h are the definition's bit for bit; then y = h K_b and the certified
+// MXFP4 step of the butterfly quantizer (kq_quant.cuh) on h, which never leaves the chip.
+//
+// Work mapping.  A CTA takes R rows per step, each on a slot of nbw = nb rounded up to a
+// multiple of 32 threads: thread t takes block column c = t % nbw of slot t / nbw (columns
+// >= nb are padding and contribute +0), so a thread keeps one block column for its life,
+// with the column's butterfly coefficients in registers, and every warp lies in one row.
+// Each thread streams its blocks of the coming steps through a private ring of
+// kAlStages 64-byte shared-memory slots (cp.async), as the butterfly kernel does.
+//
+// The pairwise tree of a row is aligned to its blocks: the first five levels sum each
+// block in registers, the next five pair the block sums of a warp by shfl_xor (fp64
+// addition is commutative, so both partners form the same sum), and the rest pair the
+// warp sums, which every warp of the slot reads from shared memory after one barrier.
+// h of each block is staged in shared memory for the warp-cooperative exact path.
+#pragma once
+
+#include "kq_quant.cuh"
+
+namespace kq {
+
+constexpr int kAlMaxThreads = 512;
+constexpr int kAlStages = 3;  // ring slots per thread (blocks of two coming steps in flight)
+
+struct AdaLnParams {
+  const uint16_t* x;      // bf16 bits [M][ldx]
+  int64_t ldx;
+  int64_t M;
+  int nb;                 // d / 32
+  int nbw;                // nb rounded up to a multiple of 32: threads per row slot
+  int tree_pad;           // smallest power of two >= nb (the row tree's width in blocks)
+  int rows;               // R: row slots per CTA
+  const uint16_t* shift;  // bf16 bits [G][nb * 32]
+  const uint16_t* scale;  // bf16 bits [G][nb * 32]
+  int64_t rows_per_group;
+  double eps;
+  const float* mats;      // fp32 [nb][32][32] (exact path)
+  const float* factored;  // [nb][48]
+  uint8_t* q;             // [M][nb * 16]
+  uint8_t* scales;        // row-major [M][nb], or tiled (scale_index)
+  double* stats;          // [M][2] (mu, rstd) or null
+};
+
+// bf16 nearest-even rounding of an fp64 value: round to odd in fp32 (truncate, then set
+// the last bit if anything was dropped), then nearest-even to bf16.  fp32 keeps at least
+// two more bits than bf16 in every binade bf16 has (16 more), so the first rounding
+// cannot change the result of the second.  NaN stays NaN, overflow becomes infinity.
+__device__ __forceinline__ uint32_t bf16_bits_of_f64(double v) {
+  float f = __double2float_rz(v);
+  if (double(f) != v && !isnan(v)) f = __uint_as_float(__float_as_uint(f) | 1u);
+  uint16_t h;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(f));
+  return h;
+}
+
+// Pairwise fp64 sum of the 32 values of one block (bf16 pairs w) after `f`.
+template <class F>
+__device__ __forceinline__ double block_pairwise(const uint32_t (&w)[16], F f) {
+  double a[16];
+#pragma unroll
+  for (int j = 0; j < 16; j++) a[j] = __dadd_rn(f(double(bf16lo(w[j]))), f(double(bf16hi(w[j]))));
+#pragma unroll
+  for (int n = 8; n >= 1; n >>= 1)
+#pragma unroll
+    for (int j = 0; j < n; j++) a[j] = __dadd_rn(a[2 * j], a[2 * j + 1]);
+  return a[0];
+}
+
+// The rest of a row's pairwise tree above the block sums v (+0 for padding columns):
+// pairs within the warp by shfl_xor (levels 6..10 of the row tree, at most log2 of the
+// tree's width), then, for rows wider than a warp, pairs of the warp sums that the slot's
+// warps leave in ws (padded with +0 to the tree's width / 32).  One barrier; every thread
+// of the slot returns the row sum.  ws must not be written again before every thread of
+// the CTA has passed the next barrier.
+__device__ __forceinline__ double row_sum(double v, int c, int nbw, int tree_pad, double* ws) {
+  const int wl = tree_pad >= 32 ? 5 : __ffs(tree_pad) - 1;
+#pragma unroll 1
+  for (int l = 0; l < wl; l++) v = __dadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, 1 << l));
+  if (tree_pad <= 32) {
+    __syncthreads();  // keeps the barrier count of every row the same
+    return __shfl_sync(0xFFFFFFFFu, v, 0);
+  }
+  const int nw = tree_pad >> 5, lane = c & 31;
+  if (lane == 0) ws[c >> 5] = v;
+  if (lane == 0 && c == 0)
+    for (int j = nbw >> 5; j < nw; j++) ws[j] = 0.0;
+  __syncthreads();
+  double u = lane < nw ? ws[lane] : 0.0;
+#pragma unroll 1
+  for (int o = 1; o < nw; o <<= 1) u = __dadd_rn(u, __shfl_xor_sync(0xFFFFFFFFu, u, o));
+  return __shfl_sync(0xFFFFFFFFu, u, 0);
+}
+
+template <int TILED>
+__global__ void __launch_bounds__(kAlMaxThreads, 1) adaln_quant_kernel(const __grid_constant__ AdaLnParams p) {
+  extern __shared__ __align__(128) uint8_t al_smem[];
+  const int R = p.rows;
+  const int nws = p.tree_pad > 32 ? (p.tree_pad >> 5) : 1;  // warp sums per row tree
+  uint8_t* ring = al_smem;                                      // [kAlStages][blockDim][64]
+  uint16_t* hx = reinterpret_cast<uint16_t*>(al_smem + size_t(kAlStages) * blockDim.x * 64);  // [blockDim][32]
+  double* ws = reinterpret_cast<double*>(al_smem + size_t(kAlStages + 1) * blockDim.x * 64);   // [2][R][nws]
+  const int t = threadIdx.x;
+  const int rho = t / p.nbw, c = t % p.nbw;
+  const bool col = c < p.nb;
+  const int cc = col ? c : 0;
+  double* ws1 = ws + size_t(rho) * nws;
+  double* ws2 = ws + size_t(R + rho) * nws;
+  const double d = double(p.nb) * kBlock;
+  uint16_t* hmine = hx + size_t(t) * kBlock;
+  const int sw = (t >> 1) & 3;
+  const uint32_t cbase = smem_addr(ring) + uint32_t(t) * 64u;
+  const uint32_t kStage = blockDim.x * 64u;
+
+  QuantParams qp = {};
+  qp.nb = p.nb;
+  qp.factored = p.factored;
+  qp.mats = p.mats;
+  grid_dependency_wait();  // inputs may come from the previous kernel in the stream
+
+  const int64_t step_rows = int64_t(gridDim.x) * R;
+  const int64_t r_first = int64_t(blockIdx.x) * R + rho;
+  const int64_t n_steps = (p.M - int64_t(blockIdx.x) * R + step_rows - 1) / step_rows;  // CTA-uniform
+  // the first kAlStages - 1 steps' blocks go in flight before anything else
+#pragma unroll
+  for (int s = 0; s < kAlStages - 1; s++) {
+    const int64_t r = r_first + s * step_rows;
+    if (col && r < p.M) copy_block_async(cbase + s * kStage, sw, p.x + r * p.ldx + int64_t(c) * kBlock);
+    copy_commit();
+  }
+  grid_launch_dependents();
+  ColCoef cf;
+  load_coef<MODE_KRON, 32>(qp, cc, cf);
+
+#pragma unroll 1
+  for (int64_t i = 0; i < n_steps; i++) {
+    const int64_t r = r_first + i * step_rows;
+    const bool act = col && r < p.M;
+    // refill the slot read one step ago with the block kAlStages - 1 steps ahead
+    {
+      const int64_t ra = r + (kAlStages - 1) * step_rows;
+      const uint32_t slot = uint32_t((i + kAlStages - 1) % kAlStages) * kStage;
+      if (col && ra < p.M) copy_block_async(cbase + slot, sw, p.x + ra * p.ldx + int64_t(c) * kBlock);
+      copy_commit();
+    }
+    copy_wait<kAlStages - 1>();  // this step's block has landed
+    uint32_t w[16];
+    read_slot(cbase + uint32_t(i % kAlStages) * kStage, sw, w);
+    if (!act) {
+#pragma unroll
+      for (int k = 0; k < 16; k++) w[k] = 0u;
+    }
+    // the modulation vectors of this row's group, in flight while the statistics run
+    const int64_t g = act ? r / p.rows_per_group : 0;
+    uint4 sv[4], hv[4];
+    {
+      const uint4* ps = reinterpret_cast<const uint4*>(p.scale + g * (int64_t(p.nb) * kBlock) + int64_t(cc) * kBlock);
+      const uint4* ph = reinterpret_cast<const uint4*>(p.shift + g * (int64_t(p.nb) * kBlock) + int64_t(cc) * kBlock);
+#pragma unroll
+      for (int k = 0; k < 4; k++) {
+        sv[k] = act ? __ldg(ps + k) : make_uint4(0u, 0u, 0u, 0u);
+        hv[k] = act ? __ldg(ph + k) : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    // statistics
+    // (padding columns and rows past M contribute +0)
+    const double b1 = act ? block_pairwise(w, [](double x) { return x; }) : 0.0;
+    const double s1 = row_sum(b1, c, p.nbw, p.tree_pad, ws1);
+    const double mu = __ddiv_rn(s1, d);
+    const double b2 = act ? block_pairwise(w,
+                                           [mu](double x) {
+                                             const double u = __dsub_rn(x, mu);
+                                             return __dmul_rn(u, u);
+                                           })
+                          : 0.0;
+    const double s2 = row_sum(b2, c, p.nbw, p.tree_pad, ws2);
+    const double var = __ddiv_rn(s2, d);
+    const double rstd = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(var, p.eps)));
+    if (act && c == 0 && p.stats != nullptr) {
+      p.stats[2 * r] = mu;
+      p.stats[2 * r + 1] = rstd;
+    }
+    // modulation, one bf16 rounding per element
+    uint32_t hw[16];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      const uint32_t s4[4] = {sv[k].x, sv[k].y, sv[k].z, sv[k].w}, b4[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
+#pragma unroll
+      for (int m = 0; m < 4; m++) {
+        uint32_t out = 0u;
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+          const uint32_t xw = w[4 * k + m];
+          const double xv = double(e ? bf16hi(xw) : bf16lo(xw));
+          const double a = __dadd_rn(1.0, double(e ? bf16hi(s4[m]) : bf16lo(s4[m])));
+          const double bv = double(e ? bf16hi(b4[m]) : bf16lo(b4[m]));
+          const double h64 = __dadd_rn(__dmul_rn(__dmul_rn(__dsub_rn(xv, mu), rstd), a), bv);
+          out |= bf16_bits_of_f64(h64) << (16 * e);
+        }
+        hw[4 * k + m] = out;
+      }
+    }
+    reinterpret_cast<uint4*>(hmine)[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    reinterpret_cast<uint4*>(hmine)[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+    reinterpret_cast<uint4*>(hmine)[2] = make_uint4(hw[8], hw[9], hw[10], hw[11]);
+    reinterpret_cast<uint4*>(hmine)[3] = make_uint4(hw[12], hw[13], hw[14], hw[15]);
+    // transform and certified MXFP4 on h
+    const int64_t rr = act ? r : 0;
+    uint8_t* qb = p.q + (rr * p.nb + cc) * 16;
+    uint8_t* sb = p.scales + scale_index(rr, cc, p.nb, TILED);
+    const bool need = quant_block<MODE_KRON, 32>(cf, hw, act, qb, sb);
+    if (__any_sync(0xFFFFFFFFu, need)) {
+      __syncwarp();  // every lane's staged h is visible to the warp
+      warp_exact_pass<KSRC_F32, 32, false>(need, hmine, p.mats + kmat_offset<32>(cc), qb, sb);
+    }
+  }
+  copy_wait<0>();  // no copy still writes the ring
+}
+
+}  // namespace kq

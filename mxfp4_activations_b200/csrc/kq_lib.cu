@@ -17,6 +17,7 @@
 
 #include "kq.h"
 #include "kq_common.cuh"
+#include "kq_adaln.cuh"
 #include "kq_expand.cuh"
 #include "kq_gemm.cuh"
 #include "kq_misc.cuh"
@@ -527,7 +528,7 @@ kq_variant resolve_variant(int64_t M, int64_t d, kq_dtype mat_dtype, bool has_fa
 
 extern "C" {
 
-int kq_abi_version(void) { return 202; }
+int kq_abi_version(void) { return 203; }
 
 const char* kq_status_string(kq_status s) {
   switch (s) {
@@ -699,6 +700,67 @@ kq_status kq_gemm_mxf4(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, c
                                  as_cuda(stream));
   }
   return launch_gemm(a_q, a_scales, M, b_q, b_scales, N, K, c, ldc, c_dtype == KQ_BF16, as_cuda(stream));
+}
+
+kq_status kq_adaln_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const void* shift, const void* scale,
+                            int64_t rows_per_group, double eps, const float* mats, const float* factored, uint8_t* q,
+                            uint8_t* scales, kq_scale_layout scale_layout, double* stats, kq_stream_t stream) {
+  if (scale_layout != KQ_SCALES_ROW_MAJOR && scale_layout != KQ_SCALES_MMA_TILED) return KQ_ERR_INVALID_ARG;
+  if (rows_per_group < 1) return KQ_ERR_INVALID_ARG;
+  kq_status st = check_x(x, M, d, ldx);
+  if (st != KQ_OK) return st;
+  if (M == 0 || d == 0) return KQ_OK;
+  const int64_t nb = d / 32;
+  if (nb > kq::kAlMaxThreads) return KQ_ERR_UNSUPPORTED;
+  st = check_out(q, scales);
+  if (st != KQ_OK) return st;
+  if (shift == nullptr || scale == nullptr || mats == nullptr || factored == nullptr) return KQ_ERR_INVALID_ARG;
+  if (!aligned(shift, 16) || !aligned(scale, 16) || !aligned(mats, 16) || !aligned(factored, 16) ||
+      (stats != nullptr && !aligned(stats, 8)))
+    return KQ_ERR_ALIGN;
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr) return cuda_fail("device query", cudaErrorInvalidDevice);
+  kq::AdaLnParams p;
+  p.x = static_cast<const uint16_t*>(x);
+  p.ldx = ldx;
+  p.M = M;
+  p.nb = int(nb);
+  p.nbw = (p.nb + 31) / 32 * 32;
+  p.tree_pad = 1;
+  while (p.tree_pad < p.nb) p.tree_pad *= 2;
+  p.rows = kq::kAlMaxThreads / p.nbw;
+  p.shift = static_cast<const uint16_t*>(shift);
+  p.scale = static_cast<const uint16_t*>(scale);
+  p.rows_per_group = rows_per_group;
+  p.eps = eps;
+  p.mats = mats;
+  p.factored = factored;
+  p.q = q;
+  p.scales = scales;
+  p.stats = stats;
+  const int threads = p.rows * p.nbw;
+  const int nws = p.tree_pad > 32 ? p.tree_pad / 32 : 1;
+  const int smem = (kq::kAlStages + 1) * threads * 64 + 2 * p.rows * nws * 8;
+  const int which = scale_layout == KQ_SCALES_MMA_TILED ? 1 : 0;
+  auto kern = which ? kq::adaln_quant_kernel<1> : kq::adaln_quant_kernel<0>;
+  // the largest configuration: 512 threads, and at most 32 warp sums per buffer
+  constexpr int kMaxSmem = (kq::kAlStages + 1) * kq::kAlMaxThreads * 64 + 2 * 32 * 8;
+  if (smem > kMaxSmem || kMaxSmem > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
+  static std::atomic<int> attr_set[2][kMaxDevices];
+  int devid = 0;
+  cudaGetDevice(&devid);
+  if (!attr_set[which][devid].load()) {
+    const cudaError_t ea = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    if (ea != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", ea);
+    attr_set[which][devid].store(1);
+  }
+  int per_sm = 0;
+  const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+  if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveBlocksPerMultiprocessor", e);
+  if (per_sm < 1) return cuda_fail("occupancy: no resident CTA", cudaErrorInvalidConfiguration);
+  const int64_t groups = (M + p.rows - 1) / p.rows;
+  const int64_t grid = std::min<int64_t>(groups, int64_t(dev->sms) * per_sm);
+  return launch_pdl(kern, dim3(unsigned(grid)), threads, smem, as_cuda(stream), "adaln_quant_kernel launch", p);
 }
 
 kq_status kq_select_gemm_kernel(int64_t M, int64_t N, int64_t K, int* two_sm) {

@@ -78,7 +78,9 @@ __device__ __forceinline__ float k_entry(const void* __restrict__ Kb, int i, int
 // a broadcast load.  The block's scale then comes from the exact maximum and
 // every code from the exact value, and lane `owner` stores them.  Must be called
 // by all 32 lanes with the same arguments (taken from the owner lane).
-template <int KSRC, int NT>
+// XG: x is in global memory (read-only path); otherwise a generic pointer, which may
+// point into shared memory.
+template <int KSRC, int NT, bool XG = true>
 __device__ __forceinline__ void exact_block_warp(const uint16_t* __restrict__ xb, const void* __restrict__ Kb,
                                               uint8_t* __restrict__ qb, uint8_t* __restrict__ sb, int owner) {
   const int lane = threadIdx.x & 31;
@@ -94,7 +96,7 @@ __device__ __forceinline__ void exact_block_warp(const uint16_t* __restrict__ xb
     uint32_t xw[8];
 #pragma unroll
     for (int k = 0; k < 2; k++) {
-      const uint4 v = __ldg(px + k);
+      const uint4 v = XG ? __ldg(px + k) : px[k];
       xw[4 * k] = v.x;
       xw[4 * k + 1] = v.y;
       xw[4 * k + 2] = v.z;
@@ -115,7 +117,7 @@ __device__ __forceinline__ void exact_block_warp(const uint16_t* __restrict__ xb
     uint32_t xw[16];
 #pragma unroll
     for (int k = 0; k < 4; k++) {
-      const uint4 v = __ldg(px + k);
+      const uint4 v = XG ? __ldg(px + k) : px[k];
       xw[4 * k] = v.x;
       xw[4 * k + 1] = v.y;
       xw[4 * k + 2] = v.z;
@@ -155,7 +157,7 @@ __device__ __forceinline__ void exact_block_warp(const uint16_t* __restrict__ xb
 
 // Every lane whose block needs the exact path hands it to the whole warp, one
 // block at a time.  Called by all 32 lanes.
-template <int KSRC, int NT = kBlock>
+template <int KSRC, int NT = kBlock, bool XG = true>
 __device__ __forceinline__ void warp_exact_pass(bool need, const uint16_t* xb, const void* Kb, uint8_t* qb,
                                                 uint8_t* sb) {
   uint32_t pending = __ballot_sync(0xFFFFFFFFu, need);
@@ -168,7 +170,7 @@ __device__ __forceinline__ void warp_exact_pass(bool need, const uint16_t* xb, c
         __shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(Kb), src));
     uint8_t* qs = reinterpret_cast<uint8_t*>(__shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(qb), src));
     uint8_t* ss = reinterpret_cast<uint8_t*>(__shfl_sync(0xFFFFFFFFu, reinterpret_cast<unsigned long long>(sb), src));
-    exact_block_warp<KSRC, NT>(xs, ks, qs, ss, src);
+    exact_block_warp<KSRC, NT, XG>(xs, ks, qs, ss, src);
   }
 }
 
