@@ -294,7 +294,7 @@ class QuantStep:
                                       q.data_ptr(), s.data_ptr(), 1, 0, self.stream)
         elif kind == "kroquant_adaln":
             st = self.lib.kq_adaln_quantize(x.data_ptr(), M, d, d, item["shift"].data_ptr(), item["scale"].data_ptr(),
-                                            (M + 1) // 2, ctypes.c_double(1e-6), item["mats"].data_ptr(),
+                                            (M + 1) // 2, ctypes.c_float(1e-6), item["mats"].data_ptr(),
                                             item["fac"].data_ptr(), q.data_ptr(), s.data_ptr(), 0, None, self.stream)
         elif kind == "smooth":
             st = self.lib.kq_ref_smooth_quantize(x.data_ptr(), M, d, d, item["inv_s"].data_ptr(), q.data_ptr(),

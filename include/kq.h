@@ -222,7 +222,8 @@ KQ_API kq_status kq_dequantize(const uint8_t* q, const uint8_t* scales, int64_t 
  * ([KQ-sum, Problem]: AdaLN blocks keep the transform from being absorbed offline;
  * [KQ-abs]: normalisation layers between blocks force it to run online).  The pages do
  * not define the normalisation; this library takes the DiT block's modulated LayerNorm
- * without a learned affine, every step one IEEE fp64 operation rounded to nearest even:
+ * without a learned affine, in fp32 as DiT models compute it, every step one IEEE binary32
+ * operation rounded to nearest even (sqrt and division correctly rounded):
  *   S1 = pairwise sum of the row's d inputs (padded with +0 to a power of two, then
  *        neighbours added level by level), mu = S1 / d,
  *   S2 = pairwise sum of (x_i - mu)^2, var = S2 / d, rstd = 1 / sqrt(var + eps),
@@ -231,16 +232,16 @@ KQ_API kq_status kq_dequantize(const uint8_t* q, const uint8_t* scales, int64_t 
  *   x             device bf16 [M][ldx], as kq_quantize (16-byte aligned, ldx % 8 == 0).
  *   shift, scale  device bf16 bits [ceil(M / rows_per_group)][d], 16-byte aligned.
  *   rows_per_group  rows that share one pair of modulation vectors (tokens per sample), >= 1.
- *   eps           added to the variance (any double).
+ *   eps           added to the variance (any float).
  *   mats, factored  fp32 [d/32][32][32] and [d/32][48], as kq_quantize's butterfly variant.
  *   q, scales, scale_layout  as kq_quantize.
- *   stats         device fp64 [M][2]: (mu, rstd) of each row, or NULL; 8-byte aligned.
+ *   stats         device fp32 [M][2]: (mu, rstd) of each row, or NULL; 8-byte aligned.
  * d must be a multiple of 32 and at most 16384 (KQ_ERR_UNSUPPORTED above).  Codes, scales
  * and statistics equal the definition bit for bit. */
 KQ_API kq_status kq_adaln_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const void* shift,
-                                   const void* scale, int64_t rows_per_group, double eps, const float* mats,
+                                   const void* scale, int64_t rows_per_group, float eps, const float* mats,
                                    const float* factored, uint8_t* q, uint8_t* scales, kq_scale_layout scale_layout,
-                                   double* stats, kq_stream_t stream);
+                                   float* stats, kq_stream_t stream);
 
 /* ---------------------------------------------------------------- consumer
  *

@@ -77,7 +77,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kq_select_variant": [I64, I64, I, I, I, P],
         "kq_gemm_mxf4": [P, P, I64, P, P, I64, I64, P, I64, I, P],
         "kq_select_gemm_kernel": [I64, I64, I64, P],
-        "kq_adaln_quantize": [P, I64, I64, I64, P, P, I64, ctypes.c_double, P, P, P, P, I, P, P],
+        "kq_adaln_quantize": [P, I64, I64, I64, P, P, I64, ctypes.c_float, P, P, P, P, I, P, P],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -261,7 +261,7 @@ def kq_adaln_quantize(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor,
     """The quantizer fused with the AdaLN-modulated LayerNorm in front of it:
     h = bf16(LN(x) (1 + scale[g]) + shift[g]) with g = row // rows_per_group, then MXFP4
     of h K per 32-element block (butterfly variant) -> (codes, scales, stats), stats the
-    fp64 (mean, 1/sqrt(var + eps)) of each row when a [M, 2] float64 tensor is given."""
+    fp32 (mean, 1/sqrt(var + eps)) of each row when a [M, 2] float32 tensor is given."""
     M, d, ldx = _rows(x)
     G = -(-M // max(1, int(rows_per_group)))
     for name, t in (("shift", shift), ("scale", scale)):
@@ -274,7 +274,7 @@ def kq_adaln_quantize(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor,
     _cuda(factored, "factored", x.device, (torch.float32,), contiguous=True, min_numel=(d // 32) * factored_floats(5))
     q, scales = _outputs(x, M, d, q, scales, scale_layout)
     if stats is not None:
-        _cuda(stats, "stats", x.device, (torch.float64,), contiguous=True, min_numel=2 * M)
+        _cuda(stats, "stats", x.device, (torch.float32,), contiguous=True, min_numel=2 * M)
     with torch.cuda.device(x.device):
         _check("kq_adaln_quantize", load().kq_adaln_quantize(_ptr(x), M, d, ldx, _ptr(shift), _ptr(scale),
                                                              int(rows_per_group), float(eps), _ptr(mats),

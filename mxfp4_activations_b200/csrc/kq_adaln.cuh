@@ -3,14 +3,17 @@
 // ...", Problem: AdaLN blocks keep the transform from being absorbed offline; the
 // KroQuant abstract: normalisation layers between blocks force it to run online).
 //
-// Per row of x (bf16, d = 32 nb):
-//   S1 = pairwise sum of the d inputs in fp64 (padded with +0 to a power of two,
-//        neighbours added level by level), mu = S1 / d
+// Per row of x (bf16, d = 32 nb), in fp32 as DiT models compute their LayerNorm:
+//   S1 = pairwise sum of the d inputs (padded with +0 to a power of two, neighbours
+//        added level by level), mu = S1 / d
 //   S2 = pairwise sum of (x_i - mu)^2, var = S2 / d, rstd = 1 / sqrt(var + eps)
 //   h_i = bf16( ((x_i - mu) * rstd) * (1 + scale[g][i]) + shift[g][i] ),  g = row / rows_per_group
-// every step one IEEE fp64 operation rounded to nearest even (no contraction), so the
-// statistics and h are the definition's bit for bit; then y = h K_b and the certified
-// MXFP4 step of the butterfly quantizer (kq_quant.cuh) on h, which never leaves the chip.
+// every step one IEEE binary32 operation rounded to nearest even (no contraction; sqrt and
+// division correctly rounded), so the statistics and h are the definition's bit for bit;
+// then y = h K_b and the certified MXFP4 step of the butterfly quantizer (kq_quant.cuh)
+// on h, which never leaves the chip.  Every step uses the scalar round-to-nearest
+// intrinsics, which the compiler never contracts: separate packed f32x2 multiplies and
+// adds were measured to be fused into one FMA.
 //
 // Work mapping.  A CTA takes R rows per step, each on a slot of nbw = nb rounded up to a
 // multiple of 32 threads: thread t takes block column c = t % nbw of slot t / nbw (columns
@@ -44,36 +47,24 @@ struct AdaLnParams {
   const uint16_t* shift;  // bf16 bits [G][nb * 32]
   const uint16_t* scale;  // bf16 bits [G][nb * 32]
   int64_t rows_per_group;
-  double eps;
+  float eps;
   const float* mats;      // fp32 [nb][32][32] (exact path)
   const float* factored;  // [nb][48]
   uint8_t* q;             // [M][nb * 16]
   uint8_t* scales;        // row-major [M][nb], or tiled (scale_index)
-  double* stats;          // [M][2] (mu, rstd) or null
+  float* stats;           // [M][2] (mu, rstd) or null
 };
 
-// bf16 nearest-even rounding of an fp64 value: round to odd in fp32 (truncate, then set
-// the last bit if anything was dropped), then nearest-even to bf16.  fp32 keeps at least
-// two more bits than bf16 in every binade bf16 has (16 more), so the first rounding
-// cannot change the result of the second.  NaN stays NaN, overflow becomes infinity.
-__device__ __forceinline__ uint32_t bf16_bits_of_f64(double v) {
-  float f = __double2float_rz(v);
-  if (double(f) != v && !isnan(v)) f = __uint_as_float(__float_as_uint(f) | 1u);
-  uint16_t h;
-  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(f));
-  return h;
-}
-
-// Pairwise fp64 sum of the 32 values of one block (bf16 pairs w) after `f`.
-template <class F>
-__device__ __forceinline__ double block_pairwise(const uint32_t (&w)[16], F f) {
-  double a[16];
+// Pairwise fp32 sum of the 32 values of one block (v_0 .. v_31): neighbours added level
+// by level.
+__device__ __forceinline__ float block_pairwise(const float (&v)[32]) {
+  float a[16];
 #pragma unroll
-  for (int j = 0; j < 16; j++) a[j] = __dadd_rn(f(double(bf16lo(w[j]))), f(double(bf16hi(w[j]))));
+  for (int j = 0; j < 16; j++) a[j] = __fadd_rn(v[2 * j], v[2 * j + 1]);
 #pragma unroll
   for (int n = 8; n >= 1; n >>= 1)
 #pragma unroll
-    for (int j = 0; j < n; j++) a[j] = __dadd_rn(a[2 * j], a[2 * j + 1]);
+    for (int j = 0; j < n; j++) a[j] = __fadd_rn(a[2 * j], a[2 * j + 1]);
   return a[0];
 }
 
@@ -83,10 +74,10 @@ __device__ __forceinline__ double block_pairwise(const uint32_t (&w)[16], F f) {
 // warps leave in ws (padded with +0 to the tree's width / 32).  One barrier; every thread
 // of the slot returns the row sum.  ws must not be written again before every thread of
 // the CTA has passed the next barrier.
-__device__ __forceinline__ double row_sum(double v, int c, int nbw, int tree_pad, double* ws) {
+__device__ __forceinline__ float row_sum(float v, int c, int nbw, int tree_pad, float* ws) {
   const int wl = tree_pad >= 32 ? 5 : __ffs(tree_pad) - 1;
 #pragma unroll 1
-  for (int l = 0; l < wl; l++) v = __dadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, 1 << l));
+  for (int l = 0; l < wl; l++) v = __fadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, 1 << l));
   if (tree_pad <= 32) {
     __syncthreads();  // keeps the barrier count of every row the same
     return __shfl_sync(0xFFFFFFFFu, v, 0);
@@ -94,11 +85,11 @@ __device__ __forceinline__ double row_sum(double v, int c, int nbw, int tree_pad
   const int nw = tree_pad >> 5, lane = c & 31;
   if (lane == 0) ws[c >> 5] = v;
   if (lane == 0 && c == 0)
-    for (int j = nbw >> 5; j < nw; j++) ws[j] = 0.0;
+    for (int j = nbw >> 5; j < nw; j++) ws[j] = 0.0f;
   __syncthreads();
-  double u = lane < nw ? ws[lane] : 0.0;
+  float u = lane < nw ? ws[lane] : 0.0f;
 #pragma unroll 1
-  for (int o = 1; o < nw; o <<= 1) u = __dadd_rn(u, __shfl_xor_sync(0xFFFFFFFFu, u, o));
+  for (int o = 1; o < nw; o <<= 1) u = __fadd_rn(u, __shfl_xor_sync(0xFFFFFFFFu, u, o));
   return __shfl_sync(0xFFFFFFFFu, u, 0);
 }
 
@@ -109,14 +100,14 @@ __global__ void __launch_bounds__(kAlMaxThreads, 1) adaln_quant_kernel(const __g
   const int nws = p.tree_pad > 32 ? (p.tree_pad >> 5) : 1;  // warp sums per row tree
   uint8_t* ring = al_smem;                                      // [kAlStages][blockDim][64]
   uint16_t* hx = reinterpret_cast<uint16_t*>(al_smem + size_t(kAlStages) * blockDim.x * 64);  // [blockDim][32]
-  double* ws = reinterpret_cast<double*>(al_smem + size_t(kAlStages + 1) * blockDim.x * 64);   // [2][R][nws]
+  float* ws = reinterpret_cast<float*>(al_smem + size_t(kAlStages + 1) * blockDim.x * 64);     // [2][R][nws]
   const int t = threadIdx.x;
   const int rho = t / p.nbw, c = t % p.nbw;
   const bool col = c < p.nb;
   const int cc = col ? c : 0;
-  double* ws1 = ws + size_t(rho) * nws;
-  double* ws2 = ws + size_t(R + rho) * nws;
-  const double d = double(p.nb) * kBlock;
+  float* ws1 = ws + size_t(rho) * nws;
+  float* ws2 = ws + size_t(R + rho) * nws;
+  const float d = float(p.nb * kBlock);
   uint16_t* hmine = hx + size_t(t) * kBlock;
   const int sw = (t >> 1) & 3;
   const uint32_t cbase = smem_addr(ring) + uint32_t(t) * 64u;
@@ -172,20 +163,28 @@ __global__ void __launch_bounds__(kAlMaxThreads, 1) adaln_quant_kernel(const __g
         hv[k] = act ? __ldg(ph + k) : make_uint4(0u, 0u, 0u, 0u);
       }
     }
-    // statistics
-    // (padding columns and rows past M contribute +0)
-    const double b1 = act ? block_pairwise(w, [](double x) { return x; }) : 0.0;
-    const double s1 = row_sum(b1, c, p.nbw, p.tree_pad, ws1);
-    const double mu = __ddiv_rn(s1, d);
-    const double b2 = act ? block_pairwise(w,
-                                           [mu](double x) {
-                                             const double u = __dsub_rn(x, mu);
-                                             return __dmul_rn(u, u);
-                                           })
-                          : 0.0;
-    const double s2 = row_sum(b2, c, p.nbw, p.tree_pad, ws2);
-    const double var = __ddiv_rn(s2, d);
-    const double rstd = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(var, p.eps)));
+    // statistics (padding columns and rows past M contribute +0)
+    float xv[32];
+#pragma unroll
+    for (int j = 0; j < 16; j++) {
+      xv[2 * j] = bf16lo(w[j]);
+      xv[2 * j + 1] = bf16hi(w[j]);
+    }
+    const float s1 = row_sum(act ? block_pairwise(xv) : 0.0f, c, p.nbw, p.tree_pad, ws1);
+    const float mu = __fdiv_rn(s1, d);
+    float b2 = 0.0f;
+    if (act) {
+      float sq[32];
+#pragma unroll
+      for (int i = 0; i < 32; i++) {
+        const float t = __fsub_rn(xv[i], mu);
+        sq[i] = __fmul_rn(t, t);
+      }
+      b2 = block_pairwise(sq);
+    }
+    const float s2 = row_sum(b2, c, p.nbw, p.tree_pad, ws2);
+    const float var = __fdiv_rn(s2, d);
+    const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, p.eps)));
     if (act && c == 0 && p.stats != nullptr) {
       p.stats[2 * r] = mu;
       p.stats[2 * r + 1] = rstd;
@@ -197,17 +196,17 @@ __global__ void __launch_bounds__(kAlMaxThreads, 1) adaln_quant_kernel(const __g
       const uint32_t s4[4] = {sv[k].x, sv[k].y, sv[k].z, sv[k].w}, b4[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
 #pragma unroll
       for (int m = 0; m < 4; m++) {
-        uint32_t out = 0u;
+        const int j = 4 * k + m;
+        float h[2];
 #pragma unroll
         for (int e = 0; e < 2; e++) {
-          const uint32_t xw = w[4 * k + m];
-          const double xv = double(e ? bf16hi(xw) : bf16lo(xw));
-          const double a = __dadd_rn(1.0, double(e ? bf16hi(s4[m]) : bf16lo(s4[m])));
-          const double bv = double(e ? bf16hi(b4[m]) : bf16lo(b4[m]));
-          const double h64 = __dadd_rn(__dmul_rn(__dmul_rn(__dsub_rn(xv, mu), rstd), a), bv);
-          out |= bf16_bits_of_f64(h64) << (16 * e);
+          const float a = __fadd_rn(1.0f, e ? bf16hi(s4[m]) : bf16lo(s4[m]));
+          const float bv = e ? bf16hi(b4[m]) : bf16lo(b4[m]);
+          h[e] = __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(xv[2 * j + e], mu), rstd), a), bv);
         }
-        hw[4 * k + m] = out;
+        uint32_t out;
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(h[1]), "f"(h[0]));
+        hw[j] = out;
       }
     }
     reinterpret_cast<uint4*>(hmine)[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);

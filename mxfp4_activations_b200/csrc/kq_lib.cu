@@ -528,7 +528,7 @@ kq_variant resolve_variant(int64_t M, int64_t d, kq_dtype mat_dtype, bool has_fa
 
 extern "C" {
 
-int kq_abi_version(void) { return 203; }
+int kq_abi_version(void) { return 204; }
 
 const char* kq_status_string(kq_status s) {
   switch (s) {
@@ -703,8 +703,8 @@ kq_status kq_gemm_mxf4(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, c
 }
 
 kq_status kq_adaln_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const void* shift, const void* scale,
-                            int64_t rows_per_group, double eps, const float* mats, const float* factored, uint8_t* q,
-                            uint8_t* scales, kq_scale_layout scale_layout, double* stats, kq_stream_t stream) {
+                            int64_t rows_per_group, float eps, const float* mats, const float* factored, uint8_t* q,
+                            uint8_t* scales, kq_scale_layout scale_layout, float* stats, kq_stream_t stream) {
   if (scale_layout != KQ_SCALES_ROW_MAJOR && scale_layout != KQ_SCALES_MMA_TILED) return KQ_ERR_INVALID_ARG;
   if (rows_per_group < 1) return KQ_ERR_INVALID_ARG;
   kq_status st = check_x(x, M, d, ldx);
@@ -740,11 +740,11 @@ kq_status kq_adaln_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, co
   p.stats = stats;
   const int threads = p.rows * p.nbw;
   const int nws = p.tree_pad > 32 ? p.tree_pad / 32 : 1;
-  const int smem = (kq::kAlStages + 1) * threads * 64 + 2 * p.rows * nws * 8;
+  const int smem = (kq::kAlStages + 1) * threads * 64 + 2 * p.rows * nws * 4;
   const int which = scale_layout == KQ_SCALES_MMA_TILED ? 1 : 0;
   auto kern = which ? kq::adaln_quant_kernel<1> : kq::adaln_quant_kernel<0>;
   // the largest configuration: 512 threads, and at most 32 warp sums per buffer
-  constexpr int kMaxSmem = (kq::kAlStages + 1) * kq::kAlMaxThreads * 64 + 2 * 32 * 8;
+  constexpr int kMaxSmem = (kq::kAlStages + 1) * kq::kAlMaxThreads * 64 + 2 * 32 * 4;
   if (smem > kMaxSmem || kMaxSmem > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
   static std::atomic<int> attr_set[2][kMaxDevices];
   int devid = 0;

@@ -395,40 +395,42 @@ void kqo_mx_gemm(const uint8_t* a_q, const uint8_t* a_scales, int64_t M, const u
 
 /* ---- the producer: AdaLN normalisation fused in front of the quantizer ------------ */
 
-/* Pairwise sum in fp64: a[0..n) padded with +0 to a power of two, then neighbours
+/* Pairwise sum in fp32: a[0..n) padded with +0 to a power of two, then neighbours
  * added level by level.  tmp holds at least that power of two. */
-static double pairwise_sum(const double* a, int64_t n, double* tmp) {
+static float pairwise_sum_f32(const float* a, int64_t n, float* tmp) {
   int64_t p = 1;
   while (p < n) p *= 2;
-  for (int64_t i = 0; i < p; i++) tmp[i] = (i < n) ? a[i] : 0.0;
+  for (int64_t i = 0; i < p; i++) tmp[i] = (i < n) ? a[i] : 0.0f;
   for (int64_t w = p; w > 1; w /= 2)
     for (int64_t j = 0; j < w / 2; j++) tmp[j] = tmp[2 * j] + tmp[2 * j + 1];
   return tmp[0];
 }
 
 /* [KQ §Problem], [KQ abstract]: the modulated LayerNorm whose output the quantizer
- * receives, in the step order stated in the header. */
+ * receives, in the step order stated in the header (every operation one IEEE binary32
+ * operation: the build keeps fp32 expressions unfused). */
 void kqo_adaln(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const uint16_t* shift,
-               const uint16_t* scale, int64_t rows_per_group, double eps, uint16_t* h, double* stats) {
+               const uint16_t* scale, int64_t rows_per_group, float eps, uint16_t* h, float* stats) {
   int64_t p = 1;
   while (p < d) p *= 2;
-  double* v = (double*)malloc(sizeof(double) * (size_t)(d > 0 ? d : 1));
-  double* tmp = (double*)malloc(sizeof(double) * (size_t)p);
+  float* v = (float*)malloc(sizeof(float) * (size_t)(d > 0 ? d : 1));
+  float* tmp = (float*)malloc(sizeof(float) * (size_t)p);
+  const float df = (float)d;
   for (int64_t r = 0; r < M; r++) {
-    for (int64_t i = 0; i < d; i++) v[i] = (double)f32_from_bf16(x[r * ldx + i]);
-    const double mu = pairwise_sum(v, d, tmp) / (double)d;
+    for (int64_t i = 0; i < d; i++) v[i] = f32_from_bf16(x[r * ldx + i]);
+    const float mu = pairwise_sum_f32(v, d, tmp) / df;
     for (int64_t i = 0; i < d; i++) {
-      const double t = v[i] - mu;
+      const float t = v[i] - mu;
       v[i] = t * t;
     }
-    const double var = pairwise_sum(v, d, tmp) / (double)d;
-    const double rstd = 1.0 / sqrt(var + eps);
+    const float var = pairwise_sum_f32(v, d, tmp) / df;
+    const float rstd = 1.0f / sqrtf(var + eps);
     const int64_t g = r / rows_per_group;
     for (int64_t i = 0; i < d; i++) {
-      const double t = (double)f32_from_bf16(x[r * ldx + i]) - mu;
-      const double a = 1.0 + (double)f32_from_bf16(scale[g * d + i]);
-      const double b = (double)f32_from_bf16(shift[g * d + i]);
-      h[r * d + i] = kqo_bf16_from_f64((t * rstd) * a + b);
+      const float t = f32_from_bf16(x[r * ldx + i]) - mu;
+      const float a = 1.0f + f32_from_bf16(scale[g * d + i]);
+      const float b = f32_from_bf16(shift[g * d + i]);
+      h[r * d + i] = kqo_bf16_from_f64((double)((t * rstd) * a + b));
     }
     if (stats != NULL) {
       stats[2 * r] = mu;
@@ -440,8 +442,8 @@ void kqo_adaln(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const uint1
 }
 
 void kqo_adaln_quantize(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const uint16_t* shift,
-                        const uint16_t* scale, int64_t rows_per_group, double eps, const void* mats,
-                        int dtype, uint8_t* q, uint8_t* scales, double* stats) {
+                        const uint16_t* scale, int64_t rows_per_group, float eps, const void* mats,
+                        int dtype, uint8_t* q, uint8_t* scales, float* stats) {
   uint16_t* h = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(M * d > 0 ? M * d : 1));
   kqo_adaln(x, M, d, ldx, shift, scale, rows_per_group, eps, h, stats);
   kqo_quantize(h, M, d, d, mats, dtype, q, scales);

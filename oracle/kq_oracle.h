@@ -111,22 +111,23 @@ void kqo_quantize_n(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const 
  * [KQ §Problem] (AdaLN blocks keep the transform from being absorbed offline) and
  * [KQ abstract] (normalisation layers between blocks force the transform to run
  * online).  The pages do not define the normalisation; this is the DiT block's
- * modulated LayerNorm without a learned affine, with every step fixed so that it is
- * reproducible bit for bit (every operation one IEEE fp64 operation, rounded to
- * nearest even):
+ * modulated LayerNorm without a learned affine, computed in fp32 as DiT models do,
+ * with every step fixed so that it is reproducible bit for bit (every operation one
+ * IEEE binary32 operation, rounded to nearest even; sqrt and division correctly
+ * rounded):
  *   S1  = pairwise sum of the row's d inputs (pad with +0 to a power of two, then add
  *         neighbours level by level: a'_j = a_2j + a_2j+1)
  *   mu  = S1 / d
  *   t_i = x_i - mu;  S2 = pairwise sum of t_i * t_i;  var = S2 / d
  *   rstd = 1 / sqrt(var + eps)
  *   h_i = bf16( ((t_i * rstd) * (1 + scale[g][i])) + shift[g][i] ),  g = row / rows_per_group
- * shift, scale: bf16 [G][d]; h: bf16 bits [M][d]; stats: fp64 [M][2] (mu, rstd) or NULL. */
+ * shift, scale: bf16 [G][d]; h: bf16 bits [M][d]; stats: fp32 [M][2] (mu, rstd) or NULL. */
 void kqo_adaln(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const uint16_t* shift,
-               const uint16_t* scale, int64_t rows_per_group, double eps, uint16_t* h, double* stats);
+               const uint16_t* scale, int64_t rows_per_group, float eps, uint16_t* h, float* stats);
 /* kqo_adaln, then kqo_quantize of h with the block matrices. */
 void kqo_adaln_quantize(const uint16_t* x, int64_t M, int64_t d, int64_t ldx, const uint16_t* shift,
-                        const uint16_t* scale, int64_t rows_per_group, double eps, const void* mats,
-                        int dtype, uint8_t* q, uint8_t* scales, double* stats);
+                        const uint16_t* scale, int64_t rows_per_group, float eps, const void* mats,
+                        int dtype, uint8_t* q, uint8_t* scales, float* stats);
 
 /* ---- the consumer: W4A4 product of two MXFP4 operands
  *

@@ -98,8 +98,8 @@ def _configure(L):
     L.kqo_fwht_quantize.argtypes = [P, I64, I64, I64, P, P]
     L.kqo_dequantize.argtypes = [P, P, I64, I64, P, I, P]
     L.kqo_mx_gemm.argtypes = [P, P, I64, P, P, I64, I64, P]
-    L.kqo_adaln.argtypes = [P, I64, I64, I64, P, P, I64, ctypes.c_double, P, P]
-    L.kqo_adaln_quantize.argtypes = [P, I64, I64, I64, P, P, I64, ctypes.c_double, P, I, P, P, P]
+    L.kqo_adaln.argtypes = [P, I64, I64, I64, P, P, I64, ctypes.c_float, P, P]
+    L.kqo_adaln_quantize.argtypes = [P, I64, I64, I64, P, P, I64, ctypes.c_float, P, I, P, P, P]
     for name in ("kqo_factor", "kqo_factor_inverse", "kqo_kron", "kqo_expand_f64", "kqo_expand",
                  "kqo_hadamard", "kqo_e2m1_pack", "kqo_transform", "kqo_mx_quantize", "kqo_quantize",
                  "kqo_smooth_quantize", "kqo_fwht_quantize", "kqo_dequantize", "kqo_mx_gemm", "kqo_adaln", "kqo_adaln_quantize"):
@@ -314,14 +314,14 @@ def mx_gemm(a_q: np.ndarray, a_scales: np.ndarray, b_q: np.ndarray, b_scales: np
 # ---- the producer: AdaLN normalisation in front of the quantizer -------------------
 
 def adaln(x: np.ndarray, shift: np.ndarray, scale: np.ndarray, rows_per_group: int, eps: float):
-    """(h bf16 bits [M, d], stats fp64 [M, 2] = (mu, rstd)) of bf16 rows x [M, d] with
+    """(h bf16 bits [M, d], stats fp32 [M, 2] = (mu, rstd)) of bf16 rows x [M, d] with
     bf16 modulation vectors shift, scale [G, d]."""
     x = _bf16_bits(x)
     M, d = x.shape
     shift, scale = _bf16_bits(shift), _bf16_bits(scale)
     assert shift.shape[1] == d and scale.shape == shift.shape and shift.shape[0] * rows_per_group >= M
     h = np.zeros((M, d), np.uint16)
-    stats = np.zeros((M, 2), np.float64)
+    stats = np.zeros((M, 2), np.float32)
     lib().kqo_adaln(_p(x), M, d, d, _p(shift), _p(scale), rows_per_group, float(eps), _p(h), _p(stats))
     return h, stats
 
@@ -335,7 +335,7 @@ def adaln_quantize(x: np.ndarray, shift: np.ndarray, scale: np.ndarray, rows_per
     mats = np.ascontiguousarray(mats)
     q = np.zeros((M, d // 2), np.uint8)
     s = np.zeros((M, d // 32), np.uint8)
-    stats = np.zeros((M, 2), np.float64)
+    stats = np.zeros((M, 2), np.float32)
     lib().kqo_adaln_quantize(_p(x), M, d, d, _p(shift), _p(scale), rows_per_group, float(eps), _p(mats),
                              _mats_dtype(mats), _p(q), _p(s), _p(stats))
     return q, s, stats

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.kq_abi_version() == 203
+    assert lib.kq_abi_version() == 204
     for code in range(8):
         s = lib.kq_status_string(code).decode()
         assert s.startswith("KQ_")

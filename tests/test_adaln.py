@@ -49,10 +49,10 @@ def run(kq, x, shift, scale, rpg, params, eps=1e-6, layout="row"):
     sv, sbuf = guarded(torch, kq.scale_bytes(M, d, layout))
     if layout == "mma":
         sv.zero_()
-    tv, tbuf = guarded(torch, M * 16)
+    tv, tbuf = guarded(torch, M * 8)
     q = qv.view(M, d // 2)
     s = sv.view(M, d // 32) if layout == "row" else sv
-    st = tv.view(torch.float64).view(M, 2)
+    st = tv.view(torch.float32).view(M, 2)
     bt.adaln_quantize(dev_bits(x), dev_bits(shift), dev_bits(scale), rpg, eps=eps, q=q, scales=s,
                       scale_layout=layout, stats=st)
     torch.cuda.synchronize()
@@ -72,7 +72,7 @@ def oracle(orc, x, shift, scale, rpg, params, eps=1e-6):
 def same_stats(a: np.ndarray, b: np.ndarray) -> bool:
     """Bit-equal, NaN payloads aside."""
     both_nan = np.isnan(a) & np.isnan(b)
-    return bool(np.all(both_nan | (a.view(np.uint64) == b.view(np.uint64))))
+    return bool(np.all(both_nan | (a.view(np.uint32) == b.view(np.uint32))))
 
 
 @pytest.mark.parametrize("d", [3072, 12288])

@@ -66,18 +66,18 @@ MUTANTS = {
     "mx_gemm_last_element_dropped": ("for (int64_t k = 0; k < K; k++)\n        acc +=",
                                      "for (int64_t k = 0; k < K - 1; k++)\n        acc +="),
     # the AdaLN normalisation in front of the quantizer
-    "adaln_unbiased_variance": ("const double var = pairwise_sum(v, d, tmp) / (double)d;",
-                                "const double var = pairwise_sum(v, d, tmp) / (double)(d - 1);"),
-    "adaln_eps_outside_sqrt": ("const double rstd = 1.0 / sqrt(var + eps);", "const double rstd = 1.0 / (sqrt(var) + eps);"),
-    "adaln_scale_without_one": ("const double a = 1.0 + (double)f32_from_bf16(scale[g * d + i]);",
-                                "const double a = (double)f32_from_bf16(scale[g * d + i]);"),
-    "adaln_shift_from_scale": ("const double b = (double)f32_from_bf16(shift[g * d + i]);",
-                               "const double b = (double)f32_from_bf16(scale[g * d + i]);"),
+    "adaln_unbiased_variance": ("const float var = pairwise_sum_f32(v, d, tmp) / df;",
+                                "const float var = pairwise_sum_f32(v, d, tmp) / (df - 1.0f);"),
+    "adaln_eps_outside_sqrt": ("const float rstd = 1.0f / sqrtf(var + eps);", "const float rstd = 1.0f / (sqrtf(var) + eps);"),
+    "adaln_scale_without_one": ("const float a = 1.0f + f32_from_bf16(scale[g * d + i]);",
+                                "const float a = f32_from_bf16(scale[g * d + i]);"),
+    "adaln_shift_from_scale": ("const float b = f32_from_bf16(shift[g * d + i]);",
+                               "const float b = f32_from_bf16(scale[g * d + i]);"),
     "adaln_group_modulo": ("const int64_t g = r / rows_per_group;", "const int64_t g = r % rows_per_group;"),
-    "adaln_pairwise_drops_last": ("for (int64_t i = 0; i < p; i++) tmp[i] = (i < n) ? a[i] : 0.0;",
-                                  "for (int64_t i = 0; i < p; i++) tmp[i] = (i < n - 1) ? a[i] : 0.0;"),
-    "adaln_mean_not_subtracted": ("      const double t = v[i] - mu;\n      v[i] = t * t;",
-                                  "      const double t = v[i];\n      v[i] = t * t;"),
+    "adaln_pairwise_drops_last": ("for (int64_t i = 0; i < p; i++) tmp[i] = (i < n) ? a[i] : 0.0f;",
+                                  "for (int64_t i = 0; i < p; i++) tmp[i] = (i < n - 1) ? a[i] : 0.0f;"),
+    "adaln_mean_not_subtracted": ("      const float t = v[i] - mu;\n      v[i] = t * t;",
+                                  "      const float t = v[i];\n      v[i] = t * t;"),
 }
 
 SKIP = {"test_e2m1_exhaustive_core_binades"}
