@@ -478,9 +478,9 @@ struct AutoRule {
   kq_variant v;
 };
 constexpr AutoRule kAutoTable[] = {
-    {1, 1152, KQ_VAR_MMA},            {1, 3072, KQ_VAR_MMA},            {1, 12288, KQ_VAR_BUTTERFLY},
+    {1, 1152, KQ_VAR_MMA},            {1, 3072, KQ_VAR_BUTTERFLY},      {1, 12288, KQ_VAR_BUTTERFLY},
     {16, 1152, KQ_VAR_BUTTERFLY},     {16, 3072, KQ_VAR_BUTTERFLY},     {16, 12288, KQ_VAR_BUTTERFLY},
-    {256, 1152, KQ_VAR_BUTTERFLY},    {256, 3072, KQ_VAR_MMA},          {256, 12288, KQ_VAR_BUTTERFLY},
+    {256, 1152, KQ_VAR_BUTTERFLY},    {256, 3072, KQ_VAR_BUTTERFLY},    {256, 12288, KQ_VAR_BUTTERFLY},
     {4096, 1152, KQ_VAR_BUTTERFLY},   {4096, 3072, KQ_VAR_BUTTERFLY},   {4096, 12288, KQ_VAR_BUTTERFLY},
     {16384, 1152, KQ_VAR_BUTTERFLY},  {16384, 3072, KQ_VAR_BUTTERFLY},  {16384, 12288, KQ_VAR_BUTTERFLY},
     {65536, 1152, KQ_VAR_BUTTERFLY},  {65536, 3072, KQ_VAR_BUTTERFLY},  {65536, 12288, KQ_VAR_BUTTERFLY},
