@@ -11,9 +11,10 @@
 // every step one IEEE binary32 operation rounded to nearest even (no contraction; sqrt and
 // division correctly rounded), so the statistics and h are the definition's bit for bit;
 // then y = h K_b and the certified MXFP4 step of the butterfly quantizer (kq_quant.cuh)
-// on h, which never leaves the chip.  Every step uses the scalar round-to-nearest
-// intrinsics, which the compiler never contracts: separate packed f32x2 multiplies and
-// adds were measured to be fused into one FMA.
+// on h, which never leaves the chip.  Steps run on packed fp32 pairs where no multiply
+// feeds a packed add; every add that follows a multiply is the scalar round-to-nearest
+// intrinsic, which the compiler never contracts (a packed multiply followed by a packed add
+// was measured to be fused into one FMA).
 //
 // Work mapping.  A CTA takes R rows per step, each on a slot of nbw = nb rounded up to a
 // multiple of 32 threads: thread t takes block column c = t % nbw of slot t / nbw (columns
@@ -163,22 +164,29 @@ __global__ void __launch_bounds__(kAlMaxThreads, 1) adaln_quant_kernel(const __g
         hv[k] = act ? __ldg(ph + k) : make_uint4(0u, 0u, 0u, 0u);
       }
     }
-    // statistics (padding columns and rows past M contribute +0)
-    float xv[32];
+    // statistics (padding columns and rows past M contribute +0).  Packed f32x2 steps are
+    // used only where no multiply feeds a packed add; every add that follows a multiply is
+    // a scalar __fadd_rn, which the compiler never contracts.
+    uint64_t X[16];
 #pragma unroll
-    for (int j = 0; j < 16; j++) {
-      xv[2 * j] = bf16lo(w[j]);
-      xv[2 * j + 1] = bf16hi(w[j]);
+    for (int j = 0; j < 16; j++) X[j] = pk2(bf16lo(w[j]), bf16hi(w[j]));
+    float b1 = 0.0f;
+    if (act) {
+      float xv[32];
+#pragma unroll
+      for (int j = 0; j < 16; j++) upk2(X[j], xv[2 * j], xv[2 * j + 1]);
+      b1 = block_pairwise(xv);
     }
-    const float s1 = row_sum(act ? block_pairwise(xv) : 0.0f, c, p.nbw, p.tree_pad, ws1);
+    const float s1 = row_sum(b1, c, p.nbw, p.tree_pad, ws1);
     const float mu = __fdiv_rn(s1, d);
+    const uint64_t MU = pk2(mu, mu);
     float b2 = 0.0f;
     if (act) {
       float sq[32];
 #pragma unroll
-      for (int i = 0; i < 32; i++) {
-        const float t = __fsub_rn(xv[i], mu);
-        sq[i] = __fmul_rn(t, t);
+      for (int j = 0; j < 16; j++) {
+        const uint64_t t = sub2_rn(X[j], MU);
+        upk2(mul2_rn(t, t), sq[2 * j], sq[2 * j + 1]);
       }
       b2 = block_pairwise(sq);
     }
@@ -190,6 +198,7 @@ __global__ void __launch_bounds__(kAlMaxThreads, 1) adaln_quant_kernel(const __g
       p.stats[2 * r + 1] = rstd;
     }
     // modulation, one bf16 rounding per element
+    const uint64_t RS = pk2(rstd, rstd), ONE = pk2(1.0f, 1.0f);
     uint32_t hw[16];
 #pragma unroll
     for (int k = 0; k < 4; k++) {
@@ -197,15 +206,12 @@ __global__ void __launch_bounds__(kAlMaxThreads, 1) adaln_quant_kernel(const __g
 #pragma unroll
       for (int m = 0; m < 4; m++) {
         const int j = 4 * k + m;
-        float h[2];
-#pragma unroll
-        for (int e = 0; e < 2; e++) {
-          const float a = __fadd_rn(1.0f, e ? bf16hi(s4[m]) : bf16lo(s4[m]));
-          const float bv = e ? bf16hi(b4[m]) : bf16lo(b4[m]);
-          h[e] = __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(xv[2 * j + e], mu), rstd), a), bv);
-        }
+        const uint64_t A = add2_rn(ONE, pk2(bf16lo(s4[m]), bf16hi(s4[m])));
+        float v0, v1;
+        upk2(mul2_rn(mul2_rn(sub2_rn(X[j], MU), RS), A), v0, v1);
+        const float h0 = __fadd_rn(v0, bf16lo(b4[m])), h1 = __fadd_rn(v1, bf16hi(b4[m]));
         uint32_t out;
-        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(h[1]), "f"(h[0]));
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(h1), "f"(h0));
         hw[j] = out;
       }
     }
