@@ -471,17 +471,20 @@ __device__ __forceinline__ void pair_commit(uint64_t* bar) {
 // 8 rows x 16 bytes stacked every 128 bytes); each row lands in one lane of every
 // lane quarter.
 template <class C>
-__device__ __forceinline__ void pair_scale_copies(uint32_t st, uint32_t sfa_col, uint32_t sfb_col) {
+__device__ __forceinline__ void pair_scale_copies(uint64_t sfa_desc, uint64_t sfb_desc, uint32_t sfa_col,
+                                                  uint32_t sfb_col) {
+  // sfa_desc / sfb_desc: descriptors of the stage's first A and B scale tiles; tiles are
+  // 512 bytes (32 in the descriptor's 16-byte address units) apart
 #pragma unroll
   for (int c = 0; c < C::kTiles; c++) {
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(sfa_col + 4 * c),
-                 "l"(gemm_sdesc(st + C::kSfaOff + 512 * c, 128, 128, 0))
+                 "l"(sfa_desc + uint64_t(32 * c))
                  : "memory");
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(sfb_col + 8 * c),
-                 "l"(gemm_sdesc(st + C::kSfbOff + 512 * c, 128, 128, 0))
+                 "l"(sfb_desc + uint64_t(32 * c))
                  : "memory");
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(sfb_col + 8 * c + 4),
-                 "l"(gemm_sdesc(st + C::kSfbOff + 512 * (C::kTiles + c), 128, 128, 0))
+                 "l"(sfb_desc + uint64_t(32 * (C::kTiles + c)))
                  : "memory");
   }
 }
@@ -574,6 +577,15 @@ __global__ void __launch_bounds__(kG2Threads, 1)
     if (rank == 0 && lane == 0) {
       int it = 0, tl = 0;
       bool ok = true;
+      // Descriptors of stage 0; another stage or K step differs only in the start-address
+      // field (16-byte units, below 2^14 for every address in this CTA's shared memory),
+      // so they are formed once and offset by an add.
+      const uint32_t st0 = smem_addr(base);
+      const uint64_t a_desc0 = gemm_sdesc(st0, 16, C::kSbo, C::kLayout);
+      const uint64_t b_desc0 = gemm_sdesc(st0 + C::kABytes, 16, C::kSbo, C::kLayout);
+      const uint64_t sfa_desc0 = gemm_sdesc(st0 + C::kSfaOff, 128, 128, 0);
+      const uint64_t sfb_desc0 = gemm_sdesc(st0 + C::kSfbOff, 128, 128, 0);
+      constexpr uint64_t kStageUnits = uint64_t(C::kStageBytes >> 4);
       for (int t = cid; t < n_tiles && ok; t += n_clusters, tl++) {
         if (tl > 0 && (*abort_flag || !mbar_wait_bounded(acc_empty, uint32_t(tl - 1) & 1u, kWaitLimitNs))) {
           *abort_flag = 1;
@@ -596,13 +608,13 @@ __global__ void __launch_bounds__(kG2Threads, 1)
           asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
           ready = kt + 1 < p.n_ktiles &&
                   mbar_test(&full[(it + 1) % C::kStages], uint32_t((it + 1) / C::kStages) & 1u);
-          const uint32_t st = smem_addr(base + s * C::kStageBytes);
+          const uint64_t so = kStageUnits * uint64_t(s);
           const uint32_t sfa_col = tmem + 256 + uint32_t(C::kSfCols * s), sfb_col = sfa_col + 4 * C::kTiles;
-          pair_scale_copies<C>(st, sfa_col, sfb_col);
+          pair_scale_copies<C>(sfa_desc0 + so, sfb_desc0 + so, sfa_col, sfb_col);
 #pragma unroll
           for (int j = 0; j < C::kMmas; j++) {
-            const uint64_t ad = gemm_sdesc(st + j * 32, 16, C::kSbo, C::kLayout);
-            const uint64_t bd = gemm_sdesc(st + C::kABytes + j * 32, 16, C::kSbo, C::kLayout);
+            const uint64_t ad = a_desc0 + so + uint64_t(2 * j);  // K step j: 32 bytes further
+            const uint64_t bd = b_desc0 + so + uint64_t(2 * j);
             const uint32_t byte = uint32_t(2 * (j & 1));
             const uint32_t accumulate = (kt > 0 || j > 0) ? 1u : 0u;
             const uint32_t sfa = (sfa_col + 4 * (j >> 1)) | (byte << 30);
