@@ -708,3 +708,61 @@ def test_adaln_symmetric_row_closed_form(orc):
     ref = sgn * a * rstd * s1 + b
     slack = 6 * 2.0**-24 * (a * rstd * np.abs(s1) + np.abs(b))
     assert _bf16_near(h[0], ref, slack).all()
+
+
+# ---------------------------------------------------------------- exhaustive sweeps of the element rules
+
+E2M1_MIDPOINTS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+
+
+def e2m1_by_midpoints(v: np.ndarray) -> np.ndarray:
+    """E2M1 code from the position of |v| among the midpoints of the grid: the number of
+    midpoints strictly below |v|, plus one at an exact midpoint whose lower code is odd
+    (ties to the even code); everything above 5 saturates to 7; sign bit from v."""
+    m = np.abs(v.astype(np.float64))
+    k = np.searchsorted(E2M1_MIDPOINTS, m, side="left")
+    tie = (k < 7) & (m == E2M1_MIDPOINTS[np.minimum(k, 6)])
+    code = k + (tie & (k % 2 == 1))
+    return code | (np.signbit(v).astype(np.int64) << 3)
+
+
+def test_e2m1_every_fp32_pattern(orc):
+    """All 2^32 fp32 bit patterns but NaN: inside [2^-3, 2^3) against the midpoint rule
+    (an independent formulation of nearest-even on the grid), outside it the two constant
+    answers (0 below 2^-3, 7 from 2^3 up, infinities included) with the sign bit."""
+    step = 1 << 24
+    lo = int(np.float32(0.125).view(np.uint32))
+    hi = int(np.float32(8.0).view(np.uint32))
+    inf = int(np.float32(np.inf).view(np.uint32))
+    for start in range(0, 1 << 31, step):
+        pos = np.arange(start, start + step, dtype=np.uint32)
+        keep = pos <= inf                                    # NaN patterns dropped
+        pos = pos[keep]
+        for sign in (0, 0x80000000):
+            bits = pos | np.uint32(sign)
+            v = bits.view(np.float32)
+            if v.size % 2:
+                v = np.append(v, v[-1])
+            packed = orc.e2m1_pack(v)
+            s = 8 if sign else 0
+            if start + step <= lo:                           # two equal nibbles per byte
+                assert np.all(packed == s * 17), start
+            elif start >= hi:
+                assert np.all(packed == (7 | s) * 17), start
+            else:
+                assert np.array_equal(unpack_nibbles(packed), e2m1_by_midpoints(v)), start
+
+
+def test_e8m0_every_positive_finite_value(orc):
+    """Every positive finite fp32 value (and +0): the byte is floor(log2 amax) - 2 + 127,
+    clamped, from the exponent field for normal values; subnormals (field 0) and zero
+    against the bit-field reference."""
+    step = 1 << 23                                           # one exponent field per chunk
+    for field in range(0, 255):
+        bits = (np.uint32(field) << np.uint32(23)) | np.arange(step, dtype=np.uint32)
+        a = bits.view(np.float32)
+        got = orc.e8m0_many(a).astype(np.int64)
+        if field == 0:
+            assert np.array_equal(got, e8m0_from_bits(a))
+        else:
+            assert np.all(got == min(max(field - 127 - 2, -127), 127) + 127), field
