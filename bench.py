@@ -274,8 +274,9 @@ class QuantStep:
             rng = np.random.default_rng([d, 77])
             mod = [torch.from_numpy(inputs.f32_to_bf16_bits((sd * rng.standard_normal((2, d))).astype(np.float32))
                                     .view(np.int16)).to(device) for sd in (0.5, 0.3)]
+            stats = torch.empty((M, 2), dtype=torch.float32, device=device)
             self.items.append(dict(d=d, M=M, params=p, mats=mats, mats16=mats16, fac=fac, x=copies, q=qs, s=ss,
-                                   inv_s=inv_s, shift=mod[0], scale=mod[1]))
+                                   inv_s=inv_s, shift=mod[0], scale=mod[1], stats=stats))
         self.n = n_copies
         self.stream = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
@@ -292,10 +293,13 @@ class QuantStep:
         elif kind == "kroquant_mma_bf16":
             st = self.lib.kq_quantize(x.data_ptr(), M, d, d, item["mats16"].data_ptr(), 1, None,
                                       q.data_ptr(), s.data_ptr(), 1, 0, self.stream)
-        elif kind == "kroquant_adaln":
+        elif kind in ("kroquant_adaln", "kroquant_adaln_fused"):
+            # with a statistics buffer: the statistics pass, then the quantizer's AdaLN form;
+            # without one: the single fused kernel
+            stats = item["stats"].data_ptr() if kind == "kroquant_adaln" else None
             st = self.lib.kq_adaln_quantize(x.data_ptr(), M, d, d, item["shift"].data_ptr(), item["scale"].data_ptr(),
                                             (M + 1) // 2, ctypes.c_float(1e-6), item["mats"].data_ptr(),
-                                            item["fac"].data_ptr(), q.data_ptr(), s.data_ptr(), 0, None, self.stream)
+                                            item["fac"].data_ptr(), q.data_ptr(), s.data_ptr(), 0, stats, self.stream)
         elif kind == "smooth":
             st = self.lib.kq_ref_smooth_quantize(x.data_ptr(), M, d, d, item["inv_s"].data_ptr(), q.data_ptr(),
                                                  s.data_ptr(), self.stream)
@@ -487,7 +491,8 @@ def run_gpu(args) -> None:
     # each shape back to back on its own
     comp = {}
     n_cmp = max(50, args.steps)
-    for kind in ("smooth", "fwht", "kroquant", "kroquant_mma", "kroquant_mma_bf16", "kroquant_adaln"):
+    for kind in ("smooth", "fwht", "kroquant", "kroquant_mma", "kroquant_mma_bf16", "kroquant_adaln",
+                 "kroquant_adaln_fused"):
         us = {str(it["d"]): timed_b2b(torch, step, j, kind, n_cmp) for j, it in enumerate(step.items)}
         comp[kind] = {"gbs": bytes_step / (sum(us.values()) * 1e-6) / 1e9, "us_per_launch": us}
 

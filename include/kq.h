@@ -236,8 +236,12 @@ KQ_API kq_status kq_dequantize(const uint8_t* q, const uint8_t* scales, int64_t 
  *   mats, factored  fp32 [d/32][32][32] and [d/32][48], as kq_quantize's butterfly variant.
  *   q, scales, scale_layout  as kq_quantize.
  *   stats         device fp32 [M][2]: (mu, rstd) of each row, or NULL; 8-byte aligned.
+ * With stats, two kernels run on the stream: a statistics pass writes (mu, rstd) of every
+ * row into stats, then the butterfly quantizer forms h from x, stats and the modulation
+ * vectors inside its row loop (the faster form).  With stats NULL, one fused kernel
+ * computes the statistics and quantizes; no memory beyond the outputs is used either way.
  * d must be a multiple of 32 and at most 16384 (KQ_ERR_UNSUPPORTED above).  Codes, scales
- * and statistics equal the definition bit for bit. */
+ * and statistics equal the definition bit for bit in both forms. */
 KQ_API kq_status kq_adaln_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, const void* shift,
                                    const void* scale, int64_t rows_per_group, float eps, const float* mats,
                                    const float* factored, uint8_t* q, uint8_t* scales, kq_scale_layout scale_layout,

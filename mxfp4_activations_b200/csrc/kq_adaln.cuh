@@ -28,6 +28,13 @@
 // addition is commutative, so both partners form the same sum), and the rest pair the
 // warp sums, which every warp of the slot reads from shared memory after one barrier.
 // h of each block is staged in shared memory for the warp-cooperative exact path.
+//
+// Two forms.  adaln_quant_kernel does everything in one kernel (kq_adaln_quantize without
+// a statistics buffer).  With one, adaln_stats_kernel writes each row's (mu, rstd) with
+// the same tree and operations, and the butterfly quantizer's ADALN form (kq_quant.cuh)
+// forms h from x, those statistics and the modulation vectors inside its own row loop:
+// the quantizer keeps its two CTAs per SM and no CTA-wide barrier, and the statistics
+// pass, free of the quantizer's registers, runs at two CTAs of up to 512 threads per SM.
 #pragma once
 
 #include "kq_quant.cuh"
@@ -94,6 +101,92 @@ __device__ __forceinline__ float row_sum(float v, int c, int nbw, int tree_pad, 
   return __shfl_sync(0xFFFFFFFFu, u, 0);
 }
 
+// The statistics of one row as its slot's threads hold it: thread c has block column c
+// as 16 bf16 words w (zero for padding columns and rows past M, act false).  Returns the
+// block's inputs as packed pairs in X and the row's mu and rstd in every thread.  Two
+// barriers (row_sum); ws1, ws2: the slot's two warp-sum buffers.
+__device__ __forceinline__ void row_stats(const uint32_t (&w)[16], bool act, int c, const AdaLnParams& p,
+                                          float* ws1, float* ws2, uint64_t (&X)[16], float& mu, float& rstd) {
+  const float d = float(p.nb * kBlock);
+#pragma unroll
+  for (int j = 0; j < 16; j++) X[j] = pk2(bf16lo(w[j]), bf16hi(w[j]));
+  float b1 = 0.0f;
+  if (act) {
+    float xv[32];
+#pragma unroll
+    for (int j = 0; j < 16; j++) upk2(X[j], xv[2 * j], xv[2 * j + 1]);
+    b1 = block_pairwise(xv);
+  }
+  const float s1 = row_sum(b1, c, p.nbw, p.tree_pad, ws1);
+  mu = __fdiv_rn(s1, d);
+  const uint64_t MU = pk2(mu, mu);
+  float b2 = 0.0f;
+  if (act) {
+    float sq[32];
+#pragma unroll
+    for (int j = 0; j < 16; j++) {
+      const uint64_t t = sub2_rn(X[j], MU);
+      upk2(mul2_rn(t, t), sq[2 * j], sq[2 * j + 1]);
+    }
+    b2 = block_pairwise(sq);
+  }
+  const float s2 = row_sum(b2, c, p.nbw, p.tree_pad, ws2);
+  const float var = __fdiv_rn(s2, d);
+  rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, p.eps)));
+}
+
+// The statistics pass of the two-kernel form (kq_adaln_quantize given stats): each
+// row's (mu, rstd), formed exactly as adaln_quant_kernel forms them, into p.stats; the
+// butterfly quantizer's ADALN form then modulates and quantizes.  Same mapping of rows
+// and block columns to threads as adaln_quant_kernel, without the quantizer, so two CTAs
+// fit on an SM; each thread loads its next step's block while this step's sums run.
+__global__ void __launch_bounds__(kAlMaxThreads, 2) adaln_stats_kernel(const __grid_constant__ AdaLnParams p) {
+  extern __shared__ __align__(16) float st_ws[];  // [2][R][nws]
+  const int R = p.rows;
+  const int nws = p.tree_pad > 32 ? (p.tree_pad >> 5) : 1;
+  const int t = threadIdx.x;
+  const int rho = t / p.nbw, c = t % p.nbw;
+  const bool col = c < p.nb;
+  float* ws1 = st_ws + size_t(rho) * nws;
+  float* ws2 = st_ws + size_t(R + rho) * nws;
+  grid_dependency_wait();  // inputs may come from the previous kernel in the stream
+  const int64_t step_rows = int64_t(gridDim.x) * R;
+  const int64_t r_first = int64_t(blockIdx.x) * R + rho;
+  const int64_t n_steps = (p.M - int64_t(blockIdx.x) * R + step_rows - 1) / step_rows;  // CTA-uniform
+  uint4 nx[4];
+#pragma unroll
+  for (int k = 0; k < 4; k++) nx[k] = make_uint4(0u, 0u, 0u, 0u);
+  if (col && r_first < p.M) {
+    const uint4* px = reinterpret_cast<const uint4*>(p.x + r_first * p.ldx + int64_t(c) * kBlock);
+#pragma unroll
+    for (int k = 0; k < 4; k++) nx[k] = __ldg(px + k);
+  }
+  grid_launch_dependents();
+#pragma unroll 1
+  for (int64_t i = 0; i < n_steps; i++) {
+    const int64_t r = r_first + i * step_rows;
+    const bool act = col && r < p.M;
+    uint32_t w[16];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      w[4 * k] = nx[k].x;
+      w[4 * k + 1] = nx[k].y;
+      w[4 * k + 2] = nx[k].z;
+      w[4 * k + 3] = nx[k].w;
+    }
+    const int64_t rn = r + step_rows;
+    if (col && rn < p.M) {
+      const uint4* px = reinterpret_cast<const uint4*>(p.x + rn * p.ldx + int64_t(c) * kBlock);
+#pragma unroll
+      for (int k = 0; k < 4; k++) nx[k] = __ldg(px + k);
+    }
+    uint64_t X[16];
+    float mu, rstd;
+    row_stats(w, act, c, p, ws1, ws2, X, mu, rstd);
+    if (act && c == 0) *reinterpret_cast<float2*>(p.stats + 2 * r) = make_float2(mu, rstd);
+  }
+}
+
 template <int TILED>
 __global__ void __launch_bounds__(kAlMaxThreads, 1) adaln_quant_kernel(const __grid_constant__ AdaLnParams p) {
   extern __shared__ __align__(128) uint8_t al_smem[];
@@ -108,7 +201,6 @@ __global__ void __launch_bounds__(kAlMaxThreads, 1) adaln_quant_kernel(const __g
   const int cc = col ? c : 0;
   float* ws1 = ws + size_t(rho) * nws;
   float* ws2 = ws + size_t(R + rho) * nws;
-  const float d = float(p.nb * kBlock);
   uint16_t* hmine = hx + size_t(t) * kBlock;
   const int sw = (t >> 1) & 3;
   const uint32_t cbase = smem_addr(ring) + uint32_t(t) * 64u;
@@ -164,57 +256,17 @@ __global__ void __launch_bounds__(kAlMaxThreads, 1) adaln_quant_kernel(const __g
         hv[k] = act ? __ldg(ph + k) : make_uint4(0u, 0u, 0u, 0u);
       }
     }
-    // statistics (padding columns and rows past M contribute +0).  Packed f32x2 steps are
-    // used only where no multiply feeds a packed add; every add that follows a multiply is
-    // a scalar __fadd_rn, which the compiler never contracts.
+    // statistics (padding columns and rows past M contribute +0)
     uint64_t X[16];
-#pragma unroll
-    for (int j = 0; j < 16; j++) X[j] = pk2(bf16lo(w[j]), bf16hi(w[j]));
-    float b1 = 0.0f;
-    if (act) {
-      float xv[32];
-#pragma unroll
-      for (int j = 0; j < 16; j++) upk2(X[j], xv[2 * j], xv[2 * j + 1]);
-      b1 = block_pairwise(xv);
-    }
-    const float s1 = row_sum(b1, c, p.nbw, p.tree_pad, ws1);
-    const float mu = __fdiv_rn(s1, d);
-    const uint64_t MU = pk2(mu, mu);
-    float b2 = 0.0f;
-    if (act) {
-      float sq[32];
-#pragma unroll
-      for (int j = 0; j < 16; j++) {
-        const uint64_t t = sub2_rn(X[j], MU);
-        upk2(mul2_rn(t, t), sq[2 * j], sq[2 * j + 1]);
-      }
-      b2 = block_pairwise(sq);
-    }
-    const float s2 = row_sum(b2, c, p.nbw, p.tree_pad, ws2);
-    const float var = __fdiv_rn(s2, d);
-    const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, p.eps)));
+    float mu, rstd;
+    row_stats(w, act, c, p, ws1, ws2, X, mu, rstd);
     if (act && c == 0 && p.stats != nullptr) {
       p.stats[2 * r] = mu;
       p.stats[2 * r + 1] = rstd;
     }
     // modulation, one bf16 rounding per element
-    const uint64_t RS = pk2(rstd, rstd), ONE = pk2(1.0f, 1.0f);
     uint32_t hw[16];
-#pragma unroll
-    for (int k = 0; k < 4; k++) {
-      const uint32_t s4[4] = {sv[k].x, sv[k].y, sv[k].z, sv[k].w}, b4[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
-#pragma unroll
-      for (int m = 0; m < 4; m++) {
-        const int j = 4 * k + m;
-        const uint64_t A = add2_rn(ONE, pk2(bf16lo(s4[m]), bf16hi(s4[m])));
-        float v0, v1;
-        upk2(mul2_rn(mul2_rn(sub2_rn(X[j], MU), RS), A), v0, v1);
-        const float h0 = __fadd_rn(v0, bf16lo(b4[m])), h1 = __fadd_rn(v1, bf16hi(b4[m]));
-        uint32_t out;
-        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(h1), "f"(h0));
-        hw[j] = out;
-      }
-    }
+    modulate(X, mu, rstd, sv, hv, hw);
     reinterpret_cast<uint4*>(hmine)[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
     reinterpret_cast<uint4*>(hmine)[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
     reinterpret_cast<uint4*>(hmine)[2] = make_uint4(hw[8], hw[9], hw[10], hw[11]);

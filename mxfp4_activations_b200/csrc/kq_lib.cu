@@ -152,26 +152,40 @@ void lane_layout(int64_t M, int64_t nb, int64_t slots, kq::QuantParams& p) {
   }
 }
 
-template <int MODE, int TILED, int NT = 32>
+// The AdaLN fields of the quantizer's ADALN form (kq_adaln_quantize given stats).
+struct AdaLnInput {
+  const float* stats = nullptr;
+  const uint16_t* shift = nullptr;
+  const uint16_t* scale = nullptr;
+  int64_t rows_per_group = 1;
+};
+
+template <int MODE, int TILED, int NT = 32, bool ADALN = false>
 kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const float* mats, const float* factored,
-                       const float* inv_s, uint8_t* q, uint8_t* scales, cudaStream_t stream) {
+                       const float* inv_s, uint8_t* q, uint8_t* scales, cudaStream_t stream,
+                       const AdaLnInput& ada = AdaLnInput()) {
   const DeviceInfo* dev = device_info();
   if (dev == nullptr) return cuda_fail("device query", cudaErrorInvalidDevice);
   int devid = 0;
   cudaGetDevice(&devid);
   const int64_t nb = d / 32;
-  void (*kern)(const kq::QuantParams) = kq::quant_kernel<MODE, TILED, NT>;
+  void (*kern)(const kq::QuantParams) = kq::quant_kernel<MODE, TILED, NT, ADALN>;
+  constexpr int smem = kq::quant_smem_bytes(ADALN);
   static std::atomic<int> attr_set[kMaxDevices];
   if (!attr_set[devid].load()) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kq::kSSmemBytes);
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
     attr_set[devid].store(1);
   }
   int per_sm = 0;
-  kq_status st = resident_ctas(reinterpret_cast<const void*>(kern), kq::kSThreads, kq::kSSmemBytes, devid, &per_sm);
+  kq_status st = resident_ctas(reinterpret_cast<const void*>(kern), kq::kSThreads, smem, devid, &per_sm);
   if (st != KQ_OK) return st;
 
   kq::QuantParams p;
+  p.stats = ada.stats;
+  p.shift = ada.shift;
+  p.scale = ada.scale;
+  p.rows_per_group = ada.rows_per_group;
   p.x = static_cast<const uint16_t*>(x);
   p.ldx = ldx;
   p.M = M;
@@ -183,7 +197,7 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   p.scales = scales;
   lane_layout(M, nb, int64_t(dev->sms) * per_sm * kq::kSThreads, p);
   const int64_t grid = (p.threads + kq::kSThreads - 1) / kq::kSThreads;
-  return launch_pdl(kern, dim3(unsigned(grid)), kq::kSThreads, kq::kSSmemBytes, stream, "quant_kernel launch", p);
+  return launch_pdl(kern, dim3(unsigned(grid)), kq::kSThreads, smem, stream, "quant_kernel launch", p);
 }
 
 // Row-tile stride for a grid of ncol column groups on sms SMs holding per_sm
@@ -740,6 +754,32 @@ kq_status kq_adaln_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, co
   p.stats = stats;
   const int threads = p.rows * p.nbw;
   const int nws = p.tree_pad > 32 ? p.tree_pad / 32 : 1;
+  int devid = 0;
+  cudaGetDevice(&devid);
+  if (stats != nullptr) {
+    // two kernels: the statistics into stats, then the butterfly quantizer's ADALN form
+    // reading them (h is formed inside it and never reaches memory)
+    const int ssmem = 2 * p.rows * nws * 4;
+    int per_sm = 0;
+    const cudaError_t eo = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kq::adaln_stats_kernel, threads, ssmem);
+    if (eo != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveBlocksPerMultiprocessor", eo);
+    if (per_sm < 1) return cuda_fail("occupancy: no resident CTA", cudaErrorInvalidConfiguration);
+    kq_status sst;
+    const int64_t sgrid = std::min<int64_t>((M + p.rows - 1) / p.rows, int64_t(dev->sms) * per_sm);
+    sst = launch_pdl(kq::adaln_stats_kernel, dim3(unsigned(sgrid)), threads, ssmem, as_cuda(stream),
+                     "adaln_stats_kernel launch", p);
+    if (sst != KQ_OK) return sst;
+    AdaLnInput ada;
+    ada.stats = stats;
+    ada.shift = p.shift;
+    ada.scale = p.scale;
+    ada.rows_per_group = rows_per_group;
+    return scale_layout == KQ_SCALES_MMA_TILED
+               ? launch_quant<kq::MODE_KRON, 1, 32, true>(x, M, d, ldx, mats, factored, nullptr, q, scales,
+                                                          as_cuda(stream), ada)
+               : launch_quant<kq::MODE_KRON, 0, 32, true>(x, M, d, ldx, mats, factored, nullptr, q, scales,
+                                                          as_cuda(stream), ada);
+  }
   const int smem = (kq::kAlStages + 1) * threads * 64 + 2 * p.rows * nws * 4;
   const int which = scale_layout == KQ_SCALES_MMA_TILED ? 1 : 0;
   auto kern = which ? kq::adaln_quant_kernel<1> : kq::adaln_quant_kernel<0>;
@@ -747,8 +787,6 @@ kq_status kq_adaln_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, co
   constexpr int kMaxSmem = (kq::kAlStages + 1) * kq::kAlMaxThreads * 64 + 2 * 32 * 4;
   if (smem > kMaxSmem || kMaxSmem > dev->smem_optin) return KQ_ERR_UNSUPPORTED;
   static std::atomic<int> attr_set[2][kMaxDevices];
-  int devid = 0;
-  cudaGetDevice(&devid);
   if (!attr_set[which][devid].load()) {
     const cudaError_t ea = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (ea != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", ea);

@@ -63,6 +63,35 @@ constexpr int kSThreads = 256;    // threads per CTA
 constexpr int kSCtasPerSm = 2;    // resident CTAs per SM the register budget is written for
 constexpr int kSStages = 4;       // 64-byte slots per thread (blocks in flight + 1)
 constexpr int kSSmemBytes = kSStages * kSThreads * 64;
+// Dynamic shared memory of quant_kernel: the rings, and with ADALN each thread's staged h
+// block (64 bytes) for the warp-cooperative exact path.
+__host__ __device__ constexpr int quant_smem_bytes(bool adaln) { return kSSmemBytes + (adaln ? kSThreads * 64 : 0); }
+
+// The AdaLN modulation of one block, every step one IEEE binary32 operation rounded to
+// nearest: h_i = bf16( ((x_i - mu) * rstd) * (1 + scale_i) + shift_i ).  X: the block's
+// inputs as packed pairs (elements 2j, 2j+1); sv, hv: its 32 scale and shift values (bf16
+// bits, 16-byte pieces in element order); hw: h as bf16 pairs.  Packed steps are used only
+// where no multiply feeds a packed add (the compiler fuses such a pair into one FMA); the
+// add of the shift is the scalar __fadd_rn, which it never contracts.
+__device__ __forceinline__ void modulate(const uint64_t (&X)[16], float mu, float rstd, const uint4 (&sv)[4],
+                                         const uint4 (&hv)[4], uint32_t (&hw)[16]) {
+  const uint64_t MU = pk2(mu, mu), RS = pk2(rstd, rstd), ONE = pk2(1.0f, 1.0f);
+#pragma unroll
+  for (int k = 0; k < 4; k++) {
+    const uint32_t s4[4] = {sv[k].x, sv[k].y, sv[k].z, sv[k].w}, b4[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
+#pragma unroll
+    for (int m = 0; m < 4; m++) {
+      const int j = 4 * k + m;
+      const uint64_t A = add2_rn(ONE, pk2(bf16lo(s4[m]), bf16hi(s4[m])));
+      float v0, v1;
+      upk2(mul2_rn(mul2_rn(sub2_rn(X[j], MU), RS), A), v0, v1);
+      const float h0 = __fadd_rn(v0, bf16lo(b4[m])), h1 = __fadd_rn(v1, bf16hi(b4[m]));
+      uint32_t out;
+      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(h1), "f"(h0));
+      hw[j] = out;
+    }
+  }
+}
 
 struct QuantParams {
   const uint16_t* x;      // bf16 bits [M][ldx]
@@ -79,6 +108,13 @@ struct QuantParams {
   const float* inv_s;     // SMOOTH: [nb*32]
   uint8_t* q;             // [M][nb*16]
   uint8_t* scales;        // row-major [M][nb], or tiled (scale_index)
+  // ADALN (the quantizer behind an AdaLN-modulated LayerNorm, kq_adaln.cuh): the input
+  // of row r's blocks is h = bf16(((x - mu) * rstd) * (1 + scale[g]) + shift[g]),
+  // g = r / rows_per_group, with (mu, rstd) = stats[r] from the statistics pass
+  const float* stats;     // [M][2]
+  const uint16_t* shift;  // bf16 bits [G][nb * 32]
+  const uint16_t* scale;  // bf16 bits [G][nb * 32]
+  int64_t rows_per_group;
 };
 
 // Coefficients of one block column, held in registers by the thread that owns it.
@@ -351,19 +387,53 @@ __device__ __forceinline__ bool quant_block(const ColCoef& cf, const uint32_t (&
 // stage from the thread's slot base), refill the slot read one step earlier with
 // the block kSStages - 1 rows ahead, quantize, and recompute exactly every block
 // of the warp that the fp32 bound could not certify.
-template <int MODE, int TILED, int NT>
+// ADALN: the block is modulated first (QuantParams); st holds this row's (mu, rstd) and
+// is replaced by the next row step's, loaded one step ahead; hst is this thread's 64-byte
+// staging of h in shared memory.
+template <int MODE, int TILED, int NT, bool ADALN = false>
 __device__ __forceinline__ void row_step(const QuantParams& p, const ColCoef& cf, uint32_t cbase, int sw,
                                          uint32_t slot, uint32_t refill, bool lane_ok, int c, int64_t r, int64_t f,
-                                         int64_t f_end, int64_t f_ahead, const uint16_t* xr, const uint16_t* xi) {
+                                         int64_t f_end, int64_t f_ahead, const uint16_t* xr, const uint16_t* xi,
+                                         float2& st, uint16_t* hst) {
+  const bool act = lane_ok && f < f_end;
+  uint4 sv[4], hv[4];
+  if (ADALN) {
+    // this row's modulation vectors (cached: every row of a group reads the same ones)
+    const int64_t g = act ? r / p.rows_per_group : 0;
+    const uint4* ps = reinterpret_cast<const uint4*>(p.scale + (g * p.nb + c) * kBlock);
+    const uint4* ph = reinterpret_cast<const uint4*>(p.shift + (g * p.nb + c) * kBlock);
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      sv[k] = __ldg(ps + k);
+      hv[k] = __ldg(ph + k);
+    }
+  }
   copy_wait<kSStages - 2>();  // this step's block has landed
   uint32_t cur[16];
   read_slot(cbase + slot, sw, cur);
   if (lane_ok && f + f_ahead < f_end) copy_block_async(cbase + refill, sw, xi);
   copy_commit();
-  const bool act = lane_ok && f < f_end;
   const int64_t fc = act ? f : c;
   uint8_t* qb = p.q + fc * 16;
   uint8_t* sb = p.scales + (TILED ? scale_index(act ? r : 0, c, p.nb, 1) : fc);
+  if (ADALN) {
+    const float2 sr = st;
+    const int64_t rn = r + p.k;  // the lane's next row
+    if (lane_ok && rn < p.M) st = __ldg(reinterpret_cast<const float2*>(p.stats) + rn);
+    uint64_t X[16];
+#pragma unroll
+    for (int j = 0; j < 16; j++) X[j] = pk2(bf16lo(cur[j]), bf16hi(cur[j]));
+    modulate(X, sr.x, sr.y, sv, hv, cur);
+    uint4* hs = reinterpret_cast<uint4*>(hst);
+#pragma unroll
+    for (int k = 0; k < 4; k++) hs[k] = make_uint4(cur[4 * k], cur[4 * k + 1], cur[4 * k + 2], cur[4 * k + 3]);
+    const bool need = quant_block<MODE, NT>(cf, cur, act, qb, sb);
+    if (__any_sync(0xFFFFFFFFu, need)) {
+      __syncwarp();  // every lane's staged h is visible to the warp
+      warp_exact_pass<KSRC_F32, NT, false>(need, hst, p.mats + kmat_offset<NT>(c), qb, sb);
+    }
+    return;
+  }
   const bool need = quant_block<MODE, NT>(cf, cur, act, qb, sb);
   if (MODE != MODE_SMOOTH && __any_sync(0xFFFFFFFFu, need)) {
     // rare: the transform block's first input and this block's columns of its matrix
@@ -377,13 +447,17 @@ __device__ __forceinline__ void row_step(const QuantParams& p, const ColCoef& cf
 // TILED: scales in the 128 x 4 tiled layout of block-scaled GEMMs (a template
 // parameter, so the row-major store costs nothing extra).  NT: transform block of
 // 16, 32, 64 or 128 elements (KRON only; n > 32 needs d % n == 0).
-template <int MODE, int TILED, int NT>
+// ADALN (KRON, 32-element blocks only): the quantizer of kq_adaln_quantize's two-kernel
+// form, on h formed from x, the statistics pass's (mu, rstd) and the modulation vectors.
+template <int MODE, int TILED, int NT, bool ADALN = false>
 __global__ void __launch_bounds__(kSThreads, kSCtasPerSm) quant_kernel(const __grid_constant__ QuantParams p) {
+  static_assert(!ADALN || (MODE == MODE_KRON && NT == kBlock), "the AdaLN prologue serves KroQuant's 32-element blocks");
   static_assert(kSStages == 4, "the row loop below is written for a ring of four slots");
   extern __shared__ __align__(128) uint8_t ring[];
   const int64_t t = int64_t(blockIdx.x) * kSThreads + threadIdx.x;
   const int sw = (threadIdx.x >> 1) & 3;
   const uint32_t cbase = smem_addr(ring) + threadIdx.x * 64u;
+  uint16_t* hst = reinterpret_cast<uint16_t*>(ring + kSSmemBytes) + threadIdx.x * kBlock;  // ADALN only
   constexpr uint32_t kStage = kSThreads * 64u;  // bytes between the stages of one thread's ring
   grid_dependency_wait();  // inputs may come from the previous kernel in the stream
   for (int pass = 0; pass < p.passes; pass++) {
@@ -407,17 +481,19 @@ __global__ void __launch_bounds__(kSThreads, kSCtasPerSm) quant_kernel(const __g
     if (pass == 0) grid_launch_dependents();
     ColCoef cf;
     load_coef<MODE, NT>(p, c, cf);
+    float2 st = make_float2(0.0f, 0.0f);  // ADALN: (mu, rstd) of the lane's current row
+    if (ADALN && lane_ok && r0 < p.M) st = __ldg(reinterpret_cast<const float2*>(p.stats) + r0);
     const int64_t f_ahead = (kSStages - 1) * fstep;
     const uint16_t* xi = xr + (kSStages - 1) * xstep;  // next block to put in flight
     // two row steps per trip: step i uses stage i & 3, so the pair (i, i + 1) uses
     // stages (h, h + 1) with h = 0 or 2 and refills (h + 3, h) & 3
     uint32_t h = 0;
     for (int64_t i = 0; i < p.n_iter; i += 2) {
-      row_step<MODE, TILED, NT>(p, cf, cbase, sw, h, (h + 3 * kStage) & (4 * kStage - 1), lane_ok, c, r, f, f_end,
-                                f_ahead, xr, xi);
+      row_step<MODE, TILED, NT, ADALN>(p, cf, cbase, sw, h, (h + 3 * kStage) & (4 * kStage - 1), lane_ok, c, r, f,
+                                       f_end, f_ahead, xr, xi, st, hst);
       if (i + 1 < p.n_iter)
-        row_step<MODE, TILED, NT>(p, cf, cbase, sw, h + kStage, h, lane_ok, c, r + p.k, f + fstep, f_end, f_ahead,
-                                  xr + xstep, xi + xstep);
+        row_step<MODE, TILED, NT, ADALN>(p, cf, cbase, sw, h + kStage, h, lane_ok, c, r + p.k, f + fstep, f_end,
+                                         f_ahead, xr + xstep, xi + xstep, st, hst);
       h ^= 2 * kStage;
       r += 2 * p.k;
       f += 2 * fstep;

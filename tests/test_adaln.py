@@ -41,8 +41,13 @@ def modulation(G: int, d: int, seed) -> tuple[np.ndarray, np.ndarray]:
     return shift, scale
 
 
-def run(kq, x, shift, scale, rpg, params, eps=1e-6, layout="row"):
-    """Device codes, scales and statistics, each inside canary bytes."""
+FORMS = ("two_kernel", "fused")
+
+
+def run(kq, x, shift, scale, rpg, params, eps=1e-6, layout="row", form="two_kernel"):
+    """Device codes, scales and statistics, each inside canary bytes.  form: "two_kernel"
+    asks for the statistics (the statistics pass, then the butterfly quantizer's AdaLN
+    form); "fused" passes none (one fused kernel), and the statistics come back None."""
     M, d = x.shape
     bt = kq.BlockTransform(torch.from_numpy(params).cuda())
     qv, qbuf = guarded(torch, M * (d // 2))
@@ -52,14 +57,14 @@ def run(kq, x, shift, scale, rpg, params, eps=1e-6, layout="row"):
     tv, tbuf = guarded(torch, M * 8)
     q = qv.view(M, d // 2)
     s = sv.view(M, d // 32) if layout == "row" else sv
-    st = tv.view(torch.float32).view(M, 2)
+    st = tv.view(torch.float32).view(M, 2) if form == "two_kernel" else None
     bt.adaln_quantize(dev_bits(x), dev_bits(shift), dev_bits(scale), rpg, eps=eps, q=q, scales=s,
                       scale_layout=layout, stats=st)
     torch.cuda.synchronize()
     for b in (qbuf, sbuf, tbuf):
         assert guards_intact(torch, b), "a kernel wrote outside its output buffer"
     assert kq.kq_get_device_error(clear=True) == 0
-    return q.cpu().numpy(), s.cpu().numpy(), st.cpu().numpy()
+    return q.cpu().numpy(), s.cpu().numpy(), None if st is None else st.cpu().numpy()
 
 
 def oracle(orc, x, shift, scale, rpg, params, eps=1e-6):
@@ -80,10 +85,11 @@ def test_adaln_flux_every_row(kq, orc, d):
     """FLUX-shaped rows (4608 tokens in two samples of 2304), every row."""
     x, params = inputs.config_case("flux", d)
     shift, scale = modulation(2, d, seed=[d, 1])
-    q, s, st = run(kq, x, shift, scale, 2304, params)
     qr, sr, str_ = oracle(orc, x, shift, scale, 2304, params)
-    assert same_stats(st, str_)
-    assert np.array_equal(s, sr) and np.array_equal(q, qr)
+    for form in FORMS:
+        q, s, st = run(kq, x, shift, scale, 2304, params, form=form)
+        assert st is None or same_stats(st, str_), form
+        assert np.array_equal(s, sr) and np.array_equal(q, qr), form
 
 
 @pytest.mark.parametrize("M,d,rpg", [(1, 32, 1), (7, 96, 3), (130, 1152, 64), (33, 2240, 5), (20, 5600, 7),
@@ -94,10 +100,11 @@ def test_adaln_ragged_shapes(kq, orc, M, d, rpg):
     x = inputs.activations(M, d, "t3", seed=[M, d, 2], outlier_frac=0.01, outlier_scale=(20.0, 100.0))
     params = inputs.lu_params(d // 32, seed=[M, d, 3])
     shift, scale = modulation(-(-M // rpg), d, seed=[M, d, 4])
-    q, s, st = run(kq, x, shift, scale, rpg, params)
     qr, sr, str_ = oracle(orc, x, shift, scale, rpg, params)
-    assert same_stats(st, str_)
-    assert np.array_equal(s, sr) and np.array_equal(q, qr)
+    for form in FORMS:
+        q, s, st = run(kq, x, shift, scale, rpg, params, form=form)
+        assert st is None or same_stats(st, str_), form
+        assert np.array_equal(s, sr) and np.array_equal(q, qr), form
 
 
 def test_adaln_tiled_scales(kq, orc):
@@ -105,9 +112,10 @@ def test_adaln_tiled_scales(kq, orc):
     x = inputs.activations(M, d, "normal", seed=5, outlier_frac=0.01)
     params = inputs.lu_params(d // 32, seed=6)
     shift, scale = modulation(3, d, seed=7)
-    q, s, _ = run(kq, x, shift, scale, rpg, params, layout="mma")
     qr, sr, _ = oracle(orc, x, shift, scale, rpg, params)
-    assert np.array_equal(q, qr) and np.array_equal(s, tiled_scales(sr))
+    for form in FORMS:
+        q, s, _ = run(kq, x, shift, scale, rpg, params, layout="mma", form=form)
+        assert np.array_equal(q, qr) and np.array_equal(s, tiled_scales(sr)), form
 
 
 def test_adaln_degenerate_rows(kq, orc):
@@ -127,10 +135,11 @@ def test_adaln_degenerate_rows(kq, orc):
     params = inputs.lu_params(d // 32, seed=9)
     shift, scale = modulation(1, d, seed=10)
     for eps in (1e-6, 0.0):
-        q, s, st = run(kq, x, shift, scale, 10, params, eps=eps)
         qr, sr, str_ = oracle(orc, x, shift, scale, 10, params, eps=eps)
-        assert same_stats(st, str_), eps
-        assert np.array_equal(s, sr) and np.array_equal(q, qr), eps
+        for form in FORMS:
+            q, s, st = run(kq, x, shift, scale, 10, params, eps=eps, form=form)
+            assert st is None or same_stats(st, str_), (eps, form)
+            assert np.array_equal(s, sr) and np.array_equal(q, qr), (eps, form)
 
 
 def test_adaln_without_stats_and_binding_checks(kq, orc):
