@@ -160,17 +160,17 @@ struct AdaLnInput {
   int64_t rows_per_group = 1;
 };
 
-template <int MODE, int TILED, int NT = 32, bool ADALN = false>
-kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const float* mats, const float* factored,
-                       const float* inv_s, uint8_t* q, uint8_t* scales, cudaStream_t stream,
-                       const AdaLnInput& ada = AdaLnInput()) {
+template <int MODE, int TILED, int NT, bool ADALN, bool GROUPED>
+kq_status launch_quant_impl(const void* x, int64_t M, int64_t d, int64_t ldx, const float* mats,
+                            const float* factored, const float* inv_s, uint8_t* q, uint8_t* scales,
+                            cudaStream_t stream, const AdaLnInput& ada) {
   const DeviceInfo* dev = device_info();
   if (dev == nullptr) return cuda_fail("device query", cudaErrorInvalidDevice);
   int devid = 0;
   cudaGetDevice(&devid);
   const int64_t nb = d / 32;
-  void (*kern)(const kq::QuantParams) = kq::quant_kernel<MODE, TILED, NT, ADALN>;
-  constexpr int smem = kq::quant_smem_bytes(ADALN);
+  void (*kern)(const kq::QuantParams) = kq::quant_kernel<MODE, TILED, NT, ADALN, GROUPED>;
+  constexpr int smem = kq::quant_smem_bytes(ADALN, GROUPED);
   static std::atomic<int> attr_set[kMaxDevices];
   if (!attr_set[devid].load()) {
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -195,9 +195,70 @@ kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const f
   p.inv_s = inv_s;
   p.q = q;
   p.scales = scales;
-  lane_layout(M, nb, int64_t(dev->sms) * per_sm * kq::kSThreads, p);
-  const int64_t grid = (p.threads + kq::kSThreads - 1) / kq::kSThreads;
+  p.cg = 0;
+  int64_t grid = 0;
+  if (GROUPED) {
+    // CTAs of 8 row residues x one group of 32 columns: fill the resident slots once
+    // (at least one CTA row), then lower the residue count k to the smallest with the same
+    // number of row steps, as lane_layout does
+    constexpr int64_t kWarps = kq::kSThreads / 32;
+    const int64_t cg = nb / 32;
+    const int64_t krow = std::max<int64_t>(1, int64_t(dev->sms) * per_sm / cg);
+    int64_t k = std::min<int64_t>(krow * kWarps, M);
+    p.n_iter = (M + k - 1) / k;
+    k = (M + p.n_iter - 1) / p.n_iter;
+    p.cg = int(cg);
+    p.k = k;
+    p.lanes = k * nb;
+    p.passes = 1;
+    grid = (k + kWarps - 1) / kWarps * cg;
+    p.threads = grid * kq::kSThreads;
+  } else {
+    lane_layout(M, nb, int64_t(dev->sms) * per_sm * kq::kSThreads, p);
+    grid = (p.threads + kq::kSThreads - 1) / kq::kSThreads;
+  }
   return launch_pdl(kern, dim3(unsigned(grid)), kq::kSThreads, smem, stream, "quant_kernel launch", p);
+}
+
+// Row steps per thread from which the grouped layout is taken.  Measured back to back at
+// M = 4608: 24 steps (d = 12288) 37.4 against 38.1 us; 6 steps (d = 3072) 17.9 against
+// 17.0 us, where the layout's start (the shared table's fill and one barrier) is not
+// amortised.  The AdaLN form was slower grouped at both widths (105.5 against 102.2 us).
+constexpr int64_t kGroupedMinSteps = 16;
+
+// The butterfly / comparison quantizer kernels.  KroQuant with 32-element blocks takes the
+// grouped layout when d is a multiple of 1024 (whole groups of 32 block columns) and each
+// thread walks at least kGroupedMinSteps rows.
+template <int MODE, int TILED, int NT = 32, bool ADALN = false>
+kq_status launch_quant(const void* x, int64_t M, int64_t d, int64_t ldx, const float* mats, const float* factored,
+                       const float* inv_s, uint8_t* q, uint8_t* scales, cudaStream_t stream,
+                       const AdaLnInput& ada = AdaLnInput()) {
+  if constexpr (MODE == kq::MODE_KRON && NT == 32 && !ADALN) {
+    const int64_t nb = d / 32;
+    const DeviceInfo* dev = device_info();
+    if (nb % 32 == 0 && dev != nullptr) {
+      int devid = 0;
+      cudaGetDevice(&devid);
+      void (*gkern)(const kq::QuantParams) = kq::quant_kernel<MODE, TILED, NT, false, true>;
+      constexpr int gsmem = kq::quant_smem_bytes(false, true);
+      static std::atomic<int> gattr_set[kMaxDevices];
+      if (!gattr_set[devid].load()) {  // before the occupancy query, which counts the shared memory
+        const cudaError_t e = cudaFuncSetAttribute(gkern, cudaFuncAttributeMaxDynamicSharedMemorySize, gsmem);
+        if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(MaxDynamicSharedMemorySize)", e);
+        gattr_set[devid].store(1);
+      }
+      int per_sm = 0;
+      const kq_status st = resident_ctas(reinterpret_cast<const void*>(gkern), kq::kSThreads, gsmem, devid, &per_sm);
+      if (st != KQ_OK) return st;
+      const int64_t krow = std::max<int64_t>(1, int64_t(dev->sms) * per_sm / (nb / 32));
+      const int64_t k = std::min<int64_t>(krow * (kq::kSThreads / 32), M);
+      if ((M + k - 1) / k >= kGroupedMinSteps)
+        return launch_quant_impl<MODE, TILED, NT, ADALN, true>(x, M, d, ldx, mats, factored, inv_s, q, scales,
+                                                               stream, ada);
+    }
+  }
+  return launch_quant_impl<MODE, TILED, NT, ADALN, false>(x, M, d, ldx, mats, factored, inv_s, q, scales, stream,
+                                                          ada);
 }
 
 // Row-tile stride for a grid of ncol column groups on sms SMs holding per_sm

@@ -63,9 +63,13 @@ constexpr int kSThreads = 256;    // threads per CTA
 constexpr int kSCtasPerSm = 2;    // resident CTAs per SM the register budget is written for
 constexpr int kSStages = 4;       // 64-byte slots per thread (blocks in flight + 1)
 constexpr int kSSmemBytes = kSStages * kSThreads * 64;
+constexpr int kDTableBytes = 32 * kBlock * 4;  // D of the 32 block columns a grouped CTA covers
 // Dynamic shared memory of quant_kernel: the rings, and with ADALN each thread's staged h
 // block (64 bytes) for the warp-cooperative exact path.
-__host__ __device__ constexpr int quant_smem_bytes(bool adaln) { return kSSmemBytes + (adaln ? kSThreads * 64 : 0); }
+// GROUPED adds the CTA's table of D (32 block columns x 32 fp32).
+__host__ __device__ constexpr int quant_smem_bytes(bool adaln, bool grouped = false) {
+  return kSSmemBytes + (adaln ? kSThreads * 64 : 0) + (grouped ? kDTableBytes : 0);
+}
 
 // The AdaLN modulation of one block, every step one IEEE binary32 operation rounded to
 // nearest: h_i = bf16( ((x_i - mu) * rstd) * (1 + scale_i) + shift_i ).  X: the block's
@@ -103,6 +107,7 @@ struct QuantParams {
   int64_t n_iter;         // row steps per lane: ceil(M / k)
   int passes;             // lanes per thread: ceil(lanes / threads)
   int nb;                 // blocks per row (d / 32)
+  int cg;                 // grouped layout (quant_kernel GROUPED): column groups of 32, nb / 32
   const float* mats;      // KRON: fp32 [nb/(NT/32)][NT][NT] (exact path)
   const float* factored;  // KRON: [nb][48]
   const float* inv_s;     // SMOOTH: [nb*32]
@@ -255,9 +260,11 @@ __device__ __forceinline__ void read_slot(uint32_t slot, int sw, uint32_t (&w)[1
 // act marks the lanes whose block is real.  Stores the fast result of a real
 // block and returns whether it must be recomputed exactly (never for SMOOTH, whose
 // fp32 product is the definition itself).
-template <int MODE, int NT>
+// DSH: D comes from the CTA's shared table (grouped layout), this lane's entries at
+// shared address dsh + 512 i (i = 0..7, 16 bytes each: D_4i .. D_4i+3), not from cf.D.
+template <int MODE, int NT, bool DSH = false>
 __device__ __forceinline__ bool quant_block(const ColCoef& cf, const uint32_t (&w)[16], bool act, uint8_t* qb,
-                                            uint8_t* sb) {
+                                            uint8_t* sb, uint32_t dsh = 0u) {
   float x[kBlock];
 #pragma unroll
   for (int h = 0; h < 16; h++) {
@@ -368,6 +375,12 @@ __device__ __forceinline__ bool quant_block(const ColCoef& cf, const uint32_t (&
     if (MODE == MODE_FWHT) {
       const float sg = (__popc(m) & 1) ? -kFwhtC : kFwhtC;
       Y[m] = mul2_rn(pk2(sg, -sg), Y[m]);
+    } else if (DSH) {
+      if ((m & 1) == 0) {
+        const uint4 v = lds128(dsh + uint32_t(m / 2) * 512u);
+        Y[m] = mul2_rn((uint64_t(v.y) << 32) | v.x, Y[m]);
+        Y[m + 1] = mul2_rn((uint64_t(v.w) << 32) | v.z, Y[m + 1]);
+      }
     } else {
       Y[m] = mul2_rn(cf.D[m], Y[m]);
     }
@@ -390,11 +403,11 @@ __device__ __forceinline__ bool quant_block(const ColCoef& cf, const uint32_t (&
 // ADALN: the block is modulated first (QuantParams); st holds this row's (mu, rstd) and
 // is replaced by the next row step's, loaded one step ahead; hst is this thread's 64-byte
 // staging of h in shared memory.
-template <int MODE, int TILED, int NT, bool ADALN = false>
+template <int MODE, int TILED, int NT, bool ADALN = false, bool GROUPED = false>
 __device__ __forceinline__ void row_step(const QuantParams& p, const ColCoef& cf, uint32_t cbase, int sw,
                                          uint32_t slot, uint32_t refill, bool lane_ok, int c, int64_t r, int64_t f,
                                          int64_t f_end, int64_t f_ahead, const uint16_t* xr, const uint16_t* xi,
-                                         float2& st, uint16_t* hst) {
+                                         float2& st, uint16_t* hst, uint32_t dsh) {
   const bool act = lane_ok && f < f_end;
   uint4 sv[4], hv[4];
   if (ADALN) {
@@ -427,14 +440,14 @@ __device__ __forceinline__ void row_step(const QuantParams& p, const ColCoef& cf
     uint4* hs = reinterpret_cast<uint4*>(hst);
 #pragma unroll
     for (int k = 0; k < 4; k++) hs[k] = make_uint4(cur[4 * k], cur[4 * k + 1], cur[4 * k + 2], cur[4 * k + 3]);
-    const bool need = quant_block<MODE, NT>(cf, cur, act, qb, sb);
+    const bool need = quant_block<MODE, NT, GROUPED>(cf, cur, act, qb, sb, dsh);
     if (__any_sync(0xFFFFFFFFu, need)) {
       __syncwarp();  // every lane's staged h is visible to the warp
       warp_exact_pass<KSRC_F32, NT, false>(need, hst, p.mats + kmat_offset<NT>(c), qb, sb);
     }
     return;
   }
-  const bool need = quant_block<MODE, NT>(cf, cur, act, qb, sb);
+  const bool need = quant_block<MODE, NT, GROUPED>(cf, cur, act, qb, sb, dsh);
   if (MODE != MODE_SMOOTH && __any_sync(0xFFFFFFFFu, need)) {
     // rare: the transform block's first input and this block's columns of its matrix
     const uint16_t* xb = xr - (c - first_column<NT>(c)) * kBlock;
@@ -449,23 +462,41 @@ __device__ __forceinline__ void row_step(const QuantParams& p, const ColCoef& cf
 // 16, 32, 64 or 128 elements (KRON only; n > 32 needs d % n == 0).
 // ADALN (KRON, 32-element blocks only): the quantizer of kq_adaln_quantize's two-kernel
 // form, on h formed from x, the statistics pass's (mu, rstd) and the modulation vectors.
-template <int MODE, int TILED, int NT, bool ADALN = false>
+// GROUPED (KRON, 32-element blocks, nb % 32 == 0): CTA b covers the 32 block columns of
+// group b % cg for 8 row residues, warp w taking residue (b / cg) 8 + w and lane l column
+// 32 (b % cg) + l, so the 8 warps share their columns' D, which one warp puts in a
+// shared table once (32 fewer live registers per thread), and their matrices for the
+// exact pass.  One lane pass per thread (passes = 1).
+template <int MODE, int TILED, int NT, bool ADALN = false, bool GROUPED = false>
 __global__ void __launch_bounds__(kSThreads, kSCtasPerSm) quant_kernel(const __grid_constant__ QuantParams p) {
   static_assert(!ADALN || (MODE == MODE_KRON && NT == kBlock), "the AdaLN prologue serves KroQuant's 32-element blocks");
+  static_assert(!GROUPED || (MODE == MODE_KRON && NT == kBlock), "the grouped layout serves KroQuant's 32-element blocks");
   static_assert(kSStages == 4, "the row loop below is written for a ring of four slots");
   extern __shared__ __align__(128) uint8_t ring[];
   const int64_t t = int64_t(blockIdx.x) * kSThreads + threadIdx.x;
   const int sw = (threadIdx.x >> 1) & 3;
   const uint32_t cbase = smem_addr(ring) + threadIdx.x * 64u;
   uint16_t* hst = reinterpret_cast<uint16_t*>(ring + kSSmemBytes) + threadIdx.x * kBlock;  // ADALN only
+  // GROUPED: this lane's column in the CTA's D table
+  const uint32_t dsh = smem_addr(ring) + uint32_t(quant_smem_bytes(ADALN)) + (threadIdx.x & 31) * 16u;
   constexpr uint32_t kStage = kSThreads * 64u;  // bytes between the stages of one thread's ring
   grid_dependency_wait();  // inputs may come from the previous kernel in the stream
   for (int pass = 0; pass < p.passes; pass++) {
-    const int64_t v = t + int64_t(pass) * p.threads;
-    const bool lane_ok = t < p.threads && v < p.lanes;
-    const int64_t vc = lane_ok ? v : 0;
-    const int c = int(vc % p.nb);
-    const int64_t r0 = vc / p.nb;
+    bool lane_ok;
+    int c;
+    int64_t r0;
+    if (GROUPED) {
+      const int64_t rr = int64_t(blockIdx.x / unsigned(p.cg)) * (kSThreads / 32) + (threadIdx.x >> 5);
+      lane_ok = rr < p.k;
+      c = int(blockIdx.x % unsigned(p.cg)) * 32 + (threadIdx.x & 31);
+      r0 = lane_ok ? rr : 0;
+    } else {
+      const int64_t v = t + int64_t(pass) * p.threads;
+      lane_ok = t < p.threads && v < p.lanes;
+      const int64_t vc = lane_ok ? v : 0;
+      c = int(vc % p.nb);
+      r0 = vc / p.nb;
+    }
     const int64_t xstep = p.k * p.ldx;
     const int64_t fstep = p.k * int64_t(p.nb);
     const int64_t f_end = p.M * int64_t(p.nb);  // row r is real iff its flat index r nb + c < f_end
@@ -481,6 +512,17 @@ __global__ void __launch_bounds__(kSThreads, kSCtasPerSm) quant_kernel(const __g
     if (pass == 0) grid_launch_dependents();
     ColCoef cf;
     load_coef<MODE, NT>(p, c, cf);
+    if (GROUPED) {
+      // every warp of the CTA has the same 32 columns: warp 0 fills the table
+      if (threadIdx.x < 32) {
+#pragma unroll
+        for (int m = 0; m < 16; m += 2)
+          asm volatile("st.shared.v2.b64 [%0], {%1, %2};" ::"r"(dsh + uint32_t(m / 2) * 512u), "l"(cf.D[m]),
+                       "l"(cf.D[m + 1])
+                       : "memory");
+      }
+      __syncthreads();
+    }
     float2 st = make_float2(0.0f, 0.0f);  // ADALN: (mu, rstd) of the lane's current row
     if (ADALN && lane_ok && r0 < p.M) st = __ldg(reinterpret_cast<const float2*>(p.stats) + r0);
     const int64_t f_ahead = (kSStages - 1) * fstep;
@@ -489,11 +531,11 @@ __global__ void __launch_bounds__(kSThreads, kSCtasPerSm) quant_kernel(const __g
     // stages (h, h + 1) with h = 0 or 2 and refills (h + 3, h) & 3
     uint32_t h = 0;
     for (int64_t i = 0; i < p.n_iter; i += 2) {
-      row_step<MODE, TILED, NT, ADALN>(p, cf, cbase, sw, h, (h + 3 * kStage) & (4 * kStage - 1), lane_ok, c, r, f,
-                                       f_end, f_ahead, xr, xi, st, hst);
+      row_step<MODE, TILED, NT, ADALN, GROUPED>(p, cf, cbase, sw, h, (h + 3 * kStage) & (4 * kStage - 1), lane_ok,
+                                                c, r, f, f_end, f_ahead, xr, xi, st, hst, dsh);
       if (i + 1 < p.n_iter)
-        row_step<MODE, TILED, NT, ADALN>(p, cf, cbase, sw, h + kStage, h, lane_ok, c, r + p.k, f + fstep, f_end,
-                                         f_ahead, xr + xstep, xi + xstep, st, hst);
+        row_step<MODE, TILED, NT, ADALN, GROUPED>(p, cf, cbase, sw, h + kStage, h, lane_ok, c, r + p.k, f + fstep,
+                                                  f_end, f_ahead, xr + xstep, xi + xstep, st, hst, dsh);
       h ^= 2 * kStage;
       r += 2 * p.k;
       f += 2 * fstep;
