@@ -36,7 +36,8 @@
 // 6 roundings on each output's path (5 FMA stages, 1 multiply by D) give 6u;
 // the fp32 coefficients (5 ratios and D_j, each rounded once) put the applied
 // matrix within 6u of K, K32 is within u of K, and y32 is one more rounding:
-// 14u in all (u = 2^-24), against C = 16u.  FWHT: 6 roundings + the final one
+// 14u in all (u = 2^-24) to first order; with the second-order terms of those products
+// of (1 + u) factors, 14u + 109u^2, against C = 14u (1 + 2^-16).  FWHT: 6 roundings + the final one
 // = 7u (its coefficients are exactly the entries of fp32(H32)), against 8u.
 // ||x||_1 is summed with upward rounding and max|K| is rounded up.  The scale is taken
 // from y_f only when max|y| +- E has one E8M0 exponent, and each code only when
@@ -54,7 +55,7 @@ namespace kq {
 
 enum Mode { MODE_KRON = 0, MODE_FWHT = 1, MODE_SMOOTH = 2 };
 
-constexpr float kKronErrC = 9.5367431640625e-07f;   // 2^-20 = 16 u (14 u needed, see above; 12 u for 16-element blocks)
+constexpr float kKronErrC = 8.344777597812936e-07f; // 14 u (1 + 2^-16), exact in fp32 (14 u + 109 u^2 needed, see above; 12 u for 16-element blocks)
 constexpr float kKronErrC64 = 1.9073486328125e-06f; // 2^-19 = 32 u for 64- and 128-element blocks (16 u, 18 u needed)
 constexpr float kFwhtErrC = 4.76837158203125e-07f;  // 2^-21 = 8 u (7 u needed)
 constexpr float kErrAbs = 7.174648137343064e-43f;   // 2^-140: FWHT subnormal-range slack
