@@ -825,10 +825,10 @@ kq_status kq_adaln_quantize(const void* x, int64_t M, int64_t d, int64_t ldx, co
     const cudaError_t eo = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kq::adaln_stats_kernel, threads, ssmem);
     if (eo != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveBlocksPerMultiprocessor", eo);
     if (per_sm < 1) return cuda_fail("occupancy: no resident CTA", cudaErrorInvalidConfiguration);
-    kq_status sst;
+    // one wave: every statistics CTA is resident before the quantizer's CTAs may launch
     const int64_t sgrid = std::min<int64_t>((M + p.rows - 1) / p.rows, int64_t(dev->sms) * per_sm);
-    sst = launch_pdl(kq::adaln_stats_kernel, dim3(unsigned(sgrid)), threads, ssmem, as_cuda(stream),
-                     "adaln_stats_kernel launch", p);
+    const kq_status sst = launch_pdl(kq::adaln_stats_kernel, dim3(unsigned(sgrid)), threads, ssmem,
+                                     as_cuda(stream), "adaln_stats_kernel launch", p);
     if (sst != KQ_OK) return sst;
     AdaLnInput ada;
     ada.stats = stats;
