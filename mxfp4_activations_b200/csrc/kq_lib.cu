@@ -553,7 +553,7 @@ struct AutoRule {
   kq_variant v;
 };
 constexpr AutoRule kAutoTable[] = {
-    {1, 1152, KQ_VAR_MMA},            {1, 3072, KQ_VAR_BUTTERFLY},      {1, 12288, KQ_VAR_BUTTERFLY},
+    {1, 1152, KQ_VAR_MMA},            {1, 3072, KQ_VAR_MMA},            {1, 12288, KQ_VAR_BUTTERFLY},
     {16, 1152, KQ_VAR_BUTTERFLY},     {16, 3072, KQ_VAR_BUTTERFLY},     {16, 12288, KQ_VAR_BUTTERFLY},
     {256, 1152, KQ_VAR_BUTTERFLY},    {256, 3072, KQ_VAR_BUTTERFLY},    {256, 12288, KQ_VAR_BUTTERFLY},
     {4096, 1152, KQ_VAR_BUTTERFLY},   {4096, 3072, KQ_VAR_BUTTERFLY},   {4096, 12288, KQ_VAR_BUTTERFLY},
